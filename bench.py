@@ -1,0 +1,400 @@
+"""Benchmark of the RG-LRU layer on B200: channel-tokens/s and achieved HBM GB/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--algo auto]
+    python bench.py --impl reference ...      # the float64 CPU oracle on a bounded sample
+
+A step is one rglru_fwd over the whole workload (Conv1D, gates, decay, scan
+and the time-split carry), inputs resident in HBM. The timed region is K
+back-to-back steps between CUDA events on the launching stream, after W
+untimed warm-up steps; each step reads and writes its own buffer set, and the
+sets rotate so that the bytes touched between two uses of one set exceed 3x
+the 126 MB L2 (no step finds its inputs in L2). Under torchrun every rank
+runs the same workload on its own GPU (weak scaling over independent
+batches, no collective on the data path); the time is the max over ranks.
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_linear_recurrence_rglru_b200.workloads import WORKLOADS, generate  # noqa: E402
+
+L2_BYTES = 126 * 2**20
+METRIC = "RG-LRU channel-tokens/s and achieved HBM GB/s vs B200 peak (1 GPU)"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# --------------------------------------------------------------- clocks ----
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu_index = gpu_index
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "power_w_max": max(power) if power else None, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------- our arm ----
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, ws: int) -> float:
+    if ws == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def fwd_bytes_per_chtok(wl) -> int:
+    """Algorithmic HBM bytes per channel-token of the fused forward: read x, write y."""
+    return 2 * (4 if wl.io == "f32" else 2)
+
+
+def run_ours(a, ws, rank, local):
+    import gated_linear_recurrence_rglru_b200 as rg
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = WORKLOADS[a.workload]
+    if wl.decode_steps:
+        raise SystemExit("--workload must be a forward workload; decode is reported as 'decode'")
+    t = generate(wl)
+    g = {k: (v.to(dev) if v is not None else None) for k, v in t.items()}
+    w = [g[k] for k in ("conv_w", "W_a", "b_a", "W_x", "b_x", "Lambda")]
+    B, T, D, H = wl.B, wl.T, wl.D, wl.H
+    esz = 4 if wl.io == "f32" else 2
+    set_bytes = 2 * B * T * D * esz
+    nsets = max(2, math.ceil(3 * L2_BYTES / set_bytes) + 1)
+    xs = [g["x"]] + [g["x"].clone() for _ in range(nsets - 1)]
+    ys = [torch.empty_like(g["x"]) for _ in range(nsets)]
+    hT = [torch.empty(B, D, device=dev) for _ in range(nsets)]
+    cs = [torch.empty(B, 3, D, device=dev, dtype=wl.dtype) for _ in range(nsets)]
+    wsb = rg.fwd_workspace_bytes(B, T, D, H, wl.dtype)
+    work = [torch.empty(max(wsb, 1), device=dev, dtype=torch.uint8) for _ in range(nsets)]
+    status = torch.zeros(1, device=dev, dtype=torch.int32)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        k = i % nsets
+        rg.rglru_fwd(xs[k], *w, h0=g["h0"], y=ys[k], h_T=hT[k], conv_state_out=cs[k],
+                     workspace=work[k], dev_status=status, algo=a.algo)
+
+    # soak (untimed) so that the clock sampler sees this load around the timed region
+    sampler = ClockSampler(local)
+    soak_t0 = time.time()
+    i = 0
+    while time.time() - soak_t0 < a.soak_s:
+        for _ in range(50):
+            step(i)
+            i += 1
+        torch.cuda.synchronize()
+    for _ in range(a.warmup):
+        step(i)
+        i += 1
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(a.steps):
+        step(i)
+        i += 1
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    ms_local = e0.elapsed_time(e1)
+    post_t0 = time.time()
+    while time.time() - post_t0 < a.soak_s:
+        for _ in range(50):
+            step(i)
+            i += 1
+        torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if int(status.item()) != 0:
+        raise SystemExit(f"device status {int(status.item())}: {rg.status_str(int(status.item()))}")
+    ms = max_over_ranks(ms_local, ws)
+    ms_step = ms / a.steps
+    chtok = B * T * D
+    value = ws * chtok * a.steps / (ms / 1e3)
+    pk = peaks()
+    bytes_step = fwd_bytes_per_chtok(wl) * chtok
+    achieved = bytes_step / (ms_step / 1e3) / 1e9
+    launches_per_step = rg.fwd_launches(B, T, D, H, wl.dtype, a.algo)
+
+    out = {
+        "metric": METRIC, "value": value, "unit": "channel-tokens/s", "n_gpus": ws,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.io, "data": "synthetic (seeded; recipe of the workload)",
+        "config": {"workload": f"{wl.name} B={B} T={T} D={D} H={H} bw={wl.bw} io={wl.io}",
+                   "algo": a.algo, "global_batch": B * ws, "seq_len": T,
+                   "parallelism": f"dp{ws} (independent batches)",
+                   "l2": f"{nsets} rotating buffer sets of {set_bytes / 1e6:.1f} MB "
+                         f"(>3x L2 between reuses)"},
+        "hbm_gbs": achieved,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                     "kernel": "whole step (all launches of one rglru_fwd)",
+                     "peak_source": pk["source"],
+                     "algorithmic_bytes_per_launch": bytes_step},
+        "gpu_launches": launches_per_step * a.steps,
+        "clocks": clocks,
+    }
+    if a.e2e:
+        out["e2e"] = run_e2e(rg, wl, g, w, dev, a)
+        # e2e of every rank is the same program; report rank-max time via value already local
+    if a.decode:
+        out["decode"] = run_decode(rg, dev, a, pk)
+    if a.cpu_baseline and ws == 1 and rank == 0:
+        out["cpu_baseline"] = cpu_baseline(wl, t, a.cpu_seconds)
+    return out
+
+
+def run_e2e(rg, wl, g, w, dev, a):
+    """Same metric through the public API with host buffers: pinned x -> device,
+    forward, y and h_T -> pinned host, every step inside the timed region."""
+    B, T, D = wl.B, wl.T, wl.D
+    x_host = g["x"].cpu().pin_memory()
+    y_host = torch.empty_like(x_host).pin_memory()
+    h_host = torch.empty(B, D).pin_memory()
+    x_dev = torch.empty_like(g["x"])
+    stream = torch.cuda.current_stream()
+
+    def step():
+        x_dev.copy_(x_host, non_blocking=True)
+        y, hT, _ = rg.rglru_fwd(x_dev, *w, h0=g["h0"], algo=a.algo, want_state=False)
+        y_host.copy_(y, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    n = max(3, min(a.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    esz = x_host.element_size()
+    return {"value": B * T * D / (ms / 1e3), "unit": "channel-tokens/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": B * T * D * esz, "d2h_bytes_per_step": B * T * D * esz,
+            "steps": n}
+
+
+def run_decode(rg, dev, a, pk):
+    """Decode workload: B=1024 sequences, one step per launch, state in place."""
+    wl = WORKLOADS["decode_batch"]
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(wl.seed)
+    B, D, H, bw = wl.B, wl.D, wl.H, wl.bw
+    dt = wl.dtype
+    steps = a.decode_steps
+    x = torch.randn(steps, B, D, generator=gen, device=dev).to(dt)
+    conv_w = (torch.randn(4, D, generator=gen, device=dev) * 0.5).to(dt)
+    W_a = (torch.randn(H, bw, bw, generator=gen, device=dev) / 8).to(dt)
+    W_x = (torch.randn(H, bw, bw, generator=gen, device=dev) / 8).to(dt)
+    b = torch.zeros(D, device=dev, dtype=dt)
+    s = torch.rand(D, generator=gen, device=dev, dtype=torch.float64) * (wl.ac_hi - wl.ac_lo) + wl.ac_lo
+    aa = s ** (1 / 8)
+    Lam = (torch.log(aa) - torch.log1p(-aa)).float()
+    h = torch.randn(B, D, generator=gen, device=dev)
+    ring = torch.randn(B, 3, D, generator=gen, device=dev).to(dt)
+    ys = torch.empty(steps, B, D, device=dev, dtype=dt)
+    stream = torch.cuda.current_stream()
+    for s_ in range(3):
+        rg.rglru_decode_step(x[s_], ring, s_, h, conv_w, W_a, b, W_x, b, Lam, y_t=ys[s_],
+                             algo=a.algo)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s_ in range(steps):
+        rg.rglru_decode_step(x[s_], ring, s_, h, conv_w, W_a, b, W_x, b, Lam, y_t=ys[s_],
+                             algo=a.algo)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    bytes_step = 20 * B * D   # x 2 + ring read 6 + ring write 2 + h read/write 8 + y 2
+    gbs = bytes_step / (ms / 1e3) / 1e9
+    return {"workload": f"decode_batch B={B} D={D} H={H} bw={bw} io=bf16, {steps} steps",
+            "value": B * D / (ms / 1e3), "unit": "channel-tokens/s", "us_per_step": ms * 1e3,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                         "algorithmic_bytes_per_launch": bytes_step},
+            "inputs": "seeded on the device with the workload's recipe",
+            "l2": "state, ring and weights total 113 MB; the state is re-read each step "
+                  "(L2 may hold part of it, as in real decoding)"}
+
+
+# ------------------------------------------------------------ CPU oracle --
+
+def oracle_sample(wl, t, seconds):
+    """Time the float64 oracle on the first rows of the workload, growing the
+    sample until it takes about `seconds` of wall time. Returns (chtok/s, desc)."""
+    from oracle import rglru_oracle as orc
+    rows = 1
+    T = wl.T
+    Tcap = T
+    while True:
+        xs = t["x"][:rows, :Tcap]
+        h0 = t["h0"][:rows] if t["h0"] is not None else None
+        t0 = time.perf_counter()
+        orc.rglru_fwd(xs, t["conv_w"], t["W_a"], t["b_a"], t["W_x"], t["b_x"], t["Lambda"],
+                      h0=h0)
+        dt = time.perf_counter() - t0
+        work = rows * Tcap * wl.D
+        if dt >= seconds or rows >= wl.B:
+            return work / dt, f"{rows} of {wl.B} batch rows x {Tcap} tokens x D={wl.D} " \
+                              f"({dt:.1f} s wall, float64 numpy oracle)"
+        grow = max(2, int(math.ceil(seconds / max(dt, 1e-3))))
+        rows = min(wl.B, rows * grow)
+
+
+def cpu_baseline(wl, t, seconds):
+    v, desc = oracle_sample(wl, t, seconds)
+    return {"value": v, "unit": "channel-tokens/s", "cores": 1, "kind": "oracle",
+            "sample": desc}
+
+
+# -------------------------------------------------------- reference arm --
+
+def run_reference(a, ws, rank):
+    if rank != 0:
+        return None
+    wl = WORKLOADS[a.workload]
+    t = generate(wl)
+    per = []
+    desc = ""
+    for _ in range(a.warmup):
+        oracle_sample(wl, t, 0.5)
+    for _ in range(a.steps):
+        v, desc = oracle_sample(wl, t, a.ref_seconds)
+        per.append(v)
+    v = statistics.median(per)
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "channel-tokens/s",
+            "n_gpus": ws, "steps": a.steps, "warmup": a.warmup, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded; recipe of the workload)",
+            "config": {"workload": f"{wl.name} B={wl.B} T={wl.T} D={wl.D} H={wl.H} "
+                                   f"bw={wl.bw} io={wl.io}", "seq_len": wl.T},
+            "cpu_baseline": {"value": v, "unit": "channel-tokens/s", "cores": 1,
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": v, "unit": "channel-tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="hawk_block", choices=sorted(WORKLOADS))
+    ap.add_argument("--algo", default="auto", choices=["auto", "generic", "tensor"])
+    ap.add_argument("--soak-s", type=float, default=1.5,
+                    help="untimed seconds of the same steps before and after the timed "
+                         "region, so the clock sampler sees the load")
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-decode", dest="decode", action="store_false")
+    ap.add_argument("--decode-steps", type=int, default=256)
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-seconds", type=float, default=5.0)
+    a = ap.parse_args(argv)
+    if a.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if a.impl == "reference":
+        out = run_reference(a, ws, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return 0
+    ws, rank, local = dist_setup()
+    out = run_ours(a, ws, rank, local)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

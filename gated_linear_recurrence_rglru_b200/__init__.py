@@ -1,0 +1,14 @@
+"""B200-native (sm_100a) RG-LRU: the recurrent core of Griffin / Hawk.
+
+The layer ("Griffin: Mixing Gated Linear Recurrences with Local Attention for
+Efficient Language Models", section "Model Architecture"): a width-4 causal
+Conv1D, block-diagonal sigmoid gates, a log-space decay a_t = a^(8 r_t) and the
+diagonal recurrence h_t = a_t h_{t-1} + sqrt(1 - a_t^2) (i_t u_t), computed by
+hand-written CUDA kernels behind a C ABI (include/rglru.h). This package is the
+thin Python binding of that library; see _abi.py.
+"""
+from ._abi import (ALGO_AUTO, ALGO_GENERIC, ALGO_TENSOR, LIB_PATH, RGLRUError,  # noqa: F401
+                   fwd_launches, fwd_workspace_bytes, rglru_decode_step, rglru_fwd, status_str, version)
+
+__all__ = ["rglru_fwd", "rglru_decode_step", "fwd_workspace_bytes", "fwd_launches", "RGLRUError",
+           "status_str", "version", "LIB_PATH"]

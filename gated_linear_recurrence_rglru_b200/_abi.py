@@ -1,0 +1,181 @@
+"""ctypes binding of librglru_b200.so (argument marshalling only).
+
+Every step of the layer runs in the library's CUDA kernels. This module turns
+torch CUDA tensors into device pointers, allocates outputs and workspace
+through torch (device memory is PyTorch's job here), passes the current torch
+stream, and raises RGLRUError on any nonzero status. If the library is
+missing, importing this module fails: there is no CPU path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librglru_b200.so")
+
+IO_F32, IO_BF16 = 0, 1
+ALGO_AUTO, ALGO_GENERIC, ALGO_TENSOR = 0, 1, 2
+ALGOS = {"auto": ALGO_AUTO, "generic": ALGO_GENERIC, "tensor": ALGO_TENSOR}
+
+EXPORTED = (
+    "rglru_status_str", "rglru_version", "rglru_fwd_workspace_bytes", "rglru_fwd",
+    "rglru_fwd_algo", "rglru_decode_step", "rglru_decode_step_algo", "rglru_fwd_launches",
+)
+
+
+class RGLRUError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_str(status)} (status {status})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python gated_linear_recurrence_rglru_b200/build.py` (there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, fp, ip, i32, sz = (ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                           ctypes.c_size_t)
+    lib.rglru_status_str.restype = ctypes.c_char_p
+    lib.rglru_status_str.argtypes = [i32]
+    lib.rglru_version.restype = i32
+    lib.rglru_version.argtypes = []
+    lib.rglru_fwd_workspace_bytes.restype = sz
+    lib.rglru_fwd_workspace_bytes.argtypes = [i32] * 5
+    lib.rglru_fwd_launches.restype = i32
+    lib.rglru_fwd_launches.argtypes = [i32] * 6
+    fwd_args = [vp] * 6 + [fp, fp, vp, vp, fp, vp] + [i32] * 5 + [vp, sz, ip, vp]
+    lib.rglru_fwd.restype = i32
+    lib.rglru_fwd.argtypes = fwd_args
+    lib.rglru_fwd_algo.restype = i32
+    lib.rglru_fwd_algo.argtypes = fwd_args + [i32]
+    dec_args = [vp, vp, i32, fp, vp] + [vp] * 5 + [fp] + [i32] * 4 + [vp]
+    lib.rglru_decode_step.restype = i32
+    lib.rglru_decode_step.argtypes = dec_args
+    lib.rglru_decode_step_algo.restype = i32
+    lib.rglru_decode_step_algo.argtypes = dec_args + [i32]
+    return lib
+
+
+LIB = _load()
+
+
+def status_str(status: int) -> str:
+    return LIB.rglru_status_str(int(status)).decode()
+
+
+def version() -> int:
+    return LIB.rglru_version()
+
+
+def _io_of(dtype: torch.dtype) -> int:
+    if dtype == torch.float32:
+        return IO_F32
+    if dtype == torch.bfloat16:
+        return IO_BF16
+    raise TypeError(f"unsupported I/O dtype {dtype} (float32 or bfloat16)")
+
+
+def _ptr(t, name, dtype=None, shape=None, optional=False):
+    if t is None:
+        if optional:
+            return None
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t.data_ptr()
+
+
+def _stream_handle(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def fwd_workspace_bytes(B: int, T: int, D: int, H: int, dtype=torch.bfloat16) -> int:
+    return int(LIB.rglru_fwd_workspace_bytes(B, T, D, H, _io_of(dtype)))
+
+
+def fwd_launches(B: int, T: int, D: int, H: int, dtype=torch.bfloat16, algo="auto") -> int:
+    """Kernel launches that one rglru_fwd call with these sizes issues."""
+    return int(LIB.rglru_fwd_launches(B, T, D, H, _io_of(dtype),
+                                      ALGOS[algo] if isinstance(algo, str) else int(algo)))
+
+
+def rglru_fwd(x, conv_w, W_a, b_a, W_x, b_x, Lambda, h0=None, conv_state_in=None, *,
+              y=None, h_T=None, conv_state_out=None, workspace=None, dev_status=None,
+              stream=None, algo="auto", want_state=True):
+    """Forward of the layer over (B, T, D). Returns (y, h_T, conv_state_out).
+
+    h_T / conv_state_out are None when want_state is False and no buffer is given.
+    """
+    if x.dim() != 3:
+        raise ValueError("x must be (B, T, D)")
+    B, T, D = x.shape
+    H = W_a.shape[0]
+    bw = D // H if H else 0
+    dt = x.dtype
+    io = _io_of(dt)
+    dev = x.device
+    if y is None:
+        y = torch.empty_like(x)
+    if want_state and h_T is None:
+        h_T = torch.empty(B, D, device=dev, dtype=torch.float32)
+    if want_state and conv_state_out is None:
+        conv_state_out = torch.empty(B, 3, D, device=dev, dtype=dt)
+    need = fwd_workspace_bytes(B, T, D, H, dt)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=dev, dtype=torch.uint8)
+    args = (
+        _ptr(x, "x", dt), _ptr(conv_w, "conv_w", dt, (4, D)),
+        _ptr(W_a, "W_a", dt, (H, bw, bw)), _ptr(b_a, "b_a", dt, (D,)),
+        _ptr(W_x, "W_x", dt, (H, bw, bw)), _ptr(b_x, "b_x", dt, (D,)),
+        _ptr(Lambda, "Lambda", torch.float32, (D,)),
+        _ptr(h0, "h0", torch.float32, (B, D), optional=True),
+        _ptr(conv_state_in, "conv_state_in", dt, (B, 3, D), optional=True),
+        _ptr(y, "y", dt, (B, T, D)),
+        _ptr(h_T, "h_T", torch.float32, (B, D), optional=True),
+        _ptr(conv_state_out, "conv_state_out", dt, (B, 3, D), optional=True),
+        B, T, D, H, io,
+        _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _ptr(dev_status, "dev_status", torch.int32, optional=True),
+        _stream_handle(stream), ALGOS[algo] if isinstance(algo, str) else int(algo),
+    )
+    st = LIB.rglru_fwd_algo(*args)
+    if st != 0:
+        raise RGLRUError(st, "rglru_fwd")
+    return y, h_T, conv_state_out
+
+
+def rglru_decode_step(x_t, conv_state, pos, h, conv_w, W_a, b_a, W_x, b_x, Lambda, *,
+                      y_t=None, stream=None, algo="auto"):
+    """One decode step: updates h and conv_state in place, returns y_t (B, D)."""
+    if x_t.dim() != 2:
+        raise ValueError("x_t must be (B, D)")
+    B, D = x_t.shape
+    H = W_a.shape[0]
+    bw = D // H if H else 0
+    dt = x_t.dtype
+    if y_t is None:
+        y_t = torch.empty_like(x_t)
+    st = LIB.rglru_decode_step_algo(
+        _ptr(x_t, "x_t", dt), _ptr(conv_state, "conv_state", dt, (B, 3, D)), int(pos),
+        _ptr(h, "h", torch.float32, (B, D)), _ptr(y_t, "y_t", dt, (B, D)),
+        _ptr(conv_w, "conv_w", dt, (4, D)), _ptr(W_a, "W_a", dt, (H, bw, bw)),
+        _ptr(b_a, "b_a", dt, (D,)), _ptr(W_x, "W_x", dt, (H, bw, bw)),
+        _ptr(b_x, "b_x", dt, (D,)), _ptr(Lambda, "Lambda", torch.float32, (D,)),
+        B, D, H, _io_of(dt), _stream_handle(stream),
+        ALGOS[algo] if isinstance(algo, str) else int(algo))
+    if st != 0:
+        raise RGLRUError(st, "rglru_decode_step")
+    return y_t

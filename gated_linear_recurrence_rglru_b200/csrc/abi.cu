@@ -1,0 +1,145 @@
+// The extern "C" boundary of the library: argument checks, algorithm choice
+// and launches on the caller's stream. See include/rglru.h for the contract.
+#include <stdint.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace rglru;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool opt_ok(const void *p) { return p == nullptr || aligned16(p); }
+
+bool overlap(const void *a, size_t na, const void *b, size_t nb) {
+  if (a == nullptr || b == nullptr || na == 0 || nb == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+int check_shape(int B, int T, int D, int H, int io) {
+  if (B < 1 || T < 1 || D < 1 || H < 1) return RGLRU_ERR_INVALID_ARG;
+  if (io != RGLRU_IO_F32 && io != RGLRU_IO_BF16) return RGLRU_ERR_INVALID_ARG;
+  if (D % H != 0 || D % 8 != 0) return RGLRU_ERR_INVALID_ARG;
+  if (D / H > 1024) return RGLRU_ERR_UNSUPPORTED;
+  if ((long long)B * D > (1ll << 31) - 1) return RGLRU_ERR_UNSUPPORTED;
+  if ((long long)B * T > (1ll << 31) - 1) return RGLRU_ERR_UNSUPPORTED;
+  return RGLRU_OK;
+}
+
+size_t io_bytes(int io) { return io == RGLRU_IO_F32 ? 4 : 2; }
+
+}  // namespace
+
+extern "C" {
+
+const char *rglru_status_str(int status) {
+  switch (status) {
+    case RGLRU_OK: return "ok";
+    case RGLRU_ERR_INVALID_ARG: return "invalid argument";
+    case RGLRU_ERR_UNSUPPORTED: return "unsupported shape, type or algorithm";
+    case RGLRU_ERR_CUDA: return "CUDA error";
+    case RGLRU_ERR_TIMEOUT: return "device-side wait timed out";
+    case RGLRU_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    default: return "unknown status";
+  }
+}
+
+int rglru_version(void) { return kVersion; }
+
+size_t rglru_fwd_workspace_bytes(int B, int T, int D, int H, int io) {
+  if (check_shape(B, T, D, H, io) != RGLRU_OK) return 0;
+  size_t need = generic_workspace_bytes(B, T, D, H);
+  return need < 256 ? 256 : need;
+}
+
+int rglru_fwd_launches(int B, int T, int D, int H, int io, int algo) {
+  if (check_shape(B, T, D, H, io) != RGLRU_OK) return 0;
+  if (algo == RGLRU_ALGO_TENSOR) return 0;
+  if (algo != RGLRU_ALGO_AUTO && algo != RGLRU_ALGO_GENERIC) return 0;
+  return generic_kernel_launches(B, T, H);
+}
+
+int rglru_fwd_algo(const void *x, const void *conv_w, const void *W_a, const void *b_a,
+                   const void *W_x, const void *b_x, const float *Lambda, const float *h0,
+                   const void *conv_state_in, void *y, float *h_T, void *conv_state_out,
+                   int B, int T, int D, int H, int io, void *workspace,
+                   size_t workspace_bytes, int *dev_status, void *stream, int algo) {
+  int st = check_shape(B, T, D, H, io);
+  if (st != RGLRU_OK) return st;
+  if (!x || !conv_w || !W_a || !b_a || !W_x || !b_x || !Lambda || !y)
+    return RGLRU_ERR_INVALID_ARG;
+  const void *req[] = {x, conv_w, W_a, b_a, W_x, b_x, Lambda, y};
+  for (const void *p : req)
+    if (!aligned16(p)) return RGLRU_ERR_INVALID_ARG;
+  if (!opt_ok(h0) || !opt_ok(conv_state_in) || !opt_ok(h_T) || !opt_ok(conv_state_out) ||
+      !opt_ok(dev_status))
+    return RGLRU_ERR_INVALID_ARG;
+  const size_t eb = io_bytes(io);
+  const size_t seq_bytes = (size_t)B * T * D * eb;
+  const size_t cs_bytes = (size_t)B * 3 * D * eb;
+  if (overlap(y, seq_bytes, x, seq_bytes)) return RGLRU_ERR_INVALID_ARG;
+  if (overlap(conv_state_out, cs_bytes, conv_state_in, cs_bytes)) return RGLRU_ERR_INVALID_ARG;
+  if (overlap(conv_state_out, cs_bytes, x, seq_bytes)) return RGLRU_ERR_INVALID_ARG;
+  if (algo != RGLRU_ALGO_AUTO && algo != RGLRU_ALGO_GENERIC && algo != RGLRU_ALGO_TENSOR)
+    return RGLRU_ERR_INVALID_ARG;
+  if (algo == RGLRU_ALGO_TENSOR) return RGLRU_ERR_UNSUPPORTED;
+
+  const size_t need = generic_workspace_bytes(B, T, D, H);
+  if (need > 0 && (workspace == nullptr || !aligned16(workspace) || workspace_bytes < need))
+    return RGLRU_ERR_WORKSPACE;
+
+  FwdArgs p{x, conv_w, W_a, b_a, W_x, b_x, Lambda, h0, conv_state_in, y, h_T, conv_state_out,
+            B, T, D, H, dev_status};
+  cudaError_t e = launch_fwd_generic(p, io, workspace, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RGLRU_OK : RGLRU_ERR_CUDA;
+}
+
+int rglru_fwd(const void *x, const void *conv_w, const void *W_a, const void *b_a,
+              const void *W_x, const void *b_x, const float *Lambda, const float *h0,
+              const void *conv_state_in, void *y, float *h_T, void *conv_state_out, int B,
+              int T, int D, int H, int io, void *workspace, size_t workspace_bytes,
+              int *dev_status, void *stream) {
+  return rglru_fwd_algo(x, conv_w, W_a, b_a, W_x, b_x, Lambda, h0, conv_state_in, y, h_T,
+                        conv_state_out, B, T, D, H, io, workspace, workspace_bytes, dev_status,
+                        stream, RGLRU_ALGO_AUTO);
+}
+
+int rglru_decode_step_algo(const void *x_t, void *conv_state, int pos, float *h, void *y_t,
+                           const void *conv_w, const void *W_a, const void *b_a,
+                           const void *W_x, const void *b_x, const float *Lambda, int B,
+                           int D, int H, int io, void *stream, int algo) {
+  int st = check_shape(B, 1, D, H, io);
+  if (st != RGLRU_OK) return st;
+  if (pos < 0) return RGLRU_ERR_INVALID_ARG;
+  if (!x_t || !conv_state || !h || !y_t || !conv_w || !W_a || !b_a || !W_x || !b_x || !Lambda)
+    return RGLRU_ERR_INVALID_ARG;
+  const void *req[] = {x_t, conv_state, h, y_t, conv_w, W_a, b_a, W_x, b_x, Lambda};
+  for (const void *p : req)
+    if (!aligned16(p)) return RGLRU_ERR_INVALID_ARG;
+  const size_t eb = io_bytes(io);
+  const size_t row_bytes = (size_t)B * D * eb;
+  if (overlap(y_t, row_bytes, x_t, row_bytes)) return RGLRU_ERR_INVALID_ARG;
+  if (overlap(y_t, row_bytes, conv_state, 3 * row_bytes)) return RGLRU_ERR_INVALID_ARG;
+  if (overlap(h, (size_t)B * D * 4, conv_state, 3 * row_bytes)) return RGLRU_ERR_INVALID_ARG;
+  if (algo != RGLRU_ALGO_AUTO && algo != RGLRU_ALGO_GENERIC && algo != RGLRU_ALGO_TENSOR)
+    return RGLRU_ERR_INVALID_ARG;
+  if (algo == RGLRU_ALGO_TENSOR) return RGLRU_ERR_UNSUPPORTED;
+  DecArgs p{x_t, conv_state, pos, h, y_t, conv_w, W_a, b_a, W_x, b_x, Lambda, B, D, H};
+  cudaError_t e = launch_decode_generic(p, io, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RGLRU_OK : RGLRU_ERR_CUDA;
+}
+
+int rglru_decode_step(const void *x_t, void *conv_state, int pos, float *h, void *y_t,
+                      const void *conv_w, const void *W_a, const void *b_a, const void *W_x,
+                      const void *b_x, const float *Lambda, int B, int D, int H, int io,
+                      void *stream) {
+  return rglru_decode_step_algo(x_t, conv_state, pos, h, y_t, conv_w, W_a, b_a, W_x, b_x,
+                                Lambda, B, D, H, io, stream, RGLRU_ALGO_AUTO);
+}
+
+}  // extern "C"

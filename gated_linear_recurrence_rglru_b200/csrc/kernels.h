@@ -1,0 +1,42 @@
+// Internal interface between the C ABI layer and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace rglru {
+
+struct FwdArgs {
+  const void *x, *conv_w, *W_a, *b_a, *W_x, *b_x;
+  const float *Lambda, *h0;
+  const void *conv_state_in;
+  void *y;
+  float *h_T;
+  void *conv_state_out;
+  int B, T, D, H;
+  int *dev_status;
+};
+
+struct DecArgs {
+  const void *x_t;
+  void *conv_state;
+  int pos;
+  float *h;
+  void *y_t;
+  const void *conv_w, *W_a, *b_a, *W_x, *b_x;
+  const float *Lambda;
+  int B, D, H;
+};
+
+struct GenericPlan {
+  int nseg;  // time segments
+  int L;     // tokens per segment (the last may be shorter)
+};
+
+GenericPlan generic_plan(int B, int T, int H);
+size_t generic_workspace_bytes(int B, int T, int D, int H);
+int generic_kernel_launches(int B, int T, int H);
+cudaError_t launch_fwd_generic(const FwdArgs &p, int io, void *ws, cudaStream_t st);
+cudaError_t launch_decode_generic(const DecArgs &p, int io, cudaStream_t st);
+
+}  // namespace rglru

@@ -1,0 +1,150 @@
+/*
+ * rglru.h -- C ABI of the B200 (sm_100a) RG-LRU library.
+ *
+ * The RG-LRU layer ("Griffin: Mixing Gated Linear Recurrences with Local
+ * Attention for Efficient Language Models", section "Model Architecture"; the
+ * recurrent gate added to a diagonal LRU and the temporal Conv1D of the
+ * recurrent block are described in S. De's thread on Griffin, "how we got
+ * there"; the gates do not read the recurrent state, "Beyond Transformer
+ * Architecture: Griffin and Google RecurrentGemma", "Core Components of
+ * Griffin", 1. RG-LRU):
+ *
+ *   u_t     = sum_{k=0..3} conv_w[k] * x_{t-3+k}          causal depthwise Conv1D, width 4
+ *   r_t     = sigmoid(u_t W_a + b_a)                       block-diagonal per head
+ *   i_t     = sigmoid(u_t W_x + b_x)                       block-diagonal per head
+ *   log a_t = -8 * r_t * softplus(-Lambda)
+ *   h_t     = a_t * h_{t-1} + sqrt(1 - a_t^2) * (i_t * u_t)
+ *   y_t     = h_t
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     allocates no memory and keeps no state between calls. Every pointer must
+ *     be 16-byte aligned. Tensors are dense and row-major in the shapes given.
+ *   - io selects the storage type of x, conv_w, W_a, W_x, b_a, b_x, y and the
+ *     conv state: RGLRU_IO_F32 (float) or RGLRU_IO_BF16 (bfloat16). Lambda and
+ *     every recurrent state (h0, h_T, h) are always float. Arithmetic is fp32.
+ *   - D = H * bw. Weights W_a, W_x have shape (H, bw, bw) with
+ *     z[h*bw + j] = sum_i u[h*bw + i] * W[h, i, j]. conv_w has shape (4, D);
+ *     tap k multiplies x_{t-3+k} (tap 3 is the current input).
+ *   - A conv state is (B, 3, D) in the I/O type. In rglru_fwd it is
+ *     chronological: slot 0 holds x_{t-3}, slot 2 holds x_{t-1}. In
+ *     rglru_decode_step it is a ring: at step pos, slot pos%3 holds x_{pos-3},
+ *     slot (pos+1)%3 holds x_{pos-2} and slot (pos+2)%3 holds x_{pos-1}; a
+ *     chronological state is the ring at pos = 0.
+ *   - stream is a cudaStream_t (NULL = the legacy default stream). Calls are
+ *     asynchronous: the return value reports argument checks and launch
+ *     errors only.
+ *   - Return values are rglru_status codes. On any nonzero return nothing was
+ *     launched (argument errors) or the launch failed (RGLRU_ERR_CUDA).
+ */
+#ifndef RGLRU_B200_H
+#define RGLRU_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RGLRU_OK = 0,
+  RGLRU_ERR_INVALID_ARG = 1,   /* NULL or misaligned pointer, non-positive or inconsistent size */
+  RGLRU_ERR_UNSUPPORTED = 2,   /* well-formed request outside what the kernels implement */
+  RGLRU_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed */
+  RGLRU_ERR_TIMEOUT = 4,       /* device side: a bounded wait expired (reported via dev_status) */
+  RGLRU_ERR_WORKSPACE = 5      /* workspace NULL, misaligned or smaller than required */
+} rglru_status;
+
+typedef enum { RGLRU_IO_F32 = 0, RGLRU_IO_BF16 = 1 } rglru_io;
+
+typedef enum {
+  RGLRU_ALGO_AUTO = 0,         /* tensor-core path when supported, else the generic path */
+  RGLRU_ALGO_GENERIC = 1,      /* CUDA-core gates, three passes over time segments */
+  RGLRU_ALGO_TENSOR = 2        /* tcgen05 gate contraction, single fused pass */
+} rglru_algo;
+
+/* Human-readable name of a status code. Never NULL. */
+const char *rglru_status_str(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int rglru_version(void);
+
+/*
+ * Bytes of device workspace that rglru_fwd / rglru_fwd_algo need for this
+ * shape, for any algorithm. Returns 0 on invalid sizes. The workspace holds
+ * the per-segment carries of the time-split scan and the scheduling counters;
+ * it needs no initialisation by the caller and may be reused across calls
+ * issued to the same stream (calls that overlap on the GPU need separate
+ * workspaces).
+ */
+size_t rglru_fwd_workspace_bytes(int B, int T, int D, int H, int io);
+
+/*
+ * Number of kernel launches one rglru_fwd_algo call with these arguments
+ * issues on its stream (0 on invalid or unsupported arguments).
+ */
+int rglru_fwd_launches(int B, int T, int D, int H, int io, int algo);
+
+/*
+ * Full-sequence forward of the layer.
+ *   x              (B, T, D)  io     input of the Conv1D
+ *   conv_w         (4, D)     io
+ *   W_a, W_x       (H, bw, bw) io    gate weights
+ *   b_a, b_x       (D)        io     gate biases
+ *   Lambda         (D)        float  a = sigmoid(Lambda)
+ *   h0             (B, D)     float  initial state, or NULL for zeros
+ *   conv_state_in  (B, 3, D)  io     chronological history, or NULL for zeros
+ *   y              (B, T, D)  io     output h_t (written)
+ *   h_T            (B, D)     float  final state (written), or NULL
+ *   conv_state_out (B, 3, D)  io     last three inputs, chronological (written), or NULL;
+ *                                    must not alias conv_state_in
+ *   workspace      device scratch of at least rglru_fwd_workspace_bytes(...)
+ *   dev_status     device int, or NULL. On a device-side failure a kernel
+ *                  stores a nonzero rglru_status there (RGLRU_ERR_TIMEOUT when
+ *                  a bounded wait for another block's carry expired; y is then
+ *                  incomplete). The library never clears it.
+ * Requirements: B, T >= 1; H >= 1; D % H == 0; D % 8 == 0; bw = D / H <= 1024.
+ */
+int rglru_fwd(const void *x, const void *conv_w, const void *W_a, const void *b_a,
+              const void *W_x, const void *b_x, const float *Lambda, const float *h0,
+              const void *conv_state_in, void *y, float *h_T, void *conv_state_out,
+              int B, int T, int D, int H, int io, void *workspace, size_t workspace_bytes,
+              int *dev_status, void *stream);
+
+/*
+ * rglru_fwd with an explicit algorithm (rglru_algo). RGLRU_ALGO_TENSOR needs
+ * io = RGLRU_IO_BF16, D % 128 == 0 and bw in {16, 32, 64, 128, 256}; otherwise
+ * it returns RGLRU_ERR_UNSUPPORTED. Both algorithms compute the same layer.
+ */
+int rglru_fwd_algo(const void *x, const void *conv_w, const void *W_a, const void *b_a,
+                   const void *W_x, const void *b_x, const float *Lambda, const float *h0,
+                   const void *conv_state_in, void *y, float *h_T, void *conv_state_out,
+                   int B, int T, int D, int H, int io, void *workspace,
+                   size_t workspace_bytes, int *dev_status, void *stream, int algo);
+
+/*
+ * One decode step for B independent sequences, state updated in place.
+ *   x_t        (B, D)     io     this step's input
+ *   conv_state (B, 3, D)  io     ring at step pos (read); slot pos%3 is overwritten with x_t
+ *   pos        >= 0              step index that places the ring (see above)
+ *   h          (B, D)     float  state h_{t-1} (read), h_t (written)
+ *   y_t        (B, D)     io     output h_t (written); must not alias x_t
+ *   conv_w, W_a, b_a, W_x, b_x, Lambda as in rglru_fwd.
+ * Requirements: B >= 1; D % H == 0; D % 8 == 0; bw <= 1024.
+ */
+int rglru_decode_step(const void *x_t, void *conv_state, int pos, float *h, void *y_t,
+                      const void *conv_w, const void *W_a, const void *b_a, const void *W_x,
+                      const void *b_x, const float *Lambda, int B, int D, int H, int io,
+                      void *stream);
+
+/* rglru_decode_step with an explicit algorithm (same rules as rglru_fwd_algo). */
+int rglru_decode_step_algo(const void *x_t, void *conv_state, int pos, float *h, void *y_t,
+                           const void *conv_w, const void *W_a, const void *b_a,
+                           const void *W_x, const void *b_x, const float *Lambda, int B,
+                           int D, int H, int io, void *stream, int algo);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RGLRU_B200_H */

@@ -1,0 +1,99 @@
+"""CPU checks of the C-ABI library: it loads without a GPU, exports every
+function include/rglru.h declares, and rejects bad arguments before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_linear_recurrence_rglru_b200 import _abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[a-z_]+\s*\*?\s*(rglru_[a-z0-9_]+)\s*\(",
+                                src, flags=re.M)
+    return names
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for n in ("rglru_fwd", "rglru_decode_step", "rglru_fwd_workspace_bytes"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(_abi.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+    assert set(_abi.EXPORTED) <= set(declared_functions())
+
+
+def test_status_strings_and_version():
+    assert _abi.status_str(0) == "ok"
+    assert "timed out" in _abi.status_str(4)
+    assert _abi.status_str(99) == "unknown status"
+    assert _abi.version() >= 100
+
+
+def test_workspace_bytes():
+    lib = _abi.LIB
+    assert lib.rglru_fwd_workspace_bytes(8, 2048, 1024, 16, 1) >= 256
+    assert lib.rglru_fwd_workspace_bytes(0, 2048, 1024, 16, 1) == 0
+    assert lib.rglru_fwd_workspace_bytes(8, 2048, 1000, 16, 1) == 0      # D % H != 0
+    assert lib.rglru_fwd_workspace_bytes(8, 2048, 1024, 16, 7) == 0      # bad io
+    # more segments (smaller B*H) never needs less than a single long segment
+    assert lib.rglru_fwd_workspace_bytes(1, 131072, 4096, 16, 1) > 0
+
+
+FAKE = 1 << 20  # 16-byte aligned non-null stand-in; never dereferenced: the checks fail first
+
+
+def fwd_call(**over):
+    a = dict(x=FAKE, conv_w=FAKE, W_a=FAKE, b_a=FAKE, W_x=FAKE, b_x=FAKE, Lambda=FAKE, h0=None,
+             csi=None, y=FAKE * 64, h_T=None, cso=None, B=2, T=16, D=64, H=2, io=1,
+             ws=FAKE * 128, ws_bytes=1 << 30, dev_status=None, stream=None, algo=0)
+    a.update(over)
+    return _abi.LIB.rglru_fwd_algo(a["x"], a["conv_w"], a["W_a"], a["b_a"], a["W_x"], a["b_x"],
+                                   a["Lambda"], a["h0"], a["csi"], a["y"], a["h_T"], a["cso"],
+                                   a["B"], a["T"], a["D"], a["H"], a["io"], a["ws"],
+                                   a["ws_bytes"], a["dev_status"], a["stream"], a["algo"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(B=0), 1), (dict(T=0), 1), (dict(H=0), 1), (dict(D=60, H=2), 1), (dict(D=63, H=1), 1),
+    (dict(io=3), 1), (dict(x=None), 1), (dict(Lambda=None), 1), (dict(y=None), 1),
+    (dict(x=FAKE + 4), 1), (dict(h0=FAKE + 8), 1), (dict(y=FAKE), 1),          # y aliases x
+    (dict(D=2048, H=1), 2), (dict(algo=9), 1),
+    (dict(B=64, T=4096, ws=None), 5), (dict(B=64, T=4096, ws_bytes=16), 5),
+])
+def test_fwd_rejects_bad_arguments(over, code):
+    assert fwd_call(**over) == code
+
+
+def test_decode_rejects_bad_arguments():
+    L = _abi.LIB
+    args = [FAKE, FAKE * 2, 0, FAKE * 4, FAKE * 8, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 64, 2, 1,
+            None, 0]
+    bad = list(args); bad[2] = -1
+    assert L.rglru_decode_step_algo(*bad) == 1                 # pos < 0
+    bad = list(args); bad[4] = FAKE                            # y_t aliases x_t
+    assert L.rglru_decode_step_algo(*bad) == 1
+    bad = list(args); bad[13] = 3                              # D % H
+    assert L.rglru_decode_step_algo(*bad) == 1
+    bad = list(args); bad[3] = None
+    assert L.rglru_decode_step_algo(*bad) == 1
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 4, 8)
+    with pytest.raises((TypeError, RuntimeError)):
+        _abi.rglru_fwd(x, torch.zeros(4, 8), torch.zeros(1, 8, 8), torch.zeros(8),
+                       torch.zeros(1, 8, 8), torch.zeros(8), torch.zeros(8))
