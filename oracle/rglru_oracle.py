@@ -79,9 +79,9 @@ def gate_preacts(u, W, b):
     B, T, D = u.shape
     H, bw, bw2 = W.shape
     assert bw == bw2 and H * bw == D
-    uh = u.reshape(B, T, H, bw)
-    z = np.einsum("bthi,hij->bthj", uh, W)
-    return z.reshape(B, T, D) + b[None, None, :]
+    uh = u.reshape(B * T, H, bw).transpose(1, 0, 2)      # (H, B*T, bw): head h's inputs
+    z = np.matmul(uh, W)                                  # z[h, n, j] = sum_i u[n, h*bw+i] W[h, i, j]
+    return z.transpose(1, 0, 2).reshape(B, T, D) + b[None, None, :]
 
 
 def sigmoid(z):
