@@ -308,22 +308,25 @@ def oracle_sample(wl, t, seconds):
     """Time the float64 oracle on the first rows of the workload, growing the
     sample until it takes about `seconds` of wall time. Returns (chtok/s, desc)."""
     from oracle import rglru_oracle as orc
-    rows = 1
-    T = wl.T
-    Tcap = T
+    rows, reps = 1, 1
+    Tcap = wl.T
     while True:
         xs = t["x"][:rows, :Tcap]
         h0 = t["h0"][:rows] if t["h0"] is not None else None
         t0 = time.perf_counter()
-        orc.rglru_fwd(xs, t["conv_w"], t["W_a"], t["b_a"], t["W_x"], t["b_x"], t["Lambda"],
-                      h0=h0)
+        for _ in range(reps):
+            orc.rglru_fwd(xs, t["conv_w"], t["W_a"], t["b_a"], t["W_x"], t["b_x"],
+                          t["Lambda"], h0=h0)
         dt = time.perf_counter() - t0
-        work = rows * Tcap * wl.D
-        if dt >= seconds or rows >= wl.B:
-            return work / dt, f"{rows} of {wl.B} batch rows x {Tcap} tokens x D={wl.D} " \
-                              f"({dt:.1f} s wall, float64 numpy oracle)"
+        work = reps * rows * Tcap * wl.D
+        if dt >= 0.8 * seconds:
+            return work / dt, (f"{reps} x ({rows} of {wl.B} batch rows x {Tcap} tokens x "
+                               f"D={wl.D}), {dt:.1f} s wall, float64 numpy oracle")
         grow = max(2, int(math.ceil(seconds / max(dt, 1e-3))))
-        rows = min(wl.B, rows * grow)
+        if rows < wl.B:
+            rows = min(wl.B, rows * grow)
+        else:
+            reps *= grow
 
 
 def cpu_baseline(wl, t, seconds):
