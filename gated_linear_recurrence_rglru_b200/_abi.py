@@ -23,7 +23,9 @@ ALGOS = {"auto": ALGO_AUTO, "generic": ALGO_GENERIC, "tensor": ALGO_TENSOR}
 EXPORTED = (
     "rglru_status_str", "rglru_version", "rglru_fwd_workspace_bytes", "rglru_fwd",
     "rglru_fwd_algo", "rglru_decode_step", "rglru_decode_step_algo", "rglru_fwd_launches",
+    "rglru_fwd_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 2 << 20  # RGLRU_NOALLOC_SCRATCH_BYTES in include/rglru.h
 
 
 class RGLRUError(RuntimeError):
@@ -53,6 +55,8 @@ def _load():
     lib.rglru_fwd.argtypes = fwd_args
     lib.rglru_fwd_algo.restype = i32
     lib.rglru_fwd_algo.argtypes = fwd_args + [i32]
+    lib.rglru_fwd_noalloc.restype = i32
+    lib.rglru_fwd_noalloc.argtypes = [vp] * 6 + [fp, fp, vp, vp, fp, vp] + [i32] * 5 + [vp]
     dec_args = [vp, vp, i32, fp, vp] + [vp] * 5 + [fp] + [i32] * 4 + [vp]
     lib.rglru_decode_step.restype = i32
     lib.rglru_decode_step.argtypes = dec_args
@@ -154,6 +158,33 @@ def rglru_fwd(x, conv_w, W_a, b_a, W_x, b_x, Lambda, h0=None, conv_state_in=None
     st = LIB.rglru_fwd_algo(*args)
     if st != 0:
         raise RGLRUError(st, "rglru_fwd")
+    return y, h_T, conv_state_out
+
+
+def rglru_fwd_noalloc(x, conv_w, W_a, b_a, W_x, b_x, Lambda, h0=None, conv_state_in=None, *,
+                      y=None, h_T=None, conv_state_out=None, stream=None):
+    """rglru_fwd without a workspace: the library's static device scratch is used.
+
+    For callers that cannot allocate device memory while running (output
+    buffers may be passed in). Returns (y, h_T, conv_state_out).
+    """
+    B, T, D = x.shape
+    H = W_a.shape[0]
+    bw = D // H if H else 0
+    dt = x.dtype
+    st = LIB.rglru_fwd_noalloc(
+        _ptr(x, "x", dt), _ptr(conv_w, "conv_w", dt, (4, D)),
+        _ptr(W_a, "W_a", dt, (H, bw, bw)), _ptr(b_a, "b_a", dt, (D,)),
+        _ptr(W_x, "W_x", dt, (H, bw, bw)), _ptr(b_x, "b_x", dt, (D,)),
+        _ptr(Lambda, "Lambda", torch.float32, (D,)),
+        _ptr(h0, "h0", torch.float32, (B, D), optional=True),
+        _ptr(conv_state_in, "conv_state_in", dt, (B, 3, D), optional=True),
+        _ptr(y, "y", dt, (B, T, D)),
+        _ptr(h_T, "h_T", torch.float32, (B, D), optional=True),
+        _ptr(conv_state_out, "conv_state_out", dt, (B, 3, D), optional=True),
+        B, T, D, H, _io_of(dt), _stream_handle(stream))
+    if st != 0:
+        raise RGLRUError(st, "rglru_fwd_noalloc")
     return y, h_T, conv_state_out
 
 

@@ -123,6 +123,45 @@ int rglru_fwd_algo(const void *x, const void *conv_w, const void *W_a, const voi
                    size_t workspace_bytes, int *dev_status, void *stream, int algo);
 
 /*
+ * Size of the library's fixed device scratch used by rglru_fwd_noalloc.
+ * Every GPU that loads the library holds this much device memory until the
+ * process exits.
+ */
+#define RGLRU_NOALLOC_SCRATCH_BYTES (2u << 20)
+
+/*
+ * rglru_fwd_noalloc: the forward of the layer (the generic algorithm, as
+ * rglru_fwd_algo with RGLRU_ALGO_GENERIC) for callers that cannot allocate
+ * device memory. The paper has no counterpart to this entry point: it exists
+ * for deployment only.
+ *
+ * Who needs it: code that must not call cudaMalloc once it is running, such
+ * as a serving loop that reserves all device memory for its own pool at
+ * start-up, or a plugin hosted by a framework that owns the allocator and
+ * gives the plugin no way to ask for scratch. rglru_fwd needs a workspace
+ * from its caller; this variant takes none. Its scratch (the per-segment
+ * carries of the time split) lives in a static device array of
+ * RGLRU_NOALLOC_SCRATCH_BYTES inside the library, and the call allocates
+ * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *
+ * Arguments, layouts and results are those of rglru_fwd without the
+ * workspace and dev_status arguments. The stream must belong to the current
+ * device. The first call on a device looks up that device's copy of the
+ * static array (cudaGetSymbolAddress, once per device, with the device
+ * current); make that first call before any stream capture. Problems whose
+ * scratch would exceed RGLRU_NOALLOC_SCRATCH_BYTES (rglru_fwd_workspace_bytes
+ * larger than it) are rejected with RGLRU_ERR_WORKSPACE before anything is
+ * launched. All calls on a device share the one array, which keeps the last
+ * call's contents (nothing in it needs to start at zero): calls that can
+ * overlap on the GPU, from different streams or threads, race on it and
+ * must be serialised by the caller.
+ */
+int rglru_fwd_noalloc(const void *x, const void *conv_w, const void *W_a, const void *b_a,
+                      const void *W_x, const void *b_x, const float *Lambda, const float *h0,
+                      const void *conv_state_in, void *y, float *h_T, void *conv_state_out,
+                      int B, int T, int D, int H, int io, void *stream);
+
+/*
  * One decode step for B independent sequences, state updated in place.
  *   x_t        (B, D)     io     this step's input
  *   conv_state (B, 3, D)  io     ring at step pos (read); slot pos%3 is overwritten with x_t
