@@ -54,14 +54,21 @@ int rglru_version(void) { return kVersion; }
 size_t rglru_fwd_workspace_bytes(int B, int T, int D, int H, int io) {
   if (check_shape(B, T, D, H, io) != RGLRU_OK) return 0;
   size_t need = generic_workspace_bytes(B, T, D, H);
+  if (tc_supported(B, T, D, H, io)) {
+    const size_t tc = tc_workspace_bytes(B, T, D, H);
+    if (tc > need) need = tc;
+  }
   return need < 256 ? 256 : need;
 }
 
 int rglru_fwd_launches(int B, int T, int D, int H, int io, int algo) {
   if (check_shape(B, T, D, H, io) != RGLRU_OK) return 0;
-  if (algo == RGLRU_ALGO_TENSOR) return 0;
-  if (algo != RGLRU_ALGO_AUTO && algo != RGLRU_ALGO_GENERIC) return 0;
-  return generic_kernel_launches(B, T, H);
+  if (algo != RGLRU_ALGO_AUTO && algo != RGLRU_ALGO_GENERIC && algo != RGLRU_ALGO_TENSOR)
+    return 0;
+  const bool tc = tc_supported(B, T, D, H, io);
+  if (algo == RGLRU_ALGO_TENSOR && !tc) return 0;
+  if (algo == RGLRU_ALGO_GENERIC || !tc) return generic_kernel_launches(B, T, H);
+  return 1;
 }
 
 int rglru_fwd_algo(const void *x, const void *conv_w, const void *W_a, const void *b_a,
@@ -87,15 +94,19 @@ int rglru_fwd_algo(const void *x, const void *conv_w, const void *W_a, const voi
   if (overlap(conv_state_out, cs_bytes, x, seq_bytes)) return RGLRU_ERR_INVALID_ARG;
   if (algo != RGLRU_ALGO_AUTO && algo != RGLRU_ALGO_GENERIC && algo != RGLRU_ALGO_TENSOR)
     return RGLRU_ERR_INVALID_ARG;
-  if (algo == RGLRU_ALGO_TENSOR) return RGLRU_ERR_UNSUPPORTED;
+  const bool tc = tc_supported(B, T, D, H, io);
+  if (algo == RGLRU_ALGO_TENSOR && !tc) return RGLRU_ERR_UNSUPPORTED;
+  const bool use_tc = tc && algo != RGLRU_ALGO_GENERIC;
 
-  const size_t need = generic_workspace_bytes(B, T, D, H);
+  const size_t need =
+      use_tc ? tc_workspace_bytes(B, T, D, H) : generic_workspace_bytes(B, T, D, H);
   if (need > 0 && (workspace == nullptr || !aligned16(workspace) || workspace_bytes < need))
     return RGLRU_ERR_WORKSPACE;
 
   FwdArgs p{x, conv_w, W_a, b_a, W_x, b_x, Lambda, h0, conv_state_in, y, h_T, conv_state_out,
             B, T, D, H, dev_status};
-  cudaError_t e = launch_fwd_generic(p, io, workspace, static_cast<cudaStream_t>(stream));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = use_tc ? launch_fwd_tc(p, workspace, s) : launch_fwd_generic(p, io, workspace, s);
   return e == cudaSuccess ? RGLRU_OK : RGLRU_ERR_CUDA;
 }
 

@@ -39,4 +39,9 @@ int generic_kernel_launches(int B, int T, int H);
 cudaError_t launch_fwd_generic(const FwdArgs &p, int io, void *ws, cudaStream_t st);
 cudaError_t launch_decode_generic(const DecArgs &p, int io, cudaStream_t st);
 
+// Tensor-core (tcgen05) fused forward, bf16 I/O.
+bool tc_supported(int B, int T, int D, int H, int io);
+size_t tc_workspace_bytes(int B, int T, int D, int H);
+cudaError_t launch_fwd_tc(const FwdArgs &p, void *ws, cudaStream_t st);
+
 }  // namespace rglru
