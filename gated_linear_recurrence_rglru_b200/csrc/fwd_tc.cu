@@ -6,24 +6,27 @@
 // state, "Beyond Transformer Architecture: Griffin and Google RecurrentGemma",
 // "Core Components of Griffin", 1. RG-LRU) is split into
 //   unit = (batch row b, group of 128 output channels), tile = 64 tokens
-//   (32 tokens when a head is 256 wide).
-// For a tile, a warpgroup computes the width-4 Conv1D of the unit's input
-// channels into a K-major bf16 operand in shared memory; one thread issues
-// the gate contraction on the tensor core with the gate weights as the A
-// operand (M = 128 output channels, MN-major, loaded by TMA) and the conv
-// output as B (N = tokens), so that TMEM lane m holds channel m's two gate
-// pre-activations along time. The same warpgroup then runs, per lane
-// (channel), the sigmoid gates, the log-space decay, sqrt(1 - a^2), and the
-// scan along time: the exact linear scan of S. De's thread ("we use linear
-// scans"), carried across tiles by a decoupled look-back over per-tile
-// (prod a, local h) aggregates and inclusive states in the workspace.
-//
-// Roles (320 threads, one CTA per SM, persistent):
-//   warp 0      producer: claims tiles (per-unit counters, stealing from other
-//               units once its own is done), TMA of x tiles and gate weights;
-//   warp 1      TMEM owner and tcgen05.mma issuer;
-//   warps 2-5   warpgroup 0, even jobs of this CTA;  warps 6-9 warpgroup 1, odd.
-// Tiles of a unit are claimed in time order by running CTAs only, so every
+//   (32 tokens when a head is 256 wide, so that its weights fit on chip).
+// Per tile
+//   1. the conv warpgroup computes the width-4 Conv1D token-major (4 channels x 8 tokens per step,
+//      vector shared-memory rows, packed fp32x2 FMAs) into the K-major bf16
+//      MMA operand and, for 128-wide channel ranges, an fp32 copy of u;
+//   2. (one thread of another warp issues tcgen05.mma with the gate weights as
+//      the A operand, M = 128 output channels, MN-major and loaded by TMA, and
+//      the conv output as B, N = tokens: TMEM lane m then holds channel m's
+//      two gate pre-activations along time);
+//   3. an epilogue warpgroup, per lane (channel): sigmoid gates, log-space decay, sqrt(1 - a^2) and a
+//      local scan along time (pass 1, results back into TMEM);
+//   4. carries the state across tiles with a decoupled look-back over per-tile
+//      (prod a, local h) aggregates and inclusive states in the workspace —
+//      the exact linear scan of S. De's thread ("linear scans instead of
+//      parallel scans"), parallel across tiles;
+//   5. rescans from the carried state and writes y (pass 2).
+// Roles: warp 0 claims tiles (per-unit counters in time order, stealing from
+// other units once its own is done) and issues TMA; warp 1 owns TMEM and
+// issues the MMAs; warps 2-5 compute the Conv1D of every job; NE epilogue
+// warpgroups take the jobs round robin, connected by mbarriers. Tiles
+// of a unit are claimed in time order by running CTAs only, so every
 // look-back waits on a tile that a running CTA owns. Every wait is bounded:
 // on expiry the kernel records RGLRU_ERR_TIMEOUT, raises an abort flag that
 // all waits observe, drains what it issued and returns.
@@ -40,12 +43,14 @@ namespace {
 using namespace tc;
 
 constexpr int kM = 128;         // output channels per unit (MMA M, TMEM lanes)
-constexpr int kJQ = 4;          // job ring depth
-constexpr int kThreads = 320;
+constexpr int kJQ = 8;          // job ring depth
 constexpr uint64_t kWaitNs = 2000000000ull;   // bound of any wait
 constexpr uint64_t kDrainNs = 200000000ull;   // bound of the drain after an abort
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
+// sqrt((1 - e^(2w)) / (-2w)) ~= 1 + w (G1 + w (G2 + w G3)) on w in [-1/8, 0]
+// (least-squares/minimax fit made for this kernel; max rel. error 7e-8 in fp32).
+constexpr float kG1 = 0.49999531f, kG2 = 0.20810417f, kG3 = 0.05930331f;
+constexpr float kFastLimit = 0.125f;          // fast path when c * softplus(-Lambda) <= 1/8
 
 struct TcParams {
   const __nv_bfloat16 *conv_w, *b_a, *b_x;
@@ -61,29 +66,38 @@ struct TcParams {
   int *dev_status;
 };
 
-template <int K, int N, int NX>
+template <int K, int N, int NX, int NE>
 struct Cfg {
+  // warps: 0 producer, 1 MMA, 2-5 conv, then NE epilogue warpgroups
+  static constexpr int kThreads = 64 + 128 + NE * 128;
   static constexpr int kXRows = N + 3;
   static constexpr int kXBytes = ((kXRows * K * 2) + 1023) / 1024 * 1024;
   static constexpr int kABytes = K * 256;          // one gate: 2 M-blocks x K rows x 128 B
-  static constexpr int kBBytes = N * K * 2;        // one slot
+  static constexpr int kBBytes = N * K * 2;        // K-major conv output, one slot
+  // fp32 u of the unit's own channels, token-major [N][128], for beta (K = 128
+  // only; with K = 256 the epilogue recomputes u from the x tile instead)
+  static constexpr bool kUTile = (K == 128);
+  static constexpr int kUBytes = kUTile ? N * kM * 4 : 0;
+  static constexpr int kNS = 2;                    // conv -> MMA / epilogue slots
+  static constexpr int kNT = 2 * NE;               // TMEM slots
   static constexpr int kOffA = 0;
   static constexpr int kOffX = 2 * kABytes;
   static constexpr int kOffB = kOffX + NX * kXBytes;
-  static constexpr int kOffBar = kOffB + 2 * kBBytes;
-  // barriers: job_full[JQ], job_empty[JQ], x_full[NX], x_empty[NX], w_full, b_full[2], acc_full[2]
-  static constexpr int kNumBars = 2 * kJQ + 2 * NX + 1 + 2 + 2;
+  static constexpr int kOffU = kOffB + kNS * kBBytes;
+  static constexpr int kOffBar = kOffU + kNS * kUBytes;
+  // job_full[JQ], job_empty[JQ], x_full[NX], x_empty[NX], w_full, w_free,
+  // b_full[NS], b_empty[NS], u_empty[NS], acc_full[NT], tmem_empty[NT]
+  static constexpr int kNumBars = 2 * kJQ + 2 * NX + 2 + 3 * kNS + 2 * kNT;
   static constexpr int kOffJobs = (kOffBar + kNumBars * 8 + 15) / 16 * 16;
   static constexpr int kOffMisc = kOffJobs + kJQ * 16;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;   // + alignment slack
-  // TMEM per slot: z_a (N columns), z_x (N), u (N); two slots.
-  static constexpr int kSlotCols = 3 * N;
-  static constexpr int kTmemCols = (2 * kSlotCols <= 128) ? 128 : (2 * kSlotCols <= 256 ? 256 : 512);
-  static constexpr int kChunks = N / 32;   // conv: 32-token chunks
-  static constexpr int kEChunks = N / 16;  // epilogue: 16-token chunks
-  static_assert(N % 32 == 0 && K % 128 == 0, "tile shape");
+  static constexpr int kSlotCols = 2 * N;                   // z_a | z_x, then a | beta
+  static constexpr int kTmemCols =
+      kNT * kSlotCols <= 128 ? 128 : (kNT * kSlotCols <= 256 ? 256 : 512);
+  static_assert((N * (K / 4)) % 128 == 0, "conv mapping");
+  static_assert(N % 16 == 0 && K % 128 == 0, "tile shape");
   static_assert(kSmemBytes <= 232448, "shared memory");
-  static_assert(2 * kSlotCols <= 512, "TMEM allocation");
+  static_assert(kNT * kSlotCols <= 512, "TMEM allocation");
 };
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -120,23 +134,64 @@ __device__ __forceinline__ void st_release(int *p, int v) {
   asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Per element, from the gate pre-activations za, zx (bias included), the conv
-// output u and nc2 = -c * softplus(-Lambda) * log2(e):
-//   r = sigmoid(za) = sqrt_r^2 with sqrt_r = (1 + e^-za)^(-1/2),
-//   i = sigmoid(zx) = (1 + tanh(zx / 2)) / 2,
-//   log2 a = nc2 * r,  a = 2^(log2 a),
-//   1 - a^2 = -expm1(2 ln a): a series in v = 2 ln a near a = 1, else 1 - a*a,
-//   beta = sqrt(1 - a^2) * i * u.
-__device__ __forceinline__ void gate_decay(float za, float zx, float u, float nc2, float &a,
-                                           float &beta, float &la2) {
-  const float e = ex2_approx(-za * kLog2e);
+__device__ __forceinline__ float2 f2(float v) { return make_float2(v, v); }
+
+// bf16 pair (low half = first element) -> two floats
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+__device__ __forceinline__ uint32_t f2_to_bf2(float2 v) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+  return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// Per-channel constants of the epilogue.
+struct ChanK {
+  float kba;    // -(b_a) log2 e
+  float hbx;    // b_x / 2
+  float nc;     // -c softplus(-Lambda): ln a_t = nc * r_t
+  float k2sp;   // 2 sqrt(softplus(-Lambda))
+  float nc2;    // nc log2 e (general path)
+};
+
+// Fast path, two tokens of one channel, valid when |nc| <= 1/8:
+//   e = 2^(-(za + ba) log2 e), sqrt_r = (1 + e)^(-1/2), r = sqrt_r^2,
+//   ln a = nc r, a = e^(ln a) (Taylor, degree 5),
+//   sqrt(1 - a^2) = sqrt(-2 ln a) sqrt(g(ln a)) = 4 sqrt(sp) sqrt_r sqrt(g),
+//   i = (1 + tanh((zx + bx) / 2)) / 2,  beta = sqrt(1 - a^2) i u.
+__device__ __forceinline__ void gate_pair_fast(float2 za, float2 zx, float2 u, const ChanK &k,
+                                               float2 &a, float2 &beta, float2 &la) {
+  const float2 earg = __ffma2_rn(za, f2(-kLog2e), f2(k.kba));
+  float2 d = make_float2(ex2_approx(earg.x), ex2_approx(earg.y));
+  d = __fadd2_rn(d, f2(1.0f));
+  const float2 q = make_float2(rsqrt_approx(d.x), rsqrt_approx(d.y));
+  la = __fmul2_rn(__fmul2_rn(q, q), f2(k.nc));
+  float2 pa = __ffma2_rn(la, f2(1.0f / 120.0f), f2(1.0f / 24.0f));
+  pa = __ffma2_rn(la, pa, f2(1.0f / 6.0f));
+  pa = __ffma2_rn(la, pa, f2(0.5f));
+  pa = __ffma2_rn(la, pa, f2(1.0f));
+  a = __ffma2_rn(la, pa, f2(1.0f));
+  float2 sg = __ffma2_rn(la, f2(kG3), f2(kG2));
+  sg = __ffma2_rn(la, sg, f2(kG1));
+  sg = __ffma2_rn(la, sg, f2(1.0f));
+  const float2 targ = __ffma2_rn(zx, f2(0.5f), f2(k.hbx));
+  const float2 t = make_float2(tanh_approx(targ.x), tanh_approx(targ.y));
+  const float2 ig = __ffma2_rn(t, f2(k.k2sp), f2(k.k2sp));   // 4 sqrt(sp) i
+  beta = __fmul2_rn(__fmul2_rn(__fmul2_rn(q, sg), ig), u);
+}
+
+// General path, one element: as above but a = 2^(log2 a) on the MUFU and
+// 1 - a^2 = -expm1(2 ln a) by its series near a = 1, else 1 - a*a.
+__device__ __forceinline__ void gate_one(float za, float zx, float u, const ChanK &k, float &a,
+                                         float &beta, float &la) {
+  const float e = ex2_approx(fmaf(za, -kLog2e, k.kba));
   const float q = rsqrt_approx(1.0f + e);
   const float r = q * q;
-  const float ig = fmaf(0.5f, tanh_approx(0.5f * zx), 0.5f);
-  la2 = nc2 * r;
+  const float ig = fmaf(0.5f, tanh_approx(fmaf(zx, 0.5f, k.hbx)), 0.5f);
+  const float la2 = k.nc2 * r;
+  la = k.nc * r;
   a = ex2_approx(la2);
-  const float v = la2 * (2.0f * kLn2);
-  // expm1(v) / v = 1 + v/2 + v^2/6 + v^3/24 + v^4/120 + v^5/720 (|v| <= 1/4)
+  const float v = 2.0f * la;
   float p = fmaf(v, 1.0f / 720.0f, 1.0f / 120.0f);
   p = fmaf(v, p, 1.0f / 24.0f);
   p = fmaf(v, p, 1.0f / 6.0f);
@@ -145,8 +200,6 @@ __device__ __forceinline__ void gate_decay(float za, float zx, float u, float nc
   const float om = (v > -0.25f) ? (-v * p) : fmaf(-a, a, 1.0f);
   beta = sqrt_approx(om) * ig * u;
 }
-
-__device__ __forceinline__ float bf2f(__nv_bfloat16 v) { return __bfloat162float(v); }
 
 __device__ void raise_abort(const TcParams &p, volatile int *cta_abort, int code) {
   if (p.dev_status) atomicCAS(p.dev_status, 0, code);
@@ -161,7 +214,7 @@ __device__ int poll_flag(const int *flag, const int *gabort, volatile int *cta_a
   if (v) return v;
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
-    __nanosleep(40);
+    __nanosleep(32);
     v = ld_acquire(flag);
     if (v) return v;
     if (*cta_abort || *(volatile const int *)gabort) return -1;
@@ -169,29 +222,92 @@ __device__ int poll_flag(const int *flag, const int *gabort, volatile int *cta_a
   }
 }
 
-template <int K, int N, int NX>
-__global__ void __launch_bounds__(kThreads, 1)
+// Conv1D of one tile, token-major. Thread t covers the 4 channels
+// [4 q, 4 q + 4) of the K range and SEG consecutive tokens; a warp covers 128
+// channels of one token segment, so that its shared-memory rows are contiguous
+// (no bank conflicts). All input rows are read before any output is written.
+// Writes the bf16 B operand (K-major, 128-byte swizzle) and, when kUTile, the
+// fp32 u of the unit's own channels token-major into ut ([N][128] floats).
+// w holds the 4 taps of the 4 channels (pairs).
+template <int K, int N, bool kUTile>
+__device__ __forceinline__ void conv_tile(const unsigned char *__restrict__ xs,
+                                          unsigned char *__restrict__ bt,
+                                          unsigned char *__restrict__ ut, const TcParams &p, int b,
+                                          int kbase, int own_lo, int tile, int nvalid,
+                                          bool last_tile, int t, const float2 (&w)[4][2]) {
+  constexpr int NQ = K / 4;                         // channel quads
+  constexpr int SEG = N * NQ / 128;                 // tokens per thread
+  const int qd = t % NQ, sg = t / NQ;
+  const int kq = qd * 4, nb = sg * SEG;
+  const bool own = (kq >= own_lo) && (kq < own_lo + kM);
+  const int chq = kbase + kq;                       // first global channel of the quad
+  uint2 rows[SEG + 3];
+#pragma unroll
+  for (int r = 0; r < SEG + 3; ++r)
+    rows[r] = *reinterpret_cast<const uint2 *>(xs + ((nb + r) * K + kq) * 2);
+  if (tile == 0 && nb == 0 && p.conv_state_in != nullptr) {
+#pragma unroll
+    for (int r = 0; r < 3; ++r)
+      rows[r] = __ldg(reinterpret_cast<const uint2 *>(p.conv_state_in +
+                                                       (static_cast<size_t>(b) * 3 + r) * p.D + chq));
+  }
+#pragma unroll
+  for (int j = 0; j < SEG; ++j) {
+    const int n = nb + j;
+    float2 u[2];
+#pragma unroll
+    for (int pp = 0; pp < 2; ++pp) {
+      const uint32_t r0 = pp ? rows[j].y : rows[j].x, r1 = pp ? rows[j + 1].y : rows[j + 1].x;
+      const uint32_t r2 = pp ? rows[j + 2].y : rows[j + 2].x, r3 = pp ? rows[j + 3].y : rows[j + 3].x;
+      float2 acc = __fmul2_rn(w[0][pp], bf2_to_f2(r0));
+      acc = __ffma2_rn(w[1][pp], bf2_to_f2(r1), acc);
+      acc = __ffma2_rn(w[2][pp], bf2_to_f2(r2), acc);
+      u[pp] = __ffma2_rn(w[3][pp], bf2_to_f2(r3), acc);
+    }
+    *reinterpret_cast<uint2 *>(bt + kmajor_sw128_offset(n, kq, N)) =
+        make_uint2(f2_to_bf2(u[0]), f2_to_bf2(u[1]));
+    if (kUTile && own)
+      *reinterpret_cast<float4 *>(ut + (n * kM + kq - own_lo) * 4) =
+          make_float4(u[0].x, u[0].y, u[1].x, u[1].y);
+    if (own && last_tile && n == nvalid - 1 && p.conv_state_out != nullptr) {
+      // the last three inputs x_{T-3}, x_{T-2}, x_{T-1} of these 4 channels
+#pragma unroll
+      for (int r = 0; r < 3; ++r)
+        *reinterpret_cast<uint2 *>(p.conv_state_out + (static_cast<size_t>(b) * 3 + r) * p.D +
+                                   chq) = rows[j + 1 + r];
+    }
+  }
+}
+
+template <int K, int N, int NX, int NE>
+__global__ void __launch_bounds__(Cfg<K, N, NX, NE>::kThreads, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_wa,
               const __grid_constant__ CUtensorMap tmap_wx, const TcParams p) {
-  using C = Cfg<K, N, NX>;
+  using C = Cfg<K, N, NX, NE>;
+  constexpr int NS = C::kNS, NT = C::kNT;
   extern __shared__ unsigned char smem_raw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   unsigned char *sA = sm + C::kOffA;
   unsigned char *sX = sm + C::kOffX;
   unsigned char *sB = sm + C::kOffB;
+  unsigned char *sU = sm + C::kOffU;
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::kOffBar);
   uint64_t *job_full = bars;
-  uint64_t *job_empty = bars + kJQ;
-  uint64_t *x_full = bars + 2 * kJQ;
+  uint64_t *job_empty = job_full + kJQ;
+  uint64_t *x_full = job_empty + kJQ;
   uint64_t *x_empty = x_full + NX;
   uint64_t *w_full = x_empty + NX;
-  uint64_t *b_full = w_full + 1;
-  uint64_t *acc_full = b_full + 2;
+  uint64_t *w_free = w_full + 1;                    // MMAs reading the old weights are done
+  uint64_t *b_full = w_free + 1;                    // [NS] conv -> MMA
+  uint64_t *b_empty = b_full + NS;                  // [NS] MMA -> conv
+  uint64_t *u_empty = b_empty + NS;                 // [NS] epilogue pass 1 -> conv
+  uint64_t *acc_full = u_empty + NS;                // [NT] MMA -> epilogue
+  uint64_t *tmem_empty = acc_full + NT;             // [NT] epilogue pass 2 -> MMA
   int4 *jobs = reinterpret_cast<int4 *>(sm + C::kOffJobs);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + C::kOffMisc);
   volatile int *cta_abort = reinterpret_cast<volatile int *>(sm + C::kOffMisc + 4);
-  volatile int *bcast = reinterpret_cast<volatile int *>(sm + C::kOffMisc + 8);  // [2]
+  volatile int *bcast = reinterpret_cast<volatile int *>(sm + C::kOffMisc + 8);  // [NE][2]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -200,20 +316,24 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
   if (tid == 0) {
     for (int i = 0; i < kJQ; ++i) {
       mbar_init(&job_full[i], 1);
-      mbar_init(&job_empty[i], 2);
+      mbar_init(&job_empty[i], 3);                  // conv, MMA, epilogue
     }
     for (int i = 0; i < NX; ++i) {
       mbar_init(&x_full[i], 1);
       mbar_init(&x_empty[i], 1);
     }
     mbar_init(w_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    mbar_init(w_free, 1);
+    for (int i = 0; i < NS; ++i) {
       mbar_init(&b_full[i], 1);
+      mbar_init(&b_empty[i], 1);
+      mbar_init(&u_empty[i], 1);
+    }
+    for (int i = 0; i < NT; ++i) {
       mbar_init(&acc_full[i], 1);
+      mbar_init(&tmem_empty[i], 1);
     }
     *cta_abort = 0;
-    bcast[0] = 0;
-    bcast[1] = 0;
     fence_mbar_init();
     prefetch_tmap(&tmap_x);
     prefetch_tmap(&tmap_wa);
@@ -221,7 +341,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
   }
   {
     uint4 *a4 = reinterpret_cast<uint4 *>(sA);
-    for (int i = tid; i < 2 * C::kABytes / 16; i += kThreads) a4[i] = make_uint4(0, 0, 0, 0);
+    for (int i = tid; i < 2 * C::kABytes / 16; i += C::kThreads) a4[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
   }
   if (warp == 1) {
@@ -234,12 +354,18 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
   const uint32_t tmem_base = *tmem_slot;
   const int R = p.bw <= 128 ? p.bw : 256;           // weight rows per TMA box
 
+#define RG_WAIT_OR_ABORT(bar, par)                                   \
+  if (!mbar_wait((bar), (par), cta_abort, kWaitNs)) {                \
+    if (!*cta_abort) raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);   \
+    break;                                                           \
+  }
+
   if (warp == 0) {
     // =============================== producer ===============================
     if (lane == 0) {
       int unit = blockIdx.x % p.n_units, scanned = 0, w_unit = -1;
       int i = 0, last_x_job = -1;
-      bool ok = true;
+      uint32_t wfree_phase = 0;
       for (;; ++i) {
         int tile = -1;
         while (unit >= 0) {
@@ -253,29 +379,27 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
         }
         if (*cta_abort) unit = -1;
         const int js = i % kJQ;
-        if (!mbar_wait(&job_empty[js], ((i / kJQ) & 1) ^ 1, cta_abort, kWaitNs)) {
-          if (!*cta_abort) raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);
-          ok = false;
-          break;
-        }
+        RG_WAIT_OR_ABORT(&job_empty[js], ((i / kJQ) & 1) ^ 1);
         const int reload = (unit >= 0 && unit != w_unit) ? 1 : 0;
         jobs[js] = make_int4(unit, tile, reload, 0);
         mbar_arrive(&job_full[js]);
         if (unit < 0) {
-          const int j2 = (i + 1) % kJQ;
-          if (mbar_wait(&job_empty[j2], (((i + 1) / kJQ) & 1) ^ 1, cta_abort, kWaitNs)) {
-            jobs[j2] = make_int4(-1, -1, 0, 0);
-            mbar_arrive(&job_full[j2]);
+          // one terminal job per epilogue warpgroup that may still wait for a job
+          for (int e = 1; e < NE; ++e) {
+            const int je = i + e;
+            if (!mbar_wait(&job_empty[je % kJQ], ((je / kJQ) & 1) ^ 1, cta_abort, kWaitNs)) break;
+            jobs[je % kJQ] = make_int4(-1, -1, 0, 0);
+            mbar_arrive(&job_full[je % kJQ]);
           }
           break;
         }
         const int b = unit / p.n_cg, cg = unit % p.n_cg;
         if (reload) {
-          if (i > 0 && !mbar_wait(&job_empty[(i - 1) % kJQ], ((i - 1) / kJQ) & 1, cta_abort,
-                                  kWaitNs)) {
-            if (!*cta_abort) raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);
-            ok = false;
-            break;
+          if (i > 0) {
+            // the MMA warp signals once the MMAs of job i-1 (the last readers of
+            // the weights in shared memory) have completed
+            RG_WAIT_OR_ABORT(w_free, wfree_phase);
+            wfree_phase ^= 1;
           }
           mbar_arrive_expect_tx(w_full, 2u * 2u * static_cast<uint32_t>(R) * 128u);
           for (int g = 0; g < 2; ++g) {
@@ -297,17 +421,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
           w_unit = unit;
         }
         const int xb = i % NX;
-        if (!mbar_wait(&x_empty[xb], ((i / NX) & 1) ^ 1, cta_abort, kWaitNs)) {
-          if (!*cta_abort) raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);
-          ok = false;
-          break;
-        }
+        RG_WAIT_OR_ABORT(&x_empty[xb], ((i / NX) & 1) ^ 1);
         const int kbase = p.bw <= 128 ? cg * kM : (cg >> 1) * 256;
         mbar_arrive_expect_tx(&x_full[xb], static_cast<uint32_t>(C::kXRows * K * 2));
         tma_load_3d(sX + xb * C::kXBytes, &tmap_x, &x_full[xb], kbase, tile * N - 3, b);
         last_x_job = i;
       }
-      if (!ok || *cta_abort) {
+      if (*cta_abort) {
         // drain: let every TMA this thread issued land before the CTA exits
         for (int j = last_x_job; j >= 0 && j > last_x_job - NX; --j)
           mbar_wait_drain(&x_full[j % NX], (j / NX) & 1, kDrainNs);
@@ -322,27 +442,25 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
       int last_commit = -1;
       for (int i = 0;; ++i) {
         const int js = i % kJQ;
-        if (!mbar_wait(&job_full[js], (i / kJQ) & 1, cta_abort, kWaitNs)) {
-          if (!*cta_abort) raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);
-          break;
-        }
+        RG_WAIT_OR_ABORT(&job_full[js], (i / kJQ) & 1);
         const int4 job = jobs[js];
         if (job.x < 0) break;
         if (job.z) {
-          if (!mbar_wait(w_full, w_phase, cta_abort, kWaitNs)) {
-            if (!*cta_abort) raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);
-            break;
+          if (last_commit >= 0) {
+            // MMAs complete in order: job i-1 done => every read of the old weights done
+            const int lc = last_commit;
+            RG_WAIT_OR_ABORT(&acc_full[lc % NT], (lc / NT) & 1);
+            mbar_arrive(w_free);
           }
+          RG_WAIT_OR_ABORT(w_full, w_phase);
           w_phase ^= 1;
         }
-        const int s = i & 1;
-        if (!mbar_wait(&b_full[s], (i >> 1) & 1, cta_abort, kWaitNs)) {
-          if (!*cta_abort) raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);
-          break;
-        }
+        const int s = i % NS, ts = i % NT;
+        RG_WAIT_OR_ABORT(&b_full[s], (i / NS) & 1);
+        RG_WAIT_OR_ABORT(&tmem_empty[ts], ((i / NT) & 1) ^ 1);
         tc_fence_after();
         const uint32_t bs = smem_u32(sB + s * C::kBBytes);
-        const uint32_t d_a = tmem_base + static_cast<uint32_t>(s * C::kSlotCols);
+        const uint32_t d_a = tmem_base + static_cast<uint32_t>(ts * C::kSlotCols);
         const uint32_t d_x = d_a + N;
 #pragma unroll
         for (int ks = 0; ks < K / 16; ++ks) {
@@ -352,215 +470,330 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
           mma_bf16(d_a, ada, bd, idesc, ks > 0 ? 1u : 0u);
           mma_bf16(d_x, adx, bd, idesc, ks > 0 ? 1u : 0u);
         }
-        mma_commit(&acc_full[s]);
+        mma_commit(&acc_full[ts]);
+        mma_commit(&b_empty[s]);
         last_commit = i;
         mbar_arrive(&job_empty[js]);
       }
       if (*cta_abort && last_commit >= 0)
-        mbar_wait_drain(&acc_full[last_commit & 1], (last_commit >> 1) & 1, kDrainNs);
+        mbar_wait_drain(&acc_full[last_commit % NT], (last_commit / NT) & 1, kDrainNs);
     }
-  } else {
-    // ============================== warpgroups ==============================
-    const int wg = (warp - 2) >> 2;               // 0 or 1
-    const int m = (warp & 3) * 32 + lane;         // TMEM lane == output channel in unit
-    const bool leader = (warp == 2 + 4 * wg) && lane == 0;
-    const int bar_id = 1 + wg;
-    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) +
-                            static_cast<uint32_t>(wg * C::kSlotCols);
-    unsigned char *bslot = sB + wg * C::kBBytes;
-    constexpr int KC = K / kM;                    // conv channels per thread (1 or 2)
+  } else if (warp < 6) {
+    // ============================ conv warpgroup ============================
+    const int wt = tid - 64;                      // 0 .. 127
+    const bool leader = (wt == 0);
     int cur_unit = -1;
-    float cw[KC][4];
-    float ba = 0.f, bx = 0.f, nc2 = 0.f;
-    int own_kk = 0;
-
-    for (int i = wg;; i += 2) {
+    float2 cwq[4][2];                             // conv taps of this thread's channel quad
+    for (int i = 0;; ++i) {
       const int js = i % kJQ;
-      if (!mbar_wait(&job_full[js], (i / kJQ) & 1, cta_abort, kWaitNs)) {
-        if (!*cta_abort) raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);
-        break;
-      }
+      RG_WAIT_OR_ABORT(&job_full[js], (i / kJQ) & 1);
       const int4 job = jobs[js];
       const int unit = job.x, tile = job.y;
       if (unit < 0) break;
       const int b = unit / p.n_cg, cg = unit % p.n_cg;
-      const int c = cg * kM + m;                  // own output channel
       const int kbase = p.bw <= 128 ? cg * kM : (cg >> 1) * 256;
+      const int own_lo = p.bw <= 128 ? 0 : (cg & 1) * kM;
+      const int nvalid = min(N, p.T - tile * N);
       if (unit != cur_unit) {
         cur_unit = unit;
-        own_kk = p.bw <= 128 ? 0 : (cg & 1);
+        const int chq = kbase + (wt % (K / 4)) * 4;
 #pragma unroll
-        for (int kk = 0; kk < KC; ++kk) {
-          const int ch = kbase + kk * kM + m;
-#pragma unroll
-          for (int tap = 0; tap < 4; ++tap) cw[kk][tap] = bf2f(p.conv_w[tap * p.D + ch]);
+        for (int tap = 0; tap < 4; ++tap) {
+          const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(p.conv_w + tap * p.D + chq));
+          cwq[tap][0] = bf2_to_f2(raw.x);
+          cwq[tap][1] = bf2_to_f2(raw.y);
         }
-        ba = bf2f(p.b_a[c]);
-        bx = bf2f(p.b_x[c]);
-        nc2 = -kDecayC * softplus_f32(-p.Lambda[c]) * kLog2e;
       }
+      const int s = i % NS, xb = i % NX;
+      RG_WAIT_OR_ABORT(&x_full[xb], (i / NX) & 1);
+      RG_WAIT_OR_ABORT(&b_empty[s], ((i / NS) & 1) ^ 1);
+      if (C::kUTile) RG_WAIT_OR_ABORT(&u_empty[s], ((i / NS) & 1) ^ 1);
+      conv_tile<K, N, C::kUTile>(sX + xb * C::kXBytes, sB + s * C::kBBytes, sU + s * C::kUBytes,
+                                 p, b, kbase, own_lo, tile, nvalid, tile == p.n_tiles - 1, wt,
+                                 cwq);
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (leader) {
+        if (C::kUTile) mbar_arrive(&x_empty[xb]);   // else the epilogue still reads x
+        mbar_arrive(&b_full[s]);
+        mbar_arrive(&job_empty[js]);
+      }
+    }
+  } else {
+    // ========================== epilogue warpgroups ==========================
+    // Epilogue warpgroup e takes jobs e, e + NE, ... Per job: pass 1 (gates,
+    // decay, local scan) and publish of the tile's aggregate; then the carry
+    // (look-back) and pass 2 of the warpgroup's previous job, whose
+    // predecessors have usually published by then.
+    const int eg = (warp - 6) >> 2;               // 0 .. NE-1
+    const int wt = tid - 192 - eg * 128;          // 0 .. 127
+    const int m = (warp & 3) * 32 + lane;         // TMEM lane == output channel in unit
+    const bool leader = (wt == 0);
+    const bool leader_warp = (wt >> 5) == 0;
+    const int bar_id = 2 + eg;
+    const uint32_t t_lane0 = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    int cur_unit = -1;
+    ChanK kc{0.f, 0.f, 0.f, 0.f, 0.f};
+    float cwo[4] = {0.f, 0.f, 0.f, 0.f};          // own channel's conv taps (K = 256)
+    bool fast = true;
+    int it_b = 0;                                 // broadcast slot parity
+    int d_i = -1, d_unit = 0, d_tile = 0;         // the deferred job
+    float d_A = 0.f, d_H = 0.f;
+
+    // ---- carry and pass 2 of the deferred job ----
+    auto phase_b = [&]() {
+      const int unit = d_unit, tile = d_tile;
+      const int b = unit / p.n_cg, cg = unit % p.n_cg;
+      const int c = cg * kM + m;
       const int n0 = tile * N;
       const int nvalid = min(N, p.T - n0);
       const bool last_tile = (tile == p.n_tiles - 1);
-
-      // ---- Conv1D into the B operand (and own channel's u in registers) ----
-      const int xb = i % NX;
-      if (!mbar_wait(&x_full[xb], (i / NX) & 1, cta_abort, kWaitNs)) {
-        if (!*cta_abort) raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);
-        break;
-      }
-      const __nv_bfloat16 *xs = reinterpret_cast<const __nv_bfloat16 *>(sX + xb * C::kXBytes);
-#pragma unroll
-      for (int kk = 0; kk < KC; ++kk) {
-        const int k = kk * kM + m;                // index within the K range
-        float xm3 = bf2f(xs[0 * K + k]), xm2 = bf2f(xs[1 * K + k]), xm1 = bf2f(xs[2 * K + k]);
-        if (tile == 0 && p.conv_state_in != nullptr) {
-          const __nv_bfloat16 *cs = p.conv_state_in + static_cast<size_t>(b) * 3 * p.D + kbase + k;
-          xm3 = bf2f(cs[0]);
-          xm2 = bf2f(cs[p.D]);
-          xm1 = bf2f(cs[2 * p.D]);
-        }
-        const bool own = (kk == own_kk);          // uniform across the warpgroup
-        // byte offsets of (row n, channel k) in the swizzled operand depend on n % 8 only,
-        // besides the n * 128 row term
-        uint32_t colo[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) colo[r] = kmajor_sw128_offset(r, k, N) - r * 128;
-#pragma unroll
-        for (int ch = 0; ch < C::kEChunks; ++ch) {
-          float uc[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = ch * 16 + j;
-            const float xv = bf2f(xs[(n + 3) * K + k]);
-            const float u =
-                fmaf(cw[kk][3], xv, fmaf(cw[kk][2], xm1, fmaf(cw[kk][1], xm2, cw[kk][0] * xm3)));
-            xm3 = xm2;
-            xm2 = xm1;
-            xm1 = xv;
-            *reinterpret_cast<__nv_bfloat16 *>(bslot + colo[n & 7] + n * 128) =
-                __float2bfloat16_rn(u);
-            uc[j] = u;
-            if (own && last_tile && n == nvalid - 1 && p.conv_state_out != nullptr) {
-              __nv_bfloat16 *co = p.conv_state_out + static_cast<size_t>(b) * 3 * p.D + c;
-              co[0] = __float2bfloat16_rn(xm3);
-              co[p.D] = __float2bfloat16_rn(xm2);
-              co[2 * p.D] = __float2bfloat16_rn(xm1);
-            }
-          }
-          if (own) tmem_st16(t_lane + 2 * N + ch * 16, uc);   // own channel's u for beta
-        }
-      }
-      tmem_wait_st();
-      fence_proxy_async_smem();
-      named_bar_sync(bar_id, 128);
-      if (leader) {
-        mbar_arrive(&x_empty[xb]);
-        mbar_arrive(&b_full[wg]);
-      }
-
-      // ---- gates, decay, local scan (pass 1) ----
-      if (!mbar_wait(&acc_full[wg], (i >> 1) & 1, cta_abort, kWaitNs)) {
-        if (!*cta_abort) raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);
-        break;
-      }
-      tc_fence_after();
-      float Hl = 0.f, S = 0.f;
-#pragma unroll
-      for (int ch = 0; ch < C::kEChunks; ++ch) {
-        float za[16], zx[16], uu[16];
-        tmem_ld16(t_lane + ch * 16, za);
-        tmem_ld16(t_lane + N + ch * 16, zx);
-        tmem_ld16(t_lane + 2 * N + ch * 16, uu);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int n = ch * 16 + j;
-          float a, beta, la2;
-          gate_decay(za[j] + ba, zx[j] + bx, uu[j], nc2, a, beta, la2);
-          if (n >= nvalid) {
-            a = 1.f;
-            beta = 0.f;
-            la2 = 0.f;
-          }
-          Hl = fmaf(a, Hl, beta);
-          S += la2;
-          za[j] = a;
-          zx[j] = beta;
-        }
-        tmem_st16(t_lane + ch * 16, za);
-        tmem_st16(t_lane + N + ch * 16, zx);
-      }
-      tmem_wait_st();
-      const float A = ex2_approx(S);
-
-      // ---- carry across tiles: decoupled look-back ----
-      const size_t tix = static_cast<size_t>(unit) * p.n_tiles + tile;
+      const int ts = d_i % NT;
+      const uint32_t t_lane = t_lane0 + static_cast<uint32_t>(ts * C::kSlotCols);
+      const size_t ubase = static_cast<size_t>(unit) * p.n_tiles;
       float h_in = 0.f;
       if (tile == 0) {
         if (p.h0 != nullptr) h_in = p.h0[static_cast<size_t>(b) * p.D + c];
       } else {
-        __stcg(p.aggA + tix * kM + m, A);
-        __stcg(p.aggH + tix * kM + m, Hl);
-        __threadfence();
-        named_bar_sync(bar_id, 128);
-        if (leader) st_release(p.flags + tix, 1);
+        // Look back over a window of up to 32 predecessors: the leader warp
+        // reads their flags at once and finds the nearest inclusive state with
+        // only aggregates after it; every thread then folds those in.
         float mult = 1.f, add = 0.f;
-        int jt = tile - 1;
+        int top = tile - 1;
         for (;;) {
-          if (leader) {
-            int f = poll_flag(p.flags + static_cast<size_t>(unit) * p.n_tiles + jt, p.abort_flag,
-                              cta_abort);
-            if (f == -2) {
-              raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);
-              f = -1;
+          const int slot = eg * 2 + (it_b & 1);
+          ++it_b;
+          if (leader_warp) {
+            const int jt = top - lane;
+            int res;
+            const uint64_t t0 = globaltimer_ns();
+            for (;;) {
+              const int f = (jt >= 0) ? ld_acquire(p.flags + ubase + jt) : 0;
+              const unsigned agg = __ballot_sync(0xffffffffu, f >= 1);
+              const unsigned inc = __ballot_sync(0xffffffffu, f == 2);
+              if (inc != 0u) {
+                const int e = __ffs(inc) - 1;     // nearest inclusive
+                const unsigned below = (e == 0) ? 0u : (0xffffffffu >> (32 - e));
+                if ((agg & below) == below) { res = e; break; }
+              } else if (agg == 0xffffffffu) {
+                res = 32;                         // 32 aggregates, no inclusive yet: fold, go on
+                break;
+              }
+              if (*cta_abort || *(volatile const int *)p.abort_flag) { res = -1; break; }
+              if (globaltimer_ns() - t0 > kWaitNs) { res = -2; break; }
+              __nanosleep(32);
             }
-            bcast[wg] = f;
+            if (lane == 0) {
+              if (res == -2) {
+                raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);
+                res = -1;
+              }
+              bcast[slot] = res;
+            }
           }
           named_bar_sync(bar_id, 128);
-          const int f = bcast[wg];
-          named_bar_sync(bar_id, 128);
-          const size_t jix = (static_cast<size_t>(unit) * p.n_tiles + jt) * kM + m;
-          if (f == 2) {
-            h_in = fmaf(mult, __ldcg(p.incH + jix), add);
-            break;
-          }
-          if (f != 1) {
+          const int e = bcast[slot];
+          if (e < 0) {
             h_in = 0.f;
             break;
           }
-          add = fmaf(mult, __ldcg(p.aggH + jix), add);
-          mult *= __ldcg(p.aggA + jix);
-          --jt;
+          const int nagg = e < 32 ? e : 32;
+          for (int k = 0; k < nagg; k += 4) {
+            float Av[4], Hv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const bool in = k + q < nagg;
+              const size_t jix = (ubase + (in ? top - k - q : top)) * kM + m;
+              Av[q] = in ? __ldcg(p.aggA + jix) : 1.f;
+              Hv[q] = in ? __ldcg(p.aggH + jix) : 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              add = fmaf(mult, Hv[q], add);
+              mult *= Av[q];
+            }
+          }
+          if (e < 32) {
+            h_in = fmaf(mult, __ldcg(p.incH + (ubase + top - e) * kM + m), add);
+            break;
+          }
+          top -= 32;
         }
+        __stcg(p.incH + (ubase + tile) * kM + m, fmaf(d_A, h_in, d_H));
+        named_bar_sync(bar_id, 128);
+        if (leader) st_release(p.flags + ubase + tile, 2);
       }
-      __stcg(p.incH + tix * kM + m, fmaf(A, h_in, Hl));
-      __threadfence();
-      named_bar_sync(bar_id, 128);
-      if (leader) st_release(p.flags + tix, 2);
-
-      // ---- final scan (pass 2): y_t = h_t ----
+      // ---- pass 2: y_t = h_t ----
       float h = h_in;
       __nv_bfloat16 *yrow = p.y + (static_cast<size_t>(b) * p.T + n0) * p.D + c;
-#pragma unroll
-      for (int ch = 0; ch < C::kEChunks; ++ch) {
+#pragma unroll 1
+      for (int ch = 0; ch < N / 16; ++ch) {
         float av[16], bv[16];
         tmem_ld16(t_lane + ch * 16, av);
         tmem_ld16(t_lane + N + ch * 16, bv);
         tmem_wait_ld();
+        __nv_bfloat16 *yc = yrow + static_cast<size_t>(ch * 16) * p.D;
+        if (ch * 16 + 16 <= nvalid) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int n = ch * 16 + j;
-          h = fmaf(av[j], h, bv[j]);
-          if (n < nvalid) yrow[static_cast<size_t>(n) * p.D] = __float2bfloat16_rn(h);
+          for (int j = 0; j < 16; ++j) {
+            h = fmaf(av[j], h, bv[j]);
+            yc[static_cast<size_t>(j) * p.D] = __float2bfloat16_rn(h);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            h = fmaf(av[j], h, bv[j]);
+            if (ch * 16 + j < nvalid) yc[static_cast<size_t>(j) * p.D] = __float2bfloat16_rn(h);
+          }
         }
       }
       if (last_tile && p.h_T != nullptr) p.h_T[static_cast<size_t>(b) * p.D + c] = h;
       tc_fence_before();
       named_bar_sync(bar_id, 128);
-      if (leader) mbar_arrive(&job_empty[js]);
+      if (leader) {
+        mbar_arrive(&tmem_empty[ts]);
+        mbar_arrive(&job_empty[d_i % kJQ]);
+      }
+      d_i = -1;
+    };
+
+    for (int i = eg;; i += NE) {
+      const int js = i % kJQ;
+      RG_WAIT_OR_ABORT(&job_full[js], (i / kJQ) & 1);
+      const int4 job = jobs[js];
+      const int unit = job.x, tile = job.y;
+      if (unit < 0) break;
+      const int b = unit / p.n_cg, cg = unit % p.n_cg;
+      const int c = cg * kM + m;                  // own output channel
+      const int own_lo = p.bw <= 128 ? 0 : (cg & 1) * kM;
+      const int nvalid = min(N, p.T - tile * N);
+      const int s = i % NS, ts = i % NT, xb = i % NX;
+      const uint32_t t_lane = t_lane0 + static_cast<uint32_t>(ts * C::kSlotCols);
+      if (unit != cur_unit) {
+        cur_unit = unit;
+        const float sp = softplus_f32(-p.Lambda[c]);
+        kc.kba = -__bfloat162float(p.b_a[c]) * kLog2e;
+        kc.hbx = 0.5f * __bfloat162float(p.b_x[c]);
+        kc.nc = -kDecayC * sp;
+        kc.nc2 = kc.nc * kLog2e;
+        kc.k2sp = 2.0f * sqrtf(sp);
+        fast = __all_sync(0xffffffffu, kDecayC * sp <= kFastLimit);
+        if (!C::kUTile) {
+#pragma unroll
+          for (int tap = 0; tap < 4; ++tap) cwo[tap] = __bfloat162float(p.conv_w[tap * p.D + c]);
+        }
+      }
+      RG_WAIT_OR_ABORT(&acc_full[ts], (i / NT) & 1);
+      tc_fence_after();
+      // own channel's u: fp32 tile from the conv warpgroup (K = 128), or
+      // recomputed from the x tile (K = 256)
+      const unsigned char *uslot = sU + s * C::kUBytes;
+      const __nv_bfloat16 *xown =
+          reinterpret_cast<const __nv_bfloat16 *>(sX + xb * C::kXBytes) + own_lo + m;
+      float xm3 = 0.f, xm2 = 0.f, xm1 = 0.f;
+      if (!C::kUTile) {
+        xm3 = __bfloat162float(xown[0]);
+        xm2 = __bfloat162float(xown[K]);
+        xm1 = __bfloat162float(xown[2 * K]);
+        if (tile == 0 && p.conv_state_in != nullptr) {
+          const __nv_bfloat16 *cs = p.conv_state_in + static_cast<size_t>(b) * 3 * p.D + c;
+          xm3 = __bfloat162float(cs[0]);
+          xm2 = __bfloat162float(cs[p.D]);
+          xm1 = __bfloat162float(cs[2 * p.D]);
+        }
+      }
+      // ---- pass 1: gates, decay, local scan ----
+      float Hl = 0.f;
+      float2 S2 = make_float2(0.f, 0.f);
+#pragma unroll 1
+      for (int ch = 0; ch < N / 16; ++ch) {
+        float za[16], zx[16];
+        tmem_ld16(t_lane + ch * 16, za);
+        tmem_ld16(t_lane + N + ch * 16, zx);
+        float uu[16];
+        if (C::kUTile) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            uu[j] = *reinterpret_cast<const float *>(uslot + ((ch * 16 + j) * kM + m) * 4);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float xv = __bfloat162float(xown[(ch * 16 + j + 3) * K]);
+            uu[j] = fmaf(cwo[3], xv, fmaf(cwo[2], xm1, fmaf(cwo[1], xm2, cwo[0] * xm3)));
+            xm3 = xm2;
+            xm2 = xm1;
+            xm1 = xv;
+          }
+        }
+        tmem_wait_ld();
+        const bool full = (ch * 16 + 16 <= nvalid);
+        if (fast) {
+#pragma unroll
+          for (int pr = 0; pr < 8; ++pr) {
+            float2 a, beta, la;
+            gate_pair_fast(make_float2(za[2 * pr], za[2 * pr + 1]),
+                           make_float2(zx[2 * pr], zx[2 * pr + 1]),
+                           make_float2(uu[2 * pr], uu[2 * pr + 1]), kc, a, beta, la);
+            if (!full) {
+              const int n = ch * 16 + 2 * pr;
+              if (n >= nvalid) a.x = 1.f, beta.x = 0.f, la.x = 0.f;
+              if (n + 1 >= nvalid) a.y = 1.f, beta.y = 0.f, la.y = 0.f;
+            }
+            Hl = fmaf(a.x, Hl, beta.x);
+            Hl = fmaf(a.y, Hl, beta.y);
+            S2 = __fadd2_rn(S2, la);
+            za[2 * pr] = a.x;
+            za[2 * pr + 1] = a.y;
+            zx[2 * pr] = beta.x;
+            zx[2 * pr + 1] = beta.y;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            float a, beta, la;
+            gate_one(za[j], zx[j], uu[j], kc, a, beta, la);
+            if (ch * 16 + j >= nvalid) a = 1.f, beta = 0.f, la = 0.f;
+            Hl = fmaf(a, Hl, beta);
+            S2.x += la;
+            za[j] = a;
+            zx[j] = beta;
+          }
+        }
+        tmem_st16(t_lane + ch * 16, za);
+        tmem_st16(t_lane + N + ch * 16, zx);
+      }
+      tmem_wait_st();
+      const float A = ex2_approx((S2.x + S2.y) * kLog2e);
+      // publish this tile's state: inclusive for the first tile of a sequence
+      // (h0 is known), else the aggregate (prod a, local h); release the u / x
+      // tile to the conv warpgroup / producer
+      {
+        const size_t tix = static_cast<size_t>(unit) * p.n_tiles + tile;
+        if (tile == 0) {
+          const float h0v = p.h0 != nullptr ? p.h0[static_cast<size_t>(b) * p.D + c] : 0.f;
+          __stcg(p.incH + tix * kM + m, fmaf(A, h0v, Hl));
+        } else {
+          __stcg(p.aggA + tix * kM + m, A);
+          __stcg(p.aggH + tix * kM + m, Hl);
+        }
+        named_bar_sync(bar_id, 128);
+        if (leader) {
+          st_release(p.flags + tix, tile == 0 ? 2 : 1);
+          if (C::kUTile) mbar_arrive(&u_empty[s]);
+          else mbar_arrive(&x_empty[xb]);
+        }
+      }
+      // ---- carry and pass 2 of the previous job, then defer this one ----
+      if (d_i >= 0) phase_b();
+      d_i = i;
+      d_unit = unit;
+      d_tile = tile;
+      d_A = A;
+      d_H = Hl;
     }
+    if (d_i >= 0 && !*cta_abort) phase_b();
   }
+#undef RG_WAIT_OR_ABORT
 
   tc_fence_before();
   __syncthreads();
@@ -609,9 +842,9 @@ TcLayout tc_layout(int B, int T, int D, int H) {
   return L;
 }
 
-template <int K, int N, int NX>
+template <int K, int N, int NX, int NE>
 cudaError_t launch_tc_t(const FwdArgs &a, const TcLayout &L, void *ws, cudaStream_t st) {
-  using C = Cfg<K, N, NX>;
+  using C = Cfg<K, N, NX, NE>;
   auto enc = encode_fn();
   if (enc == nullptr) return cudaErrorNotSupported;
   const int bw = a.D / a.H;
@@ -669,7 +902,7 @@ cudaError_t launch_tc_t(const FwdArgs &a, const TcLayout &L, void *ws, cudaStrea
 
   cudaError_t e = cudaMemsetAsync(ws, 0, L.ints_bytes, st);
   if (e != cudaSuccess) return e;
-  auto kern = fwd_tc_kernel<K, N, NX>;
+  auto kern = fwd_tc_kernel<K, N, NX, NE>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
@@ -677,7 +910,7 @@ cudaError_t launch_tc_t(const FwdArgs &a, const TcLayout &L, void *ws, cudaStrea
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long jobs = static_cast<long>(L.n_units) * L.n_tiles;
   const int grid = static_cast<int>(jobs < sms ? jobs : sms);
-  kern<<<grid, kThreads, C::kSmemBytes, st>>>(tx, twa, twx, p);
+  kern<<<grid, C::kThreads, C::kSmemBytes, st>>>(tx, twa, twx, p);
   return cudaGetLastError();
 }
 
@@ -695,8 +928,8 @@ size_t tc_workspace_bytes(int B, int T, int D, int H) { return tc_layout(B, T, D
 cudaError_t launch_fwd_tc(const FwdArgs &a, void *ws, cudaStream_t st) {
   const int bw = a.D / a.H;
   const TcLayout L = tc_layout(a.B, a.T, a.D, a.H);
-  if (bw == 256) return launch_tc_t<256, 32, 2>(a, L, ws, st);
-  return launch_tc_t<128, 64, 3>(a, L, ws, st);
+  if (bw == 256) return launch_tc_t<256, 32, 3, 2>(a, L, ws, st);
+  return launch_tc_t<128, 64, 3, 2>(a, L, ws, st);
 }
 
 }  // namespace rglru
