@@ -222,13 +222,22 @@ __device__ int poll_flag(const int *flag, const int *gabort, volatile int *cta_a
   }
 }
 
+// Offset (bytes) of (own channel c, 4-token block jb) in the fp32 u tile:
+// channel-major rows of N floats, the 16-byte blocks of a row XOR-permuted by
+// c / 4 so that both the token-major conv threads (writers) and the
+// channel-major epilogue threads (readers) spread over all banks.
+template <int N>
+__device__ __forceinline__ uint32_t u_offset(int c, int jb) {
+  return static_cast<uint32_t>(c * (N * 4) + (((jb ^ (c >> 2)) & (N / 4 - 1)) << 4));
+}
+
 // Conv1D of one tile, token-major. Thread t covers the 4 channels
 // [4 q, 4 q + 4) of the K range and SEG consecutive tokens; a warp covers 128
 // channels of one token segment, so that its shared-memory rows are contiguous
-// (no bank conflicts). All input rows are read before any output is written.
-// Writes the bf16 B operand (K-major, 128-byte swizzle) and, when kUTile, the
-// fp32 u of the unit's own channels token-major into ut ([N][128] floats).
-// w holds the 4 taps of the 4 channels (pairs).
+// (no bank conflicts). All input rows are read before any output is written,
+// and each is unpacked once. Writes the bf16 B operand (K-major, 128-byte
+// swizzle) and, when kUTile, the fp32 u of the unit's own channels
+// channel-major into ut (see u_offset). w holds the 4 taps of the 4 channels.
 template <int K, int N, bool kUTile>
 __device__ __forceinline__ void conv_tile(const unsigned char *__restrict__ xs,
                                           unsigned char *__restrict__ bt,
@@ -236,7 +245,8 @@ __device__ __forceinline__ void conv_tile(const unsigned char *__restrict__ xs,
                                           int kbase, int own_lo, int tile, int nvalid,
                                           bool last_tile, int t, const float2 (&w)[4][2]) {
   constexpr int NQ = K / 4;                         // channel quads
-  constexpr int SEG = N * NQ / 128;                 // tokens per thread
+  constexpr int SEG = N * NQ / 128;                 // tokens per thread (16)
+  static_assert(SEG % 8 == 0, "segments start on a swizzle period");
   const int qd = t % NQ, sg = t / NQ;
   const int kq = qd * 4, nb = sg * SEG;
   const bool own = (kq >= own_lo) && (kq < own_lo + kM);
@@ -251,25 +261,44 @@ __device__ __forceinline__ void conv_tile(const unsigned char *__restrict__ xs,
       rows[r] = __ldg(reinterpret_cast<const uint2 *>(p.conv_state_in +
                                                        (static_cast<size_t>(b) * 3 + r) * p.D + chq));
   }
+  // B operand offsets: row n = nb + j with n % 8 == j % 8 (nb is a multiple of 8)
+  const uint32_t bt_base = static_cast<uint32_t>((kq >> 6) * N * 128 + nb * 128 + ((kq & 7) << 1));
+  const int chunk = (kq & 63) >> 3;
+  float2 xw[4][2];
+#pragma unroll
+  for (int r = 0; r < 3; ++r) {
+    xw[r][0] = bf2_to_f2(rows[r].x);
+    xw[r][1] = bf2_to_f2(rows[r].y);
+  }
+  float uacc[4][4];                                 // u of 4 channels x 4 tokens (u tile block)
 #pragma unroll
   for (int j = 0; j < SEG; ++j) {
-    const int n = nb + j;
+    const int c3 = (j + 3) & 3;                     // window slot of token nb + j
+    xw[c3][0] = bf2_to_f2(rows[j + 3].x);
+    xw[c3][1] = bf2_to_f2(rows[j + 3].y);
     float2 u[2];
 #pragma unroll
     for (int pp = 0; pp < 2; ++pp) {
-      const uint32_t r0 = pp ? rows[j].y : rows[j].x, r1 = pp ? rows[j + 1].y : rows[j + 1].x;
-      const uint32_t r2 = pp ? rows[j + 2].y : rows[j + 2].x, r3 = pp ? rows[j + 3].y : rows[j + 3].x;
-      float2 acc = __fmul2_rn(w[0][pp], bf2_to_f2(r0));
-      acc = __ffma2_rn(w[1][pp], bf2_to_f2(r1), acc);
-      acc = __ffma2_rn(w[2][pp], bf2_to_f2(r2), acc);
-      u[pp] = __ffma2_rn(w[3][pp], bf2_to_f2(r3), acc);
+      float2 acc = __fmul2_rn(w[0][pp], xw[(j + 0) & 3][pp]);
+      acc = __ffma2_rn(w[1][pp], xw[(j + 1) & 3][pp], acc);
+      acc = __ffma2_rn(w[2][pp], xw[(j + 2) & 3][pp], acc);
+      u[pp] = __ffma2_rn(w[3][pp], xw[c3][pp], acc);
     }
-    *reinterpret_cast<uint2 *>(bt + kmajor_sw128_offset(n, kq, N)) =
+    *reinterpret_cast<uint2 *>(bt + bt_base + j * 128 + (((chunk ^ j) & 7) << 4)) =
         make_uint2(f2_to_bf2(u[0]), f2_to_bf2(u[1]));
-    if (kUTile && own)
-      *reinterpret_cast<float4 *>(ut + (n * kM + kq - own_lo) * 4) =
-          make_float4(u[0].x, u[0].y, u[1].x, u[1].y);
-    if (own && last_tile && n == nvalid - 1 && p.conv_state_out != nullptr) {
+    if (kUTile) {
+      uacc[0][j & 3] = u[0].x;
+      uacc[1][j & 3] = u[0].y;
+      uacc[2][j & 3] = u[1].x;
+      uacc[3][j & 3] = u[1].y;
+      if ((j & 3) == 3 && own) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          *reinterpret_cast<float4 *>(ut + u_offset<N>(kq - own_lo + k, (nb + j) >> 2)) =
+              make_float4(uacc[k][0], uacc[k][1], uacc[k][2], uacc[k][3]);
+      }
+    }
+    if (own && last_tile && nb + j == nvalid - 1 && p.conv_state_out != nullptr) {
       // the last three inputs x_{T-3}, x_{T-2}, x_{T-1} of these 4 channels
 #pragma unroll
       for (int r = 0; r < 3; ++r)
@@ -363,7 +392,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
   if (warp == 0) {
     // =============================== producer ===============================
     if (lane == 0) {
-      int unit = blockIdx.x % p.n_units, scanned = 0, w_unit = -1;
+      int unit = blockIdx.x % p.n_units, w_unit = -1;
       int i = 0, last_x_job = -1;
       uint32_t wfree_phase = 0;
       for (;; ++i) {
@@ -374,8 +403,16 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
             tile = t;
             break;
           }
-          if (++scanned >= p.n_units) unit = -1;
-          else unit = (unit + 1) % p.n_units;
+          // this unit is done: continue on the unit with the most tiles left
+          int best = -1, left = 0;
+          for (int u = 0; u < p.n_units; ++u) {
+            const int l = p.n_tiles - *(volatile const int *)(p.counters + u);
+            if (l > left) {
+              left = l;
+              best = u;
+            }
+          }
+          unit = best;
         }
         if (*cta_abort) unit = -1;
         const int js = i % kJQ;
@@ -713,8 +750,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
         float uu[16];
         if (C::kUTile) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            uu[j] = *reinterpret_cast<const float *>(uslot + ((ch * 16 + j) * kM + m) * 4);
+          for (int q = 0; q < 4; ++q) {
+            const float4 v = *reinterpret_cast<const float4 *>(uslot + u_offset<N>(m, ch * 4 + q));
+            uu[4 * q] = v.x;
+            uu[4 * q + 1] = v.y;
+            uu[4 * q + 2] = v.z;
+            uu[4 * q + 3] = v.w;
+          }
         } else {
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
