@@ -8,7 +8,7 @@ hand-written CUDA kernels behind a C ABI (include/rglru.h). This package is the
 thin Python binding of that library; see _abi.py.
 """
 from ._abi import (ALGO_AUTO, ALGO_GENERIC, ALGO_TENSOR, LIB_PATH, RGLRUError,  # noqa: F401
-                   fwd_launches, fwd_workspace_bytes, rglru_decode_step, rglru_fwd, status_str, version)
+                   decode_launches, fwd_launches, fwd_workspace_bytes, rglru_decode_step, rglru_fwd, status_str, version)
 
-__all__ = ["rglru_fwd", "rglru_decode_step", "fwd_workspace_bytes", "fwd_launches", "RGLRUError",
+__all__ = ["rglru_fwd", "rglru_decode_step", "fwd_workspace_bytes", "fwd_launches", "decode_launches", "RGLRUError",
            "status_str", "version", "LIB_PATH"]

@@ -23,7 +23,7 @@ ALGOS = {"auto": ALGO_AUTO, "generic": ALGO_GENERIC, "tensor": ALGO_TENSOR}
 EXPORTED = (
     "rglru_status_str", "rglru_version", "rglru_fwd_workspace_bytes", "rglru_fwd",
     "rglru_fwd_algo", "rglru_decode_step", "rglru_decode_step_algo", "rglru_fwd_launches",
-    "rglru_fwd_noalloc",
+    "rglru_fwd_noalloc", "rglru_decode_launches",
 )
 NOALLOC_SCRATCH_BYTES = 2 << 20  # RGLRU_NOALLOC_SCRATCH_BYTES in include/rglru.h
 
@@ -50,6 +50,8 @@ def _load():
     lib.rglru_fwd_workspace_bytes.argtypes = [i32] * 5
     lib.rglru_fwd_launches.restype = i32
     lib.rglru_fwd_launches.argtypes = [i32] * 6
+    lib.rglru_decode_launches.restype = i32
+    lib.rglru_decode_launches.argtypes = [i32] * 5
     fwd_args = [vp] * 6 + [fp, fp, vp, vp, fp, vp] + [i32] * 5 + [vp, sz, ip, vp]
     lib.rglru_fwd.restype = i32
     lib.rglru_fwd.argtypes = fwd_args
@@ -114,6 +116,12 @@ def fwd_launches(B: int, T: int, D: int, H: int, dtype=torch.bfloat16, algo="aut
     """Kernel launches that one rglru_fwd call with these sizes issues."""
     return int(LIB.rglru_fwd_launches(B, T, D, H, _io_of(dtype),
                                       ALGOS[algo] if isinstance(algo, str) else int(algo)))
+
+
+def decode_launches(B: int, D: int, H: int, dtype=torch.bfloat16, algo="auto") -> int:
+    """Kernel launches that one rglru_decode_step call with these sizes issues."""
+    return int(LIB.rglru_decode_launches(B, D, H, _io_of(dtype),
+                                         ALGOS[algo] if isinstance(algo, str) else int(algo)))
 
 
 def rglru_fwd(x, conv_w, W_a, b_a, W_x, b_x, Lambda, h0=None, conv_state_in=None, *,

@@ -71,6 +71,16 @@ int rglru_fwd_launches(int B, int T, int D, int H, int io, int algo) {
   return 1;
 }
 
+int rglru_decode_launches(int B, int D, int H, int io, int algo) {
+  if (check_shape(B, 1, D, H, io) != RGLRU_OK) return 0;
+  if (algo != RGLRU_ALGO_AUTO && algo != RGLRU_ALGO_GENERIC && algo != RGLRU_ALGO_TENSOR)
+    return 0;
+  const bool tc = tc_decode_supported(B, D, H, io);
+  if (algo == RGLRU_ALGO_TENSOR && !tc) return 0;
+  if (algo == RGLRU_ALGO_GENERIC || !tc) return 1;
+  return tc_decode_launches(D, H);
+}
+
 int rglru_fwd_algo(const void *x, const void *conv_w, const void *W_a, const void *b_a,
                    const void *W_x, const void *b_x, const float *Lambda, const float *h0,
                    const void *conv_state_in, void *y, float *h_T, void *conv_state_out,
@@ -139,9 +149,12 @@ int rglru_decode_step_algo(const void *x_t, void *conv_state, int pos, float *h,
   if (overlap(h, (size_t)B * D * 4, conv_state, 3 * row_bytes)) return RGLRU_ERR_INVALID_ARG;
   if (algo != RGLRU_ALGO_AUTO && algo != RGLRU_ALGO_GENERIC && algo != RGLRU_ALGO_TENSOR)
     return RGLRU_ERR_INVALID_ARG;
-  if (algo == RGLRU_ALGO_TENSOR) return RGLRU_ERR_UNSUPPORTED;
+  const bool tc = tc_decode_supported(B, D, H, io);
+  if (algo == RGLRU_ALGO_TENSOR && !tc) return RGLRU_ERR_UNSUPPORTED;
   DecArgs p{x_t, conv_state, pos, h, y_t, conv_w, W_a, b_a, W_x, b_x, Lambda, B, D, H};
-  cudaError_t e = launch_decode_generic(p, io, static_cast<cudaStream_t>(stream));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = (tc && algo != RGLRU_ALGO_GENERIC) ? launch_decode_tc(p, s)
+                                                     : launch_decode_generic(p, io, s);
   return e == cudaSuccess ? RGLRU_OK : RGLRU_ERR_CUDA;
 }
 

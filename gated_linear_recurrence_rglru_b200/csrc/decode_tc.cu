@@ -1,0 +1,535 @@
+// One RG-LRU decode step for B sequences on the tensor core (sm_100a), bf16 I/O.
+//
+// The layer at one time step ("Griffin: Mixing Gated Linear Recurrences with
+// Local Attention for Efficient Language Models", section "Model
+// Architecture"; the fixed-size state that makes decoding cheap is the point
+// of "Beyond Transformer Architecture: Griffin and Google RecurrentGemma",
+// "Core Components of Griffin", 1. RG-LRU):
+//   u = w0 x_{t-3} + w1 x_{t-2} + w2 x_{t-1} + w3 x_t      (three past inputs in a ring)
+//   [z_a | z_x] = u W (block-diagonal), gates, a, beta as in the forward
+//   h <- a h + beta,  y_t = h,  ring slot pos % 3 <- x_t
+// Jobs are (group of 128 output channels, tile of N batch rows). The gate
+// contraction runs on tcgen05 with the gate weights as A (M = 128 channels) and
+// the conv output as B (N = rows), so TMEM lane m holds channel m's gates for
+// the tile's rows; the epilogue updates h in place lane = channel, which keeps
+// its global accesses coalesced. Rows never interact, so CTAs take balanced
+// contiguous ranges of jobs and nothing waits on another CTA.
+//
+// Roles: warp 0 posts the CTA's jobs and loads gate weights by TMA; warp 1
+// owns TMEM and issues the MMAs; warps 2-5 compute the Conv1D from global
+// memory into the bf16 B operand and an fp32 u tile; two epilogue warpgroups
+// take the jobs alternately.
+//
+// Heads 256 wide are split over two channel groups whose CTAs both read all
+// 256 channels of the ring's slot pos % 3; that slot is then rewritten by a
+// separate small kernel after this one (ring_update_kernel) instead of here.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_gates.cuh"
+#include "tc_primitives.cuh"
+
+namespace rglru {
+namespace {
+
+using namespace tc;
+using namespace gates;
+
+constexpr int kM = 128;
+constexpr int kJQ = 8;
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr uint64_t kDrainNs = 200000000ull;
+
+struct DecTcParams {
+  const __nv_bfloat16 *x_t, *conv_w, *b_a, *b_x;
+  const float *Lambda;
+  __nv_bfloat16 *ring;
+  float *h;
+  __nv_bfloat16 *y_t;
+  int B, D, H, bw, pos;
+  int n_cg, n_tiles, n_jobs;
+  int write_ring;                  // 1: this kernel rewrites ring slot pos % 3
+};
+
+template <int K, int N>
+struct DCfg {
+  static constexpr int NE = 2;                     // epilogue warpgroups
+  static constexpr int kThreads = 64 + 128 + NE * 128;
+  static constexpr int kABytes = K * 256;
+  static constexpr int kBBytes = N * K * 2;
+  static constexpr int kUBytes = N * kM * 4;
+  static constexpr int kNS = 2;
+  static constexpr int kNT = 4;
+  static constexpr int kOffA = 0;
+  static constexpr int kOffB = 2 * kABytes;
+  static constexpr int kOffU = kOffB + kNS * kBBytes;
+  static constexpr int kOffBar = kOffU + kNS * kUBytes;
+  // job_full[JQ], job_empty[JQ], w_full, w_free, b_full[NS], b_empty[NS], u_empty[NS],
+  // acc_full[NT], tmem_empty[NT]
+  static constexpr int kNumBars = 2 * kJQ + 2 + 3 * kNS + 2 * kNT;
+  static constexpr int kOffJobs = (kOffBar + kNumBars * 8 + 15) / 16 * 16;
+  static constexpr int kOffMisc = kOffJobs + kJQ * 16;
+  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;
+  static constexpr int kSlotCols = 2 * N;
+  static constexpr int kTmemCols = kNT * kSlotCols <= 128 ? 128 : (kNT * kSlotCols <= 256 ? 256 : 512);
+  static_assert(kSmemBytes <= 232448, "shared memory");
+  static_assert((N * (K / 4)) % (128 * 8) == 0, "conv mapping: 8-row steps");
+};
+
+template <int N>
+__device__ __forceinline__ uint32_t u_off(int c, int jb) {
+  return static_cast<uint32_t>(c * (N * 4) + ((jb ^ ((c & 7) ^ ((c >> 3) & 7))) << 4));
+}
+
+// Conv1D of N rows x K channels from global memory. Thread t covers channel
+// quad q (4 channels) and SEG consecutive rows. Writes the bf16 K-major B
+// operand (128-byte swizzle), the fp32 u of the own channels (channel-major,
+// see u_off) and, when asked, the ring update of the own channels.
+template <int K, int N>
+__device__ __forceinline__ void dec_conv(const DecTcParams &p, unsigned char *__restrict__ bt,
+                                         unsigned char *__restrict__ ut, int kbase, int own_lo,
+                                         int r0, int t, const float2 (&w)[4][2]) {
+  constexpr int NQ = K / 4, SEG = N * NQ / 128;
+  const int qd = t % NQ, sg = t / NQ;
+  const int kq = qd * 4, nb = sg * SEG;
+  const bool own = (kq >= own_lo) && (kq < own_lo + kM);
+  const int chq = kbase + kq;
+  const int s0 = p.pos % 3, s1 = (p.pos + 1) % 3, s2 = (p.pos + 2) % 3;
+  const uint32_t bt_base = static_cast<uint32_t>((kq >> 6) * N * 128 + nb * 128 + ((kq & 7) << 1));
+  const int chunk = (kq & 63) >> 3;
+  float uacc[4][4];
+#pragma unroll
+  for (int j0 = 0; j0 < SEG; j0 += 4) {
+    uint2 xv[4], r0v[4], r1v[4], r2v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int row = r0 + nb + j0 + j;
+      if (row < p.B) {
+        const size_t rb = static_cast<size_t>(row) * 3 * p.D + chq;
+        xv[j] = __ldg(reinterpret_cast<const uint2 *>(p.x_t + static_cast<size_t>(row) * p.D + chq));
+        r0v[j] = __ldg(reinterpret_cast<const uint2 *>(p.ring + rb + static_cast<size_t>(s0) * p.D));
+        r1v[j] = __ldg(reinterpret_cast<const uint2 *>(p.ring + rb + static_cast<size_t>(s1) * p.D));
+        r2v[j] = __ldg(reinterpret_cast<const uint2 *>(p.ring + rb + static_cast<size_t>(s2) * p.D));
+      } else {
+        xv[j] = r0v[j] = r1v[j] = r2v[j] = make_uint2(0u, 0u);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int jj = j0 + j;
+      const int row = r0 + nb + jj;
+      float2 u[2];
+#pragma unroll
+      for (int pp = 0; pp < 2; ++pp) {
+        const uint32_t a0 = pp ? r0v[j].y : r0v[j].x, a1 = pp ? r1v[j].y : r1v[j].x;
+        const uint32_t a2 = pp ? r2v[j].y : r2v[j].x, a3 = pp ? xv[j].y : xv[j].x;
+        float2 acc = __fmul2_rn(w[0][pp], bf2_to_f2(a0));
+        acc = __ffma2_rn(w[1][pp], bf2_to_f2(a1), acc);
+        acc = __ffma2_rn(w[2][pp], bf2_to_f2(a2), acc);
+        u[pp] = __ffma2_rn(w[3][pp], bf2_to_f2(a3), acc);
+      }
+      *reinterpret_cast<uint2 *>(bt + bt_base + jj * 128 + (((chunk ^ jj) & 7) << 4)) =
+          make_uint2(f2_to_bf2(u[0]), f2_to_bf2(u[1]));
+      uacc[0][jj & 3] = u[0].x;
+      uacc[1][jj & 3] = u[0].y;
+      uacc[2][jj & 3] = u[1].x;
+      uacc[3][jj & 3] = u[1].y;
+      if ((jj & 3) == 3 && own) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          *reinterpret_cast<float4 *>(ut + u_off<N>(kq - own_lo + k, (nb + jj) >> 2)) =
+              make_float4(uacc[k][0], uacc[k][1], uacc[k][2], uacc[k][3]);
+      }
+      if (p.write_ring && own && row < p.B)
+        *reinterpret_cast<uint2 *>(p.ring + static_cast<size_t>(row) * 3 * p.D +
+                                   static_cast<size_t>(s0) * p.D + chq) = xv[j];
+    }
+  }
+}
+
+template <int K, int N>
+__global__ void __launch_bounds__(DCfg<K, N>::kThreads, 1)
+decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
+                 const __grid_constant__ CUtensorMap tmap_wx, const DecTcParams p) {
+  using C = DCfg<K, N>;
+  constexpr int NS = C::kNS, NT = C::kNT, NE = C::NE;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *sm = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char *sA = sm + C::kOffA;
+  unsigned char *sB = sm + C::kOffB;
+  unsigned char *sU = sm + C::kOffU;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::kOffBar);
+  uint64_t *job_full = bars;
+  uint64_t *job_empty = job_full + kJQ;
+  uint64_t *w_full = job_empty + kJQ;
+  uint64_t *w_free = w_full + 1;
+  uint64_t *b_full = w_free + 1;
+  uint64_t *b_empty = b_full + NS;
+  uint64_t *u_empty = b_empty + NS;
+  uint64_t *acc_full = u_empty + NS;
+  uint64_t *tmem_empty = acc_full + NT;
+  int4 *jobs = reinterpret_cast<int4 *>(sm + C::kOffJobs);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + C::kOffMisc);
+  volatile int *cta_abort = reinterpret_cast<volatile int *>(sm + C::kOffMisc + 4);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  // this CTA's contiguous, balanced range of jobs (job = unit * n_tiles + tile)
+  const int j_begin = static_cast<int>(static_cast<long>(p.n_jobs) * blockIdx.x / gridDim.x);
+  const int j_end = static_cast<int>(static_cast<long>(p.n_jobs) * (blockIdx.x + 1) / gridDim.x);
+
+  if (tid == 0) {
+    for (int i = 0; i < kJQ; ++i) {
+      mbar_init(&job_full[i], 1);
+      mbar_init(&job_empty[i], 6);                  // conv, MMA, 4 epilogue warps
+    }
+    mbar_init(w_full, 1);
+    mbar_init(w_free, 1);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&b_full[i], 1);
+      mbar_init(&b_empty[i], 1);
+      mbar_init(&u_empty[i], 4);
+    }
+    for (int i = 0; i < NT; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&tmem_empty[i], 4);
+    }
+    *cta_abort = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmap_wa);
+    prefetch_tmap(&tmap_wx);
+  }
+  {
+    uint4 *a4 = reinterpret_cast<uint4 *>(sA);
+    for (int i = tid; i < 2 * C::kABytes / 16; i += C::kThreads) a4[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int R = p.bw <= 128 ? p.bw : 256;
+
+#define RG_WAIT_OR_ABORT(bar, par)                   \
+  if (!mbar_wait((bar), (par), cta_abort, kWaitNs)) { \
+    *cta_abort = 1;                                  \
+    break;                                           \
+  }
+
+  if (warp == 0) {
+    // ============================== job poster ==============================
+    if (lane == 0) {
+      int w_unit = -1;
+      uint32_t wfree_phase = 0;
+      const int n = j_end - j_begin;
+      for (int i = 0; i <= n + NE - 1; ++i) {
+        const int js = i % kJQ;
+        RG_WAIT_OR_ABORT(&job_empty[js], ((i / kJQ) & 1) ^ 1);
+        if (i >= n) {                                // terminal jobs, one per epilogue warpgroup
+          jobs[js] = make_int4(-1, -1, 0, 0);
+          mbar_arrive(&job_full[js]);
+          continue;
+        }
+        const int job = j_begin + i;
+        const int unit = job / p.n_tiles, tile = job % p.n_tiles;
+        const int reload = unit != w_unit ? 1 : 0;
+        jobs[js] = make_int4(unit, tile, reload, 0);
+        mbar_arrive(&job_full[js]);
+        if (reload) {
+          if (i > 0) {
+            RG_WAIT_OR_ABORT(w_free, wfree_phase);
+            wfree_phase ^= 1;
+          }
+          const int cg = unit;
+          mbar_arrive_expect_tx(w_full, 2u * 2u * static_cast<uint32_t>(R) * 128u);
+          for (int g = 0; g < 2; ++g) {
+            const CUtensorMap *tm = g == 0 ? &tmap_wa : &tmap_wx;
+            unsigned char *dst = sA + g * C::kABytes;
+            if (p.bw == 64) {
+              for (int hh = 0; hh < 2; ++hh)
+                tma_load_2d(dst + hh * (K * 128) + hh * 64 * 128, tm, w_full, 0, (cg * 2 + hh) * 64);
+            } else if (p.bw == 128) {
+              for (int ma = 0; ma < 2; ++ma)
+                tma_load_2d(dst + ma * (K * 128), tm, w_full, 64 * ma, cg * 128);
+            } else {
+              for (int ma = 0; ma < 2; ++ma)
+                tma_load_2d(dst + ma * (K * 128), tm, w_full, (cg & 1) * 128 + 64 * ma,
+                            (cg >> 1) * 256);
+            }
+          }
+          w_unit = unit;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ============================== MMA issuer ==============================
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kM, N, true, false);
+      const uint32_t a0 = smem_u32(sA), a1 = smem_u32(sA + C::kABytes);
+      uint32_t w_phase = 0;
+      int last_commit = -1;
+      for (int i = 0;; ++i) {
+        const int js = i % kJQ;
+        RG_WAIT_OR_ABORT(&job_full[js], (i / kJQ) & 1);
+        const int4 job = jobs[js];
+        if (job.x < 0) break;
+        if (job.z) {
+          if (last_commit >= 0) {
+            const int lc = last_commit;
+            RG_WAIT_OR_ABORT(&acc_full[lc % NT], (lc / NT) & 1);
+            mbar_arrive(w_free);
+          }
+          RG_WAIT_OR_ABORT(w_full, w_phase);
+          w_phase ^= 1;
+        }
+        const int s = i % NS, ts = i % NT;
+        RG_WAIT_OR_ABORT(&b_full[s], (i / NS) & 1);
+        RG_WAIT_OR_ABORT(&tmem_empty[ts], ((i / NT) & 1) ^ 1);
+        tc_fence_after();
+        const uint32_t bs = smem_u32(sB + s * C::kBBytes);
+        const uint32_t d_a = tmem_base + static_cast<uint32_t>(ts * C::kSlotCols);
+        const uint32_t d_x = d_a + N;
+#pragma unroll
+        for (int ks = 0; ks < K / 16; ++ks) {
+          const uint64_t bd = sdesc_sw128(bs + (ks >> 2) * (N * 128) + (ks & 3) * 32, 16, 1024);
+          const uint64_t ada = sdesc_sw128(a0 + ks * 16 * 128, K * 128, 1024);
+          const uint64_t adx = sdesc_sw128(a1 + ks * 16 * 128, K * 128, 1024);
+          mma_bf16(d_a, ada, bd, idesc, ks > 0 ? 1u : 0u);
+          mma_bf16(d_x, adx, bd, idesc, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(&acc_full[ts]);
+        mma_commit(&b_empty[s]);
+        last_commit = i;
+        mbar_arrive(&job_empty[js]);
+      }
+      if (*cta_abort && last_commit >= 0)
+        mbar_wait_drain(&acc_full[last_commit % NT], (last_commit / NT) & 1, kDrainNs);
+    }
+  } else if (warp < 6) {
+    // ============================== conv warpgroup ==============================
+    const int wt = tid - 64;
+    int cur_unit = -1;
+    float2 cwq[4][2];
+    for (int i = 0;; ++i) {
+      const int js = i % kJQ;
+      RG_WAIT_OR_ABORT(&job_full[js], (i / kJQ) & 1);
+      const int4 job = jobs[js];
+      const int unit = job.x, tile = job.y;
+      if (unit < 0) break;
+      const int cg = unit;
+      const int kbase = p.bw <= 128 ? cg * kM : (cg >> 1) * 256;
+      const int own_lo = p.bw <= 128 ? 0 : (cg & 1) * kM;
+      if (unit != cur_unit) {
+        cur_unit = unit;
+        const int chq = kbase + (wt % (K / 4)) * 4;
+#pragma unroll
+        for (int tap = 0; tap < 4; ++tap) {
+          const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(p.conv_w + tap * p.D + chq));
+          cwq[tap][0] = bf2_to_f2(raw.x);
+          cwq[tap][1] = bf2_to_f2(raw.y);
+        }
+      }
+      const int s = i % NS;
+      RG_WAIT_OR_ABORT(&b_empty[s], ((i / NS) & 1) ^ 1);
+      RG_WAIT_OR_ABORT(&u_empty[s], ((i / NS) & 1) ^ 1);
+      dec_conv<K, N>(p, sB + s * C::kBBytes, sU + s * C::kUBytes, kbase, own_lo, tile * N, wt, cwq);
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (wt == 0) {
+        mbar_arrive(&b_full[s]);
+        mbar_arrive(&job_empty[js]);
+      }
+    }
+  } else {
+    // ============================ epilogue warpgroups ============================
+    const int eg = (warp - 6) >> 2;
+    const int qd = warp & 3;
+    const int m = qd * 32 + lane;
+    const uint32_t t_lane0 = tmem_base + (static_cast<uint32_t>(qd * 32) << 16);
+    int cur_unit = -1;
+    ChanK kc{0.f, 0.f, 0.f, 0.f, 0.f};
+    bool fast = true;
+    for (int i = eg;; i += NE) {
+      const int js = i % kJQ;
+      RG_WAIT_OR_ABORT(&job_full[js], (i / kJQ) & 1);
+      const int4 job = jobs[js];
+      const int unit = job.x, tile = job.y;
+      if (unit < 0) break;
+      const int c = unit * kM + m;
+      const int r0 = tile * N;
+      const int nvalid = min(N, p.B - r0);
+      const int s = i % NS, ts = i % NT;
+      if (unit != cur_unit) {
+        cur_unit = unit;
+        kc = chan_consts(__bfloat162float(p.b_a[c]), __bfloat162float(p.b_x[c]), p.Lambda[c]);
+        fast = __all_sync(0xffffffffu, chan_fast(kc));
+      }
+      RG_WAIT_OR_ABORT(&acc_full[ts], (i / NT) & 1);
+      tc_fence_after();
+      const uint32_t t_lane = t_lane0 + static_cast<uint32_t>(ts * C::kSlotCols);
+      const unsigned char *uslot = sU + s * C::kUBytes;
+#pragma unroll
+      for (int ch = 0; ch < N / 16; ++ch) {
+        // previous state of this channel for the chunk's rows (coalesced across lanes)
+        float hold[16];
+#pragma unroll
+        for (int n = 0; n < 16; ++n)
+          hold[n] = ch * 16 + n < nvalid ? p.h[static_cast<size_t>(r0 + ch * 16 + n) * p.D + c] : 0.f;
+        float za[16], zx[16], uu[16];
+        tmem_ld16(t_lane + ch * 16, za);
+        tmem_ld16(t_lane + N + ch * 16, zx);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 v = *reinterpret_cast<const float4 *>(uslot + u_off<N>(m, ch * 4 + q));
+          uu[4 * q] = v.x;
+          uu[4 * q + 1] = v.y;
+          uu[4 * q + 2] = v.z;
+          uu[4 * q + 3] = v.w;
+        }
+        tmem_wait_ld();
+#pragma unroll
+        for (int pr = 0; pr < 8; ++pr) {
+          const int n = ch * 16 + 2 * pr;
+          float2 a, beta, la;
+          if (fast) {
+            gate_pair_fast(make_float2(za[2 * pr], za[2 * pr + 1]),
+                           make_float2(zx[2 * pr], zx[2 * pr + 1]),
+                           make_float2(uu[2 * pr], uu[2 * pr + 1]), kc, a, beta, la);
+          } else {
+            gate_one(za[2 * pr], zx[2 * pr], uu[2 * pr], kc, a.x, beta.x, la.x);
+            gate_one(za[2 * pr + 1], zx[2 * pr + 1], uu[2 * pr + 1], kc, a.y, beta.y, la.y);
+          }
+          const float2 hn = __ffma2_rn(a, make_float2(hold[2 * pr], hold[2 * pr + 1]), beta);
+          if (n < nvalid) {
+            const size_t o = static_cast<size_t>(r0 + n) * p.D + c;
+            p.h[o] = hn.x;
+            p.y_t[o] = __float2bfloat16_rn(hn.x);
+          }
+          if (n + 1 < nvalid) {
+            const size_t o = static_cast<size_t>(r0 + n + 1) * p.D + c;
+            p.h[o] = hn.y;
+            p.y_t[o] = __float2bfloat16_rn(hn.y);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&u_empty[s]);
+        mbar_arrive(&tmem_empty[ts]);
+        mbar_arrive(&job_empty[js]);
+      }
+    }
+  }
+#undef RG_WAIT_OR_ABORT
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+// ring[:, pos % 3, :] <- x_t, 8 channels per thread (heads 256 wide).
+__global__ void ring_update_kernel(const __nv_bfloat16 *__restrict__ x_t,
+                                   __nv_bfloat16 *__restrict__ ring, int B, int D, int pos) {
+  const size_t n8 = static_cast<size_t>(B) * D / 8;
+  const int s0 = pos % 3;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t e = i * 8;
+    const size_t b = e / D, d = e - b * D;
+    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(x_t) + i);
+    *reinterpret_cast<uint4 *>(ring + (b * 3 + s0) * D + d) = v;
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 dec_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+template <int K, int N>
+cudaError_t launch_dec_t(const DecArgs &a, cudaStream_t st) {
+  using C = DCfg<K, N>;
+  auto enc = dec_encode_fn();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  const int bw = a.D / a.H;
+  const int R = bw <= 128 ? bw : 256;
+  CUtensorMap twa, twx;
+  for (int g = 0; g < 2; ++g) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(bw), static_cast<cuuint64_t>(a.H) * bw};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(bw) * 2};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(R)};
+    cuuint32_t es[2] = {1, 1};
+    if (enc(g == 0 ? &twa : &twx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+            const_cast<void *>(g == 0 ? a.W_a : a.W_x), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  DecTcParams p;
+  p.x_t = static_cast<const __nv_bfloat16 *>(a.x_t);
+  p.conv_w = static_cast<const __nv_bfloat16 *>(a.conv_w);
+  p.b_a = static_cast<const __nv_bfloat16 *>(a.b_a);
+  p.b_x = static_cast<const __nv_bfloat16 *>(a.b_x);
+  p.Lambda = a.Lambda;
+  p.ring = static_cast<__nv_bfloat16 *>(a.conv_state);
+  p.h = a.h;
+  p.y_t = static_cast<__nv_bfloat16 *>(a.y_t);
+  p.B = a.B;
+  p.D = a.D;
+  p.H = a.H;
+  p.bw = bw;
+  p.pos = a.pos;
+  p.n_cg = a.D / kM;
+  p.n_tiles = ceil_div(a.B, N);
+  p.n_jobs = p.n_cg * p.n_tiles;
+  p.write_ring = bw <= 128 ? 1 : 0;
+  auto kern = decode_tc_kernel<K, N>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = p.n_jobs < sms ? p.n_jobs : sms;
+  kern<<<grid, C::kThreads, C::kSmemBytes, st>>>(twa, twx, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || p.write_ring) return e;
+  const size_t n8 = static_cast<size_t>(a.B) * a.D / 8;
+  const int blocks = static_cast<int>((n8 + 255) / 256 < 4 * static_cast<size_t>(sms)
+                                          ? (n8 + 255) / 256
+                                          : 4 * static_cast<size_t>(sms));
+  ring_update_kernel<<<blocks, 256, 0, st>>>(p.x_t, p.ring, a.B, a.D, a.pos);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_decode_supported(int B, int D, int H, int io) { return tc_supported(B, 1, D, H, io); }
+
+int tc_decode_launches(int D, int H) { return D / H == 256 ? 2 : 1; }
+
+cudaError_t launch_decode_tc(const DecArgs &a, cudaStream_t st) {
+  const int bw = a.D / a.H;
+  if (bw == 256) return launch_dec_t<256, 32>(a, st);
+  return launch_dec_t<128, 32>(a, st);
+}
+
+}  // namespace rglru

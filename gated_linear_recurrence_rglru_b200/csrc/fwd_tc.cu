@@ -35,22 +35,19 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_gates.cuh"
 #include "tc_primitives.cuh"
 
 namespace rglru {
 namespace {
 
 using namespace tc;
+using namespace gates;
 
 constexpr int kM = 128;         // output channels per unit (MMA M, TMEM lanes)
 constexpr int kJQ = 8;          // job ring depth
 constexpr uint64_t kWaitNs = 2000000000ull;   // bound of any wait
 constexpr uint64_t kDrainNs = 200000000ull;   // bound of the drain after an abort
-constexpr float kLog2e = 1.4426950408889634f;
-// sqrt((1 - e^(2w)) / (-2w)) ~= 1 + w (G1 + w (G2 + w G3)) on w in [-1/8, 0]
-// (least-squares/minimax fit made for this kernel; max rel. error 7e-8 in fp32).
-constexpr float kG1 = 0.49999531f, kG2 = 0.20810417f, kG3 = 0.05930331f;
-constexpr float kFastLimit = 0.125f;          // fast path when c * softplus(-Lambda) <= 1/8
 
 struct TcParams {
   const __nv_bfloat16 *conv_w, *b_a, *b_x;
@@ -100,107 +97,6 @@ struct Cfg {
   static_assert(kNT * kSlotCols <= 512, "TMEM allocation");
 };
 
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ float rsqrt_approx(float x) {
-  float y;
-  asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ float sqrt_approx(float x) {
-  float y;
-  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ float tanh_approx(float x) {
-  float y;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-__device__ __forceinline__ void named_bar_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ int ld_acquire(const int *p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release(int *p, int v) {
-  asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ float2 f2(float v) { return make_float2(v, v); }
-
-// bf16 pair (low half = first element) -> two floats
-__device__ __forceinline__ float2 bf2_to_f2(uint32_t w) {
-  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-}
-__device__ __forceinline__ uint32_t f2_to_bf2(float2 v) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
-  return *reinterpret_cast<const uint32_t *>(&h);
-}
-
-// Per-channel constants of the epilogue.
-struct ChanK {
-  float kba;    // -(b_a) log2 e
-  float hbx;    // b_x / 2
-  float nc;     // -c softplus(-Lambda): ln a_t = nc * r_t
-  float k2sp;   // 2 sqrt(softplus(-Lambda))
-  float nc2;    // nc log2 e (general path)
-};
-
-// Fast path, two tokens of one channel, valid when |nc| <= 1/8:
-//   e = 2^(-(za + ba) log2 e), sqrt_r = (1 + e)^(-1/2), r = sqrt_r^2,
-//   ln a = nc r, a = e^(ln a) (Taylor, degree 5),
-//   sqrt(1 - a^2) = sqrt(-2 ln a) sqrt(g(ln a)) = 4 sqrt(sp) sqrt_r sqrt(g),
-//   i = (1 + tanh((zx + bx) / 2)) / 2,  beta = sqrt(1 - a^2) i u.
-__device__ __forceinline__ void gate_pair_fast(float2 za, float2 zx, float2 u, const ChanK &k,
-                                               float2 &a, float2 &beta, float2 &la) {
-  const float2 earg = __ffma2_rn(za, f2(-kLog2e), f2(k.kba));
-  float2 d = make_float2(ex2_approx(earg.x), ex2_approx(earg.y));
-  d = __fadd2_rn(d, f2(1.0f));
-  const float2 q = make_float2(rsqrt_approx(d.x), rsqrt_approx(d.y));
-  la = __fmul2_rn(__fmul2_rn(q, q), f2(k.nc));
-  float2 pa = __ffma2_rn(la, f2(1.0f / 120.0f), f2(1.0f / 24.0f));
-  pa = __ffma2_rn(la, pa, f2(1.0f / 6.0f));
-  pa = __ffma2_rn(la, pa, f2(0.5f));
-  pa = __ffma2_rn(la, pa, f2(1.0f));
-  a = __ffma2_rn(la, pa, f2(1.0f));
-  float2 sg = __ffma2_rn(la, f2(kG3), f2(kG2));
-  sg = __ffma2_rn(la, sg, f2(kG1));
-  sg = __ffma2_rn(la, sg, f2(1.0f));
-  const float2 targ = __ffma2_rn(zx, f2(0.5f), f2(k.hbx));
-  const float2 t = make_float2(tanh_approx(targ.x), tanh_approx(targ.y));
-  const float2 ig = __ffma2_rn(t, f2(k.k2sp), f2(k.k2sp));   // 4 sqrt(sp) i
-  beta = __fmul2_rn(__fmul2_rn(__fmul2_rn(q, sg), ig), u);
-}
-
-// General path, one element: as above but a = 2^(log2 a) on the MUFU and
-// 1 - a^2 = -expm1(2 ln a) by its series near a = 1, else 1 - a*a.
-__device__ __forceinline__ void gate_one(float za, float zx, float u, const ChanK &k, float &a,
-                                         float &beta, float &la) {
-  const float e = ex2_approx(fmaf(za, -kLog2e, k.kba));
-  const float q = rsqrt_approx(1.0f + e);
-  const float r = q * q;
-  const float ig = fmaf(0.5f, tanh_approx(fmaf(zx, 0.5f, k.hbx)), 0.5f);
-  const float la2 = k.nc2 * r;
-  la = k.nc * r;
-  a = ex2_approx(la2);
-  const float v = 2.0f * la;
-  float p = fmaf(v, 1.0f / 720.0f, 1.0f / 120.0f);
-  p = fmaf(v, p, 1.0f / 24.0f);
-  p = fmaf(v, p, 1.0f / 6.0f);
-  p = fmaf(v, p, 0.5f);
-  p = fmaf(v, p, 1.0f);
-  const float om = (v > -0.25f) ? (-v * p) : fmaf(-a, a, 1.0f);
-  beta = sqrt_approx(om) * ig * u;
-}
-
 __device__ void raise_abort(const TcParams &p, volatile int *cta_abort, int code) {
   if (p.dev_status) atomicCAS(p.dev_status, 0, code);
   atomicExch(p.abort_flag, 1);
@@ -223,12 +119,14 @@ __device__ int poll_flag(const int *flag, const int *gabort, volatile int *cta_a
 }
 
 // Offset (bytes) of (own channel c, 4-token block jb) in the fp32 u tile:
-// channel-major rows of N floats, the 16-byte blocks of a row XOR-permuted by
-// c / 4 so that both the token-major conv threads (writers) and the
-// channel-major epilogue threads (readers) spread over all banks.
+// channel-major rows of N floats whose 16-byte blocks are XOR-permuted by
+// (c % 8) ^ (c / 8 % 8). 16-byte accesses are served a quarter warp (8 lanes)
+// at a time; the permutation puts any 8 consecutive channels (epilogue
+// readers) and any 8 channels 4 apart (conv writers) on distinct banks.
 template <int N>
 __device__ __forceinline__ uint32_t u_offset(int c, int jb) {
-  return static_cast<uint32_t>(c * (N * 4) + (((jb ^ (c >> 2)) & (N / 4 - 1)) << 4));
+  static_assert(N >= 32, "the permutation needs 8 blocks per row");
+  return static_cast<uint32_t>(c * (N * 4) + ((jb ^ ((c & 7) ^ ((c >> 3) & 7))) << 4));
 }
 
 // Conv1D of one tile, token-major. Thread t covers the 4 channels
@@ -345,22 +243,22 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
   if (tid == 0) {
     for (int i = 0; i < kJQ; ++i) {
       mbar_init(&job_full[i], 1);
-      mbar_init(&job_empty[i], 3);                  // conv, MMA, epilogue
+      mbar_init(&job_empty[i], 6);                  // conv, MMA, 4 epilogue warps
     }
     for (int i = 0; i < NX; ++i) {
       mbar_init(&x_full[i], 1);
-      mbar_init(&x_empty[i], 1);
+      mbar_init(&x_empty[i], C::kUTile ? 1 : 4);   // conv warpgroup, or 4 epilogue warps
     }
     mbar_init(w_full, 1);
     mbar_init(w_free, 1);
     for (int i = 0; i < NS; ++i) {
       mbar_init(&b_full[i], 1);
       mbar_init(&b_empty[i], 1);
-      mbar_init(&u_empty[i], 1);
+      mbar_init(&u_empty[i], 4);                    // 4 epilogue warps
     }
     for (int i = 0; i < NT; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&tmem_empty[i], 1);
+      mbar_init(&tmem_empty[i], 4);                 // 4 epilogue warps
     }
     *cta_abort = 0;
     fence_mbar_init();
@@ -558,22 +456,19 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
     }
   } else {
     // ========================== epilogue warpgroups ==========================
-    // Epilogue warpgroup e takes jobs e, e + NE, ... Per job: pass 1 (gates,
-    // decay, local scan) and publish of the tile's aggregate; then the carry
-    // (look-back) and pass 2 of the warpgroup's previous job, whose
-    // predecessors have usually published by then.
+    // Epilogue warpgroup e takes jobs e, e + NE, ...; each of its 4 warps owns
+    // one TMEM quadrant (32 channels) and works on its own: per job, pass 1
+    // (gates, decay, local scan) and publish of its quadrant's aggregate; then
+    // the carry (look-back over its quadrant's flags) and pass 2 of the warp's
+    // previous job, whose predecessors have usually published by then.
     const int eg = (warp - 6) >> 2;               // 0 .. NE-1
-    const int wt = tid - 192 - eg * 128;          // 0 .. 127
-    const int m = (warp & 3) * 32 + lane;         // TMEM lane == output channel in unit
-    const bool leader = (wt == 0);
-    const bool leader_warp = (wt >> 5) == 0;
-    const int bar_id = 2 + eg;
-    const uint32_t t_lane0 = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const int qd = warp & 3;                      // TMEM quadrant
+    const int m = qd * 32 + lane;                 // TMEM lane == output channel in unit
+    const uint32_t t_lane0 = tmem_base + (static_cast<uint32_t>(qd * 32) << 16);
     int cur_unit = -1;
     ChanK kc{0.f, 0.f, 0.f, 0.f, 0.f};
     float cwo[4] = {0.f, 0.f, 0.f, 0.f};          // own channel's conv taps (K = 256)
     bool fast = true;
-    int it_b = 0;                                 // broadcast slot parity
     int d_i = -1, d_unit = 0, d_tile = 0;         // the deferred job
     float d_A = 0.f, d_H = 0.f;
 
@@ -592,49 +487,41 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
       if (tile == 0) {
         if (p.h0 != nullptr) h_in = p.h0[static_cast<size_t>(b) * p.D + c];
       } else {
-        // Look back over a window of up to 32 predecessors: the leader warp
-        // reads their flags at once and finds the nearest inclusive state with
-        // only aggregates after it; every thread then folds those in.
+        // Look back over a window of up to 32 predecessors: lane l reads the
+        // flag of tile top - l; the warp finds the nearest inclusive state
+        // with only aggregates after it and folds those in.
         float mult = 1.f, add = 0.f;
         int top = tile - 1;
         for (;;) {
-          const int slot = eg * 2 + (it_b & 1);
-          ++it_b;
-          if (leader_warp) {
-            const int jt = top - lane;
-            int res;
-            const uint64_t t0 = globaltimer_ns();
-            for (;;) {
-              const int f = (jt >= 0) ? ld_acquire(p.flags + ubase + jt) : 0;
-              const unsigned agg = __ballot_sync(0xffffffffu, f >= 1);
-              const unsigned inc = __ballot_sync(0xffffffffu, f == 2);
-              if (inc != 0u) {
-                const int e = __ffs(inc) - 1;     // nearest inclusive
-                const unsigned below = (e == 0) ? 0u : (0xffffffffu >> (32 - e));
-                if ((agg & below) == below) { res = e; break; }
-              } else if (agg == 0xffffffffu) {
-                res = 32;                         // 32 aggregates, no inclusive yet: fold, go on
-                break;
-              }
-              if (*cta_abort || *(volatile const int *)p.abort_flag) { res = -1; break; }
-              if (globaltimer_ns() - t0 > kWaitNs) { res = -2; break; }
-              __nanosleep(32);
+          const int jt = top - lane;
+          int res;
+          const uint64_t t0 = globaltimer_ns();
+          for (;;) {
+            const int f = (jt >= 0) ? ld_acquire(p.flags + (ubase + jt) * 4 + qd) : 0;
+            const unsigned agg = __ballot_sync(0xffffffffu, f >= 1);
+            const unsigned inc = __ballot_sync(0xffffffffu, f == 2);
+            if (inc != 0u) {
+              const int e = __ffs(inc) - 1;       // nearest inclusive
+              const unsigned below = (e == 0) ? 0u : (0xffffffffu >> (32 - e));
+              if ((agg & below) == below) { res = e; break; }
+            } else if (agg == 0xffffffffu) {
+              res = 32;                           // 32 aggregates, no inclusive yet: fold, go on
+              break;
             }
-            if (lane == 0) {
-              if (res == -2) {
-                raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);
-                res = -1;
-              }
-              bcast[slot] = res;
-            }
+            if (*cta_abort || *(volatile const int *)p.abort_flag) { res = -1; break; }
+            if (globaltimer_ns() - t0 > kWaitNs) { res = -2; break; }
+            __nanosleep(32);
           }
-          named_bar_sync(bar_id, 128);
-          const int e = bcast[slot];
-          if (e < 0) {
+          if (res == -2) {
+            if (lane == 0) raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);
+            res = -1;
+          }
+          __syncwarp();                           // order the data loads after the flags
+          if (res < 0) {
             h_in = 0.f;
             break;
           }
-          const int nagg = e < 32 ? e : 32;
+          const int nagg = res < 32 ? res : 32;
           for (int k = 0; k < nagg; k += 4) {
             float Av[4], Hv[4];
 #pragma unroll
@@ -650,15 +537,15 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
               mult *= Av[q];
             }
           }
-          if (e < 32) {
-            h_in = fmaf(mult, __ldcg(p.incH + (ubase + top - e) * kM + m), add);
+          if (res < 32) {
+            h_in = fmaf(mult, __ldcg(p.incH + (ubase + top - res) * kM + m), add);
             break;
           }
           top -= 32;
         }
         __stcg(p.incH + (ubase + tile) * kM + m, fmaf(d_A, h_in, d_H));
-        named_bar_sync(bar_id, 128);
-        if (leader) st_release(p.flags + ubase + tile, 2);
+        __syncwarp();
+        if (lane == 0) st_release(p.flags + (ubase + tile) * 4 + qd, 2);
       }
       // ---- pass 2: y_t = h_t ----
       float h = h_in;
@@ -686,8 +573,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
       }
       if (last_tile && p.h_T != nullptr) p.h_T[static_cast<size_t>(b) * p.D + c] = h;
       tc_fence_before();
-      named_bar_sync(bar_id, 128);
-      if (leader) {
+      __syncwarp();
+      if (lane == 0) {
         mbar_arrive(&tmem_empty[ts]);
         mbar_arrive(&job_empty[d_i % kJQ]);
       }
@@ -806,9 +693,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
       }
       tmem_wait_st();
       const float A = ex2_approx((S2.x + S2.y) * kLog2e);
-      // publish this tile's state: inclusive for the first tile of a sequence
-      // (h0 is known), else the aggregate (prod a, local h); release the u / x
-      // tile to the conv warpgroup / producer
+      // publish this quadrant's state: inclusive for the first tile of a
+      // sequence (h0 is known), else the aggregate (prod a, local h); release
+      // the u / x tile
       {
         const size_t tix = static_cast<size_t>(unit) * p.n_tiles + tile;
         if (tile == 0) {
@@ -818,9 +705,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
           __stcg(p.aggA + tix * kM + m, A);
           __stcg(p.aggH + tix * kM + m, Hl);
         }
-        named_bar_sync(bar_id, 128);
-        if (leader) {
-          st_release(p.flags + tix, tile == 0 ? 2 : 1);
+        __syncwarp();
+        if (lane == 0) {
+          st_release(p.flags + tix * 4 + qd, tile == 0 ? 2 : 1);
           if (C::kUTile) mbar_arrive(&u_empty[s]);
           else mbar_arrive(&x_empty[xb]);
         }
@@ -875,7 +762,8 @@ TcLayout tc_layout(int B, int T, int D, int H) {
   L.off_counters = 0;
   L.off_abort = static_cast<size_t>(L.n_units) * 4;
   L.off_flags = align_up(L.off_abort + 4, 16);
-  L.ints_bytes = align_up(L.off_flags + static_cast<size_t>(L.n_units) * L.n_tiles * 4, 256);
+  // one flag per (unit, tile, 32-channel quadrant)
+  L.ints_bytes = align_up(L.off_flags + static_cast<size_t>(L.n_units) * L.n_tiles * 16, 256);
   const size_t agg = align_up(static_cast<size_t>(L.n_units) * L.n_tiles * kM * 4, 256);
   L.off_aggA = L.ints_bytes;
   L.off_aggH = L.off_aggA + agg;

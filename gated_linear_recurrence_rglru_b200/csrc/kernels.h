@@ -44,4 +44,9 @@ bool tc_supported(int B, int T, int D, int H, int io);
 size_t tc_workspace_bytes(int B, int T, int D, int H);
 cudaError_t launch_fwd_tc(const FwdArgs &p, void *ws, cudaStream_t st);
 
+// Tensor-core decode step, bf16 I/O (same shape rules as the forward).
+bool tc_decode_supported(int B, int D, int H, int io);
+int tc_decode_launches(int D, int H);
+cudaError_t launch_decode_tc(const DecArgs &p, cudaStream_t st);
+
 }  // namespace rglru

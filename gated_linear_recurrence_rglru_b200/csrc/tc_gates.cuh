@@ -1,0 +1,140 @@
+// Device helpers shared by the tensor-core kernels: fast gate math of the
+// RG-LRU ("Griffin: Mixing Gated Linear Recurrences with Local Attention for
+// Efficient Language Models", section "Model Architecture": r = sigmoid(z_a),
+// i = sigmoid(z_x), log a = -c r softplus(-Lambda), beta = sqrt(1 - a^2) i u),
+// bf16 packing, and global-memory acquire/release accesses.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace rglru {
+namespace gates {
+
+constexpr float kLog2e = 1.4426950408889634f;
+// sqrt((1 - e^(2w)) / (-2w)) ~= 1 + w (G1 + w (G2 + w G3)) on w in [-1/8, 0]
+// (least-squares/minimax fit made for these kernels; max rel. error 7e-8 in fp32).
+constexpr float kG1 = 0.49999531f, kG2 = 0.20810417f, kG3 = 0.05930331f;
+constexpr float kFastLimit = 0.125f;          // fast path when c * softplus(-Lambda) <= 1/8
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rsqrt_approx(float x) {
+  float y;
+  asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float sqrt_approx(float x) {
+  float y;
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ int ld_acquire(const int *p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(int *p, int v) {
+  asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ float2 f2(float v) { return make_float2(v, v); }
+
+// bf16 pair (low half = first element) -> two floats
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+__device__ __forceinline__ uint32_t f2_to_bf2(float2 v) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+  return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// Per-channel constants of the epilogue.
+struct ChanK {
+  float kba;    // -(b_a) log2 e
+  float hbx;    // b_x / 2
+  float nc;     // -c softplus(-Lambda): ln a_t = nc * r_t
+  float k2sp;   // 2 sqrt(softplus(-Lambda))
+  float nc2;    // nc log2 e (general path)
+};
+
+// Fast path, two tokens of one channel, valid when |nc| <= 1/8:
+//   e = 2^(-(za + ba) log2 e), sqrt_r = (1 + e)^(-1/2), r = sqrt_r^2,
+//   ln a = nc r, a = e^(ln a) (Taylor, degree 5),
+//   sqrt(1 - a^2) = sqrt(-2 ln a) sqrt(g(ln a)) = 4 sqrt(sp) sqrt_r sqrt(g),
+//   i = (1 + tanh((zx + bx) / 2)) / 2,  beta = sqrt(1 - a^2) i u.
+__device__ __forceinline__ void gate_pair_fast(float2 za, float2 zx, float2 u, const ChanK &k,
+                                               float2 &a, float2 &beta, float2 &la) {
+  const float2 earg = __ffma2_rn(za, f2(-kLog2e), f2(k.kba));
+  float2 d = make_float2(ex2_approx(earg.x), ex2_approx(earg.y));
+  d = __fadd2_rn(d, f2(1.0f));
+  const float2 q = make_float2(rsqrt_approx(d.x), rsqrt_approx(d.y));
+  la = __fmul2_rn(__fmul2_rn(q, q), f2(k.nc));
+  float2 pa = __ffma2_rn(la, f2(1.0f / 120.0f), f2(1.0f / 24.0f));
+  pa = __ffma2_rn(la, pa, f2(1.0f / 6.0f));
+  pa = __ffma2_rn(la, pa, f2(0.5f));
+  pa = __ffma2_rn(la, pa, f2(1.0f));
+  a = __ffma2_rn(la, pa, f2(1.0f));
+  float2 sg = __ffma2_rn(la, f2(kG3), f2(kG2));
+  sg = __ffma2_rn(la, sg, f2(kG1));
+  sg = __ffma2_rn(la, sg, f2(1.0f));
+  const float2 targ = __ffma2_rn(zx, f2(0.5f), f2(k.hbx));
+  const float2 t = make_float2(tanh_approx(targ.x), tanh_approx(targ.y));
+  const float2 ig = __ffma2_rn(t, f2(k.k2sp), f2(k.k2sp));   // 4 sqrt(sp) i
+  beta = __fmul2_rn(__fmul2_rn(__fmul2_rn(q, sg), ig), u);
+}
+
+// General path, one element: as above but a = 2^(log2 a) on the MUFU and
+// 1 - a^2 = -expm1(2 ln a) by its series near a = 1, else 1 - a*a.
+__device__ __forceinline__ void gate_one(float za, float zx, float u, const ChanK &k, float &a,
+                                         float &beta, float &la) {
+  const float e = ex2_approx(fmaf(za, -kLog2e, k.kba));
+  const float q = rsqrt_approx(1.0f + e);
+  const float r = q * q;
+  const float ig = fmaf(0.5f, tanh_approx(fmaf(zx, 0.5f, k.hbx)), 0.5f);
+  const float la2 = k.nc2 * r;
+  la = k.nc * r;
+  a = ex2_approx(la2);
+  const float v = 2.0f * la;
+  float p = fmaf(v, 1.0f / 720.0f, 1.0f / 120.0f);
+  p = fmaf(v, p, 1.0f / 24.0f);
+  p = fmaf(v, p, 1.0f / 6.0f);
+  p = fmaf(v, p, 0.5f);
+  p = fmaf(v, p, 1.0f);
+  const float om = (v > -0.25f) ? (-v * p) : fmaf(-a, a, 1.0f);
+  beta = sqrt_approx(om) * ig * u;
+}
+
+
+// Per-channel constants from the channel's bias pair and Lambda.
+__device__ __forceinline__ ChanK chan_consts(float b_a, float b_x, float Lambda) {
+  const float sp = softplus_f32(-Lambda);
+  ChanK k;
+  k.kba = -b_a * kLog2e;
+  k.hbx = 0.5f * b_x;
+  k.nc = -kDecayC * sp;
+  k.nc2 = k.nc * kLog2e;
+  k.k2sp = 2.0f * sqrtf(sp);
+  return k;
+}
+
+// True when the fast path is valid for this channel (c * softplus(-Lambda) <= 1/8).
+__device__ __forceinline__ bool chan_fast(const ChanK &k) { return -k.nc <= kFastLimit; }
+
+}  // namespace gates
+}  // namespace rglru

@@ -176,6 +176,12 @@ int rglru_decode_step(const void *x_t, void *conv_state, int pos, float *h, void
                       const void *b_x, const float *Lambda, int B, int D, int H, int io,
                       void *stream);
 
+/*
+ * Number of kernel launches one rglru_decode_step_algo call with these
+ * arguments issues on its stream (0 on invalid or unsupported arguments).
+ */
+int rglru_decode_launches(int B, int D, int H, int io, int algo);
+
 /* rglru_decode_step with an explicit algorithm (same rules as rglru_fwd_algo). */
 int rglru_decode_step_algo(const void *x_t, void *conv_state, int pos, float *h, void *y_t,
                            const void *conv_w, const void *W_a, const void *b_a,

@@ -1,12 +1,14 @@
 """Error measure used to compare a result with the float64 oracle (test infrastructure).
 
 max relative error = max_i |g_i - o_i| / max(|o_i|, s_i), where s_i is the
-root-mean-square of the oracle's output over the time (or step) axis for the
-element's own (batch row, channel). A pure elementwise relative error is
-undefined where h_t crosses zero; the floor at the channel's own RMS keeps the
+root-mean-square of the oracle's output over every batch row and time (or
+decode) step of the element's own channel. A pure elementwise relative error
+is undefined where h_t crosses zero; the floor at the channel's RMS keeps the
 measure relative to the scale of that channel's state, so a wrong term, sign
 or index still shows up as an O(1) error while a correct bf16 pipeline, whose
-absolute error is a small fraction of the channel's scale, does not.
+absolute error is a small fraction of the channel's scale, does not. (One
+batch row's RMS alone is too small a floor for a few decode steps from a state
+that happens to be near zero: the step's increment then dominates the error.)
 """
 from __future__ import annotations
 
@@ -15,13 +17,19 @@ import numpy as np
 TINY = 1e-30
 
 
-def channel_rms(o: np.ndarray, time_axis: int) -> np.ndarray:
+def channel_rms(o: np.ndarray, time_axis: int = 1) -> np.ndarray:
+    """RMS of o per channel (last axis) over all other axes; keepdims.
+
+    time_axis is accepted for call sites that name it; every non-channel axis
+    (batch rows and time or decode steps) enters the RMS.
+    """
     o = np.asarray(o, dtype=np.float64)
-    return np.sqrt(np.mean(o * o, axis=time_axis, keepdims=True))
+    axes = tuple(range(o.ndim - 1))
+    return np.sqrt(np.mean(o * o, axis=axes, keepdims=True))
 
 
 def max_rel_err(g, o, scale=None, time_axis: int = 1) -> float:
-    """max |g - o| / max(|o|, scale); scale defaults to the channel RMS of o over time_axis."""
+    """max |g - o| / max(|o|, scale); scale defaults to the per-channel RMS of o."""
     g = np.asarray(g, dtype=np.float64)
     o = np.asarray(o, dtype=np.float64)
     if g.shape != o.shape:

@@ -20,7 +20,7 @@ pytestmark = pytest.mark.gpu
 
 TOL = {"f32": 1e-4, "bf16": 2e-2}
 ALGOS = ["generic", "tensor"]
-DEC_ALGOS = ["generic"]
+DEC_ALGOS = ["generic", "tensor"]
 
 
 def need_algo(wl, algo):
@@ -105,6 +105,8 @@ def test_fwd_split_composition(cuda_device, algo, io):
 
 
 def decode_run(wl, rows, dev, algo, steps):
+    if rg.decode_launches(wl.B, wl.D, wl.H, wl.dtype, algo) == 0:
+        pytest.skip(f"{algo} does not cover {wl}")
     t = generate(wl)
     g = to_dev(t, dev)
     w_dev = [g[k] for k in ("conv_w", "W_a", "b_a", "W_x", "b_x", "Lambda")]
@@ -130,6 +132,16 @@ def decode_run(wl, rows, dev, algo, steps):
 
 
 @pytest.mark.parametrize("algo", DEC_ALGOS)
+@pytest.mark.parametrize("shape", [(70, 256, 4), (33, 256, 2), (45, 512, 2), (1, 128, 1)])
+def test_decode_shapes_bf16(cuda_device, algo, shape):
+    B, D, H = shape
+    wl = WORKLOADS["decode_batch"].with_shape(B=B, D=D, H=H, decode_steps=5, bias_std=0.3,
+                                              seed=53 + B)
+    e_y, e_h = decode_run(wl, torch.arange(B), cuda_device, algo, 5)
+    assert e_y <= TOL["bf16"] and e_h <= TOL["bf16"], (e_y, e_h)
+
+
+@pytest.mark.parametrize("algo", DEC_ALGOS)
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 def test_decode_small(cuda_device, algo, io):
     wl = WORKLOADS["decode_batch"].with_shape(B=37, D=256, H=4, io=io, decode_steps=7,
@@ -140,9 +152,13 @@ def test_decode_small(cuda_device, algo, io):
 
 
 @pytest.mark.parametrize("algo", DEC_ALGOS)
-def test_decode_composes_with_fwd(cuda_device, algo):
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_decode_composes_with_fwd(cuda_device, algo, io):
     """fwd over T1 tokens then decode steps from its (h_T, conv_state_out) equals fwd over T."""
-    wl = WORKLOADS["hawk_block"].with_shape(B=3, T=20, D=256, H=2, io="f32", h0_var=0.5, seed=52)
+    wl = WORKLOADS["hawk_block"].with_shape(B=3, T=20, D=256, H=2, io=io, h0_var=0.5, seed=52)
+    if rg.decode_launches(wl.B, wl.D, wl.H, wl.dtype, algo) == 0:
+        pytest.skip(f"{algo} does not cover {wl}")
+    tol = 2e-5 if io == "f32" else 2e-2
     t = to_dev(generate(wl), cuda_device)
     w = [t[k] for k in ("conv_w", "W_a", "b_a", "W_x", "b_x", "Lambda")]
     y, hT, _ = rg.rglru_fwd(t["x"], *w, h0=t["h0"], algo=algo)
@@ -150,8 +166,8 @@ def test_decode_composes_with_fwd(cuda_device, algo):
     _, h, ring = rg.rglru_fwd(t["x"][:, :T1].contiguous(), *w, h0=t["h0"], algo=algo)
     for k, s in enumerate(range(T1, 20)):
         y_t = rg.rglru_decode_step(t["x"][:, s].contiguous(), ring, k, h, *w, algo=algo)
-        torch.testing.assert_close(y_t, y[:, s], rtol=2e-5, atol=2e-5)
-    torch.testing.assert_close(h, hT, rtol=2e-5, atol=2e-5)
+        torch.testing.assert_close(y_t.float(), y[:, s].float(), rtol=tol, atol=tol)
+    torch.testing.assert_close(h, hT, rtol=tol, atol=tol)
 
 
 # ------------------------------------------------ full-size workloads ----
