@@ -112,13 +112,19 @@ def barrier(ws):
         dist.barrier()
 
 
-def max_over_ranks(v: float, ws: int) -> float:
+def max_over_ranks(v: float, ws: int, device="cuda") -> float:
+    """The max of v over all ranks (the job's time is its slowest rank's)."""
     if ws == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], device="cuda", dtype=torch.float64)
+    t = torch.tensor([v], device=device, dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: int, steps: int, ms_max: float, ws: int) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return ws * units_per_rank * steps / (ms_max / 1e3)
 
 
 def fwd_bytes_per_chtok(wl) -> int:
@@ -191,7 +197,7 @@ def run_ours(a, ws, rank, local):
     ms = max_over_ranks(ms_local, ws)
     ms_step = ms / a.steps
     chtok = B * T * D
-    value = ws * chtok * a.steps / (ms / 1e3)
+    value = weak_scaling_value(chtok, a.steps, ms, ws)
     pk = peaks()
     bytes_step = fwd_bytes_per_chtok(wl) * chtok
     achieved = bytes_step / (ms_step / 1e3) / 1e9

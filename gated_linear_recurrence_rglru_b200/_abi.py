@@ -23,8 +23,13 @@ ALGOS = {"auto": ALGO_AUTO, "generic": ALGO_GENERIC, "tensor": ALGO_TENSOR}
 EXPORTED = (
     "rglru_status_str", "rglru_version", "rglru_fwd_workspace_bytes", "rglru_fwd",
     "rglru_fwd_algo", "rglru_decode_step", "rglru_decode_step_algo", "rglru_fwd_launches",
-    "rglru_fwd_noalloc", "rglru_decode_launches",
+    "rglru_fwd_noalloc", "rglru_decode_launches", "rglru_fwd_ex",
 )
+
+
+class FwdOptions(ctypes.Structure):
+    """rglru_fwd_options of include/rglru.h."""
+    _fields_ = [("wait_limit_ns", ctypes.c_ulonglong), ("fault_unpublished_tile", ctypes.c_int)]
 NOALLOC_SCRATCH_BYTES = 2 << 20  # RGLRU_NOALLOC_SCRATCH_BYTES in include/rglru.h
 
 
@@ -57,6 +62,8 @@ def _load():
     lib.rglru_fwd.argtypes = fwd_args
     lib.rglru_fwd_algo.restype = i32
     lib.rglru_fwd_algo.argtypes = fwd_args + [i32]
+    lib.rglru_fwd_ex.restype = i32
+    lib.rglru_fwd_ex.argtypes = fwd_args + [i32, ctypes.POINTER(FwdOptions)]
     lib.rglru_fwd_noalloc.restype = i32
     lib.rglru_fwd_noalloc.argtypes = [vp] * 6 + [fp, fp, vp, vp, fp, vp] + [i32] * 5 + [vp]
     dec_args = [vp, vp, i32, fp, vp] + [vp] * 5 + [fp] + [i32] * 4 + [vp]
@@ -126,7 +133,7 @@ def decode_launches(B: int, D: int, H: int, dtype=torch.bfloat16, algo="auto") -
 
 def rglru_fwd(x, conv_w, W_a, b_a, W_x, b_x, Lambda, h0=None, conv_state_in=None, *,
               y=None, h_T=None, conv_state_out=None, workspace=None, dev_status=None,
-              stream=None, algo="auto", want_state=True):
+              stream=None, algo="auto", want_state=True, options=None):
     """Forward of the layer over (B, T, D). Returns (y, h_T, conv_state_out).
 
     h_T / conv_state_out are None when want_state is False and no buffer is given.
@@ -163,7 +170,8 @@ def rglru_fwd(x, conv_w, W_a, b_a, W_x, b_x, Lambda, h0=None, conv_state_in=None
         _ptr(dev_status, "dev_status", torch.int32, optional=True),
         _stream_handle(stream), ALGOS[algo] if isinstance(algo, str) else int(algo),
     )
-    st = LIB.rglru_fwd_algo(*args)
+    st = (LIB.rglru_fwd_ex(*args, ctypes.byref(options)) if options is not None
+          else LIB.rglru_fwd_algo(*args))
     if st != 0:
         raise RGLRUError(st, "rglru_fwd")
     return y, h_T, conv_state_out

@@ -81,11 +81,11 @@ int rglru_decode_launches(int B, int D, int H, int io, int algo) {
   return tc_decode_launches(D, H);
 }
 
-int rglru_fwd_algo(const void *x, const void *conv_w, const void *W_a, const void *b_a,
-                   const void *W_x, const void *b_x, const float *Lambda, const float *h0,
-                   const void *conv_state_in, void *y, float *h_T, void *conv_state_out,
-                   int B, int T, int D, int H, int io, void *workspace,
-                   size_t workspace_bytes, int *dev_status, void *stream, int algo) {
+int rglru_fwd_ex(const void *x, const void *conv_w, const void *W_a, const void *b_a,
+                 const void *W_x, const void *b_x, const float *Lambda, const float *h0,
+                 const void *conv_state_in, void *y, float *h_T, void *conv_state_out, int B,
+                 int T, int D, int H, int io, void *workspace, size_t workspace_bytes,
+                 int *dev_status, void *stream, int algo, const rglru_fwd_options *opts) {
   int st = check_shape(B, T, D, H, io);
   if (st != RGLRU_OK) return st;
   if (!x || !conv_w || !W_a || !b_a || !W_x || !b_x || !Lambda || !y)
@@ -113,11 +113,24 @@ int rglru_fwd_algo(const void *x, const void *conv_w, const void *W_a, const voi
   if (need > 0 && (workspace == nullptr || !aligned16(workspace) || workspace_bytes < need))
     return RGLRU_ERR_WORKSPACE;
 
+  if (opts != nullptr && opts->wait_limit_ns > 0 && opts->wait_limit_ns < 1000000ull)
+    return RGLRU_ERR_INVALID_ARG;                // below 1 ms a healthy wait could expire
   FwdArgs p{x, conv_w, W_a, b_a, W_x, b_x, Lambda, h0, conv_state_in, y, h_T, conv_state_out,
-            B, T, D, H, dev_status};
+            B, T, D, H, dev_status,
+            opts ? opts->wait_limit_ns : 0ull, opts ? opts->fault_unpublished_tile : -1};
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = use_tc ? launch_fwd_tc(p, workspace, s) : launch_fwd_generic(p, io, workspace, s);
   return e == cudaSuccess ? RGLRU_OK : RGLRU_ERR_CUDA;
+}
+
+int rglru_fwd_algo(const void *x, const void *conv_w, const void *W_a, const void *b_a,
+                   const void *W_x, const void *b_x, const float *Lambda, const float *h0,
+                   const void *conv_state_in, void *y, float *h_T, void *conv_state_out,
+                   int B, int T, int D, int H, int io, void *workspace,
+                   size_t workspace_bytes, int *dev_status, void *stream, int algo) {
+  return rglru_fwd_ex(x, conv_w, W_a, b_a, W_x, b_x, Lambda, h0, conv_state_in, y, h_T,
+                      conv_state_out, B, T, D, H, io, workspace, workspace_bytes, dev_status,
+                      stream, algo, nullptr);
 }
 
 int rglru_fwd(const void *x, const void *conv_w, const void *W_a, const void *b_a,

@@ -183,12 +183,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
   if (tid == 0) {
     for (int i = 0; i < kJQ; ++i) {
       mbar_init(&job_full[i], 1);
-      mbar_init(&job_empty[i], 6);                  // conv, MMA, 4 epilogue warps
+      mbar_init(&job_empty[i], 9);                  // 4 conv warps, MMA, 4 epilogue warps
     }
     mbar_init(w_full, 1);
     mbar_init(w_free, 1);
     for (int i = 0; i < NS; ++i) {
-      mbar_init(&b_full[i], 1);
+      mbar_init(&b_full[i], 4);                     // 4 conv warps
       mbar_init(&b_empty[i], 1);
       mbar_init(&u_empty[i], 4);
     }
@@ -340,8 +340,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
       RG_WAIT_OR_ABORT(&u_empty[s], ((i / NS) & 1) ^ 1);
       dec_conv<K, N>(p, sB + s * C::kBBytes, sU + s * C::kUBytes, kbase, own_lo, tile * N, wt, cwq);
       fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (wt == 0) {
+      __syncwarp();
+      if (lane == 0) {                              // per warp: no barrier to strand an aborting warp at
         mbar_arrive(&b_full[s]);
         mbar_arrive(&job_empty[js]);
       }

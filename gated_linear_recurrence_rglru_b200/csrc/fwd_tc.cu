@@ -61,6 +61,8 @@ struct TcParams {
   int *counters, *abort_flag, *flags;
   float *aggA, *aggH, *incH;
   int *dev_status;
+  uint64_t wait_ns;                // bound of every wait
+  int fault_tile;                  // testing: tile of unit 0 that never publishes (-1: off)
 };
 
 template <int K, int N, int NX, int NE>
@@ -103,20 +105,6 @@ __device__ void raise_abort(const TcParams &p, volatile int *cta_abort, int code
   *cta_abort = 1;
 }
 
-// Leader-side poll of a tile flag: returns the flag (1 aggregate, 2 inclusive),
-// or -1 when another block aborted, or -2 on timeout.
-__device__ int poll_flag(const int *flag, const int *gabort, volatile int *cta_abort) {
-  int v = ld_acquire(flag);
-  if (v) return v;
-  const uint64_t t0 = globaltimer_ns();
-  for (;;) {
-    __nanosleep(32);
-    v = ld_acquire(flag);
-    if (v) return v;
-    if (*cta_abort || *(volatile const int *)gabort) return -1;
-    if (globaltimer_ns() - t0 > kWaitNs) return -2;
-  }
-}
 
 // Offset (bytes) of (own channel c, 4-token block jb) in the fp32 u tile:
 // channel-major rows of N floats whose 16-byte blocks are XOR-permuted by
@@ -243,16 +231,16 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
   if (tid == 0) {
     for (int i = 0; i < kJQ; ++i) {
       mbar_init(&job_full[i], 1);
-      mbar_init(&job_empty[i], 6);                  // conv, MMA, 4 epilogue warps
+      mbar_init(&job_empty[i], 9);                  // 4 conv warps, MMA, 4 epilogue warps
     }
     for (int i = 0; i < NX; ++i) {
       mbar_init(&x_full[i], 1);
-      mbar_init(&x_empty[i], C::kUTile ? 1 : 4);   // conv warpgroup, or 4 epilogue warps
+      mbar_init(&x_empty[i], 4);                    // 4 conv warps, or 4 epilogue warps
     }
     mbar_init(w_full, 1);
     mbar_init(w_free, 1);
     for (int i = 0; i < NS; ++i) {
-      mbar_init(&b_full[i], 1);
+      mbar_init(&b_full[i], 4);                     // 4 conv warps
       mbar_init(&b_empty[i], 1);
       mbar_init(&u_empty[i], 4);                    // 4 epilogue warps
     }
@@ -282,7 +270,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
   const int R = p.bw <= 128 ? p.bw : 256;           // weight rows per TMA box
 
 #define RG_WAIT_OR_ABORT(bar, par)                                   \
-  if (!mbar_wait((bar), (par), cta_abort, kWaitNs)) {                \
+  if (!mbar_wait((bar), (par), cta_abort, p.wait_ns)) {                \
     if (!*cta_abort) raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);   \
     break;                                                           \
   }
@@ -322,7 +310,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
           // one terminal job per epilogue warpgroup that may still wait for a job
           for (int e = 1; e < NE; ++e) {
             const int je = i + e;
-            if (!mbar_wait(&job_empty[je % kJQ], ((je / kJQ) & 1) ^ 1, cta_abort, kWaitNs)) break;
+            if (!mbar_wait(&job_empty[je % kJQ], ((je / kJQ) & 1) ^ 1, cta_abort, p.wait_ns)) break;
             jobs[je % kJQ] = make_int4(-1, -1, 0, 0);
             mbar_arrive(&job_full[je % kJQ]);
           }
@@ -416,7 +404,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
   } else if (warp < 6) {
     // ============================ conv warpgroup ============================
     const int wt = tid - 64;                      // 0 .. 127
-    const bool leader = (wt == 0);
     int cur_unit = -1;
     float2 cwq[4][2];                             // conv taps of this thread's channel quad
     for (int i = 0;; ++i) {
@@ -446,9 +433,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
       conv_tile<K, N, C::kUTile>(sX + xb * C::kXBytes, sB + s * C::kBBytes, sU + s * C::kUBytes,
                                  p, b, kbase, own_lo, tile, nvalid, tile == p.n_tiles - 1, wt,
                                  cwq);
+      // each warp hands its part over on its own: no barrier that an aborting
+      // warp could leave the others waiting at
       fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (leader) {
+      __syncwarp();
+      if (lane == 0) {
         if (C::kUTile) mbar_arrive(&x_empty[xb]);   // else the epilogue still reads x
         mbar_arrive(&b_full[s]);
         mbar_arrive(&job_empty[js]);
@@ -508,8 +497,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
               res = 32;                           // 32 aggregates, no inclusive yet: fold, go on
               break;
             }
-            if (*cta_abort || *(volatile const int *)p.abort_flag) { res = -1; break; }
-            if (globaltimer_ns() - t0 > kWaitNs) { res = -2; break; }
+            if (*cta_abort || *(volatile const int *)p.abort_flag) {
+              *cta_abort = 1;
+              res = -1;
+              break;
+            }
+            if (globaltimer_ns() - t0 > p.wait_ns) { res = -2; break; }
             __nanosleep(32);
           }
           if (res == -2) {
@@ -545,7 +538,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
         }
         __stcg(p.incH + (ubase + tile) * kM + m, fmaf(d_A, h_in, d_H));
         __syncwarp();
-        if (lane == 0) st_release(p.flags + (ubase + tile) * 4 + qd, 2);
+        if (lane == 0 && !(unit == 0 && tile == p.fault_tile))
+          st_release(p.flags + (ubase + tile) * 4 + qd, 2);
       }
       // ---- pass 2: y_t = h_t ----
       float h = h_in;
@@ -706,8 +700,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
           __stcg(p.aggH + tix * kM + m, Hl);
         }
         __syncwarp();
+        const bool silent = (unit == 0 && tile == p.fault_tile);
         if (lane == 0) {
-          st_release(p.flags + tix * 4 + qd, tile == 0 ? 2 : 1);
+          if (!silent) st_release(p.flags + tix * 4 + qd, tile == 0 ? 2 : 1);
           if (C::kUTile) mbar_arrive(&u_empty[s]);
           else mbar_arrive(&x_empty[xb]);
         }
@@ -829,6 +824,8 @@ cudaError_t launch_tc_t(const FwdArgs &a, const TcLayout &L, void *ws, cudaStrea
   p.aggH = reinterpret_cast<float *>(w + L.off_aggH);
   p.incH = reinterpret_cast<float *>(w + L.off_incH);
   p.dev_status = a.dev_status;
+  p.wait_ns = a.wait_ns ? a.wait_ns : kWaitNs;
+  p.fault_tile = a.fault_tile;
 
   cudaError_t e = cudaMemsetAsync(ws, 0, L.ints_bytes, st);
   if (e != cudaSuccess) return e;

@@ -15,6 +15,8 @@ struct FwdArgs {
   void *conv_state_out;
   int B, T, D, H;
   int *dev_status;
+  unsigned long long wait_ns;  // 0: default bound of device-side waits
+  int fault_tile;              // testing only: tile of unit 0 that never publishes (-1: off)
 };
 
 struct DecArgs {

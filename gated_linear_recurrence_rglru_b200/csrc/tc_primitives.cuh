@@ -55,17 +55,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 
 // Waits for the phase of `parity` to complete. Gives up after `limit_ns` or
 // as soon as *abort becomes nonzero; returns false then (the caller stops).
+// The result is the same for every active lane of the warp, so that a warp
+// never splits into lanes that go on and lanes that stop.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
                                           volatile int *abort, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > limit_ns) return false;
+  bool ok = mbar_try_wait(bar, parity);
+  if (!ok) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+      if (mbar_try_wait(bar, parity)) {
+        ok = true;
+        break;
+      }
+      if ((it & 63u) == 0 && (*abort || globaltimer_ns() - t0 > limit_ns)) break;
     }
   }
+  return __all_sync(__activemask(), ok);
 }
 
 // Bounded wait that ignores abort requests: used to let copies and MMAs that

@@ -123,6 +123,33 @@ int rglru_fwd_algo(const void *x, const void *conv_w, const void *W_a, const voi
                    size_t workspace_bytes, int *dev_status, void *stream, int algo);
 
 /*
+ * Options of rglru_fwd_ex. Zero-initialise, then set what is needed.
+ *   wait_limit_ns           bound of every device-side wait of the tensor-core
+ *                           forward (a CTA waiting for its predecessor's carry, or
+ *                           one of its pipeline stages); 0 = the default of 2 s.
+ *                           Values from 1 ns to 1 ms are refused (INVALID_ARG):
+ *                           healthy waits could expire.
+ *   fault_unpublished_tile  testing of the failure path: when >= 0, the tile of
+ *                           that index in the first (batch row 0, channels
+ *                           0..127) group never publishes its carry, so the
+ *                           waits of its successors run out: the call then
+ *                           reports RGLRU_ERR_TIMEOUT through dev_status and
+ *                           returns with y incomplete; the context stays usable.
+ *                           -1 = off (the default of rglru_fwd and rglru_fwd_algo).
+ */
+typedef struct {
+  unsigned long long wait_limit_ns;
+  int fault_unpublished_tile;
+} rglru_fwd_options;
+
+/* rglru_fwd_algo with options (NULL = defaults). */
+int rglru_fwd_ex(const void *x, const void *conv_w, const void *W_a, const void *b_a,
+                 const void *W_x, const void *b_x, const float *Lambda, const float *h0,
+                 const void *conv_state_in, void *y, float *h_T, void *conv_state_out, int B,
+                 int T, int D, int H, int io, void *workspace, size_t workspace_bytes,
+                 int *dev_status, void *stream, int algo, const rglru_fwd_options *opts);
+
+/*
  * Size of the library's fixed device scratch used by rglru_fwd_noalloc.
  * Every GPU that loads the library holds this much device memory until the
  * process exits.

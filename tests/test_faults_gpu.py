@@ -1,0 +1,53 @@
+"""Failure detection on the GPU without a GPU fault: a tile that never
+publishes its carry (a flag that nothing sets) makes its successors' bounded
+waits run out; the kernel must report RGLRU_ERR_TIMEOUT through the status
+word, return in bounded time, and leave the context usable."""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import gated_linear_recurrence_rglru_b200 as rg
+from gated_linear_recurrence_rglru_b200._abi import FwdOptions
+from gated_linear_recurrence_rglru_b200.workloads import WORKLOADS, generate
+from oracle import rglru_oracle as orc
+from oracle.compare import max_rel_err
+
+pytestmark = pytest.mark.gpu
+
+WL = WORKLOADS["hawk_block"].with_shape(B=1, T=64 * 12, D=128, H=2, seed=71)
+
+
+def _inputs(dev):
+    t = generate(WL)
+    return t, {k: (v.to(dev) if v is not None else None) for k, v in t.items()}
+
+
+def test_unpublished_tile_times_out_and_context_survives(cuda_device):
+    t, g = _inputs(cuda_device)
+    w = [g[k] for k in ("conv_w", "W_a", "b_a", "W_x", "b_x", "Lambda")]
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    opts = FwdOptions(wait_limit_ns=50_000_000, fault_unpublished_tile=3)
+    t0 = time.time()
+    rg.rglru_fwd(g["x"], *w, algo="tensor", dev_status=status, options=opts)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 4                  # RGLRU_ERR_TIMEOUT
+    assert time.time() - t0 < 20.0
+    # same context, normal call: correct again
+    status.zero_()
+    y, _, _ = rg.rglru_fwd(g["x"], *w, algo="tensor", dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    yo, _, _ = orc.rglru_fwd(t["x"], t["conv_w"], t["W_a"], t["b_a"], t["W_x"], t["b_x"],
+                             t["Lambda"])
+    assert max_rel_err(y.float().cpu().numpy(), yo) <= 2e-2
+
+
+def test_too_short_wait_limit_is_refused(cuda_device):
+    _, g = _inputs(cuda_device)
+    w = [g[k] for k in ("conv_w", "W_a", "b_a", "W_x", "b_x", "Lambda")]
+    with pytest.raises(rg.RGLRUError) as ei:
+        rg.rglru_fwd(g["x"], *w, algo="tensor", options=FwdOptions(wait_limit_ns=1000,
+                                                                   fault_unpublished_tile=-1))
+    assert ei.value.status == 1
