@@ -15,13 +15,16 @@
 //      the A operand, M = 128 output channels, MN-major and loaded by TMA, and
 //      the conv output as B, N = tokens: TMEM lane m then holds channel m's
 //      two gate pre-activations along time);
-//   3. an epilogue warpgroup, per lane (channel): sigmoid gates, log-space decay, sqrt(1 - a^2) and a
-//      local scan along time (pass 1, results back into TMEM);
-//   4. carries the state across tiles with a decoupled look-back over per-tile
-//      (prod a, local h) aggregates and inclusive states in the workspace —
+//   3. an epilogue warpgroup, per lane (channel): sigmoid gates, log-space
+//      decay, sqrt(1 - a^2) and a local scan along time from a zero state,
+//      keeping the running products P_t = a_1 ... a_t and local states Hl_t
+//      in TMEM (pass 1);
+//   4. carries the state across tiles with a decoupled look-back over per-tile,
+//      per-channel words (prod a, local h) / inclusive state in the workspace —
 //      the exact linear scan of S. De's thread ("linear scans instead of
 //      parallel scans"), parallel across tiles;
-//   5. rescans from the carried state and writes y (pass 2).
+//   5. writes y_t = P_t h_in + Hl_t from the carried state h_in (pass 2, no
+//      dependency between tokens).
 // Roles: warp 0 claims tiles (per-unit counters in time order, stealing from
 // other units once its own is done) and issues TMA; warp 1 owns TMEM and
 // issues the MMAs; warps 2-5 compute the Conv1D of every job; NE epilogue
@@ -58,8 +61,8 @@ struct TcParams {
   __nv_bfloat16 *conv_state_out;
   int B, T, D, H, bw;
   int n_cg, n_units, n_tiles;
-  int *counters, *abort_flag, *flags;
-  float *aggA, *aggH, *incH;
+  int *counters, *abort_flag;
+  unsigned long long *carry;       // [unit][tile][128] carry words (see carry_word)
   int *dev_status;
   uint64_t wait_ns;                // bound of every wait
   int fault_tile;                  // testing: tile of unit 0 that never publishes (-1: off)
@@ -103,6 +106,23 @@ __device__ void raise_abort(const TcParams &p, volatile int *cta_abort, int code
   if (p.dev_status) atomicCAS(p.dev_status, 0, code);
   atomicExch(p.abort_flag, 1);
   *cta_abort = 1;
+}
+
+// Carry word of one (unit, tile, channel), written with one 64-bit store:
+//   low 32 bits == 0                -> not published yet (the workspace is zeroed)
+//   low 32 bits with the sign bit   -> aggregate: A = prod a over the tile (the
+//                                      low bits with the sign cleared), H = local
+//                                      state of the tile from zero (high bits)
+//   low 32 bits == bits of +1.0f    -> inclusive: the state after the tile (high)
+// A is a product of decays in (0, 1], so its sign bit is free; the aggregate
+// of a NaN input stays a (NaN) aggregate and never reads as "not published".
+constexpr uint32_t kIncTag = 0x3F800000u;
+__device__ __forceinline__ unsigned long long carry_agg(float A, float H) {
+  return (static_cast<unsigned long long>(__float_as_uint(H)) << 32) |
+         (__float_as_uint(A) | 0x80000000u);
+}
+__device__ __forceinline__ unsigned long long carry_inc(float h) {
+  return (static_cast<unsigned long long>(__float_as_uint(h)) << 32) | kIncTag;
 }
 
 
@@ -446,9 +466,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
   } else {
     // ========================== epilogue warpgroups ==========================
     // Epilogue warpgroup e takes jobs e, e + NE, ...; each of its 4 warps owns
-    // one TMEM quadrant (32 channels) and works on its own: per job, pass 1
-    // (gates, decay, local scan) and publish of its quadrant's aggregate; then
-    // the carry (look-back over its quadrant's flags) and pass 2 of the warp's
+    // one TMEM quadrant (32 channels, one per lane) and works on its own: per
+    // job, pass 1 and the publication of each channel's aggregate; then the
+    // carry (look-back over its channels' words) and pass 2 of the warp's
     // previous job, whose predecessors have usually published by then.
     const int eg = (warp - 6) >> 2;               // 0 .. NE-1
     const int qd = warp & 3;                      // TMEM quadrant
@@ -471,101 +491,79 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
       const bool last_tile = (tile == p.n_tiles - 1);
       const int ts = d_i % NT;
       const uint32_t t_lane = t_lane0 + static_cast<uint32_t>(ts * C::kSlotCols);
-      const size_t ubase = static_cast<size_t>(unit) * p.n_tiles;
+      unsigned long long *cw = p.carry + static_cast<size_t>(unit) * p.n_tiles * kM + m;
       float h_in = 0.f;
       if (tile == 0) {
         if (p.h0 != nullptr) h_in = p.h0[static_cast<size_t>(b) * p.D + c];
       } else {
-        // Look back over a window of up to 32 predecessors: lane l reads the
-        // flag of tile top - l; the warp finds the nearest inclusive state
-        // with only aggregates after it and folds those in.
+        // Look back along this lane's channel, four words per round trip: fold
+        // aggregates until an inclusive word; an unpublished word ends the
+        // round and is read again in the next.
         float mult = 1.f, add = 0.f;
-        int top = tile - 1;
+        int k = tile - 1;                         // next tile to read
+        bool done = false;
+        const uint64_t t0 = globaltimer_ns();
         for (;;) {
-          const int jt = top - lane;
-          int res;
-          const uint64_t t0 = globaltimer_ns();
-          for (;;) {
-            const int f = (jt >= 0) ? ld_acquire(p.flags + (ubase + jt) * 4 + qd) : 0;
-            const unsigned agg = __ballot_sync(0xffffffffu, f >= 1);
-            const unsigned inc = __ballot_sync(0xffffffffu, f == 2);
-            if (inc != 0u) {
-              const int e = __ffs(inc) - 1;       // nearest inclusive
-              const unsigned below = (e == 0) ? 0u : (0xffffffffu >> (32 - e));
-              if ((agg & below) == below) { res = e; break; }
-            } else if (agg == 0xffffffffu) {
-              res = 32;                           // 32 aggregates, no inclusive yet: fold, go on
-              break;
+          if (!done) {
+            unsigned long long w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              w[q] = (k - q >= 0) ? ld_relaxed_u64(cw + static_cast<size_t>(k - q) * kM) : 0ull;
+            bool stop = false;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (stop) continue;
+              const uint32_t lo = static_cast<uint32_t>(w[q]);
+              const float hi = __uint_as_float(static_cast<uint32_t>(w[q] >> 32));
+              if (lo == 0u) {
+                stop = true;                      // not yet published: read tile k again
+              } else if (lo & 0x80000000u) {
+                add = fmaf(mult, hi, add);        // aggregate
+                mult *= __uint_as_float(lo & 0x7FFFFFFFu);
+                --k;
+              } else {
+                h_in = fmaf(mult, hi, add);       // inclusive
+                done = true;
+                stop = true;
+              }
             }
-            if (*cta_abort || *(volatile const int *)p.abort_flag) {
-              *cta_abort = 1;
-              res = -1;
-              break;
-            }
-            if (globaltimer_ns() - t0 > p.wait_ns) { res = -2; break; }
-            __nanosleep(32);
           }
-          if (res == -2) {
-            if (lane == 0) raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);
-            res = -1;
-          }
-          __syncwarp();                           // order the data loads after the flags
-          if (res < 0) {
+          if (__all_sync(0xffffffffu, done)) break;
+          const bool give_up = *cta_abort || *(volatile const int *)p.abort_flag ||
+                               (globaltimer_ns() - t0 > p.wait_ns);
+          if (__any_sync(0xffffffffu, give_up)) {
+            if (lane == 0 && !*cta_abort) raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);
+            *cta_abort = 1;
             h_in = 0.f;
             break;
           }
-          const int nagg = res < 32 ? res : 32;
-          for (int k = 0; k < nagg; k += 4) {
-            float Av[4], Hv[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const bool in = k + q < nagg;
-              const size_t jix = (ubase + (in ? top - k - q : top)) * kM + m;
-              Av[q] = in ? __ldcg(p.aggA + jix) : 1.f;
-              Hv[q] = in ? __ldcg(p.aggH + jix) : 0.f;
-            }
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              add = fmaf(mult, Hv[q], add);
-              mult *= Av[q];
-            }
-          }
-          if (res < 32) {
-            h_in = fmaf(mult, __ldcg(p.incH + (ubase + top - res) * kM + m), add);
-            break;
-          }
-          top -= 32;
+          __nanosleep(64);
         }
-        __stcg(p.incH + (ubase + tile) * kM + m, fmaf(d_A, h_in, d_H));
-        __syncwarp();
-        if (lane == 0 && !(unit == 0 && tile == p.fault_tile))
-          st_release(p.flags + (ubase + tile) * 4 + qd, 2);
+        if (!(unit == 0 && tile == p.fault_tile))
+          st_relaxed_u64(cw + static_cast<size_t>(tile) * kM, carry_inc(fmaf(d_A, h_in, d_H)));
       }
-      // ---- pass 2: y_t = h_t ----
-      float h = h_in;
+      // ---- pass 2: y_t = P_t h_in + Hl_t ----
       __nv_bfloat16 *yrow = p.y + (static_cast<size_t>(b) * p.T + n0) * p.D + c;
 #pragma unroll 1
       for (int ch = 0; ch < N / 16; ++ch) {
-        float av[16], bv[16];
-        tmem_ld16(t_lane + ch * 16, av);
-        tmem_ld16(t_lane + N + ch * 16, bv);
+        if (ch * 16 >= nvalid) break;
+        float pv[16], hv[16];
+        tmem_ld16(t_lane + ch * 16, pv);
+        tmem_ld16(t_lane + N + ch * 16, hv);
         tmem_wait_ld();
         __nv_bfloat16 *yc = yrow + static_cast<size_t>(ch * 16) * p.D;
         if (ch * 16 + 16 <= nvalid) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            h = fmaf(av[j], h, bv[j]);
-            yc[static_cast<size_t>(j) * p.D] = __float2bfloat16_rn(h);
-          }
+          for (int j = 0; j < 16; ++j)
+            yc[static_cast<size_t>(j) * p.D] = __float2bfloat16_rn(fmaf(pv[j], h_in, hv[j]));
         } else {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            h = fmaf(av[j], h, bv[j]);
-            if (ch * 16 + j < nvalid) yc[static_cast<size_t>(j) * p.D] = __float2bfloat16_rn(h);
-          }
+          for (int j = 0; j < 16; ++j)
+            if (ch * 16 + j < nvalid)
+              yc[static_cast<size_t>(j) * p.D] = __float2bfloat16_rn(fmaf(pv[j], h_in, hv[j]));
         }
       }
-      if (last_tile && p.h_T != nullptr) p.h_T[static_cast<size_t>(b) * p.D + c] = h;
+      if (last_tile && p.h_T != nullptr) p.h_T[static_cast<size_t>(b) * p.D + c] = fmaf(d_A, h_in, d_H);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -620,9 +618,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
           xm1 = __bfloat162float(cs[2 * p.D]);
         }
       }
-      // ---- pass 1: gates, decay, local scan ----
-      float Hl = 0.f;
-      float2 S2 = make_float2(0.f, 0.f);
+      // ---- pass 1: gates, decay, local scan from zero; (P_t, Hl_t) -> TMEM ----
+      // Tokens past the end of the sequence (last tile) are computed like the
+      // others (their x rows read as zeros) and never used: the tile's
+      // aggregate is read back at the last valid token.
+      float Hl = 0.f, P = 1.f;
 #pragma unroll 1
       for (int ch = 0; ch < N / 16; ++ch) {
         float za[16], zx[16];
@@ -649,7 +649,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
           }
         }
         tmem_wait_ld();
-        const bool full = (ch * 16 + 16 <= nvalid);
         if (fast) {
 #pragma unroll
           for (int pr = 0; pr < 8; ++pr) {
@@ -657,52 +656,51 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
             gate_pair_fast(make_float2(za[2 * pr], za[2 * pr + 1]),
                            make_float2(zx[2 * pr], zx[2 * pr + 1]),
                            make_float2(uu[2 * pr], uu[2 * pr + 1]), kc, a, beta, la);
-            if (!full) {
-              const int n = ch * 16 + 2 * pr;
-              if (n >= nvalid) a.x = 1.f, beta.x = 0.f, la.x = 0.f;
-              if (n + 1 >= nvalid) a.y = 1.f, beta.y = 0.f, la.y = 0.f;
-            }
             Hl = fmaf(a.x, Hl, beta.x);
+            P *= a.x;
+            za[2 * pr] = P;
+            zx[2 * pr] = Hl;
             Hl = fmaf(a.y, Hl, beta.y);
-            S2 = __fadd2_rn(S2, la);
-            za[2 * pr] = a.x;
-            za[2 * pr + 1] = a.y;
-            zx[2 * pr] = beta.x;
-            zx[2 * pr + 1] = beta.y;
+            P *= a.y;
+            za[2 * pr + 1] = P;
+            zx[2 * pr + 1] = Hl;
           }
         } else {
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             float a, beta, la;
             gate_one(za[j], zx[j], uu[j], kc, a, beta, la);
-            if (ch * 16 + j >= nvalid) a = 1.f, beta = 0.f, la = 0.f;
             Hl = fmaf(a, Hl, beta);
-            S2.x += la;
-            za[j] = a;
-            zx[j] = beta;
+            P *= a;
+            za[j] = P;
+            zx[j] = Hl;
           }
         }
         tmem_st16(t_lane + ch * 16, za);
         tmem_st16(t_lane + N + ch * 16, zx);
       }
       tmem_wait_st();
-      const float A = ex2_approx((S2.x + S2.y) * kLog2e);
-      // publish this quadrant's state: inclusive for the first tile of a
-      // sequence (h0 is known), else the aggregate (prod a, local h); release
-      // the u / x tile
+      float A = P;
+      if (nvalid < N) {
+        A = tmem_ld1(t_lane + (nvalid - 1));
+        Hl = tmem_ld1(t_lane + N + (nvalid - 1));
+        tmem_wait_ld();
+      }
+      // publish this channel's word: inclusive for the first tile of a
+      // sequence (h0 is known), else the aggregate; release the u / x tile
       {
-        const size_t tix = static_cast<size_t>(unit) * p.n_tiles + tile;
-        if (tile == 0) {
-          const float h0v = p.h0 != nullptr ? p.h0[static_cast<size_t>(b) * p.D + c] : 0.f;
-          __stcg(p.incH + tix * kM + m, fmaf(A, h0v, Hl));
-        } else {
-          __stcg(p.aggA + tix * kM + m, A);
-          __stcg(p.aggH + tix * kM + m, Hl);
+        const size_t wix = (static_cast<size_t>(unit) * p.n_tiles + tile) * kM + m;
+        const bool silent = (unit == 0 && tile == p.fault_tile);
+        if (!silent) {
+          if (tile == 0) {
+            const float h0v = p.h0 != nullptr ? p.h0[static_cast<size_t>(b) * p.D + c] : 0.f;
+            st_relaxed_u64(p.carry + wix, carry_inc(fmaf(A, h0v, Hl)));
+          } else {
+            st_relaxed_u64(p.carry + wix, carry_agg(A, Hl));
+          }
         }
         __syncwarp();
-        const bool silent = (unit == 0 && tile == p.fault_tile);
         if (lane == 0) {
-          if (!silent) st_release(p.flags + tix * 4 + qd, tile == 0 ? 2 : 1);
           if (C::kUTile) mbar_arrive(&u_empty[s]);
           else mbar_arrive(&x_empty[xb]);
         }
@@ -745,7 +743,7 @@ int tile_tokens(int bw) { return bw == 256 ? 32 : 64; }
 
 struct TcLayout {
   int n_cg, n_units, n_tiles;
-  size_t off_counters, off_abort, off_flags, off_aggA, off_aggH, off_incH, ints_bytes, total;
+  size_t off_counters, off_abort, off_carry, total;
 };
 
 TcLayout tc_layout(int B, int T, int D, int H) {
@@ -756,14 +754,9 @@ TcLayout tc_layout(int B, int T, int D, int H) {
   L.n_tiles = ceil_div(T, tile_tokens(bw));
   L.off_counters = 0;
   L.off_abort = static_cast<size_t>(L.n_units) * 4;
-  L.off_flags = align_up(L.off_abort + 4, 16);
-  // one flag per (unit, tile, 32-channel quadrant)
-  L.ints_bytes = align_up(L.off_flags + static_cast<size_t>(L.n_units) * L.n_tiles * 16, 256);
-  const size_t agg = align_up(static_cast<size_t>(L.n_units) * L.n_tiles * kM * 4, 256);
-  L.off_aggA = L.ints_bytes;
-  L.off_aggH = L.off_aggA + agg;
-  L.off_incH = L.off_aggH + agg;
-  L.total = L.off_incH + agg;
+  L.off_carry = align_up(L.off_abort + 4, 256);
+  // one 8-byte carry word per (unit, tile, channel); all of it starts at zero
+  L.total = align_up(L.off_carry + static_cast<size_t>(L.n_units) * L.n_tiles * kM * 8, 256);
   return L;
 }
 
@@ -819,15 +812,12 @@ cudaError_t launch_tc_t(const FwdArgs &a, const TcLayout &L, void *ws, cudaStrea
   p.n_tiles = L.n_tiles;
   p.counters = reinterpret_cast<int *>(w + L.off_counters);
   p.abort_flag = reinterpret_cast<int *>(w + L.off_abort);
-  p.flags = reinterpret_cast<int *>(w + L.off_flags);
-  p.aggA = reinterpret_cast<float *>(w + L.off_aggA);
-  p.aggH = reinterpret_cast<float *>(w + L.off_aggH);
-  p.incH = reinterpret_cast<float *>(w + L.off_incH);
+  p.carry = reinterpret_cast<unsigned long long *>(w + L.off_carry);
   p.dev_status = a.dev_status;
   p.wait_ns = a.wait_ns ? a.wait_ns : kWaitNs;
   p.fault_tile = a.fault_tile;
 
-  cudaError_t e = cudaMemsetAsync(ws, 0, L.ints_bytes, st);
+  cudaError_t e = cudaMemsetAsync(ws, 0, L.total, st);
   if (e != cudaSuccess) return e;
   auto kern = fwd_tc_kernel<K, N, NX, NE>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
