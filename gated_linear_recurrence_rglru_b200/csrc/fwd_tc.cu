@@ -140,9 +140,10 @@ __device__ __forceinline__ uint32_t u_offset(int c, int jb) {
 // Conv1D of one tile, token-major. Thread t covers the 4 channels
 // [4 q, 4 q + 4) of the K range and SEG consecutive tokens; a warp covers 128
 // channels of one token segment, so that its shared-memory rows are contiguous
-// (no bank conflicts). All input rows are read before any output is written,
-// and each is unpacked once. Writes the bf16 B operand (K-major, 128-byte
-// swizzle) and, when kUTile, the fp32 u of the unit's own channels
+// (no bank conflicts). The loop advances 4 tokens per iteration with a sliding
+// window of 4 input rows in registers (a compact loop: the conv shares the
+// instruction cache with the epilogue). Writes the bf16 B operand (K-major,
+// 128-byte swizzle) and, when kUTile, the fp32 u of the unit's own channels
 // channel-major into ut (see u_offset). w holds the 4 taps of the 4 channels.
 template <int K, int N, bool kUTile>
 __device__ __forceinline__ void conv_tile(const unsigned char *__restrict__ xs,
@@ -157,59 +158,84 @@ __device__ __forceinline__ void conv_tile(const unsigned char *__restrict__ xs,
   const int kq = qd * 4, nb = sg * SEG;
   const bool own = (kq >= own_lo) && (kq < own_lo + kM);
   const int chq = kbase + kq;                       // first global channel of the quad
-  uint2 rows[SEG + 3];
-#pragma unroll
-  for (int r = 0; r < SEG + 3; ++r)
-    rows[r] = *reinterpret_cast<const uint2 *>(xs + ((nb + r) * K + kq) * 2);
+  // x tile row r holds token tile * N - 3 + r: the window of output token
+  // nb + j is rows nb + j .. nb + j + 3
+  const unsigned char *xq = xs + kq * 2;
+  uint2 r0 = *reinterpret_cast<const uint2 *>(xq + (nb + 0) * K * 2);
+  uint2 r1 = *reinterpret_cast<const uint2 *>(xq + (nb + 1) * K * 2);
+  uint2 r2 = *reinterpret_cast<const uint2 *>(xq + (nb + 2) * K * 2);
   if (tile == 0 && nb == 0 && p.conv_state_in != nullptr) {
-#pragma unroll
-    for (int r = 0; r < 3; ++r)
-      rows[r] = __ldg(reinterpret_cast<const uint2 *>(p.conv_state_in +
-                                                       (static_cast<size_t>(b) * 3 + r) * p.D + chq));
+    const __nv_bfloat16 *cs = p.conv_state_in + static_cast<size_t>(b) * 3 * p.D + chq;
+    r0 = __ldg(reinterpret_cast<const uint2 *>(cs));
+    r1 = __ldg(reinterpret_cast<const uint2 *>(cs + p.D));
+    r2 = __ldg(reinterpret_cast<const uint2 *>(cs + 2 * p.D));
   }
-  // B operand offsets: row n = nb + j with n % 8 == j % 8 (nb is a multiple of 8)
-  const uint32_t bt_base = static_cast<uint32_t>((kq >> 6) * N * 128 + nb * 128 + ((kq & 7) << 1));
-  const int chunk = (kq & 63) >> 3;
   float2 xw[4][2];
+  xw[0][0] = bf2_to_f2(r0.x);
+  xw[0][1] = bf2_to_f2(r0.y);
+  xw[1][0] = bf2_to_f2(r1.x);
+  xw[1][1] = bf2_to_f2(r1.y);
+  xw[2][0] = bf2_to_f2(r2.x);
+  xw[2][1] = bf2_to_f2(r2.y);
+  // B operand: row n = nb + j of the 64-channel block kq / 64; 16-byte chunk
+  // (kq % 64) / 8 of the row, XOR-swizzled by n % 8 (= j % 8)
+  unsigned char *bq = bt + (kq >> 6) * N * 128 + nb * 128 + ((kq & 7) << 1);
+  const int chunk = (kq & 63) >> 3;
+  // u tile rows of the 4 own channels and their block permutations
+  uint32_t ubase[4], uperm[4];
 #pragma unroll
-  for (int r = 0; r < 3; ++r) {
-    xw[r][0] = bf2_to_f2(rows[r].x);
-    xw[r][1] = bf2_to_f2(rows[r].y);
+  for (int k = 0; k < 4; ++k) {
+    const int c = kq - own_lo + k;
+    ubase[k] = static_cast<uint32_t>(c * (N * 4));
+    uperm[k] = static_cast<uint32_t>((c & 7) ^ ((c >> 3) & 7));
   }
-  float uacc[4][4];                                 // u of 4 channels x 4 tokens (u tile block)
+#pragma unroll 1
+  for (int jb = 0; jb < SEG; jb += 4) {
+    uint2 nr[4];
 #pragma unroll
-  for (int j = 0; j < SEG; ++j) {
-    const int c3 = (j + 3) & 3;                     // window slot of token nb + j
-    xw[c3][0] = bf2_to_f2(rows[j + 3].x);
-    xw[c3][1] = bf2_to_f2(rows[j + 3].y);
-    float2 u[2];
+    for (int q = 0; q < 4; ++q)
+      nr[q] = *reinterpret_cast<const uint2 *>(xq + (nb + jb + 3 + q) * K * 2);
+    float uacc[4][4];                               // u of 4 channels x 4 tokens
 #pragma unroll
-    for (int pp = 0; pp < 2; ++pp) {
-      float2 acc = __fmul2_rn(w[0][pp], xw[(j + 0) & 3][pp]);
-      acc = __ffma2_rn(w[1][pp], xw[(j + 1) & 3][pp], acc);
-      acc = __ffma2_rn(w[2][pp], xw[(j + 2) & 3][pp], acc);
-      u[pp] = __ffma2_rn(w[3][pp], xw[c3][pp], acc);
-    }
-    *reinterpret_cast<uint2 *>(bt + bt_base + j * 128 + (((chunk ^ j) & 7) << 4)) =
-        make_uint2(f2_to_bf2(u[0]), f2_to_bf2(u[1]));
-    if (kUTile) {
-      uacc[0][j & 3] = u[0].x;
-      uacc[1][j & 3] = u[0].y;
-      uacc[2][j & 3] = u[1].x;
-      uacc[3][j & 3] = u[1].y;
-      if ((j & 3) == 3 && own) {
+    for (int q = 0; q < 4; ++q) {
+      const int j = jb + q;                         // j % 4 == q
+      xw[(q + 3) & 3][0] = bf2_to_f2(nr[q].x);
+      xw[(q + 3) & 3][1] = bf2_to_f2(nr[q].y);
+      float2 u[2];
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          *reinterpret_cast<float4 *>(ut + u_offset<N>(kq - own_lo + k, (nb + j) >> 2)) =
-              make_float4(uacc[k][0], uacc[k][1], uacc[k][2], uacc[k][3]);
+      for (int pp = 0; pp < 2; ++pp) {
+        float2 acc = __fmul2_rn(w[0][pp], xw[q & 3][pp]);
+        acc = __ffma2_rn(w[1][pp], xw[(q + 1) & 3][pp], acc);
+        acc = __ffma2_rn(w[2][pp], xw[(q + 2) & 3][pp], acc);
+        u[pp] = __ffma2_rn(w[3][pp], xw[(q + 3) & 3][pp], acc);
       }
+      *reinterpret_cast<uint2 *>(bq + j * 128 + (((chunk ^ j) & 7) << 4)) =
+          make_uint2(f2_to_bf2(u[0]), f2_to_bf2(u[1]));
+      uacc[0][q] = u[0].x;
+      uacc[1][q] = u[0].y;
+      uacc[2][q] = u[1].x;
+      uacc[3][q] = u[1].y;
     }
-    if (own && last_tile && nb + j == nvalid - 1 && p.conv_state_out != nullptr) {
-      // the last three inputs x_{T-3}, x_{T-2}, x_{T-1} of these 4 channels
+    if (kUTile && own) {
+      const uint32_t blk = static_cast<uint32_t>((nb + jb) >> 2);
 #pragma unroll
-      for (int r = 0; r < 3; ++r)
-        *reinterpret_cast<uint2 *>(p.conv_state_out + (static_cast<size_t>(b) * 3 + r) * p.D +
-                                   chq) = rows[j + 1 + r];
+      for (int k = 0; k < 4; ++k)
+        *reinterpret_cast<float4 *>(ut + ubase[k] + ((blk ^ uperm[k]) << 4)) =
+            make_float4(uacc[k][0], uacc[k][1], uacc[k][2], uacc[k][3]);
+    }
+  }
+  if (own && last_tile && nb == 0 && p.conv_state_out != nullptr) {
+    // the last three inputs x_{T-3}, x_{T-2}, x_{T-1}: rows nvalid .. nvalid + 2
+    // (with T < 3 the first of them are conv_state_in rows or zeros: rows 0..2
+    // hold them in the tile, or conv_state_in when this is also tile 0)
+#pragma unroll
+    for (int r = 0; r < 3; ++r) {
+      const int row = nvalid + r;
+      uint2 v = *reinterpret_cast<const uint2 *>(xq + row * K * 2);
+      if (tile == 0 && row < 3 && p.conv_state_in != nullptr)
+        v = __ldg(reinterpret_cast<const uint2 *>(p.conv_state_in +
+                                                   (static_cast<size_t>(b) * 3 + row) * p.D + chq));
+      *reinterpret_cast<uint2 *>(p.conv_state_out + (static_cast<size_t>(b) * 3 + r) * p.D + chq) = v;
     }
   }
 }
