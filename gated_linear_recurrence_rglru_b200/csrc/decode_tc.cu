@@ -353,7 +353,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
     const int m = qd * 32 + lane;
     const uint32_t t_lane0 = tmem_base + (static_cast<uint32_t>(qd * 32) << 16);
     int cur_unit = -1;
-    ChanK kc{0.f, 0.f, 0.f, 0.f, 0.f};
+    ChanK kc{0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     bool fast = true;
     for (int i = eg;; i += NE) {
       const int js = i % kJQ;

@@ -323,42 +323,78 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
 
   if (warp == 0) {
     // =============================== producer ===============================
-    if (lane == 0) {
+    // The whole warp runs this loop (all decisions are warp-uniform): all
+    // lanes wait on the ring barriers, lane 0 takes the counter, all lanes
+    // scan the other units in parallel once the current unit is done, and
+    // lane 0 alone writes the job, arrives and issues the copies. A tile is
+    // claimed only once its x slot is free, so that tiles are claimed close
+    // to the time they are processed and a look-back rarely waits on a tile
+    // that sits claimed in another CTA's queue.
+    {
       int unit = blockIdx.x % p.n_units, w_unit = -1;
       int i = 0, last_x_job = -1;
       uint32_t wfree_phase = 0;
       for (;; ++i) {
+        const int js = i % kJQ, xb = i % NX;
+        RG_WAIT_OR_ABORT(&job_empty[js], ((i / kJQ) & 1) ^ 1);
+        RG_WAIT_OR_ABORT(&x_empty[xb], ((i / NX) & 1) ^ 1);
         int tile = -1;
         while (unit >= 0) {
-          const int t = atomicAdd(&p.counters[unit], 1);
+          int t = 0;
+          if (lane == 0) t = atomicAdd(&p.counters[unit], 1);
+          t = __shfl_sync(0xffffffffu, t, 0);
           if (t < p.n_tiles) {
             tile = t;
             break;
           }
-          // this unit is done: continue on the unit with the most tiles left
-          int best = -1, left = 0;
-          for (int u = 0; u < p.n_units; ++u) {
-            const int l = p.n_tiles - *(volatile const int *)(p.counters + u);
-            if (l > left) {
-              left = l;
-              best = u;
+          // this unit is done: continue on the unit with the most tiles left,
+          // ties broken by distance from a per-CTA starting point so that the
+          // CTAs that run out at the same time spread over the units (the
+          // counters are read from L2 without ordering: a stale value only
+          // makes a worse choice, the claim itself is the atomic)
+          const int rot = static_cast<int>((blockIdx.x * 37u) % static_cast<unsigned>(p.n_units));
+          unsigned key = 0;                       // (tiles left << 16) | (65535 - distance)
+          for (int u0 = 0; u0 < p.n_units; u0 += 128) {
+            int l[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int u = u0 + q * 32 + lane;
+              l[q] = u < p.n_units ? p.n_tiles - __ldcg(p.counters + u) : 0;
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int u = u0 + q * 32 + lane;
+              if (l[q] > 0) {
+                const int dist = u >= rot ? u - rot : u + p.n_units - rot;
+                const unsigned k = (static_cast<unsigned>(min(l[q], 32767)) << 16) |
+                                   static_cast<unsigned>(65535 - min(dist, 65535));
+                key = max(key, k);
+              }
             }
           }
-          unit = best;
+          key = __reduce_max_sync(0xffffffffu, key);
+          if (key == 0) {
+            unit = -1;
+          } else {
+            const int dist = 65535 - static_cast<int>(key & 0xFFFFu);
+            unit = rot + dist < p.n_units ? rot + dist : rot + dist - p.n_units;
+          }
         }
-        if (*cta_abort) unit = -1;
-        const int js = i % kJQ;
-        RG_WAIT_OR_ABORT(&job_empty[js], ((i / kJQ) & 1) ^ 1);
+        unit = __shfl_sync(0xffffffffu, *cta_abort ? -1 : unit, 0);
         const int reload = (unit >= 0 && unit != w_unit) ? 1 : 0;
-        jobs[js] = make_int4(unit, tile, reload, 0);
-        mbar_arrive(&job_full[js]);
+        if (lane == 0) {
+          jobs[js] = make_int4(unit, tile, reload, 0);
+          mbar_arrive(&job_full[js]);
+        }
         if (unit < 0) {
           // one terminal job per epilogue warpgroup that may still wait for a job
           for (int e = 1; e < NE; ++e) {
             const int je = i + e;
             if (!mbar_wait(&job_empty[je % kJQ], ((je / kJQ) & 1) ^ 1, cta_abort, p.wait_ns)) break;
-            jobs[je % kJQ] = make_int4(-1, -1, 0, 0);
-            mbar_arrive(&job_full[je % kJQ]);
+            if (lane == 0) {
+              jobs[je % kJQ] = make_int4(-1, -1, 0, 0);
+              mbar_arrive(&job_full[je % kJQ]);
+            }
           }
           break;
         }
@@ -370,33 +406,35 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
             RG_WAIT_OR_ABORT(w_free, wfree_phase);
             wfree_phase ^= 1;
           }
-          mbar_arrive_expect_tx(w_full, 2u * 2u * static_cast<uint32_t>(R) * 128u);
-          for (int g = 0; g < 2; ++g) {
-            const CUtensorMap *tm = g == 0 ? &tmap_wa : &tmap_wx;
-            unsigned char *dst = sA + g * C::kABytes;
-            if (p.bw == 64) {
-              for (int hh = 0; hh < 2; ++hh)
-                tma_load_2d(dst + hh * (K * 128) + hh * 64 * 128, tm, w_full, 0,
-                            (cg * 2 + hh) * 64);
-            } else if (p.bw == 128) {
-              for (int ma = 0; ma < 2; ++ma)
-                tma_load_2d(dst + ma * (K * 128), tm, w_full, 64 * ma, cg * 128);
-            } else {
-              for (int ma = 0; ma < 2; ++ma)
-                tma_load_2d(dst + ma * (K * 128), tm, w_full, (cg & 1) * 128 + 64 * ma,
-                            (cg >> 1) * 256);
+          if (lane == 0) {
+            mbar_arrive_expect_tx(w_full, 2u * 2u * static_cast<uint32_t>(R) * 128u);
+            for (int g = 0; g < 2; ++g) {
+              const CUtensorMap *tm = g == 0 ? &tmap_wa : &tmap_wx;
+              unsigned char *dst = sA + g * C::kABytes;
+              if (p.bw == 64) {
+                for (int hh = 0; hh < 2; ++hh)
+                  tma_load_2d(dst + hh * (K * 128) + hh * 64 * 128, tm, w_full, 0,
+                              (cg * 2 + hh) * 64);
+              } else if (p.bw == 128) {
+                for (int ma = 0; ma < 2; ++ma)
+                  tma_load_2d(dst + ma * (K * 128), tm, w_full, 64 * ma, cg * 128);
+              } else {
+                for (int ma = 0; ma < 2; ++ma)
+                  tma_load_2d(dst + ma * (K * 128), tm, w_full, (cg & 1) * 128 + 64 * ma,
+                              (cg >> 1) * 256);
+              }
             }
           }
           w_unit = unit;
         }
-        const int xb = i % NX;
-        RG_WAIT_OR_ABORT(&x_empty[xb], ((i / NX) & 1) ^ 1);
         const int kbase = p.bw <= 128 ? cg * kM : (cg >> 1) * 256;
-        mbar_arrive_expect_tx(&x_full[xb], static_cast<uint32_t>(C::kXRows * K * 2));
-        tma_load_3d(sX + xb * C::kXBytes, &tmap_x, &x_full[xb], kbase, tile * N - 3, b);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&x_full[xb], static_cast<uint32_t>(C::kXRows * K * 2));
+          tma_load_3d(sX + xb * C::kXBytes, &tmap_x, &x_full[xb], kbase, tile * N - 3, b);
+        }
         last_x_job = i;
       }
-      if (*cta_abort) {
+      if (lane == 0 && *cta_abort) {
         // drain: let every TMA this thread issued land before the CTA exits
         for (int j = last_x_job; j >= 0 && j > last_x_job - NX; --j)
           mbar_wait_drain(&x_full[j % NX], (j / NX) & 1, kDrainNs);
@@ -501,7 +539,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
     const int m = qd * 32 + lane;                 // TMEM lane == output channel in unit
     const uint32_t t_lane0 = tmem_base + (static_cast<uint32_t>(qd * 32) << 16);
     int cur_unit = -1;
-    ChanK kc{0.f, 0.f, 0.f, 0.f, 0.f};
+    ChanK kc{0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     float cwo[4] = {0.f, 0.f, 0.f, 0.f};          // own channel's conv taps (K = 256)
     bool fast = true;
     int d_i = -1, d_unit = 0, d_tile = 0;         // the deferred job
@@ -613,13 +651,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
       const uint32_t t_lane = t_lane0 + static_cast<uint32_t>(ts * C::kSlotCols);
       if (unit != cur_unit) {
         cur_unit = unit;
-        const float sp = softplus_f32(-p.Lambda[c]);
-        kc.kba = -__bfloat162float(p.b_a[c]) * kLog2e;
-        kc.hbx = 0.5f * __bfloat162float(p.b_x[c]);
-        kc.nc = -kDecayC * sp;
-        kc.nc2 = kc.nc * kLog2e;
-        kc.k2sp = 2.0f * sqrtf(sp);
-        fast = __all_sync(0xffffffffu, kDecayC * sp <= kFastLimit);
+        kc = chan_consts(__bfloat162float(p.b_a[c]), __bfloat162float(p.b_x[c]), p.Lambda[c]);
+        fast = __all_sync(0xffffffffu, chan_fast(kc));
         if (!C::kUTile) {
 #pragma unroll
           for (int tap = 0; tap < 4; ++tap) cwo[tap] = __bfloat162float(p.conv_w[tap * p.D + c]);
@@ -674,6 +707,14 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
             xm1 = xv;
           }
         }
+        if (ch == N / 16 - 1) {
+          // the last reads of the u (x) tile are issued: hand the slot back
+          __syncwarp();
+          if (lane == 0) {
+            if (C::kUTile) mbar_arrive(&u_empty[s]);
+            else mbar_arrive(&x_empty[xb]);
+          }
+        }
         tmem_wait_ld();
         if (fast) {
 #pragma unroll
@@ -713,7 +754,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
         tmem_wait_ld();
       }
       // publish this channel's word: inclusive for the first tile of a
-      // sequence (h0 is known), else the aggregate; release the u / x tile
+      // sequence (h0 is known), else the aggregate
       {
         const size_t wix = (static_cast<size_t>(unit) * p.n_tiles + tile) * kM + m;
         const bool silent = (unit == 0 && tile == p.fault_tile);
@@ -724,11 +765,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
           } else {
             st_relaxed_u64(p.carry + wix, carry_agg(A, Hl));
           }
-        }
-        __syncwarp();
-        if (lane == 0) {
-          if (C::kUTile) mbar_arrive(&u_empty[s]);
-          else mbar_arrive(&x_empty[xb]);
         }
       }
       // ---- carry and pass 2 of the previous job, then defer this one ----
@@ -862,6 +898,8 @@ cudaError_t launch_tc_t(const FwdArgs &a, const TcLayout &L, void *ws, cudaStrea
 bool tc_supported(int B, int T, int D, int H, int io) {
   if (io != RGLRU_IO_BF16) return false;
   if (D % kM != 0 || D % H != 0) return false;
+  // the unit index of a steal decision is carried in 16 bits
+  if (static_cast<long long>(B) * (D / kM) > 65535) return false;
   const int bw = D / H;
   return bw == 64 || bw == 128 || bw == 256;
 }
@@ -872,7 +910,7 @@ cudaError_t launch_fwd_tc(const FwdArgs &a, void *ws, cudaStream_t st) {
   const int bw = a.D / a.H;
   const TcLayout L = tc_layout(a.B, a.T, a.D, a.H);
   if (bw == 256) return launch_tc_t<256, 32, 3, 2>(a, L, ws, st);
-  return launch_tc_t<128, 64, 3, 2>(a, L, ws, st);
+  return launch_tc_t<128, 64, 2, 2>(a, L, ws, st);
 }
 
 }  // namespace rglru

@@ -14,9 +14,12 @@ namespace rglru {
 namespace gates {
 
 constexpr float kLog2e = 1.4426950408889634f;
-// sqrt((1 - e^(2w)) / (-2w)) ~= 1 + w (G1 + w (G2 + w G3)) on w in [-1/8, 0]
-// (least-squares/minimax fit made for these kernels; max rel. error 7e-8 in fp32).
-constexpr float kG1 = 0.49999531f, kG2 = 0.20810417f, kG3 = 0.05930331f;
+// Polynomials on w in [-1/8, 0], least-squares fits in relative error made for
+// these kernels (constant terms pinned to 1):
+//   e^w                         ~= 1 + w (E1 + w (E2 + w (E3 + w E4)))   max rel. error 1.3e-9
+//   sqrt((1 - e^(2w)) / (-2w))  ~= 1 + w (G1 + w G2)                    max rel. error 8.0e-6
+constexpr float kE1 = 0.99999986f, kE2 = 0.49998943f, kE3 = 0.16641409f, kE4 = 0.03923329f;
+constexpr float kG1 = 0.49961998f, kG2 = 0.19817025f;
 constexpr float kFastLimit = 0.125f;          // fast path when c * softplus(-Lambda) <= 1/8
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -81,15 +84,18 @@ struct ChanK {
   float kba;    // -(b_a) log2 e
   float hbx;    // b_x / 2
   float nc;     // -c softplus(-Lambda): ln a_t = nc * r_t
-  float k2sp;   // 2 sqrt(softplus(-Lambda))
+  float s0;     // 2 sqrt(softplus(-Lambda)); s1 = s0 G1, s2 = s0 G2
+  float s1;
+  float s2;
   float nc2;    // nc log2 e (general path)
 };
 
 // Fast path, two tokens of one channel, valid when |nc| <= 1/8:
 //   e = 2^(-(za + ba) log2 e), sqrt_r = (1 + e)^(-1/2), r = sqrt_r^2,
-//   ln a = nc r, a = e^(ln a) (Taylor, degree 5),
+//   ln a = nc r, a = e^(ln a) (polynomial above),
 //   sqrt(1 - a^2) = sqrt(-2 ln a) sqrt(g(ln a)) = 4 sqrt(sp) sqrt_r sqrt(g),
-//   i = (1 + tanh((zx + bx) / 2)) / 2,  beta = sqrt(1 - a^2) i u.
+//   2 i = 1 + tanh((zx + bx) / 2),
+//   beta = sqrt(1 - a^2) i u = sqrt_r * (2 sqrt(sp) sqrt(g)) * (u (1 + tanh)).
 __device__ __forceinline__ void gate_pair_fast(float2 za, float2 zx, float2 u, const ChanK &k,
                                                float2 &a, float2 &beta, float2 &la) {
   const float2 earg = __ffma2_rn(za, f2(-kLog2e), f2(k.kba));
@@ -97,18 +103,16 @@ __device__ __forceinline__ void gate_pair_fast(float2 za, float2 zx, float2 u, c
   d = __fadd2_rn(d, f2(1.0f));
   const float2 q = make_float2(rsqrt_approx(d.x), rsqrt_approx(d.y));
   la = __fmul2_rn(__fmul2_rn(q, q), f2(k.nc));
-  float2 pa = __ffma2_rn(la, f2(1.0f / 120.0f), f2(1.0f / 24.0f));
-  pa = __ffma2_rn(la, pa, f2(1.0f / 6.0f));
-  pa = __ffma2_rn(la, pa, f2(0.5f));
-  pa = __ffma2_rn(la, pa, f2(1.0f));
+  float2 pa = __ffma2_rn(la, f2(kE4), f2(kE3));
+  pa = __ffma2_rn(la, pa, f2(kE2));
+  pa = __ffma2_rn(la, pa, f2(kE1));
   a = __ffma2_rn(la, pa, f2(1.0f));
-  float2 sg = __ffma2_rn(la, f2(kG3), f2(kG2));
-  sg = __ffma2_rn(la, sg, f2(kG1));
-  sg = __ffma2_rn(la, sg, f2(1.0f));
+  float2 sg = __ffma2_rn(la, f2(k.s2), f2(k.s1));
+  sg = __ffma2_rn(la, sg, f2(k.s0));                          // 2 sqrt(sp) sqrt(g)
   const float2 targ = __ffma2_rn(zx, f2(0.5f), f2(k.hbx));
   const float2 t = make_float2(tanh_approx(targ.x), tanh_approx(targ.y));
-  const float2 ig = __ffma2_rn(t, f2(k.k2sp), f2(k.k2sp));   // 4 sqrt(sp) i
-  beta = __fmul2_rn(__fmul2_rn(__fmul2_rn(q, sg), ig), u);
+  const float2 tu = __ffma2_rn(t, u, u);                      // 2 i u
+  beta = __fmul2_rn(__fmul2_rn(q, sg), tu);
 }
 
 // General path, one element: as above but a = 2^(log2 a) on the MUFU and
@@ -141,7 +145,9 @@ __device__ __forceinline__ ChanK chan_consts(float b_a, float b_x, float Lambda)
   k.hbx = 0.5f * b_x;
   k.nc = -kDecayC * sp;
   k.nc2 = k.nc * kLog2e;
-  k.k2sp = 2.0f * sqrtf(sp);
+  k.s0 = 2.0f * sqrtf(sp);
+  k.s1 = k.s0 * kG1;
+  k.s2 = k.s0 * kG2;
   return k;
 }
 
