@@ -68,10 +68,11 @@ struct TcParams {
   int fault_tile;                  // testing: tile of unit 0 that never publishes (-1: off)
 };
 
-template <int K, int N, int NX, int NE>
+template <int K, int N, int NX, int NE, int NU>
 struct Cfg {
-  // warps: 0 producer, 1 MMA, 2-5 conv, then NE epilogue warpgroups
-  static constexpr int kThreads = 64 + 128 + NE * 128;
+  // warps: 0 producer, 1 MMA, 2-5 conv, then NE epilogue warpgroups; the
+  // block is padded to whole warpgroups (registers are granted per warpgroup)
+  static constexpr int kThreads = (64 + 128 + NE * 128 + 127) / 128 * 128;
   static constexpr int kXRows = N + 3;
   static constexpr int kXBytes = ((kXRows * K * 2) + 1023) / 1024 * 1024;
   static constexpr int kABytes = K * 256;          // one gate: 2 M-blocks x K rows x 128 B
@@ -80,19 +81,26 @@ struct Cfg {
   // only; with K = 256 the epilogue recomputes u from the x tile instead)
   static constexpr bool kUTile = (K == 128);
   static constexpr int kUBytes = kUTile ? N * kM * 4 : 0;
-  static constexpr int kNS = 2;                    // conv -> MMA / epilogue slots
-  static constexpr int kNT = 2 * NE;               // TMEM slots
+  static constexpr int kNS = 2;                    // conv -> MMA slots (B operand)
+  // conv -> epilogue slots (u tile); with three, the conv of job i waits for
+  // pass 1 of job i - 3 rather than of job i - 2 (which ran in the same
+  // epilogue warpgroup as job i and would chain conv, MMA and pass 1 serially)
+  static constexpr int kNU = kUTile ? NU : 1;
+  // TMEM slots: one per epilogue warpgroup and one for the MMA to run ahead
+  static constexpr int kNT = NE + 1;
   static constexpr int kOffA = 0;
   static constexpr int kOffX = 2 * kABytes;
   static constexpr int kOffB = kOffX + NX * kXBytes;
   static constexpr int kOffU = kOffB + kNS * kBBytes;
-  static constexpr int kOffBar = kOffU + kNS * kUBytes;
+  static constexpr int kOffBar = kOffU + kNU * kUBytes;
   // job_full[JQ], job_empty[JQ], x_full[NX], x_empty[NX], w_full, w_free,
-  // b_full[NS], b_empty[NS], u_empty[NS], acc_full[NT], tmem_empty[NT]
-  static constexpr int kNumBars = 2 * kJQ + 2 * NX + 2 + 3 * kNS + 2 * kNT;
+  // b_full[NS], b_empty[NS], u_empty[NU], acc_full[NT], tmem_empty[NT]
+  static constexpr int kNumBars = 2 * kJQ + 2 * NX + 2 + 2 * kNS + kNU + 2 * kNT;
   static constexpr int kOffJobs = (kOffBar + kNumBars * 8 + 15) / 16 * 16;
   static constexpr int kOffMisc = kOffJobs + kJQ * 16;
-  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;   // + alignment slack
+  // the dynamic shared memory base is declared 1024-byte aligned (the kernel
+  // checks it), as the 128-byte swizzle of the TMA and MMA tiles needs
+  static constexpr int kSmemBytes = kOffMisc + 64;
   static constexpr int kSlotCols = 2 * N;                   // z_a | z_x, then a | beta
   static constexpr int kTmemCols =
       kNT * kSlotCols <= 128 ? 128 : (kNT * kSlotCols <= 256 ? 256 : 512);
@@ -240,15 +248,19 @@ __device__ __forceinline__ void conv_tile(const unsigned char *__restrict__ xs,
   }
 }
 
-template <int K, int N, int NX, int NE>
-__global__ void __launch_bounds__(Cfg<K, N, NX, NE>::kThreads, 1)
+template <int K, int N, int NX, int NE, int NU>
+__global__ void __launch_bounds__(Cfg<K, N, NX, NE, NU>::kThreads, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_wa,
               const __grid_constant__ CUtensorMap tmap_wx, const TcParams p) {
-  using C = Cfg<K, N, NX, NE>;
-  constexpr int NS = C::kNS, NT = C::kNT;
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char *sm = reinterpret_cast<unsigned char *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  using C = Cfg<K, N, NX, NE, NU>;
+  constexpr int NS = C::kNS, NT = C::kNT, NUS = C::kNU;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  if ((smem_u32(smem_raw) & 1023u) != 0u) {
+    // the layout relies on the declared alignment; refuse to run without it
+    if (threadIdx.x == 0 && p.dev_status) atomicCAS(p.dev_status, 0, RGLRU_ERR_UNSUPPORTED);
+    return;
+  }
+  unsigned char *sm = smem_raw;
   unsigned char *sA = sm + C::kOffA;
   unsigned char *sX = sm + C::kOffX;
   unsigned char *sB = sm + C::kOffB;
@@ -262,8 +274,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
   uint64_t *w_free = w_full + 1;                    // MMAs reading the old weights are done
   uint64_t *b_full = w_free + 1;                    // [NS] conv -> MMA
   uint64_t *b_empty = b_full + NS;                  // [NS] MMA -> conv
-  uint64_t *u_empty = b_empty + NS;                 // [NS] epilogue pass 1 -> conv
-  uint64_t *acc_full = u_empty + NS;                // [NT] MMA -> epilogue
+  uint64_t *u_empty = b_empty + NS;                 // [NU] epilogue pass 1 -> conv
+  uint64_t *acc_full = u_empty + NUS;               // [NT] MMA -> epilogue
   uint64_t *tmem_empty = acc_full + NT;             // [NT] epilogue pass 2 -> MMA
   int4 *jobs = reinterpret_cast<int4 *>(sm + C::kOffJobs);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + C::kOffMisc);
@@ -288,8 +300,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
     for (int i = 0; i < NS; ++i) {
       mbar_init(&b_full[i], 4);                     // 4 conv warps
       mbar_init(&b_empty[i], 1);
-      mbar_init(&u_empty[i], 4);                    // 4 epilogue warps
     }
+    for (int i = 0; i < NUS; ++i) mbar_init(&u_empty[i], 4);   // 4 epilogue warps
     for (int i = 0; i < NT; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&tmem_empty[i], 4);                 // 4 epilogue warps
@@ -510,11 +522,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
           cwq[tap][1] = bf2_to_f2(raw.y);
         }
       }
-      const int s = i % NS, xb = i % NX;
+      const int s = i % NS, xb = i % NX, us = i % NUS;
       RG_WAIT_OR_ABORT(&x_full[xb], (i / NX) & 1);
       RG_WAIT_OR_ABORT(&b_empty[s], ((i / NS) & 1) ^ 1);
-      if (C::kUTile) RG_WAIT_OR_ABORT(&u_empty[s], ((i / NS) & 1) ^ 1);
-      conv_tile<K, N, C::kUTile>(sX + xb * C::kXBytes, sB + s * C::kBBytes, sU + s * C::kUBytes,
+      if (C::kUTile) RG_WAIT_OR_ABORT(&u_empty[us], ((i / NUS) & 1) ^ 1);
+      conv_tile<K, N, C::kUTile>(sX + xb * C::kXBytes, sB + s * C::kBBytes, sU + us * C::kUBytes,
                                  p, b, kbase, own_lo, tile, nvalid, tile == p.n_tiles - 1, wt,
                                  cwq);
       // each warp hands its part over on its own: no barrier that an aborting
@@ -527,13 +539,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
         mbar_arrive(&job_empty[js]);
       }
     }
-  } else {
+  } else if (warp < 6 + 4 * NE) {
     // ========================== epilogue warpgroups ==========================
     // Epilogue warpgroup e takes jobs e, e + NE, ...; each of its 4 warps owns
     // one TMEM quadrant (32 channels, one per lane) and works on its own: per
-    // job, pass 1 and the publication of each channel's aggregate; then the
-    // carry (look-back over its channels' words) and pass 2 of the warp's
-    // previous job, whose predecessors have usually published by then.
+    // job, pass 1, the publication of each channel's aggregate, the carry
+    // (look-back over its channels' words) and pass 2. Three warpgroups keep
+    // three jobs in flight while the MMA fills the fourth TMEM slot.
     const int eg = (warp - 6) >> 2;               // 0 .. NE-1
     const int qd = warp & 3;                      // TMEM quadrant
     const int m = qd * 32 + lane;                 // TMEM lane == output channel in unit
@@ -542,100 +554,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
     ChanK kc{0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     float cwo[4] = {0.f, 0.f, 0.f, 0.f};          // own channel's conv taps (K = 256)
     bool fast = true;
-    int d_i = -1, d_unit = 0, d_tile = 0;         // the deferred job
-    float d_A = 0.f, d_H = 0.f;
-
-    // ---- carry and pass 2 of the deferred job ----
-    auto phase_b = [&]() {
-      const int unit = d_unit, tile = d_tile;
-      const int b = unit / p.n_cg, cg = unit % p.n_cg;
-      const int c = cg * kM + m;
-      const int n0 = tile * N;
-      const int nvalid = min(N, p.T - n0);
-      const bool last_tile = (tile == p.n_tiles - 1);
-      const int ts = d_i % NT;
-      const uint32_t t_lane = t_lane0 + static_cast<uint32_t>(ts * C::kSlotCols);
-      unsigned long long *cw = p.carry + static_cast<size_t>(unit) * p.n_tiles * kM + m;
-      float h_in = 0.f;
-      if (tile == 0) {
-        if (p.h0 != nullptr) h_in = p.h0[static_cast<size_t>(b) * p.D + c];
-      } else {
-        // Look back along this lane's channel, four words per round trip: fold
-        // aggregates until an inclusive word; an unpublished word ends the
-        // round and is read again in the next.
-        float mult = 1.f, add = 0.f;
-        int k = tile - 1;                         // next tile to read
-        bool done = false;
-        const uint64_t t0 = globaltimer_ns();
-        for (;;) {
-          if (!done) {
-            unsigned long long w[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              w[q] = (k - q >= 0) ? ld_relaxed_u64(cw + static_cast<size_t>(k - q) * kM) : 0ull;
-            bool stop = false;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              if (stop) continue;
-              const uint32_t lo = static_cast<uint32_t>(w[q]);
-              const float hi = __uint_as_float(static_cast<uint32_t>(w[q] >> 32));
-              if (lo == 0u) {
-                stop = true;                      // not yet published: read tile k again
-              } else if (lo & 0x80000000u) {
-                add = fmaf(mult, hi, add);        // aggregate
-                mult *= __uint_as_float(lo & 0x7FFFFFFFu);
-                --k;
-              } else {
-                h_in = fmaf(mult, hi, add);       // inclusive
-                done = true;
-                stop = true;
-              }
-            }
-          }
-          if (__all_sync(0xffffffffu, done)) break;
-          const bool give_up = *cta_abort || *(volatile const int *)p.abort_flag ||
-                               (globaltimer_ns() - t0 > p.wait_ns);
-          if (__any_sync(0xffffffffu, give_up)) {
-            if (lane == 0 && !*cta_abort) raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);
-            *cta_abort = 1;
-            h_in = 0.f;
-            break;
-          }
-          __nanosleep(64);
-        }
-        if (!(unit == 0 && tile == p.fault_tile))
-          st_relaxed_u64(cw + static_cast<size_t>(tile) * kM, carry_inc(fmaf(d_A, h_in, d_H)));
-      }
-      // ---- pass 2: y_t = P_t h_in + Hl_t ----
-      __nv_bfloat16 *yrow = p.y + (static_cast<size_t>(b) * p.T + n0) * p.D + c;
-#pragma unroll 1
-      for (int ch = 0; ch < N / 16; ++ch) {
-        if (ch * 16 >= nvalid) break;
-        float pv[16], hv[16];
-        tmem_ld16(t_lane + ch * 16, pv);
-        tmem_ld16(t_lane + N + ch * 16, hv);
-        tmem_wait_ld();
-        __nv_bfloat16 *yc = yrow + static_cast<size_t>(ch * 16) * p.D;
-        if (ch * 16 + 16 <= nvalid) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            yc[static_cast<size_t>(j) * p.D] = __float2bfloat16_rn(fmaf(pv[j], h_in, hv[j]));
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (ch * 16 + j < nvalid)
-              yc[static_cast<size_t>(j) * p.D] = __float2bfloat16_rn(fmaf(pv[j], h_in, hv[j]));
-        }
-      }
-      if (last_tile && p.h_T != nullptr) p.h_T[static_cast<size_t>(b) * p.D + c] = fmaf(d_A, h_in, d_H);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&tmem_empty[ts]);
-        mbar_arrive(&job_empty[d_i % kJQ]);
-      }
-      d_i = -1;
-    };
 
     for (int i = eg;; i += NE) {
       const int js = i % kJQ;
@@ -647,7 +565,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
       const int c = cg * kM + m;                  // own output channel
       const int own_lo = p.bw <= 128 ? 0 : (cg & 1) * kM;
       const int nvalid = min(N, p.T - tile * N);
-      const int s = i % NS, ts = i % NT, xb = i % NX;
+      const int us = i % NUS, ts = i % NT, xb = i % NX;
       const uint32_t t_lane = t_lane0 + static_cast<uint32_t>(ts * C::kSlotCols);
       if (unit != cur_unit) {
         cur_unit = unit;
@@ -662,7 +580,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
       tc_fence_after();
       // own channel's u: fp32 tile from the conv warpgroup (K = 128), or
       // recomputed from the x tile (K = 256)
-      const unsigned char *uslot = sU + s * C::kUBytes;
+      const unsigned char *uslot = sU + us * C::kUBytes;
       const __nv_bfloat16 *xown =
           reinterpret_cast<const __nv_bfloat16 *>(sX + xb * C::kXBytes) + own_lo + m;
       float xm3 = 0.f, xm2 = 0.f, xm1 = 0.f;
@@ -711,7 +629,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
           // the last reads of the u (x) tile are issued: hand the slot back
           __syncwarp();
           if (lane == 0) {
-            if (C::kUTile) mbar_arrive(&u_empty[s]);
+            if (C::kUTile) mbar_arrive(&u_empty[us]);
             else mbar_arrive(&x_empty[xb]);
           }
         }
@@ -767,15 +685,88 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
           }
         }
       }
-      // ---- carry and pass 2 of the previous job, then defer this one ----
-      if (d_i >= 0) phase_b();
-      d_i = i;
-      d_unit = unit;
-      d_tile = tile;
-      d_A = A;
-      d_H = Hl;
+      // ---- carry: the state entering this tile ----
+      unsigned long long *cw = p.carry + static_cast<size_t>(unit) * p.n_tiles * kM + m;
+      float h_in = 0.f;
+      if (tile == 0) {
+        if (p.h0 != nullptr) h_in = p.h0[static_cast<size_t>(b) * p.D + c];
+      } else {
+        // Look back along this lane's channel, four words per round trip: fold
+        // aggregates until an inclusive word; an unpublished word ends the
+        // round and is read again in the next.
+        float mult = 1.f, add = 0.f;
+        int k = tile - 1;                         // next tile to read
+        bool done = false;
+        const uint64_t t0 = globaltimer_ns();
+        for (;;) {
+          if (!done) {
+            unsigned long long w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              w[q] = (k - q >= 0) ? ld_relaxed_u64(cw + static_cast<size_t>(k - q) * kM) : 0ull;
+            bool stop = false;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (stop) continue;
+              const uint32_t lo = static_cast<uint32_t>(w[q]);
+              const float hi = __uint_as_float(static_cast<uint32_t>(w[q] >> 32));
+              if (lo == 0u) {
+                stop = true;                      // not yet published: read tile k again
+              } else if (lo & 0x80000000u) {
+                add = fmaf(mult, hi, add);        // aggregate
+                mult *= __uint_as_float(lo & 0x7FFFFFFFu);
+                --k;
+              } else {
+                h_in = fmaf(mult, hi, add);       // inclusive
+                done = true;
+                stop = true;
+              }
+            }
+          }
+          if (__all_sync(0xffffffffu, done)) break;
+          const bool give_up = *cta_abort || *(volatile const int *)p.abort_flag ||
+                               (globaltimer_ns() - t0 > p.wait_ns);
+          if (__any_sync(0xffffffffu, give_up)) {
+            if (lane == 0 && !*cta_abort) raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);
+            *cta_abort = 1;
+            h_in = 0.f;
+            break;
+          }
+          __nanosleep(64);
+        }
+        if (!(unit == 0 && tile == p.fault_tile))
+          st_relaxed_u64(cw + static_cast<size_t>(tile) * kM, carry_inc(fmaf(A, h_in, Hl)));
+      }
+      // ---- pass 2: y_t = P_t h_in + Hl_t ----
+      __nv_bfloat16 *yrow = p.y + (static_cast<size_t>(b) * p.T + tile * N) * p.D + c;
+#pragma unroll 1
+      for (int ch = 0; ch < N / 16; ++ch) {
+        if (ch * 16 >= nvalid) break;
+        float pv[16], hv[16];
+        tmem_ld16(t_lane + ch * 16, pv);
+        tmem_ld16(t_lane + N + ch * 16, hv);
+        tmem_wait_ld();
+        __nv_bfloat16 *yc = yrow + static_cast<size_t>(ch * 16) * p.D;
+        if (ch * 16 + 16 <= nvalid) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            yc[static_cast<size_t>(j) * p.D] = __float2bfloat16_rn(fmaf(pv[j], h_in, hv[j]));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (ch * 16 + j < nvalid)
+              yc[static_cast<size_t>(j) * p.D] = __float2bfloat16_rn(fmaf(pv[j], h_in, hv[j]));
+        }
+      }
+      if (tile == p.n_tiles - 1 && p.h_T != nullptr)
+        p.h_T[static_cast<size_t>(b) * p.D + c] = fmaf(A, h_in, Hl);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&tmem_empty[ts]);
+        mbar_arrive(&job_empty[js]);
+      }
     }
-    if (d_i >= 0 && !*cta_abort) phase_b();
   }
 #undef RG_WAIT_OR_ABORT
 
@@ -822,9 +813,9 @@ TcLayout tc_layout(int B, int T, int D, int H) {
   return L;
 }
 
-template <int K, int N, int NX, int NE>
+template <int K, int N, int NX, int NE, int NU>
 cudaError_t launch_tc_t(const FwdArgs &a, const TcLayout &L, void *ws, cudaStream_t st) {
-  using C = Cfg<K, N, NX, NE>;
+  using C = Cfg<K, N, NX, NE, NU>;
   auto enc = encode_fn();
   if (enc == nullptr) return cudaErrorNotSupported;
   const int bw = a.D / a.H;
@@ -881,7 +872,7 @@ cudaError_t launch_tc_t(const FwdArgs &a, const TcLayout &L, void *ws, cudaStrea
 
   cudaError_t e = cudaMemsetAsync(ws, 0, L.total, st);
   if (e != cudaSuccess) return e;
-  auto kern = fwd_tc_kernel<K, N, NX, NE>;
+  auto kern = fwd_tc_kernel<K, N, NX, NE, NU>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
@@ -909,8 +900,8 @@ size_t tc_workspace_bytes(int B, int T, int D, int H) { return tc_layout(B, T, D
 cudaError_t launch_fwd_tc(const FwdArgs &a, void *ws, cudaStream_t st) {
   const int bw = a.D / a.H;
   const TcLayout L = tc_layout(a.B, a.T, a.D, a.H);
-  if (bw == 256) return launch_tc_t<256, 32, 3, 2>(a, L, ws, st);
-  return launch_tc_t<128, 64, 2, 2>(a, L, ws, st);
+  if (bw == 256) return launch_tc_t<256, 32, 3, 3, 1>(a, L, ws, st);
+  return launch_tc_t<128, 64, 2, 3, 3>(a, L, ws, st);
 }
 
 }  // namespace rglru
