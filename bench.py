@@ -127,6 +127,39 @@ def weak_scaling_value(units_per_rank: int, steps: int, ms_max: float, ws: int) 
     return ws * units_per_rank * steps / (ms_max / 1e3)
 
 
+# DRAM traffic of the forward kernel per launch, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), stored with a hash of the
+# kernel sources it was taken on: a number taken on other sources is not reported
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+KERNEL_SOURCES = ["fwd_tc.cu", "tc_gates.cuh", "tc_primitives.cuh", "common.cuh"]
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for fn in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "gated_linear_recurrence_rglru_b200", "csrc", fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def kernel_traffic(wl, algo):
+    """(kernel name, DRAM bytes per launch or None) of the workload's forward kernel."""
+    import gated_linear_recurrence_rglru_b200 as rg
+    if not (algo in ("auto", "tensor") and rg.fwd_launches(wl.B, wl.T, wl.D, wl.H, wl.dtype, "tensor") > 0):
+        return "generic kernels (segment pass, carry, final pass)", None
+    name = "fwd_tc_kernel"
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return name, None
+    ent = rec.get("workloads", {}).get(wl.name)
+    if ent is None or rec.get("source_hash") != kernel_source_hash():
+        return name, None
+    return name, ent["dram_bytes_per_launch"]
+
+
 def fwd_bytes_per_chtok(wl) -> int:
     """Algorithmic HBM bytes per channel-token of the fused forward: read x, write y."""
     return 2 * (4 if wl.io == "f32" else 2)
@@ -155,11 +188,22 @@ def run_ours(a, ws, rank, local):
     work = [torch.empty(max(wsb, 1), device=dev, dtype=torch.uint8) for _ in range(nsets)]
     status = torch.zeros(1, device=dev, dtype=torch.int32)
     stream = torch.cuda.current_stream()
+    # per timed step, a pair of events that the library records right around its
+    # compute kernel(s) on this stream (after the workspace reset): the kernel's
+    # own launch duration for the roofline
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(a.steps)]
+    for eb, ee in kev:
+        eb.record(stream)
+        ee.record(stream)
+    torch.cuda.synchronize()
+    kopts = [rg.FwdOptions(kernel_begin_event=eb.cuda_event, kernel_end_event=ee.cuda_event)
+             for eb, ee in kev]
 
-    def step(i):
+    def step(i, opts=None):
         k = i % nsets
         rg.rglru_fwd(xs[k], *w, h0=g["h0"], y=ys[k], h_T=hT[k], conv_state_out=cs[k],
-                     workspace=work[k], dev_status=status, algo=a.algo)
+                     workspace=work[k], dev_status=status, algo=a.algo, options=opts)
 
     # soak (untimed) so that the clock sampler sees this load around the timed region
     sampler = ClockSampler(local)
@@ -178,13 +222,14 @@ def run_ours(a, ws, rank, local):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(a.steps):
-        step(i)
+    for j in range(a.steps):
+        step(i, kopts[j])
         i += 1
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(ws)
     ms_local = e0.elapsed_time(e1)
+    kernel_ms = sum(eb.elapsed_time(ee) for eb, ee in kev) / a.steps
     post_t0 = time.time()
     while time.time() - post_t0 < a.soak_s:
         for _ in range(50):
@@ -200,8 +245,10 @@ def run_ours(a, ws, rank, local):
     value = weak_scaling_value(chtok, a.steps, ms, ws)
     pk = peaks()
     bytes_step = fwd_bytes_per_chtok(wl) * chtok
-    achieved = bytes_step / (ms_step / 1e3) / 1e9
+    achieved_step = bytes_step / (ms_step / 1e3) / 1e9
+    achieved = bytes_step / (kernel_ms / 1e3) / 1e9
     launches_per_step = rg.fwd_launches(B, T, D, H, wl.dtype, a.algo)
+    kname, traffic = kernel_traffic(wl, a.algo)
 
     out = {
         "metric": METRIC, "value": value, "unit": "channel-tokens/s", "n_gpus": ws,
@@ -213,10 +260,13 @@ def run_ours(a, ws, rank, local):
                    "parallelism": f"dp{ws} (independent batches)",
                    "l2": f"{nsets} rotating buffer sets of {set_bytes / 1e6:.1f} MB "
                          f"(>3x L2 between reuses)"},
-        "hbm_gbs": achieved,
+        "hbm_gbs": achieved_step,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
-                     "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
-                     "kernel": "whole step (all launches of one rglru_fwd)",
+                     "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
+                     "kernel": kname, "kernel_ms": kernel_ms,
+                     "timing": "CUDA events recorded by the library around the kernel, "
+                               "every timed step, on the launching stream",
+                     "step_achieved": achieved_step,
                      "peak_source": pk["source"],
                      "algorithmic_bytes_per_launch": bytes_step},
         "gpu_launches": launches_per_step * a.steps,

@@ -7,8 +7,9 @@ diagonal recurrence h_t = a_t h_{t-1} + sqrt(1 - a_t^2) (i_t u_t), computed by
 hand-written CUDA kernels behind a C ABI (include/rglru.h). This package is the
 thin Python binding of that library; see _abi.py.
 """
-from ._abi import (ALGO_AUTO, ALGO_GENERIC, ALGO_TENSOR, LIB_PATH, RGLRUError,  # noqa: F401
-                   decode_launches, fwd_launches, fwd_workspace_bytes, rglru_decode_step, rglru_fwd, status_str, version)
+from ._abi import (ALGO_AUTO, ALGO_GENERIC, ALGO_TENSOR, LIB_PATH, FwdOptions,  # noqa: F401
+                   RGLRUError, decode_launches, fwd_launches, fwd_workspace_bytes, rglru_decode_step,
+                   rglru_fwd, rglru_fwd_noalloc, status_str, version)
 
-__all__ = ["rglru_fwd", "rglru_decode_step", "fwd_workspace_bytes", "fwd_launches", "decode_launches", "RGLRUError",
-           "status_str", "version", "LIB_PATH"]
+__all__ = ["rglru_fwd", "rglru_fwd_noalloc", "rglru_decode_step", "fwd_workspace_bytes", "fwd_launches",
+           "decode_launches", "FwdOptions", "RGLRUError", "status_str", "version", "LIB_PATH"]

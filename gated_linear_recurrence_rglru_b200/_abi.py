@@ -29,7 +29,8 @@ EXPORTED = (
 
 class FwdOptions(ctypes.Structure):
     """rglru_fwd_options of include/rglru.h."""
-    _fields_ = [("wait_limit_ns", ctypes.c_ulonglong), ("fault_unpublished_tile", ctypes.c_int)]
+    _fields_ = [("wait_limit_ns", ctypes.c_ulonglong), ("fault_unpublished_tile", ctypes.c_int),
+                ("kernel_begin_event", ctypes.c_void_p), ("kernel_end_event", ctypes.c_void_p)]
 NOALLOC_SCRATCH_BYTES = 2 << 20  # RGLRU_NOALLOC_SCRATCH_BYTES in include/rglru.h
 
 

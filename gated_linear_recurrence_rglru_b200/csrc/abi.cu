@@ -115,9 +115,12 @@ int rglru_fwd_ex(const void *x, const void *conv_w, const void *W_a, const void 
 
   if (opts != nullptr && opts->wait_limit_ns > 0 && opts->wait_limit_ns < 1000000ull)
     return RGLRU_ERR_INVALID_ARG;                // below 1 ms a healthy wait could expire
+  if (opts != nullptr && opts->fault_unpublished_tile < 0) return RGLRU_ERR_INVALID_ARG;
   FwdArgs p{x, conv_w, W_a, b_a, W_x, b_x, Lambda, h0, conv_state_in, y, h_T, conv_state_out,
             B, T, D, H, dev_status,
-            opts ? opts->wait_limit_ns : 0ull, opts ? opts->fault_unpublished_tile : -1};
+            opts ? opts->wait_limit_ns : 0ull, opts ? opts->fault_unpublished_tile - 1 : -1,
+            opts ? static_cast<cudaEvent_t>(opts->kernel_begin_event) : nullptr,
+            opts ? static_cast<cudaEvent_t>(opts->kernel_end_event) : nullptr};
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = use_tc ? launch_fwd_tc(p, workspace, s) : launch_fwd_generic(p, io, workspace, s);
   return e == cudaSuccess ? RGLRU_OK : RGLRU_ERR_CUDA;

@@ -880,8 +880,11 @@ cudaError_t launch_tc_t(const FwdArgs &a, const TcLayout &L, void *ws, cudaStrea
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long jobs = static_cast<long>(L.n_units) * L.n_tiles;
   const int grid = static_cast<int>(jobs < sms ? jobs : sms);
+  if (a.ev_begin != nullptr && (e = cudaEventRecord(a.ev_begin, st)) != cudaSuccess) return e;
   kern<<<grid, C::kThreads, C::kSmemBytes, st>>>(tx, twa, twx, p);
-  return cudaGetLastError();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (a.ev_end != nullptr) return cudaEventRecord(a.ev_end, st);
+  return cudaSuccess;
 }
 
 }  // namespace

@@ -294,8 +294,13 @@ static cudaError_t launch_fwd_generic_t(const FwdArgs &p, void *ws, cudaStream_t
 }
 
 cudaError_t launch_fwd_generic(const FwdArgs &p, int io, void *ws, cudaStream_t st) {
-  if (io == RGLRU_IO_F32) return launch_fwd_generic_t<float>(p, ws, st);
-  return launch_fwd_generic_t<__nv_bfloat16>(p, ws, st);
+  cudaError_t e;
+  if (p.ev_begin != nullptr && (e = cudaEventRecord(p.ev_begin, st)) != cudaSuccess) return e;
+  e = io == RGLRU_IO_F32 ? launch_fwd_generic_t<float>(p, ws, st)
+                         : launch_fwd_generic_t<__nv_bfloat16>(p, ws, st);
+  if (e != cudaSuccess) return e;
+  if (p.ev_end != nullptr) return cudaEventRecord(p.ev_end, st);
+  return cudaSuccess;
 }
 
 int generic_kernel_launches(int B, int T, int H) {

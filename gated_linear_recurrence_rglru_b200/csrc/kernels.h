@@ -17,6 +17,7 @@ struct FwdArgs {
   int *dev_status;
   unsigned long long wait_ns;  // 0: default bound of device-side waits
   int fault_tile;              // testing only: tile of unit 0 that never publishes (-1: off)
+  cudaEvent_t ev_begin, ev_end;  // recorded around the compute kernels when set
 };
 
 struct DecArgs {

@@ -53,21 +53,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may stay suspended in the instruction for
+// up to `suspend_ns` while the phase is incomplete (it resumes as soon as the
+// phase completes), so that waiting warps do not take issue slots.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t *bar, uint32_t parity,
+                                                      uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase of `parity` to complete. Gives up after `limit_ns` or
-// as soon as *abort becomes nonzero; returns false then (the caller stops).
-// The result is the same for every active lane of the warp, so that a warp
-// never splits into lanes that go on and lanes that stop.
+// as soon as *abort becomes nonzero (both checked at least every 20 us);
+// returns false then (the caller stops). The result is the same for every
+// active lane of the warp, so that a warp never splits into lanes that go on
+// and lanes that stop.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
                                           volatile int *abort, uint64_t limit_ns) {
   bool ok = mbar_try_wait(bar, parity);
   if (!ok) {
     const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-      if (mbar_try_wait(bar, parity)) {
+    for (;;) {
+      if (mbar_try_wait_suspend(bar, parity, 20000u)) {
         ok = true;
         break;
       }
-      if ((it & 63u) == 0 && (*abort || globaltimer_ns() - t0 > limit_ns)) break;
+      if (*abort || globaltimer_ns() - t0 > limit_ns) break;
     }
   }
   return __all_sync(__activemask(), ok);

@@ -129,17 +129,26 @@ int rglru_fwd_algo(const void *x, const void *conv_w, const void *W_a, const voi
  *                           one of its pipeline stages); 0 = the default of 2 s.
  *                           Values from 1 ns to 1 ms are refused (INVALID_ARG):
  *                           healthy waits could expire.
- *   fault_unpublished_tile  testing of the failure path: when >= 0, the tile of
- *                           that index in the first (batch row 0, channels
- *                           0..127) group never publishes its carry, so the
- *                           waits of its successors run out: the call then
+ *   fault_unpublished_tile  testing of the failure path: 0 = off (the default,
+ *                           and that of rglru_fwd and rglru_fwd_algo); n > 0: the
+ *                           tile of index n - 1 in the first (batch row 0,
+ *                           channels 0..127) group never publishes its carry, so
+ *                           the waits of its successors run out: the call then
  *                           reports RGLRU_ERR_TIMEOUT through dev_status and
  *                           returns with y incomplete; the context stays usable.
- *                           -1 = off (the default of rglru_fwd and rglru_fwd_algo).
+ *                           Negative values are refused (INVALID_ARG).
+ *   kernel_begin_event,     cudaEvent_t handles, or NULL: when set, recorded on the
+ *   kernel_end_event        stream right before the first and right after the last
+ *                           compute kernel of the call (after the reset of the
+ *                           workspace), so that a caller can time the kernels alone.
+ *                           The events must belong to the stream's device; the call
+ *                           neither creates nor destroys them.
  */
 typedef struct {
   unsigned long long wait_limit_ns;
   int fault_unpublished_tile;
+  void *kernel_begin_event;
+  void *kernel_end_event;
 } rglru_fwd_options;
 
 /* rglru_fwd_algo with options (NULL = defaults). */

@@ -97,3 +97,12 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises((TypeError, RuntimeError)):
         _abi.rglru_fwd(x, torch.zeros(4, 8), torch.zeros(1, 8, 8), torch.zeros(8),
                        torch.zeros(1, 8, 8), torch.zeros(8), torch.zeros(8))
+
+
+def test_options_struct_matches_header():
+    """The ctypes mirror of rglru_fwd_options has the header's fields in order."""
+    from gated_linear_recurrence_rglru_b200._abi import FwdOptions
+    hdr = open(os.path.join(ROOT, "include", "rglru.h")).read()
+    body = re.search(r"typedef struct \{([^}]*)\} rglru_fwd_options;", hdr).group(1)
+    names = re.findall(r"(\w+)\s*;", body)
+    assert names == [f[0] for f in FwdOptions._fields_]

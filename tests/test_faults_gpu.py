@@ -28,7 +28,7 @@ def test_unpublished_tile_times_out_and_context_survives(cuda_device):
     t, g = _inputs(cuda_device)
     w = [g[k] for k in ("conv_w", "W_a", "b_a", "W_x", "b_x", "Lambda")]
     status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
-    opts = FwdOptions(wait_limit_ns=50_000_000, fault_unpublished_tile=3)
+    opts = FwdOptions(wait_limit_ns=50_000_000, fault_unpublished_tile=4)   # tile 3
     t0 = time.time()
     rg.rglru_fwd(g["x"], *w, algo="tensor", dev_status=status, options=opts)
     torch.cuda.synchronize()
@@ -48,6 +48,28 @@ def test_too_short_wait_limit_is_refused(cuda_device):
     _, g = _inputs(cuda_device)
     w = [g[k] for k in ("conv_w", "W_a", "b_a", "W_x", "b_x", "Lambda")]
     with pytest.raises(rg.RGLRUError) as ei:
-        rg.rglru_fwd(g["x"], *w, algo="tensor", options=FwdOptions(wait_limit_ns=1000,
-                                                                   fault_unpublished_tile=-1))
+        rg.rglru_fwd(g["x"], *w, algo="tensor", options=FwdOptions(wait_limit_ns=1000))
     assert ei.value.status == 1
+    with pytest.raises(rg.RGLRUError) as ei:
+        rg.rglru_fwd(g["x"], *w, algo="tensor", options=FwdOptions(fault_unpublished_tile=-1))
+    assert ei.value.status == 1
+
+
+def test_zeroed_options_with_kernel_events(cuda_device):
+    """Zero-initialised options are the defaults (no fault); the kernel events
+    they carry are recorded around the compute kernel."""
+    t, g = _inputs(cuda_device)
+    w = [g[k] for k in ("conv_w", "W_a", "b_a", "W_x", "b_x", "Lambda")]
+    eb, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    eb.record()
+    ee.record()
+    torch.cuda.synchronize()
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    opts = FwdOptions(kernel_begin_event=eb.cuda_event, kernel_end_event=ee.cuda_event)
+    y, _, _ = rg.rglru_fwd(g["x"], *w, algo="tensor", dev_status=status, options=opts)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert 0.0 < eb.elapsed_time(ee) < 1000.0
+    yo, _, _ = orc.rglru_fwd(t["x"], t["conv_w"], t["W_a"], t["b_a"], t["W_x"], t["b_x"],
+                             t["Lambda"])
+    assert max_rel_err(y.float().cpu().numpy(), yo) <= 2e-2
