@@ -8,17 +8,19 @@
 //   u = w0 x_{t-3} + w1 x_{t-2} + w2 x_{t-1} + w3 x_t      (three past inputs in a ring)
 //   [z_a | z_x] = u W (block-diagonal), gates, a, beta as in the forward
 //   h <- a h + beta,  y_t = h,  ring slot pos % 3 <- x_t
-// Jobs are (group of 128 output channels, tile of N batch rows). The gate
+// Jobs are (group of 128 output channels, tile of N = 16 batch rows). The gate
 // contraction runs on tcgen05 with the gate weights as A (M = 128 channels) and
 // the conv output as B (N = rows), so TMEM lane m holds channel m's gates for
 // the tile's rows; the epilogue updates h in place lane = channel, which keeps
 // its global accesses coalesced. Rows never interact, so CTAs take balanced
 // contiguous ranges of jobs and nothing waits on another CTA.
 //
-// Roles: warp 0 posts the CTA's jobs and loads gate weights by TMA; warp 1
-// owns TMEM and issues the MMAs; warps 2-5 compute the Conv1D from global
-// memory into the bf16 B operand and an fp32 u tile; two epilogue warpgroups
-// take the jobs alternately.
+// Roles: warp 0 posts the CTA's jobs and loads by TMA the gate weights and,
+// two jobs ahead, each job's inputs (x_t and the three ring slots of its rows
+// and channels); warp 1 owns TMEM and issues the MMAs; warps 2-5 compute the
+// Conv1D from shared memory into the bf16 B operand and an fp32 u tile; two
+// epilogue warpgroups take the jobs alternately and load their rows' h before
+// waiting for the MMA.
 //
 // Heads 256 wide are split over two channel groups whose CTAs both read all
 // 256 channels of the ring's slot pos % 3; that slot is then rewritten by a
@@ -42,9 +44,10 @@ constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint64_t kDrainNs = 200000000ull;
 
 struct DecTcParams {
-  const __nv_bfloat16 *x_t, *conv_w, *b_a, *b_x;
+  const __nv_bfloat16 *conv_w, *b_a, *b_x;
   const float *Lambda;
   __nv_bfloat16 *ring;
+  const __nv_bfloat16 *x_t;
   float *h;
   __nv_bfloat16 *y_t;
   int B, D, H, bw, pos;
@@ -56,94 +59,102 @@ template <int K, int N>
 struct DCfg {
   static constexpr int NE = 2;                     // epilogue warpgroups
   static constexpr int kThreads = 64 + 128 + NE * 128;
-  static constexpr int kABytes = K * 256;
+  static constexpr int kABytes = K * 256;          // one gate: 2 M-blocks x K rows x 128 B
+  static constexpr int kInBytes = N * K * 2;       // one input tile: N rows x K channels, bf16
+  static constexpr int kXBytes = 4 * kInBytes;     // x_t and ring slots pos, pos+1, pos+2 (mod 3)
+  static constexpr int kNX = 2;                    // input slots
   static constexpr int kBBytes = N * K * 2;
   static constexpr int kUBytes = N * kM * 4;
   static constexpr int kNS = 2;
-  static constexpr int kNT = 4;
+  static constexpr int kNT = NE + 1;
   static constexpr int kOffA = 0;
-  static constexpr int kOffB = 2 * kABytes;
+  static constexpr int kOffX = 2 * kABytes;
+  static constexpr int kOffB = kOffX + kNX * kXBytes;
   static constexpr int kOffU = kOffB + kNS * kBBytes;
   static constexpr int kOffBar = kOffU + kNS * kUBytes;
-  // job_full[JQ], job_empty[JQ], w_full, w_free, b_full[NS], b_empty[NS], u_empty[NS],
-  // acc_full[NT], tmem_empty[NT]
-  static constexpr int kNumBars = 2 * kJQ + 2 + 3 * kNS + 2 * kNT;
+  // job_full[JQ], job_empty[JQ], x_full[NX], x_empty[NX], w_full, w_free,
+  // b_full[NS], b_empty[NS], u_empty[NS], acc_full[NT], tmem_empty[NT]
+  static constexpr int kNumBars = 2 * kJQ + 2 * kNX + 2 + 3 * kNS + 2 * kNT;
   static constexpr int kOffJobs = (kOffBar + kNumBars * 8 + 15) / 16 * 16;
   static constexpr int kOffMisc = kOffJobs + kJQ * 16;
-  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;
+  // the dynamic shared memory base is declared 1024-byte aligned (checked)
+  static constexpr int kSmemBytes = kOffMisc + 64;
   static constexpr int kSlotCols = 2 * N;
   static constexpr int kTmemCols = kNT * kSlotCols <= 128 ? 128 : (kNT * kSlotCols <= 256 ? 256 : 512);
+  static constexpr int NQ = K / 4;                 // conv: channel quads
+  static constexpr int SEG = N * NQ / 128;         // conv: rows per thread
   static_assert(kSmemBytes <= 232448, "shared memory");
-  static_assert((N * (K / 4)) % (128 * 8) == 0, "conv mapping: 8-row steps");
+  static_assert(N % 16 == 0 && (N * NQ) % 128 == 0 && SEG % 4 == 0, "conv mapping");
 };
 
+// Offset (bytes) of (own channel c, 4-row block jb) in the fp32 u tile:
+// channel-major rows of N floats whose 16-byte blocks are XOR-permuted so that
+// any 8 consecutive channels (a quarter warp of epilogue readers) hit distinct
+// banks: with 8 or more blocks per row by (c % 8) ^ (c / 8 % 8); with 4 blocks
+// (two rows per 128 bytes) by (c / 2) % 4.
 template <int N>
 __device__ __forceinline__ uint32_t u_off(int c, int jb) {
-  return static_cast<uint32_t>(c * (N * 4) + ((jb ^ ((c & 7) ^ ((c >> 3) & 7))) << 4));
+  static_assert(N == 16 || N >= 32, "u tile rows of 4 or of at least 8 blocks");
+  const int perm = N == 16 ? ((c >> 1) & 3) : ((c & 7) ^ ((c >> 3) & 7));
+  return static_cast<uint32_t>(c * (N * 4) + ((jb ^ perm) << 4));
 }
 
-// Conv1D of N rows x K channels from global memory. Thread t covers channel
-// quad q (4 channels) and SEG consecutive rows. Writes the bf16 K-major B
-// operand (128-byte swizzle), the fp32 u of the own channels (channel-major,
-// see u_off) and, when asked, the ring update of the own channels.
+// Conv1D of N rows x K channels from the input tile in shared memory (row-major
+// [N][K] per array: x_t, then the ring slots holding x_{t-3}, x_{t-2}, x_{t-1}).
+// Thread t covers channel quad q (4 channels) and SEG consecutive rows. Writes
+// the bf16 K-major B operand (128-byte swizzle), the fp32 u of the own channels
+// (channel-major, see u_off) and, when asked, the ring update of the own channels.
 template <int K, int N>
-__device__ __forceinline__ void dec_conv(const DecTcParams &p, unsigned char *__restrict__ bt,
+__device__ __forceinline__ void dec_conv(const DecTcParams &p, const unsigned char *__restrict__ xin,
+                                         unsigned char *__restrict__ bt,
                                          unsigned char *__restrict__ ut, int kbase, int own_lo,
                                          int r0, int t, const float2 (&w)[4][2]) {
-  constexpr int NQ = K / 4, SEG = N * NQ / 128;
+  using C = DCfg<K, N>;
+  constexpr int NQ = C::NQ, SEG = C::SEG;
   const int qd = t % NQ, sg = t / NQ;
   const int kq = qd * 4, nb = sg * SEG;
   const bool own = (kq >= own_lo) && (kq < own_lo + kM);
   const int chq = kbase + kq;
-  const int s0 = p.pos % 3, s1 = (p.pos + 1) % 3, s2 = (p.pos + 2) % 3;
-  const uint32_t bt_base = static_cast<uint32_t>((kq >> 6) * N * 128 + nb * 128 + ((kq & 7) << 1));
+  const int s0 = p.pos % 3;
+  const unsigned char *xq = xin + kq * 2;          // + array * kInBytes + row * K * 2
+  unsigned char *bq = bt + (kq >> 6) * N * 128 + ((kq & 7) << 1);
   const int chunk = (kq & 63) >> 3;
-  float uacc[4][4];
 #pragma unroll
   for (int j0 = 0; j0 < SEG; j0 += 4) {
-    uint2 xv[4], r0v[4], r1v[4], r2v[4];
+    float uacc[4][4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int row = r0 + nb + j0 + j;
-      if (row < p.B) {
-        const size_t rb = static_cast<size_t>(row) * 3 * p.D + chq;
-        xv[j] = __ldg(reinterpret_cast<const uint2 *>(p.x_t + static_cast<size_t>(row) * p.D + chq));
-        r0v[j] = __ldg(reinterpret_cast<const uint2 *>(p.ring + rb + static_cast<size_t>(s0) * p.D));
-        r1v[j] = __ldg(reinterpret_cast<const uint2 *>(p.ring + rb + static_cast<size_t>(s1) * p.D));
-        r2v[j] = __ldg(reinterpret_cast<const uint2 *>(p.ring + rb + static_cast<size_t>(s2) * p.D));
-      } else {
-        xv[j] = r0v[j] = r1v[j] = r2v[j] = make_uint2(0u, 0u);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int jj = j0 + j;
-      const int row = r0 + nb + jj;
+      const int n = nb + j0 + j;
+      const uint2 xv = *reinterpret_cast<const uint2 *>(xq + n * K * 2);
+      const uint2 r0v = *reinterpret_cast<const uint2 *>(xq + C::kInBytes + n * K * 2);
+      const uint2 r1v = *reinterpret_cast<const uint2 *>(xq + 2 * C::kInBytes + n * K * 2);
+      const uint2 r2v = *reinterpret_cast<const uint2 *>(xq + 3 * C::kInBytes + n * K * 2);
       float2 u[2];
 #pragma unroll
       for (int pp = 0; pp < 2; ++pp) {
-        const uint32_t a0 = pp ? r0v[j].y : r0v[j].x, a1 = pp ? r1v[j].y : r1v[j].x;
-        const uint32_t a2 = pp ? r2v[j].y : r2v[j].x, a3 = pp ? xv[j].y : xv[j].x;
+        const uint32_t a0 = pp ? r0v.y : r0v.x, a1 = pp ? r1v.y : r1v.x;
+        const uint32_t a2 = pp ? r2v.y : r2v.x, a3 = pp ? xv.y : xv.x;
         float2 acc = __fmul2_rn(w[0][pp], bf2_to_f2(a0));
         acc = __ffma2_rn(w[1][pp], bf2_to_f2(a1), acc);
         acc = __ffma2_rn(w[2][pp], bf2_to_f2(a2), acc);
         u[pp] = __ffma2_rn(w[3][pp], bf2_to_f2(a3), acc);
       }
-      *reinterpret_cast<uint2 *>(bt + bt_base + jj * 128 + (((chunk ^ jj) & 7) << 4)) =
+      *reinterpret_cast<uint2 *>(bq + n * 128 + (((chunk ^ n) & 7) << 4)) =
           make_uint2(f2_to_bf2(u[0]), f2_to_bf2(u[1]));
-      uacc[0][jj & 3] = u[0].x;
-      uacc[1][jj & 3] = u[0].y;
-      uacc[2][jj & 3] = u[1].x;
-      uacc[3][jj & 3] = u[1].y;
-      if ((jj & 3) == 3 && own) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          *reinterpret_cast<float4 *>(ut + u_off<N>(kq - own_lo + k, (nb + jj) >> 2)) =
-              make_float4(uacc[k][0], uacc[k][1], uacc[k][2], uacc[k][3]);
-      }
+      uacc[0][j] = u[0].x;
+      uacc[1][j] = u[0].y;
+      uacc[2][j] = u[1].x;
+      uacc[3][j] = u[1].y;
+      const int row = r0 + n;
       if (p.write_ring && own && row < p.B)
         *reinterpret_cast<uint2 *>(p.ring + static_cast<size_t>(row) * 3 * p.D +
-                                   static_cast<size_t>(s0) * p.D + chq) = xv[j];
+                                   static_cast<size_t>(s0) * p.D + chq) = xv;
+    }
+    if (own) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        *reinterpret_cast<float4 *>(ut + u_off<N>(kq - own_lo + k, (nb + j0) >> 2)) =
+            make_float4(uacc[k][0], uacc[k][1], uacc[k][2], uacc[k][3]);
     }
   }
 }
@@ -151,19 +162,24 @@ __device__ __forceinline__ void dec_conv(const DecTcParams &p, unsigned char *__
 template <int K, int N>
 __global__ void __launch_bounds__(DCfg<K, N>::kThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
-                 const __grid_constant__ CUtensorMap tmap_wx, const DecTcParams p) {
+                 const __grid_constant__ CUtensorMap tmap_wx,
+                 const __grid_constant__ CUtensorMap tmap_xt,
+                 const __grid_constant__ CUtensorMap tmap_ring, const DecTcParams p) {
   using C = DCfg<K, N>;
-  constexpr int NS = C::kNS, NT = C::kNT, NE = C::NE;
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char *sm = reinterpret_cast<unsigned char *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  constexpr int NS = C::kNS, NT = C::kNT, NE = C::NE, NX = C::kNX;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  if ((smem_u32(smem_raw) & 1023u) != 0u) return;   // the layout needs the declared alignment
+  unsigned char *sm = smem_raw;
   unsigned char *sA = sm + C::kOffA;
+  unsigned char *sX = sm + C::kOffX;
   unsigned char *sB = sm + C::kOffB;
   unsigned char *sU = sm + C::kOffU;
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::kOffBar);
   uint64_t *job_full = bars;
   uint64_t *job_empty = job_full + kJQ;
-  uint64_t *w_full = job_empty + kJQ;
+  uint64_t *x_full = job_empty + kJQ;
+  uint64_t *x_empty = x_full + NX;
+  uint64_t *w_full = x_empty + NX;
   uint64_t *w_free = w_full + 1;
   uint64_t *b_full = w_free + 1;
   uint64_t *b_empty = b_full + NS;
@@ -185,6 +201,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
       mbar_init(&job_full[i], 1);
       mbar_init(&job_empty[i], 9);                  // 4 conv warps, MMA, 4 epilogue warps
     }
+    for (int i = 0; i < NX; ++i) {
+      mbar_init(&x_full[i], 1);
+      mbar_init(&x_empty[i], 4);                    // 4 conv warps
+    }
     mbar_init(w_full, 1);
     mbar_init(w_free, 1);
     for (int i = 0; i < NS; ++i) {
@@ -200,6 +220,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
     fence_mbar_init();
     prefetch_tmap(&tmap_wa);
     prefetch_tmap(&tmap_wx);
+    prefetch_tmap(&tmap_xt);
+    prefetch_tmap(&tmap_ring);
   }
   {
     uint4 *a4 = reinterpret_cast<uint4 *>(sA);
@@ -228,6 +250,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
       int w_unit = -1;
       uint32_t wfree_phase = 0;
       const int n = j_end - j_begin;
+      int last_x_job = -1;
       for (int i = 0; i <= n + NE - 1; ++i) {
         const int js = i % kJQ;
         RG_WAIT_OR_ABORT(&job_empty[js], ((i / kJQ) & 1) ^ 1);
@@ -241,12 +264,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
         const int reload = unit != w_unit ? 1 : 0;
         jobs[js] = make_int4(unit, tile, reload, 0);
         mbar_arrive(&job_full[js]);
+        const int cg = unit;
         if (reload) {
           if (i > 0) {
             RG_WAIT_OR_ABORT(w_free, wfree_phase);
             wfree_phase ^= 1;
           }
-          const int cg = unit;
           mbar_arrive_expect_tx(w_full, 2u * 2u * static_cast<uint32_t>(R) * 128u);
           for (int g = 0; g < 2; ++g) {
             const CUtensorMap *tm = g == 0 ? &tmap_wa : &tmap_wx;
@@ -265,13 +288,30 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
           }
           w_unit = unit;
         }
+        // the job's inputs: x_t rows, then ring slots pos % 3 (x_{t-3}),
+        // (pos + 1) % 3 (x_{t-2}), (pos + 2) % 3 (x_{t-1}); rows past B read as zeros
+        const int xb = i % NX;
+        RG_WAIT_OR_ABORT(&x_empty[xb], ((i / NX) & 1) ^ 1);
+        const int kbase = p.bw <= 128 ? cg * kM : (cg >> 1) * 256;
+        unsigned char *dst = sX + xb * C::kXBytes;
+        mbar_arrive_expect_tx(&x_full[xb], static_cast<uint32_t>(C::kXBytes));
+        tma_load_2d(dst, &tmap_xt, &x_full[xb], kbase, tile * N);
+        for (int q = 0; q < 3; ++q)
+          tma_load_3d(dst + (q + 1) * C::kInBytes, &tmap_ring, &x_full[xb], kbase, (p.pos + q) % 3,
+                      tile * N);
+        last_x_job = i;
+      }
+      if (*cta_abort) {
+        for (int j = last_x_job; j >= 0 && j > last_x_job - NX; --j)
+          mbar_wait_drain(&x_full[j % NX], (j / NX) & 1, kDrainNs);
       }
     }
   } else if (warp == 1) {
     // ============================== MMA issuer ==============================
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kM, N, true, false);
-      const uint32_t a0 = smem_u32(sA), a1 = smem_u32(sA + C::kABytes);
+      const uint64_t ada0 = sdesc_sw128(smem_u32(sA), K * 128, 1024);
+      const uint64_t adx0 = sdesc_sw128(smem_u32(sA + C::kABytes), K * 128, 1024);
       uint32_t w_phase = 0;
       int last_commit = -1;
       for (int i = 0;; ++i) {
@@ -295,13 +335,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
         const uint32_t bs = smem_u32(sB + s * C::kBBytes);
         const uint32_t d_a = tmem_base + static_cast<uint32_t>(ts * C::kSlotCols);
         const uint32_t d_x = d_a + N;
+        // descriptors of K step 0; a step advances the start addresses by a
+        // constant (the address field holds address / 16, and shared-memory
+        // addresses stay below 256 KB, so the additions never carry out of it)
+        const uint64_t bd0 = sdesc_sw128(bs, 16, 1024);
 #pragma unroll
         for (int ks = 0; ks < K / 16; ++ks) {
-          const uint64_t bd = sdesc_sw128(bs + (ks >> 2) * (N * 128) + (ks & 3) * 32, 16, 1024);
-          const uint64_t ada = sdesc_sw128(a0 + ks * 16 * 128, K * 128, 1024);
-          const uint64_t adx = sdesc_sw128(a1 + ks * 16 * 128, K * 128, 1024);
-          mma_bf16(d_a, ada, bd, idesc, ks > 0 ? 1u : 0u);
-          mma_bf16(d_x, adx, bd, idesc, ks > 0 ? 1u : 0u);
+          const uint64_t bd = bd0 + static_cast<uint64_t>(((ks >> 2) * (N * 128) + (ks & 3) * 32) >> 4);
+          const uint64_t astep = static_cast<uint64_t>((ks * 16 * 128) >> 4);
+          mma_bf16(d_a, ada0 + astep, bd, idesc, ks > 0 ? 1u : 0u);
+          mma_bf16(d_x, adx0 + astep, bd, idesc, ks > 0 ? 1u : 0u);
         }
         mma_commit(&acc_full[ts]);
         mma_commit(&b_empty[s]);
@@ -335,18 +378,21 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
           cwq[tap][1] = bf2_to_f2(raw.y);
         }
       }
-      const int s = i % NS;
+      const int s = i % NS, xb = i % NX;
+      RG_WAIT_OR_ABORT(&x_full[xb], (i / NX) & 1);
       RG_WAIT_OR_ABORT(&b_empty[s], ((i / NS) & 1) ^ 1);
       RG_WAIT_OR_ABORT(&u_empty[s], ((i / NS) & 1) ^ 1);
-      dec_conv<K, N>(p, sB + s * C::kBBytes, sU + s * C::kUBytes, kbase, own_lo, tile * N, wt, cwq);
+      dec_conv<K, N>(p, sX + xb * C::kXBytes, sB + s * C::kBBytes, sU + s * C::kUBytes, kbase,
+                     own_lo, tile * N, wt, cwq);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {                              // per warp: no barrier to strand an aborting warp at
+        mbar_arrive(&x_empty[xb]);
         mbar_arrive(&b_full[s]);
         mbar_arrive(&job_empty[js]);
       }
     }
-  } else {
+  } else if (warp < 6 + 4 * NE) {
     // ============================ epilogue warpgroups ============================
     const int eg = (warp - 6) >> 2;
     const int qd = warp & 3;
@@ -370,17 +416,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
         kc = chan_consts(__bfloat162float(p.b_a[c]), __bfloat162float(p.b_x[c]), p.Lambda[c]);
         fast = __all_sync(0xffffffffu, chan_fast(kc));
       }
+      // the previous state of this channel for the job's rows, loaded while the
+      // conv and the MMA run (coalesced across lanes)
+      float hold[N];
+#pragma unroll
+      for (int n = 0; n < N; ++n)
+        hold[n] = n < nvalid ? p.h[static_cast<size_t>(r0 + n) * p.D + c] : 0.f;
       RG_WAIT_OR_ABORT(&acc_full[ts], (i / NT) & 1);
       tc_fence_after();
       const uint32_t t_lane = t_lane0 + static_cast<uint32_t>(ts * C::kSlotCols);
       const unsigned char *uslot = sU + s * C::kUBytes;
 #pragma unroll
       for (int ch = 0; ch < N / 16; ++ch) {
-        // previous state of this channel for the chunk's rows (coalesced across lanes)
-        float hold[16];
-#pragma unroll
-        for (int n = 0; n < 16; ++n)
-          hold[n] = ch * 16 + n < nvalid ? p.h[static_cast<size_t>(r0 + ch * 16 + n) * p.D + c] : 0.f;
         float za[16], zx[16], uu[16];
         tmem_ld16(t_lane + ch * 16, za);
         tmem_ld16(t_lane + N + ch * 16, zx);
@@ -405,7 +452,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
             gate_one(za[2 * pr], zx[2 * pr], uu[2 * pr], kc, a.x, beta.x, la.x);
             gate_one(za[2 * pr + 1], zx[2 * pr + 1], uu[2 * pr + 1], kc, a.y, beta.y, la.y);
           }
-          const float2 hn = __ffma2_rn(a, make_float2(hold[2 * pr], hold[2 * pr + 1]), beta);
+          const float2 hn = __ffma2_rn(a, make_float2(hold[n], hold[n + 1]), beta);
           if (n < nvalid) {
             const size_t o = static_cast<size_t>(r0 + n) * p.D + c;
             p.h[o] = hn.x;
@@ -471,7 +518,29 @@ cudaError_t launch_dec_t(const DecArgs &a, cudaStream_t st) {
   if (enc == nullptr) return cudaErrorNotSupported;
   const int bw = a.D / a.H;
   const int R = bw <= 128 ? bw : 256;
-  CUtensorMap twa, twx;
+  CUtensorMap twa, twx, txt, tring;
+  {
+    // x_t (B, D): box K channels x N rows
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.D), static_cast<cuuint64_t>(a.B)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.D) * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(K), static_cast<cuuint32_t>(N)};
+    cuuint32_t es[2] = {1, 1};
+    if (enc(&txt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(a.x_t), dims, strides,
+            box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    // ring (B, 3, D): box K channels x 1 slot x N rows
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(a.D), 3, static_cast<cuuint64_t>(a.B)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(a.D) * 2, static_cast<cuuint64_t>(a.D) * 6};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(K), 1, static_cast<cuuint32_t>(N)};
+    cuuint32_t es[3] = {1, 1, 1};
+    if (enc(&tring, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.conv_state, dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   for (int g = 0; g < 2; ++g) {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(bw), static_cast<cuuint64_t>(a.H) * bw};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(bw) * 2};
@@ -509,7 +578,7 @@ cudaError_t launch_dec_t(const DecArgs &a, cudaStream_t st) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = p.n_jobs < sms ? p.n_jobs : sms;
-  kern<<<grid, C::kThreads, C::kSmemBytes, st>>>(twa, twx, p);
+  kern<<<grid, C::kThreads, C::kSmemBytes, st>>>(twa, twx, txt, tring, p);
   e = cudaGetLastError();
   if (e != cudaSuccess || p.write_ring) return e;
   const size_t n8 = static_cast<size_t>(a.B) * a.D / 8;
@@ -528,8 +597,8 @@ int tc_decode_launches(int D, int H) { return D / H == 256 ? 2 : 1; }
 
 cudaError_t launch_decode_tc(const DecArgs &a, cudaStream_t st) {
   const int bw = a.D / a.H;
-  if (bw == 256) return launch_dec_t<256, 32>(a, st);
-  return launch_dec_t<128, 32>(a, st);
+  if (bw == 256) return launch_dec_t<256, 16>(a, st);
+  return launch_dec_t<128, 16>(a, st);
 }
 
 }  // namespace rglru

@@ -456,7 +456,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
     // ============================== MMA issuer ==============================
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kM, N, true, false);
-      const uint32_t a0 = smem_u32(sA), a1 = smem_u32(sA + C::kABytes);
+      const uint64_t ada0 = sdesc_sw128(smem_u32(sA), K * 128, 1024);
+      const uint64_t adx0 = sdesc_sw128(smem_u32(sA + C::kABytes), K * 128, 1024);
       uint32_t w_phase = 0;
       int last_commit = -1;
       for (int i = 0;; ++i) {
@@ -481,13 +482,16 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
         const uint32_t bs = smem_u32(sB + s * C::kBBytes);
         const uint32_t d_a = tmem_base + static_cast<uint32_t>(ts * C::kSlotCols);
         const uint32_t d_x = d_a + N;
+        // descriptors of K step 0; a step advances the start addresses by a
+        // constant (the address field holds address / 16, and shared-memory
+        // addresses stay below 256 KB, so the additions never carry out of it)
+        const uint64_t bd0 = sdesc_sw128(bs, 16, 1024);
 #pragma unroll
         for (int ks = 0; ks < K / 16; ++ks) {
-          const uint64_t bd = sdesc_sw128(bs + (ks >> 2) * (N * 128) + (ks & 3) * 32, 16, 1024);
-          const uint64_t ada = sdesc_sw128(a0 + ks * 16 * 128, K * 128, 1024);
-          const uint64_t adx = sdesc_sw128(a1 + ks * 16 * 128, K * 128, 1024);
-          mma_bf16(d_a, ada, bd, idesc, ks > 0 ? 1u : 0u);
-          mma_bf16(d_x, adx, bd, idesc, ks > 0 ? 1u : 0u);
+          const uint64_t bd = bd0 + static_cast<uint64_t>(((ks >> 2) * (N * 128) + (ks & 3) * 32) >> 4);
+          const uint64_t astep = static_cast<uint64_t>((ks * 16 * 128) >> 4);
+          mma_bf16(d_a, ada0 + astep, bd, idesc, ks > 0 ? 1u : 0u);
+          mma_bf16(d_x, adx0 + astep, bd, idesc, ks > 0 ? 1u : 0u);
         }
         mma_commit(&acc_full[ts]);
         mma_commit(&b_empty[s]);
