@@ -168,10 +168,11 @@ __device__ __forceinline__ void conv_tile(const unsigned char *__restrict__ xs,
   const int chq = kbase + kq;                       // first global channel of the quad
   // x tile row r holds token tile * N - 3 + r: the window of output token
   // nb + j is rows nb + j .. nb + j + 3
-  const unsigned char *xq = xs + kq * 2;
-  uint2 r0 = *reinterpret_cast<const uint2 *>(xq + (nb + 0) * K * 2);
-  uint2 r1 = *reinterpret_cast<const uint2 *>(xq + (nb + 1) * K * 2);
-  uint2 r2 = *reinterpret_cast<const uint2 *>(xq + (nb + 2) * K * 2);
+  // shared-window addresses (32-bit)
+  const uint32_t xq = smem_u32(xs) + static_cast<uint32_t>(kq * 2 + nb * K * 2);
+  uint2 r0 = lds64(xq);
+  uint2 r1 = lds64(xq + K * 2);
+  uint2 r2 = lds64(xq + 2 * K * 2);
   if (tile == 0 && nb == 0 && p.conv_state_in != nullptr) {
     const __nv_bfloat16 *cs = p.conv_state_in + static_cast<size_t>(b) * 3 * p.D + chq;
     r0 = __ldg(reinterpret_cast<const uint2 *>(cs));
@@ -187,26 +188,31 @@ __device__ __forceinline__ void conv_tile(const unsigned char *__restrict__ xs,
   xw[2][1] = bf2_to_f2(r2.y);
   // B operand: row n = nb + j of the 64-channel block kq / 64; 16-byte chunk
   // (kq % 64) / 8 of the row, XOR-swizzled by n % 8 (= j % 8)
-  unsigned char *bq = bt + (kq >> 6) * N * 128 + nb * 128 + ((kq & 7) << 1);
-  const int chunk = (kq & 63) >> 3;
-  // u tile rows of the 4 own channels and their block permutations
+  const uint32_t bq =
+      smem_u32(bt) + static_cast<uint32_t>((kq >> 6) * N * 128 + nb * 128 + ((kq & 7) << 1));
+  const uint32_t chunk = static_cast<uint32_t>((kq & 63) >> 3);
+  // u tile rows of the 4 own channels and their block permutations (x 16 bytes)
+  const uint32_t ua = smem_u32(ut);
   uint32_t ubase[4], uperm[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int c = kq - own_lo + k;
-    ubase[k] = static_cast<uint32_t>(c * (N * 4));
-    uperm[k] = static_cast<uint32_t>((c & 7) ^ ((c >> 3) & 7));
+    ubase[k] = ua + static_cast<uint32_t>(c * (N * 4));
+    uperm[k] = static_cast<uint32_t>((c & 7) ^ ((c >> 3) & 7)) << 4;
   }
 #pragma unroll 1
   for (int jb = 0; jb < SEG; jb += 4) {
+    const uint32_t xrow = xq + static_cast<uint32_t>((jb + 3) * K * 2);
     uint2 nr[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      nr[q] = *reinterpret_cast<const uint2 *>(xq + (nb + jb + 3 + q) * K * 2);
+    for (int q = 0; q < 4; ++q) nr[q] = lds64(xrow + q * K * 2);
+    // row nb + jb + q, 16-byte chunk XOR-swizzled by its row % 8; jb % 4 == 0,
+    // so (chunk ^ (jb + q)) % 8 == ((chunk ^ jb) % 8) ^ q
+    const uint32_t brow = bq + static_cast<uint32_t>(jb * 128);
+    const uint32_t cj = ((chunk ^ static_cast<uint32_t>(jb)) & 7u) << 4;
     float uacc[4][4];                               // u of 4 channels x 4 tokens
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const int j = jb + q;                         // j % 4 == q
       xw[(q + 3) & 3][0] = bf2_to_f2(nr[q].x);
       xw[(q + 3) & 3][1] = bf2_to_f2(nr[q].y);
       float2 u[2];
@@ -217,19 +223,17 @@ __device__ __forceinline__ void conv_tile(const unsigned char *__restrict__ xs,
         acc = __ffma2_rn(w[2][pp], xw[(q + 2) & 3][pp], acc);
         u[pp] = __ffma2_rn(w[3][pp], xw[(q + 3) & 3][pp], acc);
       }
-      *reinterpret_cast<uint2 *>(bq + j * 128 + (((chunk ^ j) & 7) << 4)) =
-          make_uint2(f2_to_bf2(u[0]), f2_to_bf2(u[1]));
+      sts64(brow + q * 128 + (cj ^ static_cast<uint32_t>(q << 4)), f2_to_bf2(u[0]), f2_to_bf2(u[1]));
       uacc[0][q] = u[0].x;
       uacc[1][q] = u[0].y;
       uacc[2][q] = u[1].x;
       uacc[3][q] = u[1].y;
     }
     if (kUTile && own) {
-      const uint32_t blk = static_cast<uint32_t>((nb + jb) >> 2);
+      const uint32_t blk = static_cast<uint32_t>((nb + jb) >> 2) << 4;
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        *reinterpret_cast<float4 *>(ut + ubase[k] + ((blk ^ uperm[k]) << 4)) =
-            make_float4(uacc[k][0], uacc[k][1], uacc[k][2], uacc[k][3]);
+        sts128f(ubase[k] + (blk ^ uperm[k]), uacc[k][0], uacc[k][1], uacc[k][2], uacc[k][3]);
     }
   }
   if (own && last_tile && nb == 0 && p.conv_state_out != nullptr) {
@@ -239,7 +243,7 @@ __device__ __forceinline__ void conv_tile(const unsigned char *__restrict__ xs,
 #pragma unroll
     for (int r = 0; r < 3; ++r) {
       const int row = nvalid + r;
-      uint2 v = *reinterpret_cast<const uint2 *>(xq + row * K * 2);
+      uint2 v = lds64(xq + static_cast<uint32_t>((row - nb) * K * 2));
       if (tile == 0 && row < 3 && p.conv_state_in != nullptr)
         v = __ldg(reinterpret_cast<const uint2 *>(p.conv_state_in +
                                                    (static_cast<size_t>(b) * 3 + row) * p.D + chq));
@@ -584,7 +588,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
       tc_fence_after();
       // own channel's u: fp32 tile from the conv warpgroup (K = 128), or
       // recomputed from the x tile (K = 256)
-      const unsigned char *uslot = sU + us * C::kUBytes;
+      // this channel's row of the u tile and its block permutation (x 16 bytes)
+      const uint32_t urow = smem_u32(sU + us * C::kUBytes) + static_cast<uint32_t>(m * (N * 4));
+      const uint32_t uperm = static_cast<uint32_t>((m & 7) ^ ((m >> 3) & 7)) << 4;
       const __nv_bfloat16 *xown =
           reinterpret_cast<const __nv_bfloat16 *>(sX + xb * C::kXBytes) + own_lo + m;
       float xm3 = 0.f, xm2 = 0.f, xm1 = 0.f;
@@ -613,7 +619,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
         if (C::kUTile) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const float4 v = *reinterpret_cast<const float4 *>(uslot + u_offset<N>(m, ch * 4 + q));
+            const float4 v = lds128f(urow + (static_cast<uint32_t>((ch * 4 + q) << 4) ^ uperm));
             uu[4 * q] = v.x;
             uu[4 * q + 1] = v.y;
             uu[4 * q + 2] = v.z;
