@@ -27,6 +27,8 @@
 // separate small kernel after this one (ring_update_kernel) instead of here.
 #include <cudaTypedefs.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_gates.cuh"
@@ -571,12 +573,21 @@ cudaError_t launch_dec_t(const DecArgs &a, cudaStream_t st) {
   p.n_jobs = p.n_cg * p.n_tiles;
   p.write_ring = bw <= 128 ? 1 : 0;
   auto kern = decode_tc_kernel<K, N>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  // per device, once: the kernel's shared-memory opt-in and the SM count (no
+  // attribute call on later steps, which may be captured in a CUDA graph)
+  constexpr int kMaxDev = 64;
+  static std::atomic<int> sms_of[kMaxDev];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int sms = dev < kMaxDev ? sms_of[dev].load(std::memory_order_acquire) : 0;
+  if (sms == 0) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return e;
+    if (dev < kMaxDev) sms_of[dev].store(sms, std::memory_order_release);
+  }
   const int grid = p.n_jobs < sms ? p.n_jobs : sms;
   kern<<<grid, C::kThreads, C::kSmemBytes, st>>>(twa, twx, txt, tring, p);
   e = cudaGetLastError();

@@ -34,6 +34,7 @@
 // on expiry the kernel records RGLRU_ERR_TIMEOUT, raises an abort flag that
 // all waits observe, drains what it issued and returns.
 #include <cudaTypedefs.h>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -883,11 +884,19 @@ cudaError_t launch_tc_t(const FwdArgs &a, const TcLayout &L, void *ws, cudaStrea
   cudaError_t e = cudaMemsetAsync(ws, 0, L.total, st);
   if (e != cudaSuccess) return e;
   auto kern = fwd_tc_kernel<K, N, NX, NE, NU>;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-  if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // per device, once: the kernel's shared-memory opt-in and the SM count
+  constexpr int kMaxDev = 64;
+  static std::atomic<int> sms_of[kMaxDev];
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  int sms = dev < kMaxDev ? sms_of[dev].load(std::memory_order_acquire) : 0;
+  if (sms == 0) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return e;
+    if (dev < kMaxDev) sms_of[dev].store(sms, std::memory_order_release);
+  }
   const long jobs = static_cast<long>(L.n_units) * L.n_tiles;
   const int grid = static_cast<int>(jobs < sms ? jobs : sms);
   if (a.ev_begin != nullptr && (e = cudaEventRecord(a.ev_begin, st)) != cudaSuccess) return e;
