@@ -8,8 +8,10 @@ hand-written CUDA kernels behind a C ABI (include/rglru.h). This package is the
 thin Python binding of that library; see _abi.py.
 """
 from ._abi import (ALGO_AUTO, ALGO_GENERIC, ALGO_TENSOR, LIB_PATH, FwdOptions,  # noqa: F401
-                   RGLRUError, decode_launches, fwd_launches, fwd_workspace_bytes, rglru_decode_step,
-                   rglru_fwd, rglru_fwd_noalloc, status_str, version)
+                   RGLRUError, bwd_launches, bwd_workspace_bytes, decode_launches, fwd_launches,
+                   fwd_workspace_bytes, rglru_bwd, rglru_decode_step, rglru_fwd, rglru_fwd_noalloc,
+                   status_str, version)
 
-__all__ = ["rglru_fwd", "rglru_fwd_noalloc", "rglru_decode_step", "fwd_workspace_bytes", "fwd_launches",
-           "decode_launches", "FwdOptions", "RGLRUError", "status_str", "version", "LIB_PATH"]
+__all__ = ["rglru_fwd", "rglru_fwd_noalloc", "rglru_decode_step", "rglru_bwd", "fwd_workspace_bytes",
+           "bwd_workspace_bytes", "fwd_launches", "bwd_launches", "decode_launches", "FwdOptions",
+           "RGLRUError", "status_str", "version", "LIB_PATH"]

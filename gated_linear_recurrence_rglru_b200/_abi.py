@@ -23,7 +23,8 @@ ALGOS = {"auto": ALGO_AUTO, "generic": ALGO_GENERIC, "tensor": ALGO_TENSOR}
 EXPORTED = (
     "rglru_status_str", "rglru_version", "rglru_fwd_workspace_bytes", "rglru_fwd",
     "rglru_fwd_algo", "rglru_decode_step", "rglru_decode_step_algo", "rglru_fwd_launches",
-    "rglru_fwd_noalloc", "rglru_decode_launches", "rglru_fwd_ex",
+    "rglru_fwd_noalloc", "rglru_decode_launches", "rglru_fwd_ex", "rglru_bwd",
+    "rglru_bwd_workspace_bytes", "rglru_bwd_launches",
 )
 
 
@@ -72,6 +73,13 @@ def _load():
     lib.rglru_decode_step.argtypes = dec_args
     lib.rglru_decode_step_algo.restype = i32
     lib.rglru_decode_step_algo.argtypes = dec_args + [i32]
+    lib.rglru_bwd_workspace_bytes.restype = sz
+    lib.rglru_bwd_workspace_bytes.argtypes = [i32] * 5
+    lib.rglru_bwd_launches.restype = i32
+    lib.rglru_bwd_launches.argtypes = [i32] * 5
+    lib.rglru_bwd.restype = i32
+    lib.rglru_bwd.argtypes = ([vp] * 6 + [fp, fp, vp, vp, fp, vp] + [fp] * 8 + [i32] * 5
+                              + [vp, sz, vp])
     return lib
 
 
@@ -227,3 +235,60 @@ def rglru_decode_step(x_t, conv_state, pos, h, conv_w, W_a, b_a, W_x, b_x, Lambd
     if st != 0:
         raise RGLRUError(st, "rglru_decode_step")
     return y_t
+
+
+def bwd_workspace_bytes(B: int, T: int, D: int, H: int, dtype=torch.bfloat16) -> int:
+    return int(LIB.rglru_bwd_workspace_bytes(B, T, D, H, _io_of(dtype)))
+
+
+def bwd_launches(B: int, T: int, D: int, H: int, dtype=torch.bfloat16) -> int:
+    """Kernel launches that one rglru_bwd call with these sizes issues."""
+    return int(LIB.rglru_bwd_launches(B, T, D, H, _io_of(dtype)))
+
+
+def rglru_bwd(x, conv_w, W_a, b_a, W_x, b_x, Lambda, dy, h0=None, conv_state_in=None,
+              dh_T=None, *, want_dh0=True, want_dconv_state=False, workspace=None, out=None,
+              stream=None):
+    """Backward of the layer: gradients of <dy, y> + <dh_T, h_T> with respect to the
+    forward inputs (include/rglru.h, rglru_bwd). Returns a dict with dx (the I/O
+    dtype), dconv_w, dW_a, db_a, dW_x, db_x, dLambda (fp32), and dh0 / dconv_state
+    (fp32, or None when not wanted). `out` may hold preallocated outputs by name."""
+    B, T, D = x.shape
+    H = W_a.shape[0]
+    bw = D // H
+    dt = x.dtype
+    dev = x.device
+    f32 = torch.float32
+    o = dict(out or {})
+
+    def buf(name, shape, dtype):
+        t = o.get(name)
+        return t if t is not None else torch.empty(shape, device=dev, dtype=dtype)
+
+    g = dict(dx=buf("dx", (B, T, D), dt), dconv_w=buf("dconv_w", (4, D), f32),
+             dW_a=buf("dW_a", (H, bw, bw), f32), db_a=buf("db_a", (D,), f32),
+             dW_x=buf("dW_x", (H, bw, bw), f32), db_x=buf("db_x", (D,), f32),
+             dLambda=buf("dLambda", (D,), f32),
+             dh0=buf("dh0", (B, D), f32) if want_dh0 else None,
+             dconv_state=buf("dconv_state", (B, 3, D), f32) if want_dconv_state else None)
+    if workspace is None:
+        workspace = torch.empty(max(bwd_workspace_bytes(B, T, D, H, dt), 256), device=dev,
+                                dtype=torch.uint8)
+    st = LIB.rglru_bwd(
+        _ptr(x, "x", dt, (B, T, D)), _ptr(conv_w, "conv_w", dt, (4, D)),
+        _ptr(W_a, "W_a", dt, (H, bw, bw)), _ptr(b_a, "b_a", dt, (D,)),
+        _ptr(W_x, "W_x", dt, (H, bw, bw)), _ptr(b_x, "b_x", dt, (D,)),
+        _ptr(Lambda, "Lambda", f32, (D,)), _ptr(h0, "h0", f32, (B, D), optional=True),
+        _ptr(conv_state_in, "conv_state_in", dt, (B, 3, D), optional=True),
+        _ptr(dy, "dy", dt, (B, T, D)), _ptr(dh_T, "dh_T", f32, (B, D), optional=True),
+        _ptr(g["dx"], "dx", dt, (B, T, D)), _ptr(g["dconv_w"], "dconv_w", f32, (4, D)),
+        _ptr(g["dW_a"], "dW_a", f32, (H, bw, bw)), _ptr(g["db_a"], "db_a", f32, (D,)),
+        _ptr(g["dW_x"], "dW_x", f32, (H, bw, bw)), _ptr(g["db_x"], "db_x", f32, (D,)),
+        _ptr(g["dLambda"], "dLambda", f32, (D,)),
+        _ptr(g["dh0"], "dh0", f32, (B, D), optional=True),
+        _ptr(g["dconv_state"], "dconv_state", f32, (B, 3, D), optional=True),
+        B, T, D, H, _io_of(dt), _ptr(workspace, "workspace"), workspace.numel(),
+        _stream_handle(stream))
+    if st != 0:
+        raise RGLRUError(st, "rglru_bwd")
+    return g

@@ -183,3 +183,54 @@ int rglru_decode_step(const void *x_t, void *conv_state, int pos, float *h, void
 }
 
 }  // extern "C"
+
+extern "C" {
+
+size_t rglru_bwd_workspace_bytes(int B, int T, int D, int H, int io) {
+  if (check_shape(B, T, D, H, io) != RGLRU_OK) return 0;
+  return bwd_workspace_bytes(B, T, D, H);
+}
+
+int rglru_bwd_launches(int B, int T, int D, int H, int io) {
+  if (check_shape(B, T, D, H, io) != RGLRU_OK) return 0;
+  return bwd_launches();
+}
+
+int rglru_bwd(const void *x, const void *conv_w, const void *W_a, const void *b_a,
+              const void *W_x, const void *b_x, const float *Lambda, const float *h0,
+              const void *conv_state_in, const void *dy, const float *dh_T, void *dx,
+              float *dconv_w, float *dW_a, float *db_a, float *dW_x, float *db_x,
+              float *dLambda, float *dh0, float *dconv_state_in, int B, int T, int D, int H,
+              int io, void *workspace, size_t workspace_bytes, void *stream) {
+  int st = check_shape(B, T, D, H, io);
+  if (st != RGLRU_OK) return st;
+  const void *req[] = {x, conv_w, W_a, b_a, W_x, b_x, Lambda, dy, dx,
+                       dconv_w, dW_a, db_a, dW_x, db_x, dLambda};
+  for (const void *p : req)
+    if (p == nullptr || !aligned16(p)) return RGLRU_ERR_INVALID_ARG;
+  if (!opt_ok(h0) || !opt_ok(conv_state_in) || !opt_ok(dh_T) || !opt_ok(dh0) ||
+      !opt_ok(dconv_state_in))
+    return RGLRU_ERR_INVALID_ARG;
+  const size_t eb = io_bytes(io);
+  const size_t seq = (size_t)B * T * D * eb;
+  const size_t bw = (size_t)D / H;
+  // outputs must not overlap the inputs they are computed from
+  const void *ins[] = {x, dy, conv_w, W_a, W_x};
+  const size_t in_n[] = {seq, seq, 4 * (size_t)D * eb, (size_t)D * bw * eb, (size_t)D * bw * eb};
+  const void *outs[] = {dx, dconv_w, dW_a, dW_x, db_a, db_x, dLambda, dh0, dconv_state_in};
+  const size_t out_n[] = {seq, 16 * (size_t)D, 4 * (size_t)D * bw, 4 * (size_t)D * bw,
+                          4 * (size_t)D, 4 * (size_t)D, 4 * (size_t)D, 4 * (size_t)B * D,
+                          12 * (size_t)B * D};
+  for (int i = 0; i < 5; ++i)
+    for (int o = 0; o < 9; ++o)
+      if (overlap(ins[i], in_n[i], outs[o], out_n[o])) return RGLRU_ERR_INVALID_ARG;
+  const size_t need = bwd_workspace_bytes(B, T, D, H);
+  if (workspace == nullptr || !aligned16(workspace) || workspace_bytes < need)
+    return RGLRU_ERR_WORKSPACE;
+  BwdArgs p{x, conv_w, W_a, b_a, W_x, b_x, Lambda, h0, conv_state_in, dy, dh_T, dx,
+            dconv_w, dW_a, db_a, dW_x, db_x, dLambda, dh0, dconv_state_in, B, T, D, H};
+  const cudaError_t e = launch_bwd(p, io, workspace, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RGLRU_OK : RGLRU_ERR_CUDA;
+}
+
+}  // extern "C"

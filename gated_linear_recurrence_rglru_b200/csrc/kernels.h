@@ -20,6 +20,16 @@ struct FwdArgs {
   cudaEvent_t ev_begin, ev_end;  // recorded around the compute kernels when set
 };
 
+struct BwdArgs {
+  const void *x, *conv_w, *W_a, *b_a, *W_x, *b_x;
+  const float *Lambda, *h0;
+  const void *conv_state_in, *dy;
+  const float *dh_T;
+  void *dx;
+  float *dconv_w, *dW_a, *db_a, *dW_x, *db_x, *dLambda, *dh0, *dconv_state_in;
+  int B, T, D, H;
+};
+
 struct DecArgs {
   const void *x_t;
   void *conv_state;
@@ -39,6 +49,9 @@ struct GenericPlan {
 GenericPlan generic_plan(int B, int T, int H);
 size_t generic_workspace_bytes(int B, int T, int D, int H);
 int generic_kernel_launches(int B, int T, int H);
+size_t bwd_workspace_bytes(int B, int T, int D, int H);
+int bwd_launches();
+cudaError_t launch_bwd(const BwdArgs &p, int io, void *ws, cudaStream_t st);
 cudaError_t launch_fwd_generic(const FwdArgs &p, int io, void *ws, cudaStream_t st);
 cudaError_t launch_decode_generic(const DecArgs &p, int io, cudaStream_t st);
 

@@ -224,6 +224,51 @@ int rglru_decode_step_algo(const void *x_t, void *conv_state, int pos, float *h,
                            const void *W_x, const void *b_x, const float *Lambda, int B,
                            int D, int H, int io, void *stream, int algo);
 
+/*
+ * Backward of the layer (the gradient of a scalar loss through one forward
+ * call). The forward is the layer of "Griffin: Mixing Gated Linear
+ * Recurrences with Local Attention for Efficient Language Models", section
+ * "Model Architecture"; the backward is the chain rule through it: with
+ * dy = dL/dy (B, T, D) and dh_T = dL/dh_T (B, D, or NULL for zeros) it returns
+ * the gradients of L with respect to every forward input, recomputing the
+ * forward from its inputs (nothing is saved between the calls). Time is cut
+ * into segments of at most 512 tokens whose carries run in both time
+ * directions, so the result does not depend on the batch or sequence size
+ * beyond fp32 rounding.
+ *
+ * Inputs (as for rglru_fwd, same dtypes, layouts and alignment): x, conv_w,
+ * W_a, b_a, W_x, b_x, Lambda, h0 (or NULL), conv_state_in (or NULL), and dy
+ * (B, T, D) in the I/O dtype, dh_T fp32 (B, D) or NULL.
+ * Outputs (device memory, caller-owned, not aliasing any input):
+ *   dx              (B, T, D), the I/O dtype
+ *   dconv_w         (4, D) fp32
+ *   dW_a, dW_x      (H, bw, bw) fp32
+ *   db_a, db_x      (D) fp32
+ *   dLambda         (D) fp32
+ *   dh0             (B, D) fp32, or NULL (not computed)
+ *   dconv_state_in  (B, 3, D) fp32 (gradient with respect to the chronological
+ *                   conv history, zeros if conv_state_in is NULL), or NULL
+ * The library zeroes and accumulates the fp32 parameter gradients itself
+ * (the call overwrites them; it does not add to their contents).
+ * workspace: device memory of rglru_bwd_workspace_bytes(B, T, D, H, io) bytes,
+ * 16-byte aligned, not shared with a concurrent call.
+ * Arithmetic is fp32 on CUDA cores for both I/O types; any head width up to
+ * 1024 that divides D. Returns RGLRU_OK, INVALID_ARG (shapes, NULL required
+ * pointers, alignment, overlaps), WORKSPACE or CUDA. Nothing in the backward
+ * waits on another block, so it has no device-side status.
+ */
+size_t rglru_bwd_workspace_bytes(int B, int T, int D, int H, int io);
+
+int rglru_bwd(const void *x, const void *conv_w, const void *W_a, const void *b_a,
+              const void *W_x, const void *b_x, const float *Lambda, const float *h0,
+              const void *conv_state_in, const void *dy, const float *dh_T, void *dx,
+              float *dconv_w, float *dW_a, float *db_a, float *dW_x, float *db_x,
+              float *dLambda, float *dh0, float *dconv_state_in, int B, int T, int D, int H,
+              int io, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Number of kernel launches of one rglru_bwd call (0 on invalid arguments). */
+int rglru_bwd_launches(int B, int T, int D, int H, int io);
+
 #ifdef __cplusplus
 }
 #endif

@@ -106,3 +106,17 @@ def test_options_struct_matches_header():
     body = re.search(r"typedef struct \{([^}]*)\} rglru_fwd_options;", hdr).group(1)
     names = re.findall(r"(\w+)\s*;", body)
     assert names == [f[0] for f in FwdOptions._fields_]
+
+
+def test_bwd_refuses_bad_arguments_before_launch():
+    """rglru_bwd (28 arguments) checks shapes and pointers on the host."""
+    L = _abi.LIB
+    null = [None] * 20
+    # null required pointers
+    assert L.rglru_bwd(*null, 2, 8, 64, 2, 0, None, 0, None) == 1
+    # bad shapes: D not a multiple of H, bad io
+    assert L.rglru_bwd(*null, 2, 8, 65, 2, 0, None, 0, None) == 1
+    assert L.rglru_bwd(*null, 2, 8, 64, 2, 7, None, 0, None) == 1
+    assert L.rglru_bwd_workspace_bytes(2, 8, 64, 2, 0) > 0
+    assert L.rglru_bwd_workspace_bytes(2, 8, 65, 2, 0) == 0
+    assert L.rglru_bwd_launches(2, 8, 64, 2, 1) == 5
