@@ -285,6 +285,8 @@ def run_ours(a, ws, rank, local):
         # e2e of every rank is the same program; report rank-max time via value already local
     if a.decode:
         out["decode"] = run_decode(rg, dev, a, pk)
+    if a.backward:
+        out["backward"] = run_backward(rg, wl, g, w, dev, a, pk)
     if a.cpu_baseline and ws == 1 and rank == 0:
         out["cpu_baseline"] = cpu_baseline(wl, t, a.cpu_seconds)
     return out
@@ -320,6 +322,48 @@ def run_e2e(rg, wl, g, w, dev, a):
     return {"value": B * T * D / (ms / 1e3), "unit": "channel-tokens/s", "ms_per_step": ms,
             "h2d_bytes_per_step": B * T * D * esz, "d2h_bytes_per_step": B * T * D * esz,
             "steps": n}
+
+
+def run_backward(rg, wl, g, w, dev, a, pk):
+    """Backward of the same workload: gradients of <dy, y> + <dh_T, h_T> for every
+    input, one rglru_bwd per step, inputs resident, rotating dy / dx sets."""
+    B, T, D, H = wl.B, wl.T, wl.D, wl.H
+    esz = 4 if wl.io == "f32" else 2
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(wl.seed + 1000)
+    nsets = 3
+    dys = [torch.randn(B, T, D, generator=gen, device=dev).to(wl.dtype) for _ in range(nsets)]
+    dh_T = torch.randn(B, D, generator=gen, device=dev)
+    ws = torch.empty(rg.bwd_workspace_bytes(B, T, D, H, wl.dtype), device=dev, dtype=torch.uint8)
+    outs = [None] * nsets
+
+    def step(i):
+        k = i % nsets
+        outs[k] = rg.rglru_bwd(g["x"], *w, dys[k], h0=g["h0"], dh_T=dh_T, workspace=ws,
+                               out=outs[k])
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    steps = max(5, min(a.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    bytes_step = 3 * esz * B * T * D    # read x and dy, write dx
+    gbs = bytes_step / (ms / 1e3) / 1e9
+    return {"workload": f"{wl.name} backward B={B} T={T} D={D} H={H} io={wl.io}",
+            "value": B * T * D / (ms / 1e3), "unit": "channel-tokens/s", "ms_per_step": ms,
+            "steps": steps, "gpu_launches_per_step": rg.bwd_launches(B, T, D, H, wl.dtype),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                         "algorithmic_bytes_per_launch": bytes_step,
+                         "note": "step time of all five launches; fp32 CUDA-core arithmetic, "
+                                 "16 B per channel-token of fp32 intermediates in a workspace "
+                                 "(not algorithmic)"}}
 
 
 def run_decode(rg, dev, a, pk):
@@ -461,6 +505,7 @@ def main(argv=None):
                          "region, so the clock sampler sees the load")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-decode", dest="decode", action="store_false")
+    ap.add_argument("--no-backward", dest="backward", action="store_false")
     ap.add_argument("--decode-steps", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
