@@ -65,15 +65,37 @@ __device__ __forceinline__ ChanC chan_c(const BwdArgs &p, int d) {
   return c;
 }
 
+// Gate weight (i, jj) of the head: from shared memory (fp32 rows of stride
+// bw + 1, when kSW) or through L1 from global memory.
+template <typename T, bool kSW>
+__device__ __forceinline__ float w_at(const T *W, const float *Ws, int bw, int i, int jj) {
+  return kSW ? Ws[i * (bw + 1) + jj] : ldg_f32(W + (size_t)i * bw + jj);
+}
+
+// Stages both gate weights of the head in shared memory, fp32, rows padded to
+// bw + 1 floats: the gate contraction reads row i across the threads and the
+// transposed one reads row j along a thread, both without bank conflicts.
+template <typename T>
+__device__ __forceinline__ void stage_weights(const T *Wa, const T *Wx, float *Wsa, float *Wsx,
+                                              int bw) {
+  for (int idx = threadIdx.x; idx < bw * bw; idx += blockDim.x) {
+    const int i = idx / bw, jj = idx - (idx / bw) * bw;
+    Wsa[i * (bw + 1) + jj] = ldg_f32(Wa + idx);
+    Wsx[i * (bw + 1) + jj] = ldg_f32(Wx + idx);
+  }
+  __syncthreads();
+}
+
 // One group of kTB tokens from tb (own channel): Conv1D outputs u (the window
 // xm3, xm2, xm1 = x_{tb-3..tb-1} advances), the head's u staged in u_s, then
 // both gate pre-activations through the head's weights. Tokens at or past t1
 // get u = 0 and are not used. Must be reached by every thread of the block.
-template <typename T>
+template <typename T, bool kSW>
 __device__ __forceinline__ void group_preacts(const T *xb, int D, int tb, int t1, int j, int bw,
                                               bool active, int d, const ChanC &c, float &xm3,
                                               float &xm2, float &xm1, float *u_s, const T *Wa,
-                                              const T *Wx, float (&u)[kTB], float (&za)[kTB],
+                                              const T *Wx, const float *Wsa, const float *Wsx,
+                                              float (&u)[kTB], float (&za)[kTB],
                                               float (&zx)[kTB]) {
 #pragma unroll
   for (int k = 0; k < kTB; ++k) {
@@ -97,8 +119,8 @@ __device__ __forceinline__ void group_preacts(const T *xb, int D, int tb, int t1
   }
   if (active) {
     for (int i = 0; i < bw; ++i) {
-      const float wa = ldg_f32(Wa + (size_t)i * bw + j);
-      const float wx = ldg_f32(Wx + (size_t)i * bw + j);
+      const float wa = w_at<T, kSW>(Wa, Wsa, bw, i, j);
+      const float wx = w_at<T, kSW>(Wx, Wsx, bw, i, j);
 #pragma unroll
       for (int k = 0; k < kTB; ++k) {
         const float ui = u_s[k * bw + i];
@@ -110,12 +132,15 @@ __device__ __forceinline__ void group_preacts(const T *xb, int D, int tb, int t1
   __syncthreads();
 }
 
-template <typename T>
+template <typename T, bool kSW>
 __global__ void __launch_bounds__(1024)
 bwd_aggregate_kernel(BwdArgs p, int L, int nseg, float *__restrict__ ws_A,
                      float *__restrict__ ws_H, float *__restrict__ ws_R) {
-  extern __shared__ float u_s[];  // [kTB][bw]
+  extern __shared__ float smem_a[];
   const int bw = p.D / p.H, D = p.D;
+  float *u_s = smem_a;                            // [kTB][bw]
+  float *Wsa = u_s + kTB * bw;                    // [bw][bw + 1] when kSW
+  float *Wsx = Wsa + (kSW ? bw * (bw + 1) : 0);
   const int j = threadIdx.x;
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const bool active = j < bw;
@@ -127,6 +152,7 @@ bwd_aggregate_kernel(BwdArgs p, int L, int nseg, float *__restrict__ ws_A,
   const T *dyb = static_cast<const T *>(p.dy) + (size_t)b * p.T * D;
   const T *Wa = static_cast<const T *>(p.W_a) + (size_t)h * bw * bw;
   const T *Wx = static_cast<const T *>(p.W_x) + (size_t)h * bw * bw;
+  if (kSW) stage_weights<T>(Wa, Wx, Wsa, Wsx, bw);
   ChanC c{0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   float xm3 = 0.f, xm2 = 0.f, xm1 = 0.f;
   if (active) {
@@ -139,7 +165,8 @@ bwd_aggregate_kernel(BwdArgs p, int L, int nseg, float *__restrict__ ws_A,
   float P = 1.f, Hl = 0.f, R = 0.f;
   for (int tb = t0; tb < t1; tb += kTB) {
     float u[kTB], za[kTB], zx[kTB];
-    group_preacts<T>(xb, D, tb, t1, j, bw, active, d, c, xm3, xm2, xm1, u_s, Wa, Wx, u, za, zx);
+    group_preacts<T, kSW>(xb, D, tb, t1, j, bw, active, d, c, xm3, xm2, xm1, u_s, Wa, Wx, Wsa,
+                          Wsx, u, za, zx);
     if (active) {
 #pragma unroll
       for (int k = 0; k < kTB; ++k) {
@@ -184,7 +211,7 @@ __global__ void bwd_carry_kernel(int B, int D, int nseg, const float *__restrict
   if (dh0) dh0[idx] = cc;
 }
 
-template <typename T>
+template <typename T, bool kSW>
 __global__ void __launch_bounds__(1024)
 bwd_final_kernel(BwdArgs p, int L, int nseg, const float *__restrict__ ws_hin,
                  const float *__restrict__ ws_C, float *__restrict__ ws_u,
@@ -195,7 +222,9 @@ bwd_final_kernel(BwdArgs p, int L, int nseg, const float *__restrict__ ws_hin,
   float *u_s = smem;                    // [kTB][bw]
   float *dza_s = u_s + kTB * bw;        // [kTB][bw]
   float *dzx_s = dza_s + kTB * bw;      // [kTB][bw]
-  float *hb_s = dzx_s + kTB * bw;       // [nsub][bw] state at each group start
+  float *Wsa = dzx_s + kTB * bw;        // [bw][bw + 1] when kSW
+  float *Wsx = Wsa + (kSW ? bw * (bw + 1) : 0);
+  float *hb_s = Wsx + (kSW ? bw * (bw + 1) : 0);   // [nsub][bw] state at each group start
   const int j = threadIdx.x;
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const bool active = j < bw;
@@ -209,6 +238,7 @@ bwd_final_kernel(BwdArgs p, int L, int nseg, const float *__restrict__ ws_hin,
   const T *Wa = static_cast<const T *>(p.W_a) + (size_t)h * bw * bw;
   const T *Wx = static_cast<const T *>(p.W_x) + (size_t)h * bw * bw;
   const size_t seg = ((size_t)b * nseg + s) * D + d;
+  if (kSW) stage_weights<T>(Wa, Wx, Wsa, Wsx, bw);
   ChanC c{0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (active) c = chan_c<T>(p, d);
   const float neg_c_sp = -kDecayC * c.sp;
@@ -225,7 +255,8 @@ bwd_final_kernel(BwdArgs p, int L, int nseg, const float *__restrict__ ws_hin,
     const int tb = t0 + g * kTB;
     if (active) hb_s[g * bw + j] = hcur;
     float u[kTB], za[kTB], zx[kTB];
-    group_preacts<T>(xb, D, tb, t1, j, bw, active, d, c, xm3, xm2, xm1, u_s, Wa, Wx, u, za, zx);
+    group_preacts<T, kSW>(xb, D, tb, t1, j, bw, active, d, c, xm3, xm2, xm1, u_s, Wa, Wx, Wsa,
+                          Wsx, u, za, zx);
     if (active) {
 #pragma unroll
       for (int k = 0; k < kTB; ++k) {
@@ -251,7 +282,8 @@ bwd_final_kernel(BwdArgs p, int L, int nseg, const float *__restrict__ ws_hin,
       w1 = hist_x(xb, cs_in_b, tb - 1, D, d);
     }
     float u[kTB], za[kTB], zx[kTB];
-    group_preacts<T>(xb, D, tb, t1, j, bw, active, d, c, w3, w2, w1, u_s, Wa, Wx, u, za, zx);
+    group_preacts<T, kSW>(xb, D, tb, t1, j, bw, active, d, c, w3, w2, w1, u_s, Wa, Wx, Wsa, Wsx,
+                          u, za, zx);
     float du_own[kTB];
     if (active) {
       float a[kTB], r[kTB], ig[kTB], gg[kTB], hp[kTB];
@@ -301,8 +333,8 @@ bwd_final_kernel(BwdArgs p, int L, int nseg, const float *__restrict__ ws_hin,
 #pragma unroll
       for (int k = 0; k < kTB; ++k) acc[k] = du_own[k];
       for (int m = 0; m < bw; ++m) {
-        const float wa = ldg_f32(Wa + (size_t)j * bw + m);
-        const float wx = ldg_f32(Wx + (size_t)j * bw + m);
+        const float wa = w_at<T, kSW>(Wa, Wsa, bw, j, m);
+        const float wx = w_at<T, kSW>(Wx, Wsx, bw, j, m);
 #pragma unroll
         for (int k = 0; k < kTB; ++k)
           acc[k] = fmaf(dza_s[k * bw + m], wa, fmaf(dzx_s[k * bw + m], wx, acc[k]));
@@ -444,7 +476,7 @@ BwdLayout bwd_layout(int B, int T, int D, int H) {
   return L;
 }
 
-template <typename T>
+template <typename T, bool kSW>
 cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
   const int bw = p.D / p.H;
   const BwdPlan pl = bwd_plan(p.B, p.T, p.H);
@@ -468,24 +500,28 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
 
   const int threads = ceil_div(bw, 32) * 32;
   const dim3 grid(pl.nseg, p.H, p.B);
-  const size_t smem1 = (size_t)kTB * bw * sizeof(float);
+  const size_t wsm = kSW ? 2 * (size_t)bw * (bw + 1) * sizeof(float) : 0;
+  const size_t smem1 = (size_t)kTB * bw * sizeof(float) + wsm;
   const int nsub_max = ceil_div(pl.L, kTB);
-  const size_t smem3 = (size_t)(3 * kTB + nsub_max) * bw * sizeof(float);
+  const size_t smem3 = (size_t)(3 * kTB + nsub_max) * bw * sizeof(float) + wsm;
   if (smem1 > 48 * 1024 &&
-      (e = cudaFuncSetAttribute(bwd_aggregate_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem1)) != cudaSuccess)
+      (e = cudaFuncSetAttribute(bwd_aggregate_kernel<T, kSW>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1)) !=
+          cudaSuccess)
     return e;
   if (smem3 > 48 * 1024 &&
-      (e = cudaFuncSetAttribute(bwd_final_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem3)) != cudaSuccess)
+      (e = cudaFuncSetAttribute(bwd_final_kernel<T, kSW>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3)) !=
+          cudaSuccess)
     return e;
-  bwd_aggregate_kernel<T><<<grid, threads, smem1, st>>>(p, pl.L, pl.nseg, A, Hh, R);
+  bwd_aggregate_kernel<T, kSW><<<grid, threads, smem1, st>>>(p, pl.L, pl.nseg, A, Hh, R);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int bd = p.B * p.D;
   bwd_carry_kernel<<<ceil_div(bd, 256), 256, 0, st>>>(p.B, p.D, pl.nseg, A, Hh, R, p.h0, p.dh_T,
                                                       hin, C, p.dh0);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  bwd_final_kernel<T><<<grid, threads, smem3, st>>>(p, pl.L, pl.nseg, hin, C, U, dza, dzx, du);
+  bwd_final_kernel<T, kSW><<<grid, threads, smem3, st>>>(p, pl.L, pl.nseg, hin, C, U, dza, dzx,
+                                                          du);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int N = p.B * p.T;
   const int tiles = ceil_div(bw, 32);
@@ -506,8 +542,12 @@ size_t bwd_workspace_bytes(int B, int T, int D, int H) { return bwd_layout(B, T,
 int bwd_launches() { return 5; }
 
 cudaError_t launch_bwd(const BwdArgs &p, int io, void *ws, cudaStream_t st) {
-  if (io == RGLRU_IO_F32) return launch_bwd_t<float>(p, ws, st);
-  return launch_bwd_t<__nv_bfloat16>(p, ws, st);
+  // both gate weights in shared memory (fp32) up to 128-wide heads: 2 x 129 x 128 x 4 B
+  const bool sw = p.D / p.H <= 128;
+  if (io == RGLRU_IO_F32)
+    return sw ? launch_bwd_t<float, true>(p, ws, st) : launch_bwd_t<float, false>(p, ws, st);
+  return sw ? launch_bwd_t<__nv_bfloat16, true>(p, ws, st)
+            : launch_bwd_t<__nv_bfloat16, false>(p, ws, st);
 }
 
 }  // namespace rglru
