@@ -5,26 +5,33 @@
 // linear scans in both time directions, the forward's scheme in S. De's
 // thread). fp32 arithmetic on CUDA cores for any I/O type.
 //
-// Time is cut into segments of at most kMaxSeg tokens; one block per
-// (segment, head, batch row), thread j owning channel h*bw + j:
-//   K1 aggregate  per segment: A = prod a_t, H = local state from zero and
-//                 R = sum_t P_t dy_t with P_t = a_t0 ... a_t (the segment's
-//                 contribution to the state gradient that leaves it leftwards);
+// Time is cut into segments of L tokens (L a multiple of the 8-token group);
+// a block holds S segments of one head and batch row, thread (sl, j) owning
+// channel h*bw + j of segment sl, with the head's gate weights staged once in
+// shared memory for all of them:
+//   K1 gates      per segment, in time order: Conv1D u, both gate
+//                 pre-activations (z_a, z_x -> fp32 workspace), the local scan
+//                 from zero, whose (prod a, state) at each group start also go
+//                 to the workspace, and the aggregates A = prod a_t,
+//                 H = local end state and R = sum_t P_t dy_t with
+//                 P_t = a_t0 ... a_t (the segment's contribution to the state
+//                 gradient that leaves it leftwards);
 //   K2 carry      per (b, channel): h_in of each segment in time order from h0,
 //                 and C_s, the state gradient entering segment s from the right
 //                 (dh_T for the last), in reverse order: C_{s-1} = R_s + A_s C_s,
 //                 dh0 = R_0 + A_0 C_0;
-//   K3 final      per segment: a forward sweep from h_in keeps the state at every
-//                 8-token boundary in shared memory; a reverse sweep over the
-//                 8-token groups recomputes each group (conv, gates), rebuilds
-//                 h_{t-1}, runs G_t = dy_t + a_{t+1} G_{t+1} from C_s and forms
-//                 d a = G h_{t-1}, d beta = G, g = sqrt(1 - a^2),
-//                 d g = G i u, d i = G g u, d u = G g i + d z_a W_a^T + d z_x W_x^T,
+//   K3 final      per segment, groups in reverse order: the group's start state
+//                 (prod a) h_in + (local state) and its stored z_a, z_x give
+//                 h_{t-1}, a and beta for its 8 tokens; then G_t = dy_t +
+//                 a_{t+1} G_{t+1} from C_s and d a = G h_{t-1}, d beta = G,
+//                 g = sqrt(1 - a^2), d g = G i u, d i = G g u,
+//                 d u = G g i + d z_a W_a^T + d z_x W_x^T,
 //                 d la = d a a - d g a^2 / g, la = -c r sp, z -> r, i by sigmoid;
 //                 it accumulates d b_a, d b_x and d Lambda per channel and writes
-//                 u, d z_a, d z_x and d u to an fp32 workspace;
-//   K4 weights    d W[h] = U_h^T dZ_h for both gates (32 x 32 tiles, the token
-//                 sum split over blocks and combined with atomics);
+//                 u, d z_a, d z_x (over z_a, z_x) and d u to the workspace;
+//   K4 weights    d W[h] = U_h^T dZ_h for both gates (64 x 64 tiles, 4 x 4 per
+//                 thread, the token sum split over blocks and combined with
+//                 atomics);
 //   K5 conv       d x_t = sum_k w[k] d u_{t+3-k} (t < 0: the conv history's
 //                 gradient) and d w[k] = sum_t x_{t-3+k} d u_t.
 // The path of d z_a through g carries r / g, which tends to 0 with r
@@ -36,8 +43,36 @@ namespace rglru {
 
 namespace {
 
-constexpr int kTB = 8;         // tokens per group
-constexpr int kMaxSeg = 512;   // tokens per segment: at most 64 boundary states per channel
+constexpr int kTB = 8;       // tokens per group
+constexpr int kRow = 12;     // floats per (channel, group) row in shared memory: 8 tokens and
+                             // 4 pad, so 8 consecutive rows start on distinct 16-byte bank groups
+constexpr int kMinSeg = 32;  // shortest segment the plan makes (unless T is shorter)
+// threads the plan aims for: about four waves of 1024 threads on 148 SMs (any
+// SM count works; the figure only sets the segment length)
+constexpr long kTargetThreads = 4L * 148 * 1024;
+
+struct BwdPlan {
+  int L;      // tokens per segment, a multiple of kTB (the last segment may be shorter)
+  int nseg;   // segments per sequence
+  int S;      // segments per block
+  int bwp;    // threads per segment: bw rounded up to a warp
+};
+
+BwdPlan bwd_plan(int B, int T, int D, int H) {
+  const int bw = D / H;
+  BwdPlan pl;
+  pl.bwp = ceil_div(bw, 32) * 32;
+  pl.S = (bw <= 64 ? 256 : 512) / pl.bwp;
+  if (pl.S < 1) pl.S = 1;
+  const long chans = (long)B * D;
+  long nseg = (kTargetThreads + chans - 1) / chans;
+  const long max_seg = ceil_div(T, kMinSeg);
+  if (nseg > max_seg) nseg = max_seg;
+  if (nseg < 1) nseg = 1;
+  pl.L = ceil_div(ceil_div(T, (int)nseg), kTB) * kTB;
+  pl.nseg = ceil_div(T, pl.L);
+  return pl;
+}
 
 template <typename T>
 __device__ __forceinline__ float hist_x(const T *xb, const T *cs_in_b, int t, int D, int d) {
@@ -65,6 +100,25 @@ __device__ __forceinline__ ChanC chan_c(const BwdArgs &p, int d) {
   return c;
 }
 
+// Conv1D outputs of channel d for the group of kTB tokens from tb; tokens at
+// or past t1 give 0.
+template <typename T>
+__device__ __forceinline__ void conv_group(const T *xb, const T *cs_in_b, int D, int d, int tb,
+                                           int t1, const ChanC &c, float (&u)[kTB]) {
+  float xm3 = hist_x(xb, cs_in_b, tb - 3, D, d);
+  float xm2 = hist_x(xb, cs_in_b, tb - 2, D, d);
+  float xm1 = hist_x(xb, cs_in_b, tb - 1, D, d);
+#pragma unroll
+  for (int k = 0; k < kTB; ++k) {
+    const int t = tb + k;
+    const float xv = t < t1 ? ldg_f32(xb + (size_t)t * D + d) : 0.f;
+    u[k] = t < t1 ? fmaf(c.w3, xv, fmaf(c.w2, xm1, fmaf(c.w1, xm2, c.w0 * xm3))) : 0.f;
+    xm3 = xm2;
+    xm2 = xm1;
+    xm1 = xv;
+  }
+}
+
 // Gate weight (i, jj) of the head: from shared memory (fp32 rows of stride
 // bw + 1, when kSW) or through L1 from global memory.
 template <typename T, bool kSW>
@@ -86,66 +140,43 @@ __device__ __forceinline__ void stage_weights(const T *Wa, const T *Wx, float *W
   __syncthreads();
 }
 
-// One group of kTB tokens from tb (own channel): Conv1D outputs u (the window
-// xm3, xm2, xm1 = x_{tb-3..tb-1} advances), the head's u staged in u_s, then
-// both gate pre-activations through the head's weights. Tokens at or past t1
-// get u = 0 and are not used. Must be reached by every thread of the block.
-template <typename T, bool kSW>
-__device__ __forceinline__ void group_preacts(const T *xb, int D, int tb, int t1, int j, int bw,
-                                              bool active, int d, const ChanC &c, float &xm3,
-                                              float &xm2, float &xm1, float *u_s, const T *Wa,
-                                              const T *Wx, const float *Wsa, const float *Wsx,
-                                              float (&u)[kTB], float (&za)[kTB],
-                                              float (&zx)[kTB]) {
-#pragma unroll
-  for (int k = 0; k < kTB; ++k) {
-    const int t = tb + k;
-    float uv = 0.f;
-    if (active && t < t1) {
-      const float xv = ldg_f32(xb + (size_t)t * D + d);
-      uv = fmaf(c.w3, xv, fmaf(c.w2, xm1, fmaf(c.w1, xm2, c.w0 * xm3)));
-      xm3 = xm2;
-      xm2 = xm1;
-      xm1 = xv;
-    }
-    u[k] = uv;
-    if (active) u_s[k * bw + j] = uv;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int k = 0; k < kTB; ++k) {
-    za[k] = c.ba;
-    zx[k] = c.bx;
-  }
-  if (active) {
-    for (int i = 0; i < bw; ++i) {
-      const float wa = w_at<T, kSW>(Wa, Wsa, bw, i, j);
-      const float wx = w_at<T, kSW>(Wx, Wsx, bw, i, j);
-#pragma unroll
-      for (int k = 0; k < kTB; ++k) {
-        const float ui = u_s[k * bw + i];
-        za[k] = fmaf(ui, wa, za[k]);
-        zx[k] = fmaf(ui, wx, zx[k]);
-      }
-    }
-  }
-  __syncthreads();
+__device__ __forceinline__ void store_row(float *row, const float (&v)[kTB]) {
+  reinterpret_cast<float4 *>(row)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4 *>(row)[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
 
-template <typename T, bool kSW>
-__global__ void __launch_bounds__(1024)
-bwd_aggregate_kernel(BwdArgs p, int L, int nseg, float *__restrict__ ws_A,
-                     float *__restrict__ ws_H, float *__restrict__ ws_R) {
-  extern __shared__ float smem_a[];
-  const int bw = p.D / p.H, D = p.D;
-  float *u_s = smem_a;                            // [kTB][bw]
-  float *Wsa = u_s + kTB * bw;                    // [bw][bw + 1] when kSW
+// One (segment, channel) thread of a block. Threads of segments past the end,
+// and the pad threads of a head narrower than its warps, are inactive but
+// take every barrier.
+struct BwdThread {
+  int sl, j, s, d, t0, t1;
+  bool active;
+};
+
+__device__ __forceinline__ BwdThread bwd_thread(const BwdArgs &p, const BwdPlan &pl, int bw) {
+  BwdThread th;
+  th.sl = threadIdx.x / pl.bwp;
+  th.j = threadIdx.x - th.sl * pl.bwp;
+  th.s = blockIdx.x * pl.S + th.sl;
+  th.t0 = min(p.T, th.s * pl.L);
+  th.t1 = min(p.T, th.t0 + pl.L);
+  th.active = th.j < bw && th.t0 < th.t1;
+  th.d = blockIdx.y * bw + (th.j < bw ? th.j : 0);
+  return th;
+}
+
+template <typename T, bool kSW, int kMaxT>
+__global__ void __launch_bounds__(kMaxT, kMaxT == 256 ? 3 : 1)
+bwd_gates_kernel(BwdArgs p, BwdPlan pl, float *__restrict__ ws_A, float *__restrict__ ws_H,
+                 float *__restrict__ ws_R, float *__restrict__ ws_gP, float *__restrict__ ws_gH,
+                 float *__restrict__ ws_za, float *__restrict__ ws_zx) {
+  extern __shared__ float4 smem_g[];
+  const int bw = p.D / p.H, D = p.D, h = blockIdx.y, b = blockIdx.z;
+  const int seg_floats = pl.S * bw * kRow;
+  float *u_s = reinterpret_cast<float *>(smem_g);   // [2][S][bw][kRow], double-buffered
+  float *Wsa = u_s + 2 * seg_floats;                // [bw][bw + 1] when kSW
   float *Wsx = Wsa + (kSW ? bw * (bw + 1) : 0);
-  const int j = threadIdx.x;
-  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const bool active = j < bw;
-  const int d = h * bw + (active ? j : 0);
-  const int t0 = s * L, t1 = min(p.T, t0 + L);
+  const BwdThread th = bwd_thread(p, pl, bw);
   const T *xb = static_cast<const T *>(p.x) + (size_t)b * p.T * D;
   const T *cs_in_b =
       p.conv_state_in ? static_cast<const T *>(p.conv_state_in) + (size_t)b * 3 * D : nullptr;
@@ -154,35 +185,67 @@ bwd_aggregate_kernel(BwdArgs p, int L, int nseg, float *__restrict__ ws_A,
   const T *Wx = static_cast<const T *>(p.W_x) + (size_t)h * bw * bw;
   if (kSW) stage_weights<T>(Wa, Wx, Wsa, Wsx, bw);
   ChanC c{0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  float xm3 = 0.f, xm2 = 0.f, xm1 = 0.f;
-  if (active) {
-    c = chan_c<T>(p, d);
-    xm3 = hist_x(xb, cs_in_b, t0 - 3, D, d);
-    xm2 = hist_x(xb, cs_in_b, t0 - 2, D, d);
-    xm1 = hist_x(xb, cs_in_b, t0 - 1, D, d);
-  }
+  if (th.active) c = chan_c<T>(p, th.d);
   const float neg_c_sp = -kDecayC * c.sp;
+  const int ngt = ceil_div(p.T, kTB);
+  const int jr = th.j < bw ? th.j : 0;
   float P = 1.f, Hl = 0.f, R = 0.f;
-  for (int tb = t0; tb < t1; tb += kTB) {
-    float u[kTB], za[kTB], zx[kTB];
-    group_preacts<T, kSW>(xb, D, tb, t1, j, bw, active, d, c, xm3, xm2, xm1, u_s, Wa, Wx, Wsa,
-                          Wsx, u, za, zx);
-    if (active) {
+  const int ng = pl.L / kTB;
+  for (int g = 0; g < ng; ++g) {
+    const int tb = th.t0 + g * kTB;
+    const bool live = th.active && tb < th.t1;
+    const float *useg = u_s + (g & 1) * seg_floats + th.sl * bw * kRow;
+    float u[kTB];
+    if (live) {
+      const size_t go = ((size_t)b * ngt + tb / kTB) * D + th.d;
+      ws_gP[go] = P;
+      ws_gH[go] = Hl;
+      conv_group<T>(xb, cs_in_b, D, th.d, tb, th.t1, c, u);
+    } else {
+#pragma unroll
+      for (int k = 0; k < kTB; ++k) u[k] = 0.f;
+    }
+    if (th.j < bw) store_row(const_cast<float *>(useg) + jr * kRow, u);
+    __syncthreads();
+    if (live) {
+      float za[kTB], zx[kTB];
+#pragma unroll
+      for (int k = 0; k < kTB; ++k) {
+        za[k] = c.ba;
+        zx[k] = c.bx;
+      }
+      // z_j = b_j + sum_i u_i W[i, j]: the 8 tokens of u_i in two 16-byte reads
+#pragma unroll 8
+      for (int i = 0; i < bw; ++i) {
+        const float4 u0 = reinterpret_cast<const float4 *>(useg + i * kRow)[0];
+        const float4 u1 = reinterpret_cast<const float4 *>(useg + i * kRow)[1];
+        const float wa = w_at<T, kSW>(Wa, Wsa, bw, i, th.j);
+        const float wx = w_at<T, kSW>(Wx, Wsx, bw, i, th.j);
+        const float uv[kTB] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+        for (int k = 0; k < kTB; ++k) {
+          za[k] = fmaf(uv[k], wa, za[k]);
+          zx[k] = fmaf(uv[k], wx, zx[k]);
+        }
+      }
 #pragma unroll
       for (int k = 0; k < kTB; ++k) {
         const int t = tb + k;
-        if (t < t1) {
+        if (t < th.t1) {
           float a, beta, la;
           decay_and_input(za[k], zx[k], u[k], neg_c_sp, a, beta, la);
           Hl = fmaf(a, Hl, beta);
           P *= a;
-          R = fmaf(P, ldg_f32(dyb + (size_t)t * D + d), R);
+          R = fmaf(P, ldg_f32(dyb + (size_t)t * D + th.d), R);
+          const size_t o = ((size_t)b * p.T + t) * D + th.d;
+          ws_za[o] = za[k];
+          ws_zx[o] = zx[k];
         }
       }
     }
   }
-  if (!active) return;
-  const size_t o = ((size_t)b * nseg + s) * D + d;
+  if (!th.active) return;
+  const size_t o = ((size_t)b * pl.nseg + th.s) * D + th.d;
   ws_A[o] = P;
   ws_H[o] = Hl;
   ws_R[o] = R;
@@ -197,12 +260,14 @@ __global__ void bwd_carry_kernel(int B, int D, int nseg, const float *__restrict
   if (idx >= B * D) return;
   const int b = idx / D, d = idx - (idx / D) * D;
   float hh = h0 ? h0[idx] : 0.f;
+#pragma unroll 8
   for (int s = 0; s < nseg; ++s) {
     const size_t o = ((size_t)b * nseg + s) * D + d;
     ws_hin[o] = hh;
     hh = fmaf(ws_A[o], hh, ws_H[o]);
   }
   float cc = dh_T ? dh_T[idx] : 0.f;
+#pragma unroll 8
   for (int s = nseg - 1; s >= 0; --s) {
     const size_t o = ((size_t)b * nseg + s) * D + d;
     ws_C[o] = cc;
@@ -211,87 +276,62 @@ __global__ void bwd_carry_kernel(int B, int D, int nseg, const float *__restrict
   if (dh0) dh0[idx] = cc;
 }
 
-template <typename T, bool kSW>
-__global__ void __launch_bounds__(1024)
-bwd_final_kernel(BwdArgs p, int L, int nseg, const float *__restrict__ ws_hin,
-                 const float *__restrict__ ws_C, float *__restrict__ ws_u,
-                 float *__restrict__ ws_dza, float *__restrict__ ws_dzx,
+template <typename T, bool kSW, int kMaxT>
+__global__ void __launch_bounds__(kMaxT, kMaxT == 256 ? 3 : 1)
+bwd_final_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
+                 const float *__restrict__ ws_C, const float *__restrict__ ws_gP,
+                 const float *__restrict__ ws_gH, float *__restrict__ ws_za,
+                 float *__restrict__ ws_zx, float *__restrict__ ws_u,
                  float *__restrict__ ws_du) {
-  extern __shared__ float smem[];
-  const int bw = p.D / p.H, D = p.D;
-  float *u_s = smem;                    // [kTB][bw]
-  float *dza_s = u_s + kTB * bw;        // [kTB][bw]
-  float *dzx_s = dza_s + kTB * bw;      // [kTB][bw]
-  float *Wsa = dzx_s + kTB * bw;        // [bw][bw + 1] when kSW
+  extern __shared__ float4 smem_f[];
+  const int bw = p.D / p.H, D = p.D, h = blockIdx.y, b = blockIdx.z;
+  float *dz_s = reinterpret_cast<float *>(smem_f);   // [S][2][bw][kRow]: d z_a, d z_x rows
+  float *Wsa = dz_s + 2 * pl.S * bw * kRow;          // [bw][bw + 1] when kSW
   float *Wsx = Wsa + (kSW ? bw * (bw + 1) : 0);
-  float *hb_s = Wsx + (kSW ? bw * (bw + 1) : 0);   // [nsub][bw] state at each group start
-  const int j = threadIdx.x;
-  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const bool active = j < bw;
-  const int d = h * bw + (active ? j : 0);
-  const int t0 = s * L, t1 = min(p.T, t0 + L);
-  const int nsub = (t1 - t0 + kTB - 1) / kTB;
+  const BwdThread th = bwd_thread(p, pl, bw);
   const T *xb = static_cast<const T *>(p.x) + (size_t)b * p.T * D;
   const T *cs_in_b =
       p.conv_state_in ? static_cast<const T *>(p.conv_state_in) + (size_t)b * 3 * D : nullptr;
   const T *dyb = static_cast<const T *>(p.dy) + (size_t)b * p.T * D;
   const T *Wa = static_cast<const T *>(p.W_a) + (size_t)h * bw * bw;
   const T *Wx = static_cast<const T *>(p.W_x) + (size_t)h * bw * bw;
-  const size_t seg = ((size_t)b * nseg + s) * D + d;
   if (kSW) stage_weights<T>(Wa, Wx, Wsa, Wsx, bw);
   ChanC c{0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  if (active) c = chan_c<T>(p, d);
-  const float neg_c_sp = -kDecayC * c.sp;
-
-  // ---- forward sweep: the state at every group start ----
-  float xm3 = 0.f, xm2 = 0.f, xm1 = 0.f, hcur = 0.f;
-  if (active) {
-    xm3 = hist_x(xb, cs_in_b, t0 - 3, D, d);
-    xm2 = hist_x(xb, cs_in_b, t0 - 2, D, d);
-    xm1 = hist_x(xb, cs_in_b, t0 - 1, D, d);
-    hcur = ws_hin[seg];
+  float h_in = 0.f, gc = 0.f;   // gc: a_{t+1} G_{t+1} for the token being processed
+  if (th.active) {
+    c = chan_c<T>(p, th.d);
+    const size_t seg = ((size_t)b * pl.nseg + th.s) * D + th.d;
+    h_in = ws_hin[seg];
+    gc = ws_C[seg];
   }
-  for (int g = 0; g < nsub; ++g) {
-    const int tb = t0 + g * kTB;
-    if (active) hb_s[g * bw + j] = hcur;
-    float u[kTB], za[kTB], zx[kTB];
-    group_preacts<T, kSW>(xb, D, tb, t1, j, bw, active, d, c, xm3, xm2, xm1, u_s, Wa, Wx, Wsa,
-                          Wsx, u, za, zx);
-    if (active) {
-#pragma unroll
-      for (int k = 0; k < kTB; ++k) {
-        if (tb + k < t1) {
-          float a, beta, la;
-          decay_and_input(za[k], zx[k], u[k], neg_c_sp, a, beta, la);
-          hcur = fmaf(a, hcur, beta);
-        }
-      }
-    }
-  }
-
-  // ---- reverse sweep over the groups ----
-  float gc = active ? ws_C[seg] : 0.f;   // a_{t+1} G_{t+1} for the token being processed
+  const float neg_c_sp = -kDecayC * c.sp, csp = kDecayC * c.sp;
+  const int ngt = ceil_div(p.T, kTB);
+  const int jr = th.j < bw ? th.j : 0;
+  float *dza_row = dz_s + ((th.sl * 2 + 0) * bw + jr) * kRow;
+  float *dzx_row = dz_s + ((th.sl * 2 + 1) * bw + jr) * kRow;
+  const float *dza_seg = dz_s + (th.sl * 2 + 0) * bw * kRow;
+  const float *dzx_seg = dz_s + (th.sl * 2 + 1) * bw * kRow;
   float acc_sp = 0.f, acc_ba = 0.f, acc_bx = 0.f;
-  const float csp = kDecayC * c.sp;
-  for (int g = nsub - 1; g >= 0; --g) {
-    const int tb = t0 + g * kTB;
-    float w3 = 0.f, w2 = 0.f, w1 = 0.f;
-    if (active) {
-      w3 = hist_x(xb, cs_in_b, tb - 3, D, d);
-      w2 = hist_x(xb, cs_in_b, tb - 2, D, d);
-      w1 = hist_x(xb, cs_in_b, tb - 1, D, d);
-    }
-    float u[kTB], za[kTB], zx[kTB];
-    group_preacts<T, kSW>(xb, D, tb, t1, j, bw, active, d, c, w3, w2, w1, u_s, Wa, Wx, Wsa, Wsx,
-                          u, za, zx);
-    float du_own[kTB];
-    if (active) {
+  for (int g = pl.L / kTB - 1; g >= 0; --g) {
+    const int tb = th.t0 + g * kTB;
+    const bool live = th.active && tb < th.t1;
+    float dub[kTB];
+#pragma unroll
+    for (int k = 0; k < kTB; ++k) dub[k] = 0.f;
+    if (live) {
+      float u[kTB];
+      conv_group<T>(xb, cs_in_b, D, th.d, tb, th.t1, c, u);
       float a[kTB], r[kTB], ig[kTB], gg[kTB], hp[kTB];
-      float hh = hb_s[g * bw + j];
+      const size_t go = ((size_t)b * ngt + tb / kTB) * D + th.d;
+      float hh = fmaf(ws_gP[go], h_in, ws_gH[go]);
 #pragma unroll
       for (int k = 0; k < kTB; ++k) {
-        r[k] = sigmoid_f32(za[k]);
-        ig[k] = sigmoid_f32(zx[k]);
+        const int t = tb + k;
+        const size_t o = ((size_t)b * p.T + t) * D + th.d;
+        const float za = t < th.t1 ? ws_za[o] : 0.f;
+        const float zx = t < th.t1 ? ws_zx[o] : 0.f;
+        r[k] = sigmoid_f32(za);
+        ig[k] = sigmoid_f32(zx);
         const float la = neg_c_sp * r[k];
         a[k] = expf(la);
         gg[k] = sqrtf(-expm1f(2.0f * la));
@@ -301,13 +341,13 @@ bwd_final_kernel(BwdArgs p, int L, int nseg, const float *__restrict__ ws_hin,
 #pragma unroll
       for (int k = kTB - 1; k >= 0; --k) {
         const int t = tb + k;
-        float dza = 0.f, dzx = 0.f, dub = 0.f;
-        if (t < t1) {
-          const float G = ldg_f32(dyb + (size_t)t * D + d) + gc;
+        float dza = 0.f, dzx = 0.f;
+        if (t < th.t1) {
+          const float G = ldg_f32(dyb + (size_t)t * D + th.d) + gc;
           const float da = G * hp[k];
           const float dg = G * ig[k] * u[k];
           const float di = G * gg[k] * u[k];
-          dub = G * gg[k] * ig[k];
+          dub[k] = G * gg[k] * ig[k];
           const float rog = gg[k] > 0.f ? r[k] / gg[k] : 0.f;
           const float aa = a[k] * a[k];
           dza = -csp * da * a[k] * r[k] * (1.f - r[k]) + csp * aa * (1.f - r[k]) * dg * rog;
@@ -316,151 +356,162 @@ bwd_final_kernel(BwdArgs p, int L, int nseg, const float *__restrict__ ws_hin,
           acc_ba += dza;
           acc_bx += dzx;
           gc = a[k] * G;
-          const size_t o = ((size_t)b * p.T + t) * D + d;
+          const size_t o = ((size_t)b * p.T + t) * D + th.d;
           ws_u[o] = u[k];
-          ws_dza[o] = dza;
-          ws_dzx[o] = dzx;
+          ws_za[o] = dza;
+          ws_zx[o] = dzx;
         }
-        dza_s[k * bw + j] = dza;
-        dzx_s[k * bw + j] = dzx;
-        du_own[k] = dub;
+        dza_row[k] = dza;
+        dzx_row[k] = dzx;
       }
+    } else if (th.j < bw) {
+      store_row(dza_row, dub);   // zeros
+      store_row(dzx_row, dub);
     }
     __syncthreads();
-    if (active) {
+    if (live) {
       // d u_j += sum_m d z_a[m] W_a[j, m] + d z_x[m] W_x[j, m]
-      float acc[kTB];
-#pragma unroll
-      for (int k = 0; k < kTB; ++k) acc[k] = du_own[k];
+#pragma unroll 8
       for (int m = 0; m < bw; ++m) {
-        const float wa = w_at<T, kSW>(Wa, Wsa, bw, j, m);
-        const float wx = w_at<T, kSW>(Wx, Wsx, bw, j, m);
+        const float4 a0 = reinterpret_cast<const float4 *>(dza_seg + m * kRow)[0];
+        const float4 a1 = reinterpret_cast<const float4 *>(dza_seg + m * kRow)[1];
+        const float4 x0 = reinterpret_cast<const float4 *>(dzx_seg + m * kRow)[0];
+        const float4 x1 = reinterpret_cast<const float4 *>(dzx_seg + m * kRow)[1];
+        const float wa = w_at<T, kSW>(Wa, Wsa, bw, th.j, m);
+        const float wx = w_at<T, kSW>(Wx, Wsx, bw, th.j, m);
+        const float av[kTB] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float xv[kTB] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
-        for (int k = 0; k < kTB; ++k)
-          acc[k] = fmaf(dza_s[k * bw + m], wa, fmaf(dzx_s[k * bw + m], wx, acc[k]));
+        for (int k = 0; k < kTB; ++k) dub[k] = fmaf(av[k], wa, fmaf(xv[k], wx, dub[k]));
       }
 #pragma unroll
       for (int k = 0; k < kTB; ++k)
-        if (tb + k < t1) ws_du[((size_t)b * p.T + tb + k) * D + d] = acc[k];
+        if (tb + k < th.t1) ws_du[((size_t)b * p.T + tb + k) * D + th.d] = dub[k];
     }
     __syncthreads();
   }
-  if (!active) return;
-  atomicAdd(p.dLambda + d, acc_sp * (-sigmoid_f32(-__ldg(p.Lambda + d))));
-  atomicAdd(p.db_a + d, acc_ba);
-  atomicAdd(p.db_x + d, acc_bx);
+  if (!th.active) return;
+  atomicAdd(p.dLambda + th.d, acc_sp * (-sigmoid_f32(-__ldg(p.Lambda + th.d))));
+  atomicAdd(p.db_a + th.d, acc_ba);
+  atomicAdd(p.db_x + th.d, acc_bx);
 }
 
 // d W[h, i, j] += sum_n U[n, h bw + i] dZ[n, h bw + j] over one chunk of
-// tokens; a 32 x 32 tile of (i, j) per block, 8 rows of threads.
-__global__ void __launch_bounds__(256)
+// tokens: a 64 x 64 tile of (i, j) of one gate and head per block, 4 x 4 per
+// thread, 32 tokens of both operands staged in shared memory at a time.
+constexpr int kDwTile = 64, kDwRows = 32, kDwThreads = 256;
+
+__global__ void __launch_bounds__(kDwThreads)
 bwd_dw_kernel(const float *__restrict__ U, const float *__restrict__ dZa,
               const float *__restrict__ dZx, float *__restrict__ dWa, float *__restrict__ dWx,
               int N, int D, int H, int chunk) {
-  __shared__ float us[32][33];
-  __shared__ float zs[32][33];
+  __shared__ __align__(16) float us[kDwRows][kDwTile];
+  __shared__ __align__(16) float zs[kDwRows][kDwTile];
   const int bw = D / H;
-  const int tiles = (bw + 31) / 32;
+  const int tiles = ceil_div(bw, kDwTile);
   int tile = blockIdx.x;
-  const int gate = tile % 2;
-  tile /= 2;
+  const int gate = tile & 1;
+  tile >>= 1;
   const int ti = tile % tiles, tj = (tile / tiles) % tiles, h = tile / (tiles * tiles);
   const float *Z = gate == 0 ? dZa : dZx;
   float *dW = gate == 0 ? dWa : dWx;
-  const int tx = threadIdx.x, ty = threadIdx.y;   // 32 x 8
-  const int i0 = ti * 32, j0 = tj * 32;
+  const int tid = threadIdx.x;
+  const int ri = tid >> 4, rj = tid & 15;   // this thread's rows 4 ri.., columns 4 rj..
+  const int lc = tid & 63, lr = tid >> 6;   // loader: column lc, rows lr + 4 q
+  const int i0 = ti * kDwTile, j0 = tj * kDwTile;
+  const bool iok = i0 + lc < bw, jok = j0 + lc < bw;
+  const float *Uc = U + (size_t)h * bw + i0 + lc;
+  const float *Zc = Z + (size_t)h * bw + j0 + lc;
   const int n_begin = blockIdx.y * chunk, n_end = min(N, n_begin + chunk);
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int n0 = n_begin; n0 < n_end; n0 += 32) {
+  float acc[4][4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int n = n0 + ty + 8 * q;
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[a][e] = 0.f;
+  for (int n0 = n_begin; n0 < n_end; n0 += kDwRows) {
+#pragma unroll
+    for (int q = 0; q < kDwRows / 4; ++q) {
+      const int n = n0 + lr + 4 * q;
       const bool ok = n < n_end;
-      us[ty + 8 * q][tx] =
-          ok && i0 + tx < bw ? U[(size_t)n * D + h * bw + i0 + tx] : 0.f;
-      zs[ty + 8 * q][tx] =
-          ok && j0 + tx < bw ? Z[(size_t)n * D + h * bw + j0 + tx] : 0.f;
+      us[lr + 4 * q][lc] = ok && iok ? Uc[(size_t)n * D] : 0.f;
+      zs[lr + 4 * q][lc] = ok && jok ? Zc[(size_t)n * D] : 0.f;
     }
     __syncthreads();
-#pragma unroll 8
-    for (int nn = 0; nn < 32; ++nn) {
-      const float z = zs[nn][tx];
+#pragma unroll 4
+    for (int nn = 0; nn < kDwRows; ++nn) {
+      const float4 uv = *reinterpret_cast<const float4 *>(&us[nn][4 * ri]);
+      const float4 zv = *reinterpret_cast<const float4 *>(&zs[nn][4 * rj]);
+      const float ua[4] = {uv.x, uv.y, uv.z, uv.w};
+      const float za[4] = {zv.x, zv.y, zv.z, zv.w};
 #pragma unroll
-      for (int q = 0; q < 4; ++q) acc[q] = fmaf(us[nn][ty + 8 * q], z, acc[q]);
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[a][e] = fmaf(ua[a], za[e], acc[a][e]);
     }
     __syncthreads();
   }
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int i = i0 + ty + 8 * q, jj = j0 + tx;
-    if (i < bw && jj < bw) atomicAdd(dW + ((size_t)h * bw + i) * bw + jj, acc[q]);
-  }
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = i0 + 4 * ri + a, jj = j0 + 4 * rj + e;
+      if (i < bw && jj < bw) atomicAdd(dW + ((size_t)h * bw + i) * bw + jj, acc[a][e]);
+    }
 }
 
-// d x (and the conv history's gradient) from d u, and d w per channel for one
-// chunk of tokens of one batch row; thread per channel.
+// d x (and the conv history's gradient) from d u, and d w per channel, for one
+// chunk of kConvChunk extended positions m (x_{m-3}) of one batch row; thread
+// per channel, the last three d u values in registers:
+//   d x_{m-3} = sum_k w[k] d u_{m-k},  d w[k] += x_{m-3} d u_{m-k}  (0 <= m-k < T).
+constexpr int kConvChunk = 64, kConvThreads = 256;
+
 template <typename T>
-__global__ void bwd_conv_kernel(BwdArgs p, const float *__restrict__ du, int chunk) {
+__global__ void __launch_bounds__(kConvThreads)
+bwd_conv_kernel(BwdArgs p, const float *__restrict__ du) {
   const int D = p.D;
-  const int d = blockIdx.x * blockDim.x + threadIdx.x;
+  const int d = blockIdx.x * kConvThreads + threadIdx.x;
   const int b = blockIdx.y;
   if (d >= D) return;
-  const int m_begin = blockIdx.z * chunk, m_end = min(p.T + 3, m_begin + chunk);
+  const int m_begin = blockIdx.z * kConvChunk, m_end = min(p.T + 3, m_begin + kConvChunk);
   const T *cw = static_cast<const T *>(p.conv_w);
   float w[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) w[k] = ldg_f32(cw + (size_t)k * D + d);
-  const float *dub = du + (size_t)b * p.T * D;
+  const float *dub = du + (size_t)b * p.T * D + d;
   const T *xb = static_cast<const T *>(p.x) + (size_t)b * p.T * D;
   const T *cs_in_b =
       p.conv_state_in ? static_cast<const T *>(p.conv_state_in) + (size_t)b * 3 * D : nullptr;
-  T *dxb = static_cast<T *>(p.dx) + (size_t)b * p.T * D;
+  T *dxb = static_cast<T *>(p.dx) + (size_t)b * p.T * D + d;
+  auto du_at = [&](int t) { return (t >= 0 && t < p.T) ? dub[(size_t)t * D] : 0.f; };
+  float g1 = du_at(m_begin - 1), g2 = du_at(m_begin - 2), g3 = du_at(m_begin - 3);
   float dw[4] = {0.f, 0.f, 0.f, 0.f};
-  // extended index m: x_{m-3}; d xe[m] = sum_k w[k] d u[m - k]; d w[k] += xe[m] d u[m - k]
+#pragma unroll 4
   for (int m = m_begin; m < m_end; ++m) {
+    const float g0 = du_at(m);
     const float xv = hist_x(xb, cs_in_b, m - 3, D, d);
-    float acc = 0.f;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int t = m - k;
-      if (t >= 0 && t < p.T) {
-        const float g = dub[(size_t)t * D + d];
-        acc = fmaf(w[k], g, acc);
-        dw[k] = fmaf(xv, g, dw[k]);
-      }
-    }
-    if (m >= 3) dxb[(size_t)(m - 3) * D + d] = from_f32<T>(acc);
+    const float acc = fmaf(w[0], g0, fmaf(w[1], g1, fmaf(w[2], g2, w[3] * g3)));
+    dw[0] = fmaf(xv, g0, dw[0]);
+    dw[1] = fmaf(xv, g1, dw[1]);
+    dw[2] = fmaf(xv, g2, dw[2]);
+    dw[3] = fmaf(xv, g3, dw[3]);
+    if (m >= 3) dxb[(size_t)(m - 3) * D] = from_f32<T>(acc);
     else if (p.dconv_state_in) p.dconv_state_in[((size_t)b * 3 + m) * D + d] = acc;
+    g3 = g2;
+    g2 = g1;
+    g1 = g0;
   }
 #pragma unroll
   for (int k = 0; k < 4; ++k) atomicAdd(p.dconv_w + (size_t)k * D + d, dw[k]);
 }
 
-struct BwdPlan {
-  int L, nseg;
-};
-
-BwdPlan bwd_plan(int B, int T, int H) {
-  constexpr int kTargetBlocks = 296, kMinSeg = 16;
-  const long units = (long)B * H;
-  int nseg = (int)((kTargetBlocks + units - 1) / units);
-  const int max_seg = ceil_div(T, kMinSeg);
-  if (nseg > max_seg) nseg = max_seg;
-  if (nseg < ceil_div(T, kMaxSeg)) nseg = ceil_div(T, kMaxSeg);
-  if (nseg < 1) nseg = 1;
-  BwdPlan pl;
-  pl.L = ceil_div(T, nseg);
-  pl.nseg = ceil_div(T, pl.L);
-  return pl;
-}
-
 struct BwdLayout {
-  size_t off_A, off_H, off_R, off_hin, off_C, off_u, off_dza, off_dzx, off_du, total;
+  size_t off_A, off_H, off_R, off_hin, off_C, off_gP, off_gH, off_za, off_zx, off_u, off_du, total;
 };
 
 BwdLayout bwd_layout(int B, int T, int D, int H) {
-  const BwdPlan pl = bwd_plan(B, T, H);
+  const BwdPlan pl = bwd_plan(B, T, D, H);
   const size_t seg = align_up((size_t)B * pl.nseg * D * sizeof(float), 256);
+  const size_t grp = align_up((size_t)B * ceil_div(T, kTB) * D * sizeof(float), 256);
   const size_t tok = align_up((size_t)B * T * D * sizeof(float), 256);
   BwdLayout L{};
   L.off_A = 0;
@@ -468,26 +519,26 @@ BwdLayout bwd_layout(int B, int T, int D, int H) {
   L.off_R = L.off_H + seg;
   L.off_hin = L.off_R + seg;
   L.off_C = L.off_hin + seg;
-  L.off_u = L.off_C + seg;
-  L.off_dza = L.off_u + tok;
-  L.off_dzx = L.off_dza + tok;
-  L.off_du = L.off_dzx + tok;
+  L.off_gP = L.off_C + seg;
+  L.off_gH = L.off_gP + grp;
+  L.off_za = L.off_gH + grp;
+  L.off_zx = L.off_za + tok;
+  L.off_u = L.off_zx + tok;
+  L.off_du = L.off_u + tok;
   L.total = L.off_du + tok;
   return L;
 }
 
-template <typename T, bool kSW>
+template <typename T, bool kSW, int kMaxT>
 cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
   const int bw = p.D / p.H;
-  const BwdPlan pl = bwd_plan(p.B, p.T, p.H);
+  const BwdPlan pl = bwd_plan(p.B, p.T, p.D, p.H);
   const BwdLayout Ly = bwd_layout(p.B, p.T, p.D, p.H);
   unsigned char *w = static_cast<unsigned char *>(ws);
-  float *A = reinterpret_cast<float *>(w + Ly.off_A), *Hh = reinterpret_cast<float *>(w + Ly.off_H);
-  float *R = reinterpret_cast<float *>(w + Ly.off_R), *hin = reinterpret_cast<float *>(w + Ly.off_hin);
-  float *C = reinterpret_cast<float *>(w + Ly.off_C), *U = reinterpret_cast<float *>(w + Ly.off_u);
-  float *dza = reinterpret_cast<float *>(w + Ly.off_dza);
-  float *dzx = reinterpret_cast<float *>(w + Ly.off_dzx);
-  float *du = reinterpret_cast<float *>(w + Ly.off_du);
+  auto at = [w](size_t off) { return reinterpret_cast<float *>(w + off); };
+  float *A = at(Ly.off_A), *Hh = at(Ly.off_H), *R = at(Ly.off_R);
+  float *hin = at(Ly.off_hin), *C = at(Ly.off_C), *gP = at(Ly.off_gP), *gH = at(Ly.off_gH);
+  float *za = at(Ly.off_za), *zx = at(Ly.off_zx), *U = at(Ly.off_u), *du = at(Ly.off_du);
   const size_t D = p.D;
   cudaError_t e;
   // the accumulated gradients start at zero
@@ -498,41 +549,53 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
   if ((e = cudaMemsetAsync(p.db_x, 0, D * sizeof(float), st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(p.dLambda, 0, D * sizeof(float), st)) != cudaSuccess) return e;
 
-  const int threads = ceil_div(bw, 32) * 32;
-  const dim3 grid(pl.nseg, p.H, p.B);
+  const int threads = pl.S * pl.bwp;
+  const dim3 grid(ceil_div(pl.nseg, pl.S), p.H, p.B);
   const size_t wsm = kSW ? 2 * (size_t)bw * (bw + 1) * sizeof(float) : 0;
-  const size_t smem1 = (size_t)kTB * bw * sizeof(float) + wsm;
-  const int nsub_max = ceil_div(pl.L, kTB);
-  const size_t smem3 = (size_t)(3 * kTB + nsub_max) * bw * sizeof(float) + wsm;
-  if (smem1 > 48 * 1024 &&
-      (e = cudaFuncSetAttribute(bwd_aggregate_kernel<T, kSW>,
+  // K1: double-buffered u rows; K3: d z_a and d z_x rows; both [S][bw][kRow]
+  const size_t smem1 = 2 * (size_t)pl.S * bw * kRow * sizeof(float) + wsm;
+  const size_t smem3 = smem1;
+  if ((e = cudaFuncSetAttribute(bwd_gates_kernel<T, kSW, kMaxT>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1)) !=
-          cudaSuccess)
+      cudaSuccess)
     return e;
-  if (smem3 > 48 * 1024 &&
-      (e = cudaFuncSetAttribute(bwd_final_kernel<T, kSW>,
+  if ((e = cudaFuncSetAttribute(bwd_final_kernel<T, kSW, kMaxT>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3)) !=
-          cudaSuccess)
+      cudaSuccess)
     return e;
-  bwd_aggregate_kernel<T, kSW><<<grid, threads, smem1, st>>>(p, pl.L, pl.nseg, A, Hh, R);
+  bwd_gates_kernel<T, kSW, kMaxT><<<grid, threads, smem1, st>>>(p, pl, A, Hh, R, gP, gH, za, zx);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int bd = p.B * p.D;
   bwd_carry_kernel<<<ceil_div(bd, 256), 256, 0, st>>>(p.B, p.D, pl.nseg, A, Hh, R, p.h0, p.dh_T,
                                                       hin, C, p.dh0);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  bwd_final_kernel<T, kSW><<<grid, threads, smem3, st>>>(p, pl.L, pl.nseg, hin, C, U, dza, dzx,
-                                                          du);
+  bwd_final_kernel<T, kSW, kMaxT><<<grid, threads, smem3, st>>>(p, pl, hin, C, gP, gH, za, zx,
+                                                                 U, du);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // K4: about 8 blocks of 256 threads per SM of a 148-SM part over the token chunks
   const int N = p.B * p.T;
-  const int tiles = ceil_div(bw, 32);
-  const int chunk = 1024;
-  bwd_dw_kernel<<<dim3(2 * tiles * tiles * p.H, ceil_div(N, chunk)), dim3(32, 8), 0, st>>>(
-      U, dza, dzx, p.dW_a, p.dW_x, N, p.D, p.H, chunk);
+  const int tiles = ceil_div(bw, kDwTile);
+  const int tile_blocks = 2 * tiles * tiles * p.H;
+  const int nchunk = ceil_div(8 * 148, tile_blocks);
+  const int chunk = ceil_div(ceil_div(N, nchunk), kDwRows) * kDwRows;
+  bwd_dw_kernel<<<dim3(tile_blocks, ceil_div(N, chunk)), kDwThreads, 0, st>>>(
+      U, za, zx, p.dW_a, p.dW_x, N, p.D, p.H, chunk);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const int cchunk = 256;
-  bwd_conv_kernel<T><<<dim3(ceil_div(p.D, 128), p.B, ceil_div(p.T + 3, cchunk)), 128, 0, st>>>(
-      p, du, cchunk);
+  bwd_conv_kernel<T><<<dim3(ceil_div(p.D, kConvThreads), p.B, ceil_div(p.T + 3, kConvChunk)),
+                       kConvThreads, 0, st>>>(p, du);
   return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_bwd_io(const BwdArgs &p, void *ws, cudaStream_t st) {
+  const int bw = p.D / p.H;
+  // both gate weights in shared memory (fp32) up to 128-wide heads: 2 x 129 x 128 x 4 B;
+  // a segment's threads (bw rounded up to a warp) fit a 512-thread block up to 512-wide
+  // heads; heads up to 64 wide run 256-thread blocks, several per SM
+  if (bw <= 64) return launch_bwd_t<T, true, 256>(p, ws, st);
+  if (bw <= 128) return launch_bwd_t<T, true, 512>(p, ws, st);
+  if (bw <= 512) return launch_bwd_t<T, false, 512>(p, ws, st);
+  return launch_bwd_t<T, false, 1024>(p, ws, st);
 }
 
 }  // namespace
@@ -542,12 +605,8 @@ size_t bwd_workspace_bytes(int B, int T, int D, int H) { return bwd_layout(B, T,
 int bwd_launches() { return 5; }
 
 cudaError_t launch_bwd(const BwdArgs &p, int io, void *ws, cudaStream_t st) {
-  // both gate weights in shared memory (fp32) up to 128-wide heads: 2 x 129 x 128 x 4 B
-  const bool sw = p.D / p.H <= 128;
-  if (io == RGLRU_IO_F32)
-    return sw ? launch_bwd_t<float, true>(p, ws, st) : launch_bwd_t<float, false>(p, ws, st);
-  return sw ? launch_bwd_t<__nv_bfloat16, true>(p, ws, st)
-            : launch_bwd_t<__nv_bfloat16, false>(p, ws, st);
+  if (io == RGLRU_IO_F32) return launch_bwd_io<float>(p, ws, st);
+  return launch_bwd_io<__nv_bfloat16>(p, ws, st);
 }
 
 }  // namespace rglru

@@ -5,8 +5,9 @@ Bars: fp32 I/O 1e-4, bf16 I/O 2e-2, as for the forward. dx and the conv
 history's gradient use the forward's metric: max |g - o| / max(|o|, per-channel
 RMS of o); dh0 is floored at its RMS over the whole tensor. Parameter gradients,
 which sum over every token, use the norm-wise max |g - o| / max |o| per tensor.
-Cases span several 8-token groups, a ragged tail, one and several 512-token
-segments, h0, a conv history and a state-gradient input dh_T.
+Cases span several 8-token groups, a ragged tail, one and many segments,
+heads from 32 to 1024 channels (every block shape the launcher picks), h0, a
+conv history and a state-gradient input dh_T.
 """
 import numpy as np
 import pytest
@@ -27,6 +28,12 @@ CASES = [
     WORKLOADS["hawk_block"].with_shape(B=2, T=301, D=128, H=2, h0_var=0.5, bias_std=0.5, seed=43),
     WORKLOADS["hawk_block"].with_shape(B=1, T=1100, D=256, H=1, h0_var=0.1, seed=44),
     WORKLOADS["griffin2b"].with_shape(B=1, T=200, D=512, H=2, h0_var=0.1, seed=45),
+    # 128-wide heads (4 segments of 128 threads per block), 1024-wide heads
+    # (one 1024-thread segment per block) and the hawk_block head layout at full
+    # length (64 segments of 32 tokens per sequence, 4 per block)
+    WORKLOADS["hawk_block"].with_shape(B=1, T=700, D=256, H=2, h0_var=0.5, seed=46),
+    WORKLOADS["tiny_f32"].with_shape(B=1, T=90, D=1024, H=1, h0_var=0.5, seed=47),
+    WORKLOADS["hawk_block"].with_shape(B=2, T=2048, D=1024, H=16, h0_var=0.1, seed=48),
 ]
 
 
