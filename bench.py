@@ -392,9 +392,10 @@ def run_backward(rg, wl, g, w, dev, a, pk):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "traffic": None,
                          "algorithmic_bytes_per_launch": bytes_step,
-                         "note": "step time of all five launches; fp32 CUDA-core arithmetic, "
-                                 "16 B per channel-token of fp32 intermediates in a workspace "
-                                 "(not algorithmic)"}}
+                         "note": "step time of all five launches; fp32 CUDA-core arithmetic "
+                                 "(three gate contractions of 2 bw MACs per channel-token); "
+                                 "fp32 intermediates in a workspace (z_a, z_x, u, d u: 16 B "
+                                 "per channel-token written and re-read) are not algorithmic"}}
 
 
 def run_decode(rg, dev, a, pk):

@@ -398,7 +398,8 @@ bwd_final_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
 
 // d W[h, i, j] += sum_n U[n, h bw + i] dZ[n, h bw + j] over one chunk of
 // tokens: a 64 x 64 tile of (i, j) of one gate and head per block, 4 x 4 per
-// thread, 32 tokens of both operands staged in shared memory at a time.
+// thread, 32 tokens of both operands staged in shared memory at a time (the
+// next 32 already in flight to registers).
 constexpr int kDwTile = 64, kDwRows = 32, kDwThreads = 256;
 
 __global__ void __launch_bounds__(kDwThreads)
@@ -428,15 +429,26 @@ bwd_dw_kernel(const float *__restrict__ U, const float *__restrict__ dZa,
   for (int a = 0; a < 4; ++a)
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[a][e] = 0.f;
-  for (int n0 = n_begin; n0 < n_end; n0 += kDwRows) {
+  // the next 32 tokens' loads are issued before this tile's FMAs (register prefetch)
+  float pu[kDwRows / 4], pz[kDwRows / 4];
+  auto fetch = [&](int n0) {
 #pragma unroll
     for (int q = 0; q < kDwRows / 4; ++q) {
       const int n = n0 + lr + 4 * q;
       const bool ok = n < n_end;
-      us[lr + 4 * q][lc] = ok && iok ? Uc[(size_t)n * D] : 0.f;
-      zs[lr + 4 * q][lc] = ok && jok ? Zc[(size_t)n * D] : 0.f;
+      pu[q] = ok && iok ? Uc[(size_t)n * D] : 0.f;
+      pz[q] = ok && jok ? Zc[(size_t)n * D] : 0.f;
+    }
+  };
+  fetch(n_begin);
+  for (int n0 = n_begin; n0 < n_end; n0 += kDwRows) {
+#pragma unroll
+    for (int q = 0; q < kDwRows / 4; ++q) {
+      us[lr + 4 * q][lc] = pu[q];
+      zs[lr + 4 * q][lc] = pz[q];
     }
     __syncthreads();
+    if (n0 + kDwRows < n_end) fetch(n0 + kDwRows);
 #pragma unroll 4
     for (int nn = 0; nn < kDwRows; ++nn) {
       const float4 uv = *reinterpret_cast<const float4 *>(&us[nn][4 * ri]);
