@@ -36,6 +36,8 @@
 //                 gradient) and d w[k] = sum_t x_{t-3+k} d u_t.
 // The path of d z_a through g carries r / g, which tends to 0 with r
 // (1 - a^2 ~ 2 c sp r); it is formed as that ratio (0 where g = 0).
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -165,6 +167,76 @@ __device__ __forceinline__ BwdThread bwd_thread(const BwdArgs &p, const BwdPlan 
   return th;
 }
 
+// ---- warp-level bf16 tensor-core MMA (m16n8k16, fp32 accumulate) ----
+// Fragment layouts (PTX ISA, mma.m16n8k16 with .bf16): lane l, g = l / 4,
+// q = l % 4. A (16 x 16, row-major): a0 = (g, 2q..2q+1), a1 = (g + 8, 2q..),
+// a2 = (g, 2q + 8..), a3 = (g + 8, 2q + 8..). B (16 x 8): b0 = (k = 2q..2q+1,
+// n = g), b1 = (k = 2q + 8.., n = g). C (16 x 8): c0, c1 = (g, 2q), (g, 2q + 1);
+// c2, c3 = (g + 8, 2q), (g + 8, 2q + 1). Each pair holds the lower k (column)
+// in its low half.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&a)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t shared_addr(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(unsigned short lo, unsigned short hi) {
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+// Geometry of the tensor-core kernels for a head width kBW in {32, 64, 128}:
+// S segments of kBW threads per block, the block's M = 8 S tokens of a group
+// as MT m-tiles of 16, kBW / 8 n-tiles of 8 channels, kBW / 16 k-steps. Warp w
+// owns n-tile 2w / MT and the m-tiles 2w % MT and the next one.
+template <int kBW>
+struct TcGeo {
+  static constexpr int kThreads = kBW == 128 ? 512 : 256;
+  static constexpr int S = kThreads / kBW;
+  static constexpr int M = S * kTB;
+  static constexpr int MT = M / 16;
+  static constexpr int NKS = kBW / 16;
+  static constexpr int kStride = kBW + 8;   // bf16 per A row: 16-byte rows on distinct bank groups
+  static_assert(MT % 2 == 0 && MT * (kBW / 8) == 2 * (kThreads / 32), "two tiles per warp");
+};
+
+// The post-contraction part of a K1 group: decay, input, the local scan and
+// the running R; z_a, z_x of the live tokens to the workspace.
+template <typename T>
+__device__ __forceinline__ void gates_scan_group(const float (&za)[kTB], const float (&zx)[kTB],
+                                                 const float (&u)[kTB], int tb, int t1,
+                                                 float neg_c_sp, const T *dyb, size_t orow,
+                                                 int D, float &P, float &Hl, float &R,
+                                                 float *__restrict__ ws_za,
+                                                 float *__restrict__ ws_zx) {
+#pragma unroll
+  for (int k = 0; k < kTB; ++k) {
+    const int t = tb + k;
+    if (t < t1) {
+      float a, beta, la;
+      decay_and_input(za[k], zx[k], u[k], neg_c_sp, a, beta, la);
+      Hl = fmaf(a, Hl, beta);
+      P *= a;
+      const size_t o = orow + (size_t)t * D;
+      R = fmaf(P, ldg_f32(dyb + o), R);
+      ws_za[o] = za[k];
+      ws_zx[o] = zx[k];
+    }
+  }
+}
+
 template <typename T, bool kSW, int kMaxT>
 __global__ void __launch_bounds__(kMaxT, kMaxT == 256 ? 3 : 1)
 bwd_gates_kernel(BwdArgs p, BwdPlan pl, float *__restrict__ ws_A, float *__restrict__ ws_H,
@@ -180,7 +252,7 @@ bwd_gates_kernel(BwdArgs p, BwdPlan pl, float *__restrict__ ws_A, float *__restr
   const T *xb = static_cast<const T *>(p.x) + (size_t)b * p.T * D;
   const T *cs_in_b =
       p.conv_state_in ? static_cast<const T *>(p.conv_state_in) + (size_t)b * 3 * D : nullptr;
-  const T *dyb = static_cast<const T *>(p.dy) + (size_t)b * p.T * D;
+  const T *dyb = static_cast<const T *>(p.dy);
   const T *Wa = static_cast<const T *>(p.W_a) + (size_t)h * bw * bw;
   const T *Wx = static_cast<const T *>(p.W_x) + (size_t)h * bw * bw;
   if (kSW) stage_weights<T>(Wa, Wx, Wsa, Wsx, bw);
@@ -189,6 +261,7 @@ bwd_gates_kernel(BwdArgs p, BwdPlan pl, float *__restrict__ ws_A, float *__restr
   const float neg_c_sp = -kDecayC * c.sp;
   const int ngt = ceil_div(p.T, kTB);
   const int jr = th.j < bw ? th.j : 0;
+  const size_t orow = (size_t)b * p.T * D + th.d;
   float P = 1.f, Hl = 0.f, R = 0.f;
   const int ng = pl.L / kTB;
   for (int g = 0; g < ng; ++g) {
@@ -228,20 +301,127 @@ bwd_gates_kernel(BwdArgs p, BwdPlan pl, float *__restrict__ ws_A, float *__restr
           zx[k] = fmaf(uv[k], wx, zx[k]);
         }
       }
+      gates_scan_group<T>(za, zx, u, tb, th.t1, neg_c_sp, dyb, orow, D, P, Hl, R, ws_za, ws_zx);
+    }
+  }
+  if (!th.active) return;
+  const size_t o = ((size_t)b * pl.nseg + th.s) * D + th.d;
+  ws_A[o] = P;
+  ws_H[o] = Hl;
+  ws_R[o] = R;
+}
+
+// K1 for bf16 I/O and kBW in {32, 64, 128}: the gate contraction of each group
+// on the tensor cores. u goes to shared memory as bf16 rows (token-major), each
+// warp multiplies its two 16-token m-tiles by its 8 columns of W_a and W_x
+// (fragments held in registers for the whole kernel), scatters the fp32
+// results into (segment, channel) rows, and each thread reads back its own
+// channel's 8 tokens for the scan.
+template <int kBW>
+__global__ void __launch_bounds__(TcGeo<kBW>::kThreads, kBW == 128 ? 1 : 3)
+bwd_gates_tc_kernel(BwdArgs p, BwdPlan pl, float *__restrict__ ws_A, float *__restrict__ ws_H,
+                    float *__restrict__ ws_R, float *__restrict__ ws_gP,
+                    float *__restrict__ ws_gH, float *__restrict__ ws_za,
+                    float *__restrict__ ws_zx) {
+  using T = __nv_bfloat16;
+  using G = TcGeo<kBW>;
+  extern __shared__ float4 smem_gt[];
+  float *z_s = reinterpret_cast<float *>(smem_gt);                        // [S][2][kBW][kRow]
+  T *u_s = reinterpret_cast<T *>(z_s + G::S * 2 * kBW * kRow);            // [M][kStride]
+  const int D = p.D, h = blockIdx.y, b = blockIdx.z;
+  const BwdThread th = bwd_thread(p, pl, kBW);
+  const T *xb = static_cast<const T *>(p.x) + (size_t)b * p.T * D;
+  const T *cs_in_b =
+      p.conv_state_in ? static_cast<const T *>(p.conv_state_in) + (size_t)b * 3 * D : nullptr;
+  const T *dyb = static_cast<const T *>(p.dy);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nt = (2 * warp) / G::MT, mt0 = (2 * warp) % G::MT;
+  const int fg = lane >> 2, fq = lane & 3;
+  // B[k = i][n = j] = W[i, j] for this warp's columns nt*8 + fg, all k-steps
+  uint32_t bA[G::NKS][2], bX[G::NKS][2];
+  {
+    const unsigned short *wa =
+        reinterpret_cast<const unsigned short *>(p.W_a) + (size_t)h * kBW * kBW + nt * 8 + fg;
+    const unsigned short *wx =
+        reinterpret_cast<const unsigned short *>(p.W_x) + (size_t)h * kBW * kBW + nt * 8 + fg;
 #pragma unroll
-      for (int k = 0; k < kTB; ++k) {
-        const int t = tb + k;
-        if (t < th.t1) {
-          float a, beta, la;
-          decay_and_input(za[k], zx[k], u[k], neg_c_sp, a, beta, la);
-          Hl = fmaf(a, Hl, beta);
-          P *= a;
-          R = fmaf(P, ldg_f32(dyb + (size_t)t * D + th.d), R);
-          const size_t o = ((size_t)b * p.T + t) * D + th.d;
-          ws_za[o] = za[k];
-          ws_zx[o] = zx[k];
-        }
+    for (int ks = 0; ks < G::NKS; ++ks)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int kk = ks * 16 + 2 * fq + 8 * hf;
+        bA[ks][hf] = pack_bf16(__ldg(wa + (size_t)kk * kBW), __ldg(wa + (size_t)(kk + 1) * kBW));
+        bX[ks][hf] = pack_bf16(__ldg(wx + (size_t)kk * kBW), __ldg(wx + (size_t)(kk + 1) * kBW));
       }
+  }
+  // ldmatrix.x4 row address of this lane: row (l % 8) + 8 ((l / 8) % 2), column 8 (l / 16)
+  const uint32_t a_lane = shared_addr(u_s) +
+                          (((lane & 7) + ((lane >> 3) & 1) * 8) * G::kStride + (lane >> 4) * 8) * 2;
+  ChanC c{0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (th.active) c = chan_c<T>(p, th.d);
+  const float neg_c_sp = -kDecayC * c.sp;
+  const int ngt = ceil_div(p.T, kTB);
+  const size_t orow = (size_t)b * p.T * D + th.d;
+  const float *za_row = z_s + ((th.sl * 2 + 0) * kBW + th.j) * kRow;
+  const float *zx_row = z_s + ((th.sl * 2 + 1) * kBW + th.j) * kRow;
+  T *u_col = u_s + th.sl * kTB * G::kStride + th.j;
+  float P = 1.f, Hl = 0.f, R = 0.f;
+  const int ng = pl.L / kTB;
+  for (int g = 0; g < ng; ++g) {
+    const int tb = th.t0 + g * kTB;
+    const bool live = th.active && tb < th.t1;
+    float u[kTB];
+    if (live) {
+      const size_t go = ((size_t)b * ngt + tb / kTB) * D + th.d;
+      ws_gP[go] = P;
+      ws_gH[go] = Hl;
+      conv_group<T>(xb, cs_in_b, D, th.d, tb, th.t1, c, u);
+    } else {
+#pragma unroll
+      for (int k = 0; k < kTB; ++k) u[k] = 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < kTB; ++k) u_col[k * G::kStride] = __float2bfloat16_rn(u[k]);
+    __syncthreads();
+    float acc[2][2][4];
+#pragma unroll
+    for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mi][0][e] = acc[mi][1][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < G::NKS; ++ks)
+#pragma unroll
+      for (int mi = 0; mi < 2; ++mi) {
+        uint32_t a[4];
+        ldsm_x4(a_lane + ((mt0 + mi) * 16 * G::kStride + ks * 16) * 2, a);
+        mma_bf16(acc[mi][0], a, bA[ks][0], bA[ks][1]);
+        mma_bf16(acc[mi][1], a, bX[ks][0], bX[ks][1]);
+      }
+#pragma unroll
+    for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = (mt0 + mi) * 16 + fg + (e >= 2 ? 8 : 0);
+        const int col = nt * 8 + 2 * fq + (e & 1);
+        z_s[(((r >> 3) * 2 + 0) * kBW + col) * kRow + (r & 7)] = acc[mi][0][e];
+        z_s[(((r >> 3) * 2 + 1) * kBW + col) * kRow + (r & 7)] = acc[mi][1][e];
+      }
+    __syncthreads();
+    if (live) {
+      float za[kTB], zx[kTB];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const float4 va = reinterpret_cast<const float4 *>(za_row)[q];
+        const float4 vx = reinterpret_cast<const float4 *>(zx_row)[q];
+        za[4 * q] = va.x + c.ba;
+        za[4 * q + 1] = va.y + c.ba;
+        za[4 * q + 2] = va.z + c.ba;
+        za[4 * q + 3] = va.w + c.ba;
+        zx[4 * q] = vx.x + c.bx;
+        zx[4 * q + 1] = vx.y + c.bx;
+        zx[4 * q + 2] = vx.z + c.bx;
+        zx[4 * q + 3] = vx.w + c.bx;
+      }
+      gates_scan_group<T>(za, zx, u, tb, th.t1, neg_c_sp, dyb, orow, D, P, Hl, R, ws_za, ws_zx);
     }
   }
   if (!th.active) return;
@@ -276,6 +456,77 @@ __global__ void bwd_carry_kernel(int B, int D, int nseg, const float *__restrict
   if (dh0) dh0[idx] = cc;
 }
 
+// The per-thread part of a K3 group (a live thread only): the group's start
+// state from (prod a, local state) and h_in, the stored z, then the reverse
+// chain over its tokens. With G_t the state gradient at token t, every
+// gradient of the token is G_t times a factor known in time order:
+//   d z_a = G c sp (1 - r) Q,  d Lambda-sum term = G c Q,
+//   Q = a (a i u (r / g) - h_{t-1} r),
+//   d z_x = G g u i (1 - i),   own part of d u = G g i,
+// so the forward part keeps five factors per token and the reverse part is a
+// handful of multiplies. It writes u, d z_a, d z_x over the workspace, passes
+// each token's (d z_a, d z_x) to sink(k, ...) (zeros past t1), leaves the own
+// part of d u in dub and advances gc and the per-channel sums (acc_q sums
+// G Q; the caller scales it by c).
+template <typename T, typename Sink>
+__device__ __forceinline__ void final_group(const BwdThread &th, const ChanC &c, const T *xb,
+                                            const T *cs_in_b, const T *dyb, size_t orow, int D,
+                                            int tb, size_t go, float h_in,
+                                            const float *__restrict__ ws_gP,
+                                            const float *__restrict__ ws_gH,
+                                            float *__restrict__ ws_za, float *__restrict__ ws_zx,
+                                            float *__restrict__ ws_u, float &gc, float &acc_q,
+                                            float &acc_ba, float &acc_bx, float (&dub)[kTB],
+                                            Sink sink) {
+  const float neg_c_sp = -kDecayC * c.sp, csp = kDecayC * c.sp;
+  float u[kTB];
+  conv_group<T>(xb, cs_in_b, D, th.d, tb, th.t1, c, u);
+  float fa[kTB], fza[kTB], fq[kTB], fzx[kTB], fu[kTB];
+  float hh = fmaf(ws_gP[go], h_in, ws_gH[go]);
+#pragma unroll
+  for (int k = 0; k < kTB; ++k) {
+    const int t = tb + k;
+    const size_t o = orow + (size_t)t * D;
+    const bool in = t < th.t1;
+    const float za = in ? ws_za[o] : 0.f;
+    const float zx = in ? ws_zx[o] : 0.f;
+    if (in) ws_u[o] = u[k];
+    const float r = sigmoid_f32(za);
+    const float ig = sigmoid_f32(zx);
+    const float la = neg_c_sp * r;
+    const float a = expf(la);
+    const float gg = sqrtf(-expm1f(2.0f * la));
+    const float rog = gg > 0.f ? r / gg : 0.f;
+    const float q = a * (a * ig * u[k] * rog - hh * r);
+    fa[k] = a;
+    fq[k] = q;
+    fza[k] = csp * (1.f - r) * q;
+    fzx[k] = gg * u[k] * ig * (1.f - ig);
+    fu[k] = gg * ig;
+    hh = fmaf(a, hh, gg * ig * u[k]);
+  }
+#pragma unroll
+  for (int k = kTB - 1; k >= 0; --k) {
+    const int t = tb + k;
+    float dza = 0.f, dzx = 0.f;
+    dub[k] = 0.f;
+    if (t < th.t1) {
+      const size_t o = orow + (size_t)t * D;
+      const float G = ldg_f32(dyb + o) + gc;
+      dza = G * fza[k];
+      dzx = G * fzx[k];
+      dub[k] = G * fu[k];
+      acc_q = fmaf(G, fq[k], acc_q);
+      acc_ba += dza;
+      acc_bx += dzx;
+      gc = fa[k] * G;
+      ws_za[o] = dza;
+      ws_zx[o] = dzx;
+    }
+    sink(k, dza, dzx);
+  }
+}
+
 template <typename T, bool kSW, int kMaxT>
 __global__ void __launch_bounds__(kMaxT, kMaxT == 256 ? 3 : 1)
 bwd_final_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
@@ -292,7 +543,7 @@ bwd_final_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
   const T *xb = static_cast<const T *>(p.x) + (size_t)b * p.T * D;
   const T *cs_in_b =
       p.conv_state_in ? static_cast<const T *>(p.conv_state_in) + (size_t)b * 3 * D : nullptr;
-  const T *dyb = static_cast<const T *>(p.dy) + (size_t)b * p.T * D;
+  const T *dyb = static_cast<const T *>(p.dy);
   const T *Wa = static_cast<const T *>(p.W_a) + (size_t)h * bw * bw;
   const T *Wx = static_cast<const T *>(p.W_x) + (size_t)h * bw * bw;
   if (kSW) stage_weights<T>(Wa, Wx, Wsa, Wsx, bw);
@@ -304,69 +555,32 @@ bwd_final_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
     h_in = ws_hin[seg];
     gc = ws_C[seg];
   }
-  const float neg_c_sp = -kDecayC * c.sp, csp = kDecayC * c.sp;
   const int ngt = ceil_div(p.T, kTB);
   const int jr = th.j < bw ? th.j : 0;
+  const size_t orow = (size_t)b * p.T * D + th.d;
   float *dza_row = dz_s + ((th.sl * 2 + 0) * bw + jr) * kRow;
   float *dzx_row = dz_s + ((th.sl * 2 + 1) * bw + jr) * kRow;
   const float *dza_seg = dz_s + (th.sl * 2 + 0) * bw * kRow;
   const float *dzx_seg = dz_s + (th.sl * 2 + 1) * bw * kRow;
-  float acc_sp = 0.f, acc_ba = 0.f, acc_bx = 0.f;
+  float acc_q = 0.f, acc_ba = 0.f, acc_bx = 0.f;
   for (int g = pl.L / kTB - 1; g >= 0; --g) {
     const int tb = th.t0 + g * kTB;
     const bool live = th.active && tb < th.t1;
     float dub[kTB];
-#pragma unroll
-    for (int k = 0; k < kTB; ++k) dub[k] = 0.f;
     if (live) {
-      float u[kTB];
-      conv_group<T>(xb, cs_in_b, D, th.d, tb, th.t1, c, u);
-      float a[kTB], r[kTB], ig[kTB], gg[kTB], hp[kTB];
       const size_t go = ((size_t)b * ngt + tb / kTB) * D + th.d;
-      float hh = fmaf(ws_gP[go], h_in, ws_gH[go]);
+      final_group<T>(th, c, xb, cs_in_b, dyb, orow, D, tb, go, h_in, ws_gP, ws_gH, ws_za, ws_zx,
+                     ws_u, gc, acc_q, acc_ba, acc_bx, dub, [&](int k, float dza, float dzx) {
+                       dza_row[k] = dza;
+                       dzx_row[k] = dzx;
+                     });
+    } else {
 #pragma unroll
-      for (int k = 0; k < kTB; ++k) {
-        const int t = tb + k;
-        const size_t o = ((size_t)b * p.T + t) * D + th.d;
-        const float za = t < th.t1 ? ws_za[o] : 0.f;
-        const float zx = t < th.t1 ? ws_zx[o] : 0.f;
-        r[k] = sigmoid_f32(za);
-        ig[k] = sigmoid_f32(zx);
-        const float la = neg_c_sp * r[k];
-        a[k] = expf(la);
-        gg[k] = sqrtf(-expm1f(2.0f * la));
-        hp[k] = hh;
-        hh = fmaf(a[k], hh, gg[k] * ig[k] * u[k]);
+      for (int k = 0; k < kTB; ++k) dub[k] = 0.f;
+      if (th.j < bw) {
+        store_row(dza_row, dub);   // zeros
+        store_row(dzx_row, dub);
       }
-#pragma unroll
-      for (int k = kTB - 1; k >= 0; --k) {
-        const int t = tb + k;
-        float dza = 0.f, dzx = 0.f;
-        if (t < th.t1) {
-          const float G = ldg_f32(dyb + (size_t)t * D + th.d) + gc;
-          const float da = G * hp[k];
-          const float dg = G * ig[k] * u[k];
-          const float di = G * gg[k] * u[k];
-          dub[k] = G * gg[k] * ig[k];
-          const float rog = gg[k] > 0.f ? r[k] / gg[k] : 0.f;
-          const float aa = a[k] * a[k];
-          dza = -csp * da * a[k] * r[k] * (1.f - r[k]) + csp * aa * (1.f - r[k]) * dg * rog;
-          acc_sp += -kDecayC * da * a[k] * r[k] + kDecayC * aa * dg * rog;
-          dzx = di * ig[k] * (1.f - ig[k]);
-          acc_ba += dza;
-          acc_bx += dzx;
-          gc = a[k] * G;
-          const size_t o = ((size_t)b * p.T + t) * D + th.d;
-          ws_u[o] = u[k];
-          ws_za[o] = dza;
-          ws_zx[o] = dzx;
-        }
-        dza_row[k] = dza;
-        dzx_row[k] = dzx;
-      }
-    } else if (th.j < bw) {
-      store_row(dza_row, dub);   // zeros
-      store_row(dzx_row, dub);
     }
     __syncthreads();
     if (live) {
@@ -386,12 +600,139 @@ bwd_final_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
       }
 #pragma unroll
       for (int k = 0; k < kTB; ++k)
-        if (tb + k < th.t1) ws_du[((size_t)b * p.T + tb + k) * D + th.d] = dub[k];
+        if (tb + k < th.t1) ws_du[orow + (size_t)(tb + k) * D] = dub[k];
     }
     __syncthreads();
   }
   if (!th.active) return;
-  atomicAdd(p.dLambda + th.d, acc_sp * (-sigmoid_f32(-__ldg(p.Lambda + th.d))));
+  atomicAdd(p.dLambda + th.d, kDecayC * acc_q * (-sigmoid_f32(-__ldg(p.Lambda + th.d))));
+  atomicAdd(p.db_a + th.d, acc_ba);
+  atomicAdd(p.db_x + th.d, acc_bx);
+}
+
+// K3 for bf16 I/O and kBW in {32, 64, 128}: the transposed contraction
+// d u += d z_a W_a^T + d z_x W_x^T of each group on the tensor cores. The
+// threads put their d z as bf16 rows (token-major) in shared memory, each warp
+// multiplies its two m-tiles by its 8 columns of W_a^T and W_x^T into one
+// accumulator, scatters it into (segment, channel) rows, and each thread adds
+// its channel's 8 tokens to its own part of d u.
+template <int kBW>
+__global__ void __launch_bounds__(TcGeo<kBW>::kThreads, kBW == 128 ? 1 : 3)
+bwd_final_tc_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
+                    const float *__restrict__ ws_C, const float *__restrict__ ws_gP,
+                    const float *__restrict__ ws_gH, float *__restrict__ ws_za,
+                    float *__restrict__ ws_zx, float *__restrict__ ws_u,
+                    float *__restrict__ ws_du) {
+  using T = __nv_bfloat16;
+  using G = TcGeo<kBW>;
+  extern __shared__ float4 smem_ft[];
+  float *du_s = reinterpret_cast<float *>(smem_ft);                  // [S][kBW][kRow]
+  T *a_s = reinterpret_cast<T *>(du_s + G::S * kBW * kRow);          // [2][M][kStride]
+  T *w_s = a_s + 2 * G::M * G::kStride;                              // [2][kBW][kStride]
+  const int D = p.D, h = blockIdx.y, b = blockIdx.z;
+  const BwdThread th = bwd_thread(p, pl, kBW);
+  const T *xb = static_cast<const T *>(p.x) + (size_t)b * p.T * D;
+  const T *cs_in_b =
+      p.conv_state_in ? static_cast<const T *>(p.conv_state_in) + (size_t)b * 3 * D : nullptr;
+  const T *dyb = static_cast<const T *>(p.dy);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nt = (2 * warp) / G::MT, mt0 = (2 * warp) % G::MT;
+  const int fg = lane >> 2, fq = lane & 3;
+  // The head's W_a and W_x as bf16 rows j (m contiguous, stride kStride) in
+  // shared memory: B[k = m][n = j] = W[j, m], so the k pairs of column
+  // j = nt*8 + fg are adjacent in row j; read per k-step (2 words per gate).
+  {
+    const uint32_t *wa = reinterpret_cast<const uint32_t *>(static_cast<const T *>(p.W_a) +
+                                                            (size_t)h * kBW * kBW);
+    const uint32_t *wx = reinterpret_cast<const uint32_t *>(static_cast<const T *>(p.W_x) +
+                                                            (size_t)h * kBW * kBW);
+    uint32_t *ws32 = reinterpret_cast<uint32_t *>(w_s);
+    for (int idx = threadIdx.x; idx < kBW * kBW / 2; idx += G::kThreads) {
+      const int row = idx / (kBW / 2), cw = idx - row * (kBW / 2);
+      ws32[row * (G::kStride / 2) + cw] = __ldg(wa + idx);
+      ws32[(kBW + row) * (G::kStride / 2) + cw] = __ldg(wx + idx);
+    }
+  }
+  const uint32_t *wfa =
+      reinterpret_cast<const uint32_t *>(w_s) + (nt * 8 + fg) * (G::kStride / 2) + fq;
+  const uint32_t *wfx = wfa + kBW * (G::kStride / 2);
+  const uint32_t a_lane = shared_addr(a_s) +
+                          (((lane & 7) + ((lane >> 3) & 1) * 8) * G::kStride + (lane >> 4) * 8) * 2;
+  constexpr uint32_t kGateBytes = G::M * G::kStride * 2;   // d z_x rows follow d z_a rows
+  ChanC c{0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float h_in = 0.f, gc = 0.f;   // gc: a_{t+1} G_{t+1} for the token being processed
+  if (th.active) {
+    c = chan_c<T>(p, th.d);
+    const size_t seg = ((size_t)b * pl.nseg + th.s) * D + th.d;
+    h_in = ws_hin[seg];
+    gc = ws_C[seg];
+  }
+  const int ngt = ceil_div(p.T, kTB);
+  const size_t orow = (size_t)b * p.T * D + th.d;
+  T *dza_col = a_s + th.sl * kTB * G::kStride + th.j;
+  T *dzx_col = dza_col + G::M * G::kStride;
+  const float *du_row = du_s + (th.sl * kBW + th.j) * kRow;
+  float acc_q = 0.f, acc_ba = 0.f, acc_bx = 0.f;
+  for (int g = pl.L / kTB - 1; g >= 0; --g) {
+    const int tb = th.t0 + g * kTB;
+    const bool live = th.active && tb < th.t1;
+    float dub[kTB];
+    if (live) {
+      const size_t go = ((size_t)b * ngt + tb / kTB) * D + th.d;
+      final_group<T>(th, c, xb, cs_in_b, dyb, orow, D, tb, go, h_in, ws_gP, ws_gH, ws_za, ws_zx,
+                     ws_u, gc, acc_q, acc_ba, acc_bx, dub, [&](int k, float dza, float dzx) {
+                       dza_col[k * G::kStride] = __float2bfloat16_rn(dza);
+                       dzx_col[k * G::kStride] = __float2bfloat16_rn(dzx);
+                     });
+    } else {
+#pragma unroll
+      for (int k = 0; k < kTB; ++k) {
+        dub[k] = 0.f;
+        dza_col[k * G::kStride] = __float2bfloat16_rn(0.f);
+        dzx_col[k * G::kStride] = __float2bfloat16_rn(0.f);
+      }
+    }
+    __syncthreads();
+    float acc[2][4];
+#pragma unroll
+    for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mi][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < G::NKS; ++ks) {
+      // elements ks*16 + 2 fq + 8 hf of row j: words ks*8 + fq + 4 hf
+      const uint32_t ba0 = wfa[ks * 8], ba1 = wfa[ks * 8 + 4];
+      const uint32_t bx0 = wfx[ks * 8], bx1 = wfx[ks * 8 + 4];
+#pragma unroll
+      for (int mi = 0; mi < 2; ++mi) {
+        const uint32_t off = ((mt0 + mi) * 16 * G::kStride + ks * 16) * 2;
+        uint32_t a[4];
+        ldsm_x4(a_lane + off, a);
+        mma_bf16(acc[mi], a, ba0, ba1);
+        ldsm_x4(a_lane + kGateBytes + off, a);
+        mma_bf16(acc[mi], a, bx0, bx1);
+      }
+    }
+#pragma unroll
+    for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = (mt0 + mi) * 16 + fg + (e >= 2 ? 8 : 0);
+        const int col = nt * 8 + 2 * fq + (e & 1);
+        du_s[((r >> 3) * kBW + col) * kRow + (r & 7)] = acc[mi][e];
+      }
+    __syncthreads();
+    if (live) {
+      const float4 v0 = reinterpret_cast<const float4 *>(du_row)[0];
+      const float4 v1 = reinterpret_cast<const float4 *>(du_row)[1];
+      const float dv[kTB] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+      for (int k = 0; k < kTB; ++k)
+        if (tb + k < th.t1) ws_du[orow + (size_t)(tb + k) * D] = dub[k] + dv[k];
+    }
+  }
+  if (!th.active) return;
+  atomicAdd(p.dLambda + th.d, kDecayC * acc_q * (-sigmoid_f32(-__ldg(p.Lambda + th.d))));
   atomicAdd(p.db_a + th.d, acc_ba);
   atomicAdd(p.db_x + th.d, acc_bx);
 }
@@ -541,7 +882,8 @@ BwdLayout bwd_layout(int B, int T, int D, int H) {
   return L;
 }
 
-template <typename T, bool kSW, int kMaxT>
+// kTcBW > 0: bf16 I/O with heads kTcBW wide, K1 and K3 on the tensor cores.
+template <typename T, bool kSW, int kMaxT, int kTcBW>
 cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
   const int bw = p.D / p.H;
   const BwdPlan pl = bwd_plan(p.B, p.T, p.D, p.H);
@@ -563,27 +905,54 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
 
   const int threads = pl.S * pl.bwp;
   const dim3 grid(ceil_div(pl.nseg, pl.S), p.H, p.B);
-  const size_t wsm = kSW ? 2 * (size_t)bw * (bw + 1) * sizeof(float) : 0;
-  // K1: double-buffered u rows; K3: d z_a and d z_x rows; both [S][bw][kRow]
-  const size_t smem1 = 2 * (size_t)pl.S * bw * kRow * sizeof(float) + wsm;
-  const size_t smem3 = smem1;
-  if ((e = cudaFuncSetAttribute(bwd_gates_kernel<T, kSW, kMaxT>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1)) !=
-      cudaSuccess)
-    return e;
-  if ((e = cudaFuncSetAttribute(bwd_final_kernel<T, kSW, kMaxT>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3)) !=
-      cudaSuccess)
-    return e;
-  bwd_gates_kernel<T, kSW, kMaxT><<<grid, threads, smem1, st>>>(p, pl, A, Hh, R, gP, gH, za, zx);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int bd = p.B * p.D;
-  bwd_carry_kernel<<<ceil_div(bd, 256), 256, 0, st>>>(p.B, p.D, pl.nseg, A, Hh, R, p.h0, p.dh_T,
-                                                      hin, C, p.dh0);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  bwd_final_kernel<T, kSW, kMaxT><<<grid, threads, smem3, st>>>(p, pl, hin, C, gP, gH, za, zx,
-                                                                 U, du);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if constexpr (kTcBW > 0) {
+    using G = TcGeo<kTcBW>;
+    // K1: fp32 z rows [S][2][bw][kRow] and bf16 u rows [M][kStride];
+    // K3: fp32 d u rows [S][bw][kRow], bf16 d z_a, d z_x rows [2][M][kStride] and
+    //     bf16 W_a, W_x rows [2][bw][kStride]
+    const size_t smem1 = (size_t)G::S * 2 * kTcBW * kRow * 4 + (size_t)G::M * G::kStride * 2;
+    const size_t smem3 = (size_t)G::S * kTcBW * kRow * 4 + 2 * (size_t)G::M * G::kStride * 2 +
+                         2 * (size_t)kTcBW * G::kStride * 2;   // + bf16 W_a, W_x rows
+    if ((e = cudaFuncSetAttribute(bwd_gates_tc_kernel<kTcBW>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1)) !=
+        cudaSuccess)
+      return e;
+    if ((e = cudaFuncSetAttribute(bwd_final_tc_kernel<kTcBW>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3)) !=
+        cudaSuccess)
+      return e;
+    bwd_gates_tc_kernel<kTcBW><<<grid, G::kThreads, smem1, st>>>(p, pl, A, Hh, R, gP, gH, za, zx);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    bwd_carry_kernel<<<ceil_div(bd, 256), 256, 0, st>>>(p.B, p.D, pl.nseg, A, Hh, R, p.h0,
+                                                        p.dh_T, hin, C, p.dh0);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    bwd_final_tc_kernel<kTcBW><<<grid, G::kThreads, smem3, st>>>(p, pl, hin, C, gP, gH, za, zx,
+                                                                  U, du);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  } else {
+    const size_t wsm = kSW ? 2 * (size_t)bw * (bw + 1) * sizeof(float) : 0;
+    // K1: double-buffered u rows; K3: d z_a and d z_x rows; both [S][bw][kRow]
+    const size_t smem1 = 2 * (size_t)pl.S * bw * kRow * sizeof(float) + wsm;
+    const size_t smem3 = smem1;
+    if ((e = cudaFuncSetAttribute(bwd_gates_kernel<T, kSW, kMaxT>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1)) !=
+        cudaSuccess)
+      return e;
+    if ((e = cudaFuncSetAttribute(bwd_final_kernel<T, kSW, kMaxT>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3)) !=
+        cudaSuccess)
+      return e;
+    bwd_gates_kernel<T, kSW, kMaxT><<<grid, threads, smem1, st>>>(p, pl, A, Hh, R, gP, gH, za,
+                                                                   zx);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    bwd_carry_kernel<<<ceil_div(bd, 256), 256, 0, st>>>(p.B, p.D, pl.nseg, A, Hh, R, p.h0,
+                                                        p.dh_T, hin, C, p.dh0);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    bwd_final_kernel<T, kSW, kMaxT><<<grid, threads, smem3, st>>>(p, pl, hin, C, gP, gH, za, zx,
+                                                                   U, du);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   // K4: about 8 blocks of 256 threads per SM of a 148-SM part over the token chunks
   const int N = p.B * p.T;
   const int tiles = ceil_div(bw, kDwTile);
@@ -601,13 +970,19 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
 template <typename T>
 cudaError_t launch_bwd_io(const BwdArgs &p, void *ws, cudaStream_t st) {
   const int bw = p.D / p.H;
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    // bf16 operands for the two in-loop gate contractions (tensor cores)
+    if (bw == 32) return launch_bwd_t<T, false, 256, 32>(p, ws, st);
+    if (bw == 64) return launch_bwd_t<T, false, 256, 64>(p, ws, st);
+    if (bw == 128) return launch_bwd_t<T, false, 512, 128>(p, ws, st);
+  }
   // both gate weights in shared memory (fp32) up to 128-wide heads: 2 x 129 x 128 x 4 B;
   // a segment's threads (bw rounded up to a warp) fit a 512-thread block up to 512-wide
   // heads; heads up to 64 wide run 256-thread blocks, several per SM
-  if (bw <= 64) return launch_bwd_t<T, true, 256>(p, ws, st);
-  if (bw <= 128) return launch_bwd_t<T, true, 512>(p, ws, st);
-  if (bw <= 512) return launch_bwd_t<T, false, 512>(p, ws, st);
-  return launch_bwd_t<T, false, 1024>(p, ws, st);
+  if (bw <= 64) return launch_bwd_t<T, true, 256, 0>(p, ws, st);
+  if (bw <= 128) return launch_bwd_t<T, true, 512, 0>(p, ws, st);
+  if (bw <= 512) return launch_bwd_t<T, false, 512, 0>(p, ws, st);
+  return launch_bwd_t<T, false, 1024, 0>(p, ws, st);
 }
 
 }  // namespace

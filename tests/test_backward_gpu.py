@@ -1,7 +1,9 @@
 """GPU parity of the backward (rglru_bwd through the C ABI) against the float64
 backward oracle (oracle/rglru_backward.py, itself pinned by finite differences).
 
-Bars: fp32 I/O 1e-4, bf16 I/O 2e-2, as for the forward. dx and the conv
+Bars: fp32 I/O 1e-4, bf16 I/O 2e-2, as for the forward. For bf16 I/O and heads
+32, 64 or 128 wide the two in-loop gate contractions run on the tensor cores
+with bf16 operands (u and d z rounded like the forward's u), the rest in fp32. dx and the conv
 history's gradient use the forward's metric: max |g - o| / max(|o|, per-channel
 RMS of o); dh0 is floored at its RMS over the whole tensor. Parameter gradients,
 which sum over every token, use the norm-wise max |g - o| / max |o| per tensor.
@@ -34,6 +36,10 @@ CASES = [
     WORKLOADS["hawk_block"].with_shape(B=1, T=700, D=256, H=2, h0_var=0.5, seed=46),
     WORKLOADS["tiny_f32"].with_shape(B=1, T=90, D=1024, H=1, h0_var=0.5, seed=47),
     WORKLOADS["hawk_block"].with_shape(B=2, T=2048, D=1024, H=16, h0_var=0.1, seed=48),
+    # 32-wide heads (8 segments per block) and 96-wide heads (5 segments of 96
+    # threads, weights in shared memory, CUDA-core contractions)
+    WORKLOADS["hawk_block"].with_shape(B=2, T=77, D=128, H=4, h0_var=0.5, bias_std=0.5, seed=49),
+    WORKLOADS["hawk_block"].with_shape(B=1, T=50, D=192, H=2, h0_var=0.5, seed=50),
 ]
 
 
