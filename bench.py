@@ -392,8 +392,10 @@ def run_backward(rg, wl, g, w, dev, a, pk):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "traffic": None,
                          "algorithmic_bytes_per_launch": bytes_step,
-                         "note": "step time of all five launches; fp32 CUDA-core arithmetic "
-                                 "(three gate contractions of 2 bw MACs per channel-token); "
+                         "note": "step time of all five launches; the three gate "
+                                 "contractions (2 bw MACs per channel-token each) on the "
+                                 "tensor cores (bf16 operands, fp32 accumulate) for bf16 I/O "
+                                 "with 32/64/128-wide heads, the rest fp32 on CUDA cores; "
                                  "fp32 intermediates in a workspace (z_a, z_x, u, d u: 16 B "
                                  "per channel-token written and re-read) are not algorithmic"}}
 

@@ -3,7 +3,10 @@
 // Attention for Efficient Language Models", section "Model Architecture"
 // defines the forward; the backward is the chain rule through it, run as
 // linear scans in both time directions, the forward's scheme in S. De's
-// thread). fp32 arithmetic on CUDA cores for any I/O type.
+// thread). fp32 arithmetic, except that for bf16 I/O with heads 32, 64 or
+// 128 wide the three gate contractions run on the tensor cores (warp-level
+// bf16 MMA with fp32 accumulation, operands rounded to bf16 like the forward's
+// u); fp32 I/O keeps them on CUDA cores.
 //
 // Time is cut into segments of L tokens (L a multiple of the 8-token group);
 // a block holds S segments of one head and batch row, thread (sl, j) owning
@@ -29,9 +32,9 @@
 //                 d la = d a a - d g a^2 / g, la = -c r sp, z -> r, i by sigmoid;
 //                 it accumulates d b_a, d b_x and d Lambda per channel and writes
 //                 u, d z_a, d z_x (over z_a, z_x) and d u to the workspace;
-//   K4 weights    d W[h] = U_h^T dZ_h for both gates (64 x 64 tiles, 4 x 4 per
-//                 thread, the token sum split over blocks and combined with
-//                 atomics);
+//   K4 weights    d W[h] = U_h^T dZ_h for both gates (64 x 64 tiles, the token
+//                 sum split over blocks and combined with atomics; tensor cores
+//                 or 4 x 4 FFMA tiles per thread);
 //   K5 conv       d x_t = sum_k w[k] d u_{t+3-k} (t < 0: the conv history's
 //                 gradient) and d w[k] = sum_t x_{t-3+k} d u_t.
 // The path of d z_a through g carries r / g, which tends to 0 with r
@@ -212,6 +215,43 @@ struct TcGeo {
   static_assert(MT % 2 == 0 && MT * (kBW / 8) == 2 * (kThreads / 32), "two tiles per warp");
 };
 
+// Gate math of the backward in fp32 with about 1e-6 relative error: sigmoid
+// and exp through the hardware base-2 exponential, approximate reciprocal and
+// reciprocal square root; 1 - a^2 = -expm1(2 log a) by its Taylor series
+// -x (1 + x/2 + x^2/6 + ... + x^6/5040) for |x| < 0.5 (truncation below 3e-7
+// relative) and as 1 - e^x beyond (no cancellation there).
+__device__ __forceinline__ float sigmoid_fast(float z) {
+  return __fdividef(1.0f, 1.0f + __expf(-z));
+}
+
+__device__ __forceinline__ float neg_expm1_fast(float x) {   // x <= 0
+  float p = fmaf(x, 1.f / 5040.f, 1.f / 720.f);
+  p = fmaf(x, p, 1.f / 120.f);
+  p = fmaf(x, p, 1.f / 24.f);
+  p = fmaf(x, p, 1.f / 6.f);
+  p = fmaf(x, p, 0.5f);
+  p = fmaf(x, p, 1.0f);
+  return x > -0.5f ? -x * p : 1.0f - __expf(x);
+}
+
+// r, i, a = e^(log a), g = sqrt(1 - a^2) and r / g (0 where g = 0) of one token.
+struct TokGates {
+  float r, i, a, g, rog;
+};
+
+__device__ __forceinline__ TokGates tok_gates(float za, float zx, float neg_c_sp) {
+  TokGates t;
+  t.r = sigmoid_fast(za);
+  t.i = sigmoid_fast(zx);
+  const float la = neg_c_sp * t.r;
+  t.a = __expf(la);
+  const float om = neg_expm1_fast(2.0f * la);
+  const float rs = om > 0.f ? rsqrtf(om) : 0.f;
+  t.g = om * rs;
+  t.rog = t.r * rs;
+  return t;
+}
+
 // The post-contraction part of a K1 group: decay, input, the local scan and
 // the running R; z_a, z_x of the live tokens to the workspace.
 template <typename T>
@@ -225,10 +265,9 @@ __device__ __forceinline__ void gates_scan_group(const float (&za)[kTB], const f
   for (int k = 0; k < kTB; ++k) {
     const int t = tb + k;
     if (t < t1) {
-      float a, beta, la;
-      decay_and_input(za[k], zx[k], u[k], neg_c_sp, a, beta, la);
-      Hl = fmaf(a, Hl, beta);
-      P *= a;
+      const TokGates q = tok_gates(za[k], zx[k], neg_c_sp);
+      Hl = fmaf(q.a, Hl, q.g * (q.i * u[k]));
+      P *= q.a;
       const size_t o = orow + (size_t)t * D;
       R = fmaf(P, ldg_f32(dyb + o), R);
       ws_za[o] = za[k];
@@ -491,12 +530,8 @@ __device__ __forceinline__ void final_group(const BwdThread &th, const ChanC &c,
     const float za = in ? ws_za[o] : 0.f;
     const float zx = in ? ws_zx[o] : 0.f;
     if (in) ws_u[o] = u[k];
-    const float r = sigmoid_f32(za);
-    const float ig = sigmoid_f32(zx);
-    const float la = neg_c_sp * r;
-    const float a = expf(la);
-    const float gg = sqrtf(-expm1f(2.0f * la));
-    const float rog = gg > 0.f ? r / gg : 0.f;
+    const TokGates tg = tok_gates(za, zx, neg_c_sp);
+    const float r = tg.r, ig = tg.i, a = tg.a, gg = tg.g, rog = tg.rog;
     const float q = a * (a * ig * u[k] * rog - hh * r);
     fa[k] = a;
     fq[k] = q;
@@ -812,6 +847,110 @@ bwd_dw_kernel(const float *__restrict__ U, const float *__restrict__ dZa,
     }
 }
 
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&a)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ uint2 f4_to_bf16x4(float4 v) {
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
+  const __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
+  return make_uint2(*reinterpret_cast<const uint32_t *>(&lo),
+                    *reinterpret_cast<const uint32_t *>(&hi));
+}
+
+// d W on the tensor cores (bf16 I/O, heads a multiple of 64 wide): the same
+// 64 x 64 (i, j) tiles and token chunks as bwd_dw_kernel, 4 warps each a
+// 32 x 32 quarter. 32 tokens of U and dZ are staged as bf16 token-major rows
+// (padded by 8 elements); with A[i][n] = U[n][i] and B[n][j] = dZ[n][j], both
+// fragments come from ldmatrix .trans of those rows (a thread receives stored
+// elements (2q, g) and (2q + 1, g) of each 8 x 8 block: the k pairs of column
+// g). The next 32 tokens are in flight to registers during the MMAs.
+constexpr int kDwTcThreads = 128, kDwTcStride = kDwTile + 8;
+
+__global__ void __launch_bounds__(kDwTcThreads)
+bwd_dw_tc_kernel(const float *__restrict__ U, const float *__restrict__ dZa,
+                 const float *__restrict__ dZx, float *__restrict__ dWa, float *__restrict__ dWx,
+                 int N, int D, int H, int chunk) {
+  __shared__ __align__(16) __nv_bfloat16 us[kDwRows][kDwTcStride];
+  __shared__ __align__(16) __nv_bfloat16 zs[kDwRows][kDwTcStride];
+  const int bw = D / H;
+  const int tiles = bw / kDwTile;
+  int tile = blockIdx.x;
+  const int gate = tile & 1;
+  tile >>= 1;
+  const int ti = tile % tiles, tj = (tile / tiles) % tiles, h = tile / (tiles * tiles);
+  const float *Z = gate == 0 ? dZa : dZx;
+  float *dW = gate == 0 ? dWa : dWx;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int wi = (warp & 1) * 32, wj = (warp >> 1) * 32;
+  const int i0 = ti * kDwTile, j0 = tj * kDwTile;
+  // loader: rows lr + 8 q, columns lc .. lc + 3 (16-byte fp32 loads)
+  const int lr = tid >> 4, lc = (tid & 15) * 4;
+  const float *Uc = U + (size_t)h * bw + i0 + lc;
+  const float *Zc = Z + (size_t)h * bw + j0 + lc;
+  const int n_begin = blockIdx.y * chunk, n_end = min(N, n_begin + chunk);
+  float4 pu[kDwRows / 8], pz[kDwRows / 8];
+  auto fetch = [&](int n0) {
+#pragma unroll
+    for (int q = 0; q < kDwRows / 8; ++q) {
+      const int n = n0 + lr + 8 * q;
+      const bool ok = n < n_end;
+      pu[q] = ok ? *reinterpret_cast<const float4 *>(Uc + (size_t)n * D) : make_float4(0, 0, 0, 0);
+      pz[q] = ok ? *reinterpret_cast<const float4 *>(Zc + (size_t)n * D) : make_float4(0, 0, 0, 0);
+    }
+  };
+  // ldmatrix lane rows: A blocks (n-block q / 2, i-block q % 2), B blocks (n-block q % 2,
+  // j-block q / 2), q = lane / 8
+  const int lq = lane >> 3, lrow = lane & 7;
+  const uint32_t a_lane = shared_addr(&us[lrow + (lq >> 1) * 8][wi + (lq & 1) * 8]);
+  const uint32_t b_lane = shared_addr(&zs[lrow + (lq & 1) * 8][wj + (lq >> 1) * 8]);
+  constexpr uint32_t kRowBytes = kDwTcStride * 2;
+  float acc[2][4][4];
+#pragma unroll
+  for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mi][nt][e] = 0.f;
+  fetch(n_begin);
+  for (int n0 = n_begin; n0 < n_end; n0 += kDwRows) {
+#pragma unroll
+    for (int q = 0; q < kDwRows / 8; ++q) {
+      *reinterpret_cast<uint2 *>(&us[lr + 8 * q][lc]) = f4_to_bf16x4(pu[q]);
+      *reinterpret_cast<uint2 *>(&zs[lr + 8 * q][lc]) = f4_to_bf16x4(pz[q]);
+    }
+    __syncthreads();
+    if (n0 + kDwRows < n_end) fetch(n0 + kDwRows);
+#pragma unroll
+    for (int ks = 0; ks < kDwRows / 16; ++ks) {
+      uint32_t a[2][4], b[2][4];
+#pragma unroll
+      for (int mi = 0; mi < 2; ++mi) ldsm_x4_trans(a_lane + ks * 16 * kRowBytes + mi * 32, a[mi]);
+#pragma unroll
+      for (int np = 0; np < 2; ++np) ldsm_x4_trans(b_lane + ks * 16 * kRowBytes + np * 32, b[np]);
+#pragma unroll
+      for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+          mma_bf16(acc[mi][nt], a[mi], b[nt >> 1][(nt & 1) * 2], b[nt >> 1][(nt & 1) * 2 + 1]);
+    }
+    __syncthreads();
+  }
+  const int fg = lane >> 2, fq = lane & 3;
+#pragma unroll
+  for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = i0 + wi + mi * 16 + fg + (e >= 2 ? 8 : 0);
+        const int jj = j0 + wj + nt * 8 + 2 * fq + (e & 1);
+        atomicAdd(dW + ((size_t)h * bw + i) * bw + jj, acc[mi][nt][e]);
+      }
+}
+
 // d x (and the conv history's gradient) from d u, and d w per channel, for one
 // chunk of kConvChunk extended positions m (x_{m-3}) of one batch row; thread
 // per channel, the last three d u values in registers:
@@ -959,8 +1098,12 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
   const int tile_blocks = 2 * tiles * tiles * p.H;
   const int nchunk = ceil_div(8 * 148, tile_blocks);
   const int chunk = ceil_div(ceil_div(N, nchunk), kDwRows) * kDwRows;
-  bwd_dw_kernel<<<dim3(tile_blocks, ceil_div(N, chunk)), kDwThreads, 0, st>>>(
-      U, za, zx, p.dW_a, p.dW_x, N, p.D, p.H, chunk);
+  if (kTcBW > 0 && bw % kDwTile == 0)
+    bwd_dw_tc_kernel<<<dim3(tile_blocks, ceil_div(N, chunk)), kDwTcThreads, 0, st>>>(
+        U, za, zx, p.dW_a, p.dW_x, N, p.D, p.H, chunk);
+  else
+    bwd_dw_kernel<<<dim3(tile_blocks, ceil_div(N, chunk)), kDwThreads, 0, st>>>(
+        U, za, zx, p.dW_a, p.dW_x, N, p.D, p.H, chunk);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   bwd_conv_kernel<T><<<dim3(ceil_div(p.D, kConvThreads), p.B, ceil_div(p.T + 3, kConvChunk)),
                        kConvThreads, 0, st>>>(p, du);
