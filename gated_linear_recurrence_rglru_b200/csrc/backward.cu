@@ -215,6 +215,11 @@ struct TcGeo {
   static_assert(MT % 2 == 0 && MT * (kBW / 8) == 2 * (kThreads / 32), "two tiles per warp");
 };
 
+// Brings the line holding p into L1 ahead of its load (a hint: no result, no fault).
+__device__ __forceinline__ void prefetch_l1(const void *p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
 // Gate math of the backward in fp32 with about 1e-6 relative error: sigmoid
 // and exp through the hardware base-2 exponential, approximate reciprocal and
 // reciprocal square root; 1 - a^2 = -expm1(2 log a) by its Taylor series
@@ -414,6 +419,12 @@ bwd_gates_tc_kernel(BwdArgs p, BwdPlan pl, float *__restrict__ ws_A, float *__re
       ws_gP[go] = P;
       ws_gH[go] = Hl;
       conv_group<T>(xb, cs_in_b, D, th.d, tb, th.t1, c, u);
+      // this group's dy rows and the next group's x rows
+#pragma unroll
+      for (int k = 0; k < kTB; ++k) {
+        if (tb + k < th.t1) prefetch_l1(dyb + orow + (size_t)(tb + k) * D);
+        if (tb + kTB + k < th.t1) prefetch_l1(xb + (size_t)(tb + kTB + k) * D + th.d);
+      }
     } else {
 #pragma unroll
       for (int k = 0; k < kTB; ++k) u[k] = 0.f;
@@ -518,6 +529,18 @@ __device__ __forceinline__ void final_group(const BwdThread &th, const ChanC &c,
                                             float &acc_ba, float &acc_bx, float (&dub)[kTB],
                                             Sink sink) {
   const float neg_c_sp = -kDecayC * c.sp, csp = kDecayC * c.sp;
+  if (tb - kTB >= th.t0) {
+    // the group processed next (8 tokens earlier): its z and dy rows
+    const float *pza = ws_za + orow + (size_t)(tb - kTB) * D;
+    const float *pzx = ws_zx + orow + (size_t)(tb - kTB) * D;
+    const T *pdy = dyb + orow + (size_t)(tb - kTB) * D;
+#pragma unroll
+    for (int k = 0; k < kTB; ++k) {
+      prefetch_l1(pza + (size_t)k * D);
+      prefetch_l1(pzx + (size_t)k * D);
+      prefetch_l1(pdy + (size_t)k * D);
+    }
+  }
   float u[kTB];
   conv_group<T>(xb, cs_in_b, D, th.d, tb, th.t1, c, u);
   float fa[kTB], fza[kTB], fq[kTB], fzx[kTB], fu[kTB];

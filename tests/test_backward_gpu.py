@@ -40,6 +40,8 @@ CASES = [
     # threads, weights in shared memory, CUDA-core contractions)
     WORKLOADS["hawk_block"].with_shape(B=2, T=77, D=128, H=4, h0_var=0.5, bias_std=0.5, seed=49),
     WORKLOADS["hawk_block"].with_shape(B=1, T=50, D=192, H=2, h0_var=0.5, seed=50),
+    # the bench workload itself (B=8, T=2048, D=1024, H=16, bf16), every output
+    WORKLOADS["hawk_block"],
 ]
 
 
