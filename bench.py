@@ -287,6 +287,8 @@ def run_ours(a, ws, rank, local):
         out["decode"] = run_decode(rg, dev, a, pk)
     if a.backward:
         out["backward"] = run_backward(rg, wl, g, w, dev, a, pk)
+    if a.block:
+        out["block"] = run_block(rg, wl, dev, a, pk)
     if a.cpu_baseline and ws == 1 and rank == 0:
         out["cpu_baseline"] = cpu_baseline(wl, t, a.cpu_seconds)
     return out
@@ -398,6 +400,52 @@ def run_backward(rg, wl, g, w, dev, a, pk):
                                  "with 32/64/128-wide heads, the rest fp32 on CUDA cores; "
                                  "fp32 intermediates in a workspace (z_a, z_x, u, d u: 16 B "
                                  "per channel-token written and re-read) are not algorithmic"}}
+
+
+def run_block(rg, wl, dev, a, pk):
+    """The recurrent block around the layer on the same workload (Dm = D): input and
+    gate projections, the layer, GeLU gating and the output projection, one
+    rglru_block_fwd per step, inputs resident, three rotating x / out sets."""
+    from gated_linear_recurrence_rglru_b200.workloads import generate_block
+    B, T, D, H = wl.B, wl.T, wl.D, wl.H
+    Dm = D
+    t = generate_block(wl, Dm)
+    gd = {k: (v.to(dev) if v is not None else None) for k, v in t.items()}
+    wts = [gd[k] for k in ("W_in", "W_gate", "W_out", "conv_w", "W_a", "b_a", "W_x", "b_x",
+                           "Lambda")]
+    nsets = 3
+    xs = [gd["x"]] + [torch.randn_like(gd["x"], dtype=torch.float32).to(wl.dtype)
+                      for _ in range(nsets - 1)]
+    outs = [torch.empty_like(gd["x"]) for _ in range(nsets)]
+    ws = torch.empty(rg.block_fwd_workspace_bytes(B, T, Dm, D, H, wl.dtype), device=dev,
+                     dtype=torch.uint8)
+
+    def step(i):
+        k = i % nsets
+        rg.rglru_block_fwd(xs[k], *wts, h0=gd["h0"], out=outs[k], workspace=ws,
+                           want_state=False)
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    steps = max(5, min(a.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    flops = 3 * 2 * B * T * Dm * D
+    tfs = flops / (ms / 1e3) / 1e12
+    return {"workload": f"{wl.name} recurrent block B={B} T={T} Dm={Dm} D={D} H={H} io={wl.io}",
+            "value": B * T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+            "roofline": {"bound": "tensor", "achieved": tfs, "peak": pk["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": tfs / pk["bf16_tflops"], "traffic": None,
+                         "algorithmic_flops_per_step": flops,
+                         "note": "three dense projections (cuBLAS, bf16, fp32 accumulate) "
+                                 "over the step time, which also holds the layer and the "
+                                 "GeLU gating (HBM-bound, about 45 and 15 us)"}}
 
 
 def run_decode(rg, dev, a, pk):
@@ -540,6 +588,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-decode", dest="decode", action="store_false")
     ap.add_argument("--no-backward", dest="backward", action="store_false")
+    ap.add_argument("--no-block", dest="block", action="store_false")
     ap.add_argument("--decode-steps", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

@@ -24,7 +24,8 @@ EXPORTED = (
     "rglru_status_str", "rglru_version", "rglru_fwd_workspace_bytes", "rglru_fwd",
     "rglru_fwd_algo", "rglru_decode_step", "rglru_decode_step_algo", "rglru_fwd_launches",
     "rglru_fwd_noalloc", "rglru_decode_launches", "rglru_fwd_ex", "rglru_bwd",
-    "rglru_bwd_workspace_bytes", "rglru_bwd_launches",
+    "rglru_bwd_workspace_bytes", "rglru_bwd_launches", "rglru_block_fwd",
+    "rglru_block_fwd_workspace_bytes",
 )
 
 
@@ -80,6 +81,11 @@ def _load():
     lib.rglru_bwd.restype = i32
     lib.rglru_bwd.argtypes = ([vp] * 6 + [fp, fp, vp, vp, fp, vp] + [fp] * 8 + [i32] * 5
                               + [vp, sz, vp])
+    lib.rglru_block_fwd_workspace_bytes.restype = sz
+    lib.rglru_block_fwd_workspace_bytes.argtypes = [i32] * 6
+    lib.rglru_block_fwd.restype = i32
+    lib.rglru_block_fwd.argtypes = ([vp] * 9 + [fp, fp, vp, vp, fp, vp] + [i32] * 6
+                                    + [vp, sz, ip, vp])
     return lib
 
 
@@ -292,3 +298,56 @@ def rglru_bwd(x, conv_w, W_a, b_a, W_x, b_x, Lambda, dy, h0=None, conv_state_in=
     if st != 0:
         raise RGLRUError(st, "rglru_bwd")
     return g
+
+
+def block_fwd_workspace_bytes(B: int, T: int, Dm: int, D: int, H: int,
+                              dtype=torch.bfloat16) -> int:
+    """Workspace of rglru_block_fwd (include/rglru.h)."""
+    n = LIB.rglru_block_fwd_workspace_bytes(B, T, Dm, D, H, _io_of(dtype))
+    if n == 0:
+        raise RGLRUError(1, "rglru_block_fwd_workspace_bytes")
+    return n
+
+
+def rglru_block_fwd(x, W_in, W_gate, W_out, conv_w, W_a, b_a, W_x, b_x, Lambda, h0=None,
+                    conv_state_in=None, *, out=None, h_T=None, conv_state_out=None,
+                    workspace=None, dev_status=None, stream=None, want_state=True):
+    """Recurrent block around the layer (include/rglru.h, rglru_block_fwd):
+    out = (layer(x W_in) * GeLU(x W_gate)) W_out over x (B, T, Dm).
+    Returns (out, h_T, conv_state_out) of the layer inside."""
+    if x.dim() != 3:
+        raise ValueError("x must be (B, T, Dm)")
+    B, T, Dm = x.shape
+    D = W_in.shape[1]
+    H = W_a.shape[0]
+    bw = D // H if H else 0
+    dt = x.dtype
+    io = _io_of(dt)
+    dev = x.device
+    if out is None:
+        out = torch.empty_like(x)
+    if want_state and h_T is None:
+        h_T = torch.empty(B, D, device=dev, dtype=torch.float32)
+    if want_state and conv_state_out is None:
+        conv_state_out = torch.empty(B, 3, D, device=dev, dtype=dt)
+    if workspace is None:
+        workspace = torch.empty(block_fwd_workspace_bytes(B, T, Dm, D, H, dt), device=dev,
+                                dtype=torch.uint8)
+    st = LIB.rglru_block_fwd(
+        _ptr(x, "x", dt), _ptr(W_in, "W_in", dt, (Dm, D)), _ptr(W_gate, "W_gate", dt, (Dm, D)),
+        _ptr(W_out, "W_out", dt, (D, Dm)), _ptr(conv_w, "conv_w", dt, (4, D)),
+        _ptr(W_a, "W_a", dt, (H, bw, bw)), _ptr(b_a, "b_a", dt, (D,)),
+        _ptr(W_x, "W_x", dt, (H, bw, bw)), _ptr(b_x, "b_x", dt, (D,)),
+        _ptr(Lambda, "Lambda", torch.float32, (D,)),
+        _ptr(h0, "h0", torch.float32, (B, D), optional=True),
+        _ptr(conv_state_in, "conv_state_in", dt, (B, 3, D), optional=True),
+        _ptr(out, "out", dt, (B, T, Dm)),
+        _ptr(h_T, "h_T", torch.float32, (B, D), optional=True),
+        _ptr(conv_state_out, "conv_state_out", dt, (B, 3, D), optional=True),
+        B, T, Dm, D, H, io,
+        _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _ptr(dev_status, "dev_status", torch.int32, optional=True), _stream_handle(stream))
+    if st != 0:
+        raise RGLRUError(st, "rglru_block_fwd")
+    return out, h_T, conv_state_out
+

@@ -234,3 +234,46 @@ int rglru_bwd(const void *x, const void *conv_w, const void *W_a, const void *b_
 }
 
 }  // extern "C"
+
+extern "C" {
+
+size_t rglru_block_fwd_workspace_bytes(int B, int T, int Dm, int D, int H, int io) {
+  if (check_shape(B, T, D, H, io) != RGLRU_OK || Dm < 8 || Dm % 8 != 0) return 0;
+  return block_layout(B, T, D, io, rglru_fwd_workspace_bytes(B, T, D, H, io)).total;
+}
+
+int rglru_block_fwd(const void *x, const void *W_in, const void *W_gate, const void *W_out,
+                    const void *conv_w, const void *W_a, const void *b_a, const void *W_x,
+                    const void *b_x, const float *Lambda, const float *h0,
+                    const void *conv_state_in, void *out, float *h_T, void *conv_state_out,
+                    int B, int T, int Dm, int D, int H, int io, void *workspace,
+                    size_t workspace_bytes, int *dev_status, void *stream) {
+  int st = check_shape(B, T, D, H, io);
+  if (st != RGLRU_OK) return st;
+  if (Dm < 8 || Dm % 8 != 0) return RGLRU_ERR_INVALID_ARG;
+  const void *req[] = {x, W_in, W_gate, W_out, out};
+  for (const void *p : req)
+    if (p == nullptr || !aligned16(p)) return RGLRU_ERR_INVALID_ARG;
+  const size_t eb = io_bytes(io);
+  if (overlap(out, (size_t)B * T * Dm * eb, x, (size_t)B * T * Dm * eb))
+    return RGLRU_ERR_INVALID_ARG;
+  const size_t fwd_ws = rglru_fwd_workspace_bytes(B, T, D, H, io);
+  const BlockLayout L = block_layout(B, T, D, io, fwd_ws);
+  if (workspace == nullptr || !aligned16(workspace) || workspace_bytes < L.total)
+    return RGLRU_ERR_WORKSPACE;
+  unsigned char *w = static_cast<unsigned char *>(workspace);
+  void *xr = w + L.off_xr, *g = w + L.off_g, *y = w + L.off_y, *fw = w + L.off_fwd;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int M = B * T;
+  if ((st = launch_block_gemm(io, M, D, Dm, x, W_in, xr, s)) != RGLRU_OK) return st;
+  if ((st = launch_block_gemm(io, M, D, Dm, x, W_gate, g, s)) != RGLRU_OK) return st;
+  st = rglru_fwd(xr, conv_w, W_a, b_a, W_x, b_x, Lambda, h0, conv_state_in, y, h_T,
+                 conv_state_out, B, T, D, H, io, fw, workspace_bytes - L.off_fwd, dev_status,
+                 stream);
+  if (st != RGLRU_OK) return st;
+  if (launch_gelu_gate(io, y, g, (size_t)M * D, s) != cudaSuccess) return RGLRU_ERR_CUDA;
+  return launch_block_gemm(io, M, Dm, D, y, W_out, out, s);
+}
+
+}  // extern "C"
+

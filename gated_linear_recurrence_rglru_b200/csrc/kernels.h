@@ -52,6 +52,17 @@ int generic_kernel_launches(int B, int T, int H);
 size_t bwd_workspace_bytes(int B, int T, int D, int H);
 int bwd_launches();
 cudaError_t launch_bwd(const BwdArgs &p, int io, void *ws, cudaStream_t st);
+
+// Recurrent block around the layer (block.cu): workspace offsets of x W_in,
+// x W_gate, the layer output y and the layer's own forward workspace.
+struct BlockLayout {
+  size_t off_xr, off_g, off_y, off_fwd, total;
+};
+BlockLayout block_layout(int B, int T, int D, int io, size_t fwd_ws);
+// Row-major C[M x N] = A[M x K] B[K x N] in the I/O type (cuBLAS); an RGLRU_* status.
+int launch_block_gemm(int io, int M, int N, int K, const void *A, const void *B, void *C,
+                      cudaStream_t st);
+cudaError_t launch_gelu_gate(int io, void *y, const void *g, size_t n, cudaStream_t st);
 cudaError_t launch_fwd_generic(const FwdArgs &p, int io, void *ws, cudaStream_t st);
 cudaError_t launch_decode_generic(const DecArgs &p, int io, cudaStream_t st);
 

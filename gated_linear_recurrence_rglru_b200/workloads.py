@@ -27,6 +27,9 @@ Recipe (every workload, in this draw order from one torch CPU generator):
 Lambda, h0 and every recurrent state are fp32 whatever the I/O dtype.
 The decode workload then draws h ~ N(0, 1), the conv ring ~ N(0, 1) and the
 256 per-step inputs x_t ~ N(0, 1).
+The recurrent block around the layer (generate_block) adds, from a second
+generator, the block input x (B, T, Dm) ~ N(0, 1) and its projections W_in,
+W_gate (Dm, D) ~ N(0, 1/Dm) and W_out (D, Dm) ~ N(0, 1/D).
 """
 from __future__ import annotations
 
@@ -129,3 +132,23 @@ def generate(wl: Workload) -> dict:
         out["b_a"] = _normal(gen, (D,), wl.bias_std, dt)
         out["b_x"] = _normal(gen, (D,), wl.bias_std, dt)
     return out
+
+
+def generate_block(wl: Workload, Dm: int) -> dict:
+    """Inputs of the recurrent block around the layer: the layer's parameters of
+    generate(wl) (its x unused), the block input x (B, T, Dm) ~ N(0, 1) and the
+    projections W_in, W_gate (Dm, D) ~ N(0, 1/Dm), W_out (D, Dm) ~ N(0, 1/D)
+    (variance 1/fan-in), drawn in that order from a second generator seeded
+    with seed + 7919."""
+    out = generate(wl)
+    out.pop("x", None)
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(wl.seed + 7919)
+    B, T, D = wl.B, wl.T, wl.D
+    dt = wl.dtype
+    out["x"] = _normal(gen, (B, T, Dm), 1.0, dt)
+    out["W_in"] = _normal(gen, (Dm, D), 1.0 / math.sqrt(Dm), dt)
+    out["W_gate"] = _normal(gen, (Dm, D), 1.0 / math.sqrt(Dm), dt)
+    out["W_out"] = _normal(gen, (D, Dm), 1.0 / math.sqrt(D), dt)
+    return out
+

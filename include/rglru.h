@@ -252,8 +252,10 @@ int rglru_decode_step_algo(const void *x_t, void *conv_state, int pos, float *h,
  * (the call overwrites them; it does not add to their contents).
  * workspace: device memory of rglru_bwd_workspace_bytes(B, T, D, H, io) bytes,
  * 16-byte aligned, not shared with a concurrent call.
- * Arithmetic is fp32 on CUDA cores for both I/O types; any head width up to
- * 1024 that divides D. Returns RGLRU_OK, INVALID_ARG (shapes, NULL required
+ * Arithmetic is fp32, except that for bf16 I/O with heads 32, 64 or 128 wide
+ * the three gate contractions (z = u W, d z W^T, U^T dZ) run on the tensor
+ * cores with bf16 operands and fp32 accumulation; any head width up to 1024
+ * that divides D. Returns RGLRU_OK, INVALID_ARG (shapes, NULL required
  * pointers, alignment, overlaps), WORKSPACE or CUDA. Nothing in the backward
  * waits on another block, so it has no device-side status.
  */
@@ -268,6 +270,36 @@ int rglru_bwd(const void *x, const void *conv_w, const void *W_a, const void *b_
 
 /* Number of kernel launches of one rglru_bwd call (0 on invalid arguments). */
 int rglru_bwd_launches(int B, int T, int D, int H, int io);
+
+/*
+ * Recurrent block around the layer ("Griffin: Mixing Gated Linear Recurrences
+ * with Local Attention for Efficient Language Models", section "Model
+ * Architecture": a temporal Conv1D and the RG-LRU inside a recurrent block;
+ * the model's MLP is GeLU-gated). Read as two branches of the block
+ * input x (B, T, Dm):
+ *   g   = GeLU(x W_gate)              GeLU(v) = v (1 + erf(v / sqrt 2)) / 2
+ *   y   = rglru_fwd(x W_in)           the layer above, with h0 / conv_state_in
+ *   out = (y * g) W_out               (B, T, Dm)
+ * Shapes (row-major, the I/O dtype): x (B, T, Dm), W_in and W_gate (Dm, D),
+ * W_out (D, Dm), out (B, T, Dm); the layer's parameters, h0, conv_state_in,
+ * h_T and conv_state_out as for rglru_fwd (the state and conv history are the
+ * layer's, over D channels). Dm >= 8 and a multiple of 8.
+ * The three projections are dense GEMMs run by cuBLAS with fp32 accumulation
+ * (fp32 I/O: no TF32); x W_in, x W_gate and y are kept in the I/O dtype in
+ * the workspace; GeLU and the product are one kernel of this library.
+ * workspace: rglru_block_fwd_workspace_bytes(...) bytes of device memory,
+ * 16-byte aligned. out must not overlap x. dev_status as for rglru_fwd.
+ * Returns RGLRU_OK, INVALID_ARG, UNSUPPORTED, WORKSPACE or CUDA (including a
+ * cuBLAS failure).
+ */
+size_t rglru_block_fwd_workspace_bytes(int B, int T, int Dm, int D, int H, int io);
+
+int rglru_block_fwd(const void *x, const void *W_in, const void *W_gate, const void *W_out,
+                    const void *conv_w, const void *W_a, const void *b_a, const void *W_x,
+                    const void *b_x, const float *Lambda, const float *h0,
+                    const void *conv_state_in, void *out, float *h_T, void *conv_state_out,
+                    int B, int T, int Dm, int D, int H, int io, void *workspace,
+                    size_t workspace_bytes, int *dev_status, void *stream);
 
 #ifdef __cplusplus
 }
