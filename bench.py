@@ -397,7 +397,7 @@ def run_backward(rg, wl, g, w, dev, a, pk):
                          "note": "step time of all five launches; the three gate "
                                  "contractions (2 bw MACs per channel-token each) on the "
                                  "tensor cores (bf16 operands, fp32 accumulate) for bf16 I/O "
-                                 "with 32/64/128-wide heads, the rest fp32 on CUDA cores; "
+                                 "with 64/128-wide heads, the rest fp32 on CUDA cores; "
                                  "fp32 intermediates in a workspace (z_a, z_x, u, d u: 16 B "
                                  "per channel-token written and re-read) are not algorithmic"}}
 

@@ -4,14 +4,17 @@
 // defines the forward; the backward is the chain rule through it, run as
 // linear scans in both time directions, the forward's scheme in S. De's
 // thread). fp32 arithmetic, except that for bf16 I/O with heads 32, 64 or
-// 128 wide the three gate contractions run on the tensor cores (warp-level
-// bf16 MMA with fp32 accumulation, operands rounded to bf16 like the forward's
-// u); fp32 I/O keeps them on CUDA cores.
+// 128 wide the two in-loop gate contractions (z = u W in K1, d z W^T in K3),
+// and d W = U^T dZ for heads 64 or 128 wide, run on the tensor cores
+// (warp-level bf16 MMA with fp32 accumulation, operands rounded to bf16 like
+// the forward's u); fp32 I/O keeps them on CUDA cores.
 //
 // Time is cut into segments of L tokens (L a multiple of the 8-token group);
 // a block holds S segments of one head and batch row, thread (sl, j) owning
-// channel h*bw + j of segment sl, with the head's gate weights staged once in
-// shared memory for all of them:
+// channel h*bw + j of segment sl, with the head's gate weights loaded once
+// per block for all of them (fp32 rows in shared memory for the CUDA-core
+// contractions; MMA fragments in registers in K1, bf16 rows in shared memory
+// in K3 for the tensor-core ones):
 //   K1 gates      per segment, in time order: Conv1D u, both gate
 //                 pre-activations (z_a, z_x -> fp32 workspace), the local scan
 //                 from zero, whose (prod a, state) at each group start also go

@@ -253,9 +253,9 @@ int rglru_decode_step_algo(const void *x_t, void *conv_state, int pos, float *h,
  * workspace: device memory of rglru_bwd_workspace_bytes(B, T, D, H, io) bytes,
  * 16-byte aligned, not shared with a concurrent call.
  * Arithmetic is fp32, except that for bf16 I/O with heads 32, 64 or 128 wide
- * the three gate contractions (z = u W, d z W^T, U^T dZ) run on the tensor
- * cores with bf16 operands and fp32 accumulation; any head width up to 1024
- * that divides D. Returns RGLRU_OK, INVALID_ARG (shapes, NULL required
+ * the gate contractions z = u W and d z W^T (and U^T dZ for heads 64 or 128
+ * wide) run on the tensor cores with bf16 operands and fp32 accumulation; any
+ * head width up to 1024 that divides D. Returns RGLRU_OK, INVALID_ARG (shapes, NULL required
  * pointers, alignment, overlaps), WORKSPACE or CUDA. Nothing in the backward
  * waits on another block, so it has no device-side status.
  */
