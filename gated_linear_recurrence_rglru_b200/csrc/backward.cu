@@ -977,9 +977,33 @@ bwd_dw_tc_kernel(const float *__restrict__ U, const float *__restrict__ dZa,
       }
 }
 
+// Two adjacent channels of the I/O type as floats (p 2-element aligned), and back.
+template <typename T>
+__device__ __forceinline__ float2 ldg_pair(const T *p);
+template <>
+__device__ __forceinline__ float2 ldg_pair<float>(const float *p) {
+  return __ldg(reinterpret_cast<const float2 *>(p));
+}
+template <>
+__device__ __forceinline__ float2 ldg_pair<__nv_bfloat16>(const __nv_bfloat16 *p) {
+  const unsigned int w = __ldg(reinterpret_cast<const unsigned int *>(p));
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w));
+}
+template <typename T>
+__device__ __forceinline__ void st_pair(T *p, float2 v);
+template <>
+__device__ __forceinline__ void st_pair<float>(float *p, float2 v) {
+  *reinterpret_cast<float2 *>(p) = v;
+}
+template <>
+__device__ __forceinline__ void st_pair<__nv_bfloat16>(__nv_bfloat16 *p, float2 v) {
+  *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(v.x, v.y);
+}
+
 // d x (and the conv history's gradient) from d u, and d w per channel, for one
 // chunk of kConvChunk extended positions m (x_{m-3}) of one batch row; thread
-// per channel, the last three d u values in registers:
+// per two adjacent channels (paired 8-byte d u and 4- or 8-byte x loads), the
+// last three d u values in registers:
 //   d x_{m-3} = sum_k w[k] d u_{m-k},  d w[k] += x_{m-3} d u_{m-k}  (0 <= m-k < T).
 constexpr int kConvChunk = 64, kConvThreads = 256;
 
@@ -987,39 +1011,60 @@ template <typename T>
 __global__ void __launch_bounds__(kConvThreads)
 bwd_conv_kernel(BwdArgs p, const float *__restrict__ du) {
   const int D = p.D;
-  const int d = blockIdx.x * kConvThreads + threadIdx.x;
+  const int d = 2 * (blockIdx.x * kConvThreads + threadIdx.x);   // D is a multiple of 8
   const int b = blockIdx.y;
   if (d >= D) return;
   const int m_begin = blockIdx.z * kConvChunk, m_end = min(p.T + 3, m_begin + kConvChunk);
   const T *cw = static_cast<const T *>(p.conv_w);
-  float w[4];
+  float2 w[4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) w[k] = ldg_f32(cw + (size_t)k * D + d);
+  for (int k = 0; k < 4; ++k) w[k] = ldg_pair<T>(cw + (size_t)k * D + d);
   const float *dub = du + (size_t)b * p.T * D + d;
-  const T *xb = static_cast<const T *>(p.x) + (size_t)b * p.T * D;
-  const T *cs_in_b =
-      p.conv_state_in ? static_cast<const T *>(p.conv_state_in) + (size_t)b * 3 * D : nullptr;
+  const T *xb = static_cast<const T *>(p.x) + (size_t)b * p.T * D + d;
+  const T *csb = p.conv_state_in
+                     ? static_cast<const T *>(p.conv_state_in) + (size_t)b * 3 * D + d
+                     : nullptr;
   T *dxb = static_cast<T *>(p.dx) + (size_t)b * p.T * D + d;
-  auto du_at = [&](int t) { return (t >= 0 && t < p.T) ? dub[(size_t)t * D] : 0.f; };
-  float g1 = du_at(m_begin - 1), g2 = du_at(m_begin - 2), g3 = du_at(m_begin - 3);
-  float dw[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
+  auto du_at = [&](int t) {
+    return (t >= 0 && t < p.T) ? __ldg(reinterpret_cast<const float2 *>(dub + (size_t)t * D))
+                               : make_float2(0.f, 0.f);
+  };
+  auto x_at = [&](int t) {   // x_t, t >= -3 (t < 0: the conv history, or zeros)
+    if (t >= 0) return ldg_pair<T>(xb + (size_t)t * D);
+    if (csb != nullptr) return ldg_pair<T>(csb + (size_t)(3 + t) * D);
+    return make_float2(0.f, 0.f);
+  };
+  float2 g1 = du_at(m_begin - 1), g2 = du_at(m_begin - 2), g3 = du_at(m_begin - 3);
+  float2 dw[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) dw[k] = make_float2(0.f, 0.f);
+#pragma unroll 8
   for (int m = m_begin; m < m_end; ++m) {
-    const float g0 = du_at(m);
-    const float xv = hist_x(xb, cs_in_b, m - 3, D, d);
-    const float acc = fmaf(w[0], g0, fmaf(w[1], g1, fmaf(w[2], g2, w[3] * g3)));
-    dw[0] = fmaf(xv, g0, dw[0]);
-    dw[1] = fmaf(xv, g1, dw[1]);
-    dw[2] = fmaf(xv, g2, dw[2]);
-    dw[3] = fmaf(xv, g3, dw[3]);
-    if (m >= 3) dxb[(size_t)(m - 3) * D] = from_f32<T>(acc);
-    else if (p.dconv_state_in) p.dconv_state_in[((size_t)b * 3 + m) * D + d] = acc;
+    const float2 g0 = du_at(m);
+    const float2 xv = x_at(m - 3);
+    float2 acc;
+    acc.x = fmaf(w[0].x, g0.x, fmaf(w[1].x, g1.x, fmaf(w[2].x, g2.x, w[3].x * g3.x)));
+    acc.y = fmaf(w[0].y, g0.y, fmaf(w[1].y, g1.y, fmaf(w[2].y, g2.y, w[3].y * g3.y)));
+    dw[0].x = fmaf(xv.x, g0.x, dw[0].x);
+    dw[0].y = fmaf(xv.y, g0.y, dw[0].y);
+    dw[1].x = fmaf(xv.x, g1.x, dw[1].x);
+    dw[1].y = fmaf(xv.y, g1.y, dw[1].y);
+    dw[2].x = fmaf(xv.x, g2.x, dw[2].x);
+    dw[2].y = fmaf(xv.y, g2.y, dw[2].y);
+    dw[3].x = fmaf(xv.x, g3.x, dw[3].x);
+    dw[3].y = fmaf(xv.y, g3.y, dw[3].y);
+    if (m >= 3) st_pair<T>(dxb + (size_t)(m - 3) * D, acc);
+    else if (p.dconv_state_in)
+      *reinterpret_cast<float2 *>(p.dconv_state_in + ((size_t)b * 3 + m) * D + d) = acc;
     g3 = g2;
     g2 = g1;
     g1 = g0;
   }
 #pragma unroll
-  for (int k = 0; k < 4; ++k) atomicAdd(p.dconv_w + (size_t)k * D + d, dw[k]);
+  for (int k = 0; k < 4; ++k) {
+    atomicAdd(p.dconv_w + (size_t)k * D + d, dw[k].x);
+    atomicAdd(p.dconv_w + (size_t)k * D + d + 1, dw[k].y);
+  }
 }
 
 struct BwdLayout {
@@ -1131,7 +1176,8 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
     bwd_dw_kernel<<<dim3(tile_blocks, ceil_div(N, chunk)), kDwThreads, 0, st>>>(
         U, za, zx, p.dW_a, p.dW_x, N, p.D, p.H, chunk);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  bwd_conv_kernel<T><<<dim3(ceil_div(p.D, kConvThreads), p.B, ceil_div(p.T + 3, kConvChunk)),
+  bwd_conv_kernel<T><<<dim3(ceil_div(p.D, 2 * kConvThreads), p.B,
+                            ceil_div(p.T + 3, kConvChunk)),
                        kConvThreads, 0, st>>>(p, du);
   return cudaGetLastError();
 }
