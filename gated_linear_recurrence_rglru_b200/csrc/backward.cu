@@ -223,6 +223,21 @@ __device__ __forceinline__ void prefetch_l1(const void *p) {
   asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
 }
 
+// 16-byte asynchronous global -> shared copy (zero-filled when !full: nothing is
+// read from src then, which must still be a valid address); completed by
+// cp_async_wait_all on the issuing thread, published to the block by a barrier.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, bool full) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(shared_addr(dst)),
+               "l"(src), "r"(full ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // Gate math of the backward in fp32 with about 1e-6 relative error: sigmoid
 // and exp through the hardware base-2 exponential, approximate reciprocal and
 // reciprocal square root; 1 - a^2 = -expm1(2 log a) by its Taylor series
@@ -521,7 +536,11 @@ __global__ void bwd_carry_kernel(int B, int D, int nseg, const float *__restrict
 // each token's (d z_a, d z_x) to sink(k, ...) (zeros past t1), leaves the own
 // part of d u in dub and advances gc and the per-channel sums (acc_q sums
 // G Q; the caller scales it by c).
-template <typename T, typename Sink>
+// kStaged: the group's z_a, z_x and dy rows were copied to shared memory ahead
+// of time (sza, szx, sdy: this thread's channel at token 0 of the group, rows
+// sstride elements apart, zeros past t1); else they are read from the
+// workspace and dy in global memory, with an L1 prefetch of the next group.
+template <typename T, bool kStaged, typename Sink>
 __device__ __forceinline__ void final_group(const BwdThread &th, const ChanC &c, const T *xb,
                                             const T *cs_in_b, const T *dyb, size_t orow, int D,
                                             int tb, size_t go, float h_in,
@@ -530,9 +549,10 @@ __device__ __forceinline__ void final_group(const BwdThread &th, const ChanC &c,
                                             float *__restrict__ ws_za, float *__restrict__ ws_zx,
                                             float *__restrict__ ws_u, float &gc, float &acc_q,
                                             float &acc_ba, float &acc_bx, float (&dub)[kTB],
-                                            Sink sink) {
+                                            const float *sza, const float *szx, const T *sdy,
+                                            int sstride, Sink sink) {
   const float neg_c_sp = -kDecayC * c.sp, csp = kDecayC * c.sp;
-  if (tb - kTB >= th.t0) {
+  if (!kStaged && tb - kTB >= th.t0) {
     // the group processed next (8 tokens earlier): its z and dy rows
     const float *pza = ws_za + orow + (size_t)(tb - kTB) * D;
     const float *pzx = ws_zx + orow + (size_t)(tb - kTB) * D;
@@ -553,8 +573,14 @@ __device__ __forceinline__ void final_group(const BwdThread &th, const ChanC &c,
     const int t = tb + k;
     const size_t o = orow + (size_t)t * D;
     const bool in = t < th.t1;
-    const float za = in ? ws_za[o] : 0.f;
-    const float zx = in ? ws_zx[o] : 0.f;
+    float za, zx;
+    if constexpr (kStaged) {
+      za = sza[k * sstride];
+      zx = szx[k * sstride];
+    } else {
+      za = in ? ws_za[o] : 0.f;
+      zx = in ? ws_zx[o] : 0.f;
+    }
     if (in) ws_u[o] = u[k];
     const TokGates tg = tok_gates(za, zx, neg_c_sp);
     const float r = tg.r, ig = tg.i, a = tg.a, gg = tg.g, rog = tg.rog;
@@ -573,7 +599,10 @@ __device__ __forceinline__ void final_group(const BwdThread &th, const ChanC &c,
     dub[k] = 0.f;
     if (t < th.t1) {
       const size_t o = orow + (size_t)t * D;
-      const float G = ldg_f32(dyb + o) + gc;
+      float dy;
+      if constexpr (kStaged) dy = to_f32<T>(sdy[k * sstride]);
+      else dy = ldg_f32(dyb + o);
+      const float G = dy + gc;
       dza = G * fza[k];
       dzx = G * fzx[k];
       dub[k] = G * fu[k];
@@ -630,11 +659,12 @@ bwd_final_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
     float dub[kTB];
     if (live) {
       const size_t go = ((size_t)b * ngt + tb / kTB) * D + th.d;
-      final_group<T>(th, c, xb, cs_in_b, dyb, orow, D, tb, go, h_in, ws_gP, ws_gH, ws_za, ws_zx,
-                     ws_u, gc, acc_q, acc_ba, acc_bx, dub, [&](int k, float dza, float dzx) {
-                       dza_row[k] = dza;
-                       dzx_row[k] = dzx;
-                     });
+      final_group<T, false>(th, c, xb, cs_in_b, dyb, orow, D, tb, go, h_in, ws_gP, ws_gH, ws_za,
+                            ws_zx, ws_u, gc, acc_q, acc_ba, acc_bx, dub, nullptr, nullptr,
+                            nullptr, 0, [&](int k, float dza, float dzx) {
+                              dza_row[k] = dza;
+                              dzx_row[k] = dzx;
+                            });
     } else {
 #pragma unroll
       for (int k = 0; k < kTB; ++k) dub[k] = 0.f;
@@ -678,7 +708,7 @@ bwd_final_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
 // accumulator, scatters it into (segment, channel) rows, and each thread adds
 // its channel's 8 tokens to its own part of d u.
 template <int kBW>
-__global__ void __launch_bounds__(TcGeo<kBW>::kThreads, kBW == 128 ? 1 : 3)
+__global__ void __launch_bounds__(TcGeo<kBW>::kThreads, kBW == 128 ? 1 : 2)
 bwd_final_tc_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
                     const float *__restrict__ ws_C, const float *__restrict__ ws_gP,
                     const float *__restrict__ ws_gH, float *__restrict__ ws_za,
@@ -690,6 +720,10 @@ bwd_final_tc_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
   float *du_s = reinterpret_cast<float *>(smem_ft);                  // [S][kBW][kRow]
   T *a_s = reinterpret_cast<T *>(du_s + G::S * kBW * kRow);          // [2][M][kStride]
   T *w_s = a_s + 2 * G::M * G::kStride;                              // [2][kBW][kStride]
+  // z_a, z_x and dy rows of a group, double-buffered: [2][S][kTB][kBW]
+  float *za_st = reinterpret_cast<float *>(w_s + 2 * kBW * G::kStride);
+  float *zx_st = za_st + 2 * G::S * kTB * kBW;
+  T *dy_st = reinterpret_cast<T *>(zx_st + 2 * G::S * kTB * kBW);
   const int D = p.D, h = blockIdx.y, b = blockIdx.z;
   const BwdThread th = bwd_thread(p, pl, kBW);
   const T *xb = static_cast<const T *>(p.x) + (size_t)b * p.T * D;
@@ -734,17 +768,48 @@ bwd_final_tc_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
   T *dzx_col = dza_col + G::M * G::kStride;
   const float *du_row = du_s + (th.sl * kBW + th.j) * kRow;
   float acc_q = 0.f, acc_ba = 0.f, acc_bx = 0.f;
-  for (int g = pl.L / kTB - 1; g >= 0; --g) {
+  // Staging of group g's rows into buffer buf: 16-byte copies spread over the
+  // block (per segment and token: kBW/4 chunks of z_a, kBW/4 of z_x, kBW/8 of
+  // dy). Rows past a segment's end are zero-filled; segments with no live
+  // token in the group are skipped (no thread reads them).
+  constexpr int CZ = kBW / 4, CY = kBW / 8, CR = 2 * CZ + CY;
+  auto stage = [&](int g, int buf) {
+    for (int ci = threadIdx.x; ci < G::S * kTB * CR; ci += G::kThreads) {
+      const int rowid = ci / CR, w = ci - rowid * CR;
+      const int sl = rowid / kTB, k = rowid - sl * kTB;
+      const int s0 = min(p.T, (blockIdx.x * G::S + sl) * pl.L), s1 = min(p.T, s0 + pl.L);
+      const int tb = s0 + g * kTB;
+      if (tb >= s1) continue;
+      const bool in = tb + k < s1;
+      const size_t grow = ((size_t)b * p.T + (in ? tb + k : tb)) * D + (size_t)h * kBW;
+      const int slot = ((buf * G::S + sl) * kTB + k) * kBW;
+      if (w < CZ) cp_async16(za_st + slot + w * 4, ws_za + grow + w * 4, in);
+      else if (w < 2 * CZ) cp_async16(zx_st + slot + (w - CZ) * 4, ws_zx + grow + (w - CZ) * 4, in);
+      else cp_async16(dy_st + slot + (w - 2 * CZ) * 8, dyb + grow + (w - 2 * CZ) * 8, in);
+    }
+    cp_async_commit();
+  };
+  const int ng = pl.L / kTB;
+  stage(ng - 1, 0);
+  cp_async_wait_all();
+  __syncthreads();
+  for (int g = ng - 1; g >= 0; --g) {
     const int tb = th.t0 + g * kTB;
     const bool live = th.active && tb < th.t1;
+    const int buf = (ng - 1 - g) & 1;
+    // the next group's rows land while this group is computed (its buffer was
+    // last read before the previous iteration's barriers)
+    if (g > 0) stage(g - 1, buf ^ 1);
     float dub[kTB];
     if (live) {
       const size_t go = ((size_t)b * ngt + tb / kTB) * D + th.d;
-      final_group<T>(th, c, xb, cs_in_b, dyb, orow, D, tb, go, h_in, ws_gP, ws_gH, ws_za, ws_zx,
-                     ws_u, gc, acc_q, acc_ba, acc_bx, dub, [&](int k, float dza, float dzx) {
-                       dza_col[k * G::kStride] = __float2bfloat16_rn(dza);
-                       dzx_col[k * G::kStride] = __float2bfloat16_rn(dzx);
-                     });
+      const int srow = ((buf * G::S + th.sl) * kTB) * kBW + th.j;
+      final_group<T, true>(th, c, xb, cs_in_b, dyb, orow, D, tb, go, h_in, ws_gP, ws_gH, ws_za,
+                           ws_zx, ws_u, gc, acc_q, acc_ba, acc_bx, dub, za_st + srow,
+                           zx_st + srow, dy_st + srow, kBW, [&](int k, float dza, float dzx) {
+                             dza_col[k * G::kStride] = __float2bfloat16_rn(dza);
+                             dzx_col[k * G::kStride] = __float2bfloat16_rn(dzx);
+                           });
     } else {
 #pragma unroll
       for (int k = 0; k < kTB; ++k) {
@@ -782,6 +847,7 @@ bwd_final_tc_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
         const int col = nt * 8 + 2 * fq + (e & 1);
         du_s[((r >> 3) * kBW + col) * kRow + (r & 7)] = acc[mi][e];
       }
+    cp_async_wait_all();   // the next group's rows: published by the barrier below
     __syncthreads();
     if (live) {
       const float4 v0 = reinterpret_cast<const float4 *>(du_row)[0];
@@ -1119,11 +1185,13 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
   if constexpr (kTcBW > 0) {
     using G = TcGeo<kTcBW>;
     // K1: fp32 z rows [S][2][bw][kRow] and bf16 u rows [M][kStride];
-    // K3: fp32 d u rows [S][bw][kRow], bf16 d z_a, d z_x rows [2][M][kStride] and
-    //     bf16 W_a, W_x rows [2][bw][kStride]
+    // K3: fp32 d u rows [S][bw][kRow], bf16 d z_a, d z_x rows [2][M][kStride],
+    //     bf16 W_a, W_x rows [2][bw][kStride] and the staged z_a, z_x (fp32) and dy
+    //     (bf16) rows [2][S][kTB][bw]
     const size_t smem1 = (size_t)G::S * 2 * kTcBW * kRow * 4 + (size_t)G::M * G::kStride * 2;
     const size_t smem3 = (size_t)G::S * kTcBW * kRow * 4 + 2 * (size_t)G::M * G::kStride * 2 +
-                         2 * (size_t)kTcBW * G::kStride * 2;   // + bf16 W_a, W_x rows
+                         2 * (size_t)kTcBW * G::kStride * 2 +   // + bf16 W_a, W_x rows
+                         2 * (size_t)G::S * kTB * kTcBW * (4 + 4 + 2);   // + staged rows
     if ((e = cudaFuncSetAttribute(bwd_gates_tc_kernel<kTcBW>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1)) !=
         cudaSuccess)
