@@ -120,3 +120,29 @@ def test_bwd_refuses_bad_arguments_before_launch():
     assert L.rglru_bwd_workspace_bytes(2, 8, 64, 2, 0) > 0
     assert L.rglru_bwd_workspace_bytes(2, 8, 65, 2, 0) == 0
     assert L.rglru_bwd_launches(2, 8, 64, 2, 1) == 5
+
+
+def test_block_refuses_bad_arguments_before_launch():
+    """rglru_block_fwd (25 arguments) checks shapes, pointers, overlaps and the
+    workspace on the host, before any CUDA call."""
+    L = _abi.LIB
+    B, T, Dm, D, H, io = 2, 8, 64, 64, 2, 0
+    # x, W_in, W_gate, W_out, conv_w, W_a, b_a, W_x, b_x, Lambda, h0, conv_state_in, out, h_T,
+    # conv_state_out: distinct 16-byte aligned stand-ins 1 MiB apart (never dereferenced)
+    ptrs = [FAKE * (k + 1) for k in range(15)]
+    ptrs[10] = ptrs[11] = ptrs[13] = ptrs[14] = None          # optional ones absent
+    ws_need = L.rglru_block_fwd_workspace_bytes(B, T, Dm, D, H, io)
+    assert ws_need > 0
+    assert L.rglru_block_fwd_workspace_bytes(B, T, 12, D, H, io) == 0      # Dm % 8
+    assert L.rglru_block_fwd_workspace_bytes(B, T, Dm, 65, H, io) == 0     # D % H
+
+    def call(p=ptrs, dims=(B, T, Dm, D, H, io), ws=None, ws_bytes=0):
+        return L.rglru_block_fwd(*p, *dims, ws, ws_bytes, None, None)
+
+    assert call(p=[None] * 15) == 1                              # null required pointers
+    assert call(dims=(B, T, 12, D, H, io)) == 1                  # Dm not a multiple of 8
+    assert call(dims=(B, T, Dm, D, H, 7)) == 1                   # bad io
+    bad = list(ptrs); bad[12] = ptrs[0]                          # out aliases x
+    assert call(p=bad) == 1
+    assert call() == 5                                           # no workspace
+    assert call(ws=FAKE * 64, ws_bytes=ws_need - 16) == 5        # workspace too small
