@@ -4,7 +4,11 @@
     python bench.py --impl reference ...      # the float64 CPU oracle on a bounded sample
 
 A step is one rglru_fwd over the whole workload (Conv1D, gates, decay, scan
-and the time-split carry), inputs resident in HBM. The timed region is K
+and the time-split carry), inputs resident in HBM. The headline workload is
+long_context (B=1, T=131072, D=4096, H=16, bf16: the largest configuration);
+the other forward workloads (hawk_block, griffin2b) are timed the same way as
+`legs`, and decode_batch, the backward and the recurrent block (both on
+hawk_block) as their own keys. The timed region is K
 back-to-back steps between CUDA events on the launching stream, after W
 untimed warm-up steps; each step reads and writes its own buffer set, and the
 sets rotate so that the bytes touched between two uses of one set exceed 3x
@@ -134,12 +138,25 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
 KERNEL_SOURCES = ["fwd_tc.cu", "tc_gates.cuh", "tc_primitives.cuh", "common.cuh"]
 
 
-def kernel_source_hash() -> str:
+def _code_only(src: str) -> str:
+    """C++ source without comments and blank space (comment edits keep the hash)."""
+    import re
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
+def kernel_source_hash(texts=None) -> str:
+    """Hash of the code (comments and spacing removed) of the forward kernel's sources."""
     import hashlib
     h = hashlib.sha256()
     for fn in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, "gated_linear_recurrence_rglru_b200", "csrc", fn), "rb") as f:
-            h.update(f.read())
+        if texts is not None:
+            src = texts[fn]
+        else:
+            with open(os.path.join(ROOT, "gated_linear_recurrence_rglru_b200", "csrc", fn)) as f:
+                src = f.read()
+        h.update(_code_only(src).encode())
     return h.hexdigest()[:16]
 
 
@@ -165,21 +182,34 @@ def fwd_bytes_per_chtok(wl) -> int:
     return 2 * (4 if wl.io == "f32" else 2)
 
 
-def run_ours(a, ws, rank, local):
-    import gated_linear_recurrence_rglru_b200 as rg
+def config_of(wl, ws, algo):
+    """The config dict of a forward workload (the same for both arms of the bench)."""
+    esz = 4 if wl.io == "f32" else 2
+    set_bytes = 2 * wl.B * wl.T * wl.D * esz
+    nsets = n_buffer_sets(set_bytes)
+    return {"workload": f"{wl.name} B={wl.B} T={wl.T} D={wl.D} H={wl.H} bw={wl.bw} io={wl.io}",
+            "algo": algo, "global_batch": wl.B * ws, "seq_len": wl.T,
+            "parallelism": f"dp{ws} (independent batches)",
+            "l2": f"{nsets} rotating buffer sets of {set_bytes / 1e6:.1f} MB "
+                  f"(>3x L2 between reuses)"}
 
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    wl = WORKLOADS[a.workload]
-    if wl.decode_steps:
-        raise SystemExit("--workload must be a forward workload; decode is reported as 'decode'")
+
+def n_buffer_sets(set_bytes):
+    """Buffer sets rotated so that >3x L2 is touched between two uses of one set."""
+    return max(2, math.ceil(3 * L2_BYTES / set_bytes) + 1)
+
+
+def time_forward(rg, wl, dev, steps, warmup, algo, pk, soak_s=0.0, ws=1):
+    """Time rglru_fwd on a workload: `steps` back-to-back steps between CUDA events
+    on the launching stream after `warmup` untimed ones, then the same steps again
+    with the kernel events that the library records around its compute kernel.
+    Returns the leg's figures (times are this rank's)."""
     t = generate(wl)
     g = {k: (v.to(dev) if v is not None else None) for k, v in t.items()}
     w = [g[k] for k in ("conv_w", "W_a", "b_a", "W_x", "b_x", "Lambda")]
     B, T, D, H = wl.B, wl.T, wl.D, wl.H
     esz = 4 if wl.io == "f32" else 2
-    set_bytes = 2 * B * T * D * esz
-    nsets = max(2, math.ceil(3 * L2_BYTES / set_bytes) + 1)
+    nsets = n_buffer_sets(2 * B * T * D * esz)
     xs = [g["x"]] + [g["x"].clone() for _ in range(nsets - 1)]
     ys = [torch.empty_like(g["x"]) for _ in range(nsets)]
     hT = [torch.empty(B, D, device=dev) for _ in range(nsets)]
@@ -189,10 +219,9 @@ def run_ours(a, ws, rank, local):
     status = torch.zeros(1, device=dev, dtype=torch.int32)
     stream = torch.cuda.current_stream()
     # per timed step, a pair of events that the library records right around its
-    # compute kernel(s) on this stream (after the workspace reset): the kernel's
-    # own launch duration for the roofline
+    # compute kernel(s) on this stream: the kernel's own launch duration
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(a.steps)]
+           for _ in range(steps)]
     for eb, ee in kev:
         eb.record(stream)
         ee.record(stream)
@@ -203,18 +232,16 @@ def run_ours(a, ws, rank, local):
     def step(i, opts=None):
         k = i % nsets
         rg.rglru_fwd(xs[k], *w, h0=g["h0"], y=ys[k], h_T=hT[k], conv_state_out=cs[k],
-                     workspace=work[k], dev_status=status, algo=a.algo, options=opts)
+                     workspace=work[k], dev_status=status, algo=algo, options=opts)
 
-    # soak (untimed) so that the clock sampler sees this load around the timed region
-    sampler = ClockSampler(local)
-    soak_t0 = time.time()
     i = 0
-    while time.time() - soak_t0 < a.soak_s:
-        for _ in range(50):
+    soak_t0 = time.time()
+    while time.time() - soak_t0 < soak_s:         # untimed load around the timed region
+        for _ in range(20):
             step(i)
             i += 1
         torch.cuda.synchronize()
-    for _ in range(a.warmup):
+    for _ in range(warmup):
         step(i)
         i += 1
     torch.cuda.synchronize()
@@ -222,75 +249,104 @@ def run_ours(a, ws, rank, local):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(a.steps):
+    for _ in range(steps):
         step(i)
         i += 1
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(ws)
     ms_local = e0.elapsed_time(e1)
-    # the same K steps again, each with the pair of events that the library
-    # records around its compute kernel: the kernel's own launch durations
-    # (a separate pass, so that the event records do not slow the steps above)
-    for j in range(a.steps):
+    for j in range(steps):
         step(i, kopts[j])
         i += 1
     torch.cuda.synchronize()
-    kernel_ms = sum(eb.elapsed_time(ee) for eb, ee in kev) / a.steps
+    kernel_ms = sum(eb.elapsed_time(ee) for eb, ee in kev) / steps
     post_t0 = time.time()
-    while time.time() - post_t0 < a.soak_s:
-        for _ in range(50):
+    while time.time() - post_t0 < soak_s:
+        for _ in range(20):
             step(i)
             i += 1
         torch.cuda.synchronize()
-    clocks = sampler.stop()
     if int(status.item()) != 0:
         raise SystemExit(f"device status {int(status.item())}: {rg.status_str(int(status.item()))}")
-    ms = max_over_ranks(ms_local, ws)
-    ms_step = ms / a.steps
     chtok = B * T * D
-    value = weak_scaling_value(chtok, a.steps, ms, ws)
-    pk = peaks()
     bytes_step = fwd_bytes_per_chtok(wl) * chtok
-    achieved_step = bytes_step / (ms_step / 1e3) / 1e9
+    kname, traffic = kernel_traffic(wl, algo)
+    ms_step = ms_local / steps
     achieved = bytes_step / (kernel_ms / 1e3) / 1e9
-    launches_per_step = rg.fwd_launches(B, T, D, H, wl.dtype, a.algo)
-    kname, traffic = kernel_traffic(wl, a.algo)
+    achieved_step = bytes_step / (ms_step / 1e3) / 1e9
+    leg = {"workload": config_of(wl, ws, algo)["workload"], "steps": steps,
+           "ms_per_step": ms_step, "value": chtok / (ms_step / 1e3), "unit": "channel-tokens/s",
+           "hbm_gbs": achieved_step,
+           "gpu_launches_per_step": rg.fwd_launches(B, T, D, H, wl.dtype, algo),
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
+                        "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
+                        "kernel": kname, "kernel_ms": kernel_ms,
+                        "timing": "CUDA events recorded by the library around the kernel on "
+                                  "the launching stream, every step of a second pass of the "
+                                  "same K steps right after the timed one",
+                        "step_achieved": achieved_step, "peak_source": pk["source"],
+                        "algorithmic_bytes_per_launch": bytes_step}}
+    leg["_ms_total"] = ms_local
+    leg["_inputs"] = (t, g, w)
+    return leg
 
+
+FWD_LEGS = ("hawk_block", "griffin2b", "long_context")
+
+
+def run_ours(a, ws, rank, local):
+    import gated_linear_recurrence_rglru_b200 as rg
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = WORKLOADS[a.workload]
+    if wl.decode_steps:
+        raise SystemExit("--workload must be a forward workload; decode is reported as 'decode'")
+    pk = peaks()
+    sampler = ClockSampler(local)
+    head = time_forward(rg, wl, dev, a.steps, a.warmup, a.algo, pk, soak_s=a.soak_s, ws=ws)
+    clocks = sampler.stop()
+    ms = max_over_ranks(head.pop("_ms_total"), ws)
+    t, g, w = head.pop("_inputs")
+    ms_step = ms / a.steps
+    chtok = wl.B * wl.T * wl.D
+    value = weak_scaling_value(chtok, a.steps, ms, ws)
     out = {
         "metric": METRIC, "value": value, "unit": "channel-tokens/s", "n_gpus": ws,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": wl.io, "data": "synthetic (seeded; recipe of the workload)",
-        "config": {"workload": f"{wl.name} B={B} T={T} D={D} H={H} bw={wl.bw} io={wl.io}",
-                   "algo": a.algo, "global_batch": B * ws, "seq_len": T,
-                   "parallelism": f"dp{ws} (independent batches)",
-                   "l2": f"{nsets} rotating buffer sets of {set_bytes / 1e6:.1f} MB "
-                         f"(>3x L2 between reuses)"},
-        "hbm_gbs": achieved_step,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
-                     "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
-                     "kernel": kname, "kernel_ms": kernel_ms,
-                     "timing": "CUDA events recorded by the library around the kernel on "
-                               "the launching stream, every step of a second pass of the "
-                               "same K steps right after the timed one",
-                     "step_achieved": achieved_step,
-                     "peak_source": pk["source"],
-                     "algorithmic_bytes_per_launch": bytes_step},
-        "gpu_launches": launches_per_step * a.steps,
+        "config": config_of(wl, ws, a.algo),
+        "hbm_gbs": fwd_bytes_per_chtok(wl) * chtok / (ms_step / 1e3) / 1e9,
+        "roofline": head["roofline"],
+        "gpu_launches": head["gpu_launches_per_step"] * a.steps,
         "clocks": clocks,
     }
+    if a.legs:
+        # the other forward workloads, each timed and measured the same way (this rank)
+        legs = {}
+        for name in FWD_LEGS:
+            if name == wl.name:
+                continue
+            leg = time_forward(rg, WORKLOADS[name], dev, min(a.steps, 100), a.warmup, a.algo,
+                               pk, ws=ws)
+            leg.pop("_ms_total")
+            leg.pop("_inputs")
+            legs[name] = leg
+        out["legs"] = legs
     if a.e2e:
         out["e2e"] = run_e2e(rg, wl, g, w, dev, a)
-        # e2e of every rank is the same program; report rank-max time via value already local
+    if a.cpu_baseline and ws == 1 and rank == 0:
+        out["cpu_baseline"] = cpu_baseline(wl, a.cpu_seconds, t)
+    del t, g, w
+    torch.cuda.empty_cache()
     if a.decode:
         out["decode"] = run_decode(rg, dev, a, pk)
     if a.backward:
-        out["backward"] = run_backward(rg, wl, g, w, dev, a, pk)
+        out["backward"] = run_backward(rg, WORKLOADS["hawk_block"], dev, a, pk)
     if a.block:
-        out["block"] = run_block(rg, wl, dev, a, pk)
-    if a.cpu_baseline and ws == 1 and rank == 0:
-        out["cpu_baseline"] = cpu_baseline(wl, t, a.cpu_seconds)
+        out["block"] = run_block(rg, WORKLOADS["hawk_block"], dev, a, pk)
     return out
 
 
@@ -302,7 +358,7 @@ def run_e2e(rg, wl, g, w, dev, a):
     the copy-in of step i+1 and the copy-out of step i-1 overlap the forward of
     step i (every copy still belongs to exactly one step)."""
     B, T, D, H = wl.B, wl.T, wl.D, wl.H
-    nbuf = 3
+    nbuf = 3 if g["x"].numel() * g["x"].element_size() < 2**29 else 2
     x_host = [g["x"].cpu().pin_memory() for _ in range(nbuf)]
     y_host = [torch.empty_like(x_host[0]).pin_memory() for _ in range(nbuf)]
     x_dev = [torch.empty_like(g["x"]) for _ in range(nbuf)]
@@ -336,10 +392,10 @@ def run_e2e(rg, wl, g, w, dev, a):
             out_done[k].record(s_out)
         used[k] = True
 
-    for i in range(3):
+    for i in range(nbuf):
         step(i)
     torch.cuda.synchronize()
-    n = max(6, min(a.steps, 30))
+    n = max(6, min(a.steps, 30 if nbuf == 3 else 10))
     main = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(main)
@@ -354,13 +410,16 @@ def run_e2e(rg, wl, g, w, dev, a):
     esz = x_host[0].element_size()
     return {"value": B * T * D / (ms / 1e3), "unit": "channel-tokens/s", "ms_per_step": ms,
             "h2d_bytes_per_step": B * T * D * esz, "d2h_bytes_per_step": B * T * D * esz,
-            "steps": n, "pipelining": "3 buffer sets, copy-in / forward / copy-out streams"}
+            "steps": n, "pipelining": f"{nbuf} buffer sets, copy-in / forward / copy-out streams"}
 
 
-def run_backward(rg, wl, g, w, dev, a, pk):
-    """Backward of the same workload: gradients of <dy, y> + <dh_T, h_T> for every
+def run_backward(rg, wl, dev, a, pk):
+    """Backward of a workload: gradients of <dy, y> + <dh_T, h_T> for every
     input, one rglru_bwd per step, inputs resident, rotating dy / dx sets."""
     B, T, D, H = wl.B, wl.T, wl.D, wl.H
+    t = generate(wl)
+    g = {k: (v.to(dev) if v is not None else None) for k, v in t.items()}
+    w = [g[k] for k in ("conv_w", "W_a", "b_a", "W_x", "b_x", "Lambda")]
     esz = 4 if wl.io == "f32" else 2
     gen = torch.Generator(device=dev)
     gen.manual_seed(wl.seed + 1000)
@@ -449,34 +508,32 @@ def run_block(rg, wl, dev, a, pk):
 
 
 def run_decode(rg, dev, a, pk):
-    """Decode workload: B=1024 sequences, one step per launch, state in place."""
+    """Decode workload: B=1024 sequences, one step per launch, state in place. The
+    inputs are the workload's own seeded draws (the ones the parity tests check)."""
     wl = WORKLOADS["decode_batch"]
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(wl.seed)
-    B, D, H, bw = wl.B, wl.D, wl.H, wl.bw
-    dt = wl.dtype
     steps = a.decode_steps
-    x = torch.randn(steps, B, D, generator=gen, device=dev).to(dt)
-    conv_w = (torch.randn(4, D, generator=gen, device=dev) * 0.5).to(dt)
-    W_a = (torch.randn(H, bw, bw, generator=gen, device=dev) / 8).to(dt)
-    W_x = (torch.randn(H, bw, bw, generator=gen, device=dev) / 8).to(dt)
-    b = torch.zeros(D, device=dev, dtype=dt)
-    s = torch.rand(D, generator=gen, device=dev, dtype=torch.float64) * (wl.ac_hi - wl.ac_lo) + wl.ac_lo
-    aa = s ** (1 / 8)
-    Lam = (torch.log(aa) - torch.log1p(-aa)).float()
-    h = torch.randn(B, D, generator=gen, device=dev)
-    ring = torch.randn(B, 3, D, generator=gen, device=dev).to(dt)
-    ys = torch.empty(steps, B, D, device=dev, dtype=dt)
+    t = generate(wl.with_shape(decode_steps=max(steps, 1)))
+    B, D, H, bw = wl.B, wl.D, wl.H, wl.bw
+    x = t["x_steps"].to(dev)
+    conv_w, W_a, b_a, W_x, b_x, Lam = (t[k].to(dev) for k in ("conv_w", "W_a", "b_a", "W_x",
+                                                               "b_x", "Lambda"))
+    h = t["h"].to(dev)
+    ring = t["conv_state"].to(dev)
+    del t
+    ys = torch.empty(steps, B, D, device=dev, dtype=wl.dtype)
     stream = torch.cuda.current_stream()
-    for s_ in range(3):
-        rg.rglru_decode_step(x[s_], ring, s_, h, conv_w, W_a, b, W_x, b, Lam, y_t=ys[s_],
+
+    def one(s_):
+        rg.rglru_decode_step(x[s_], ring, s_, h, conv_w, W_a, b_a, W_x, b_x, Lam, y_t=ys[s_],
                              algo=a.algo)
+
+    for s_ in range(3):
+        one(s_)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for s_ in range(steps):
-        rg.rglru_decode_step(x[s_], ring, s_, h, conv_w, W_a, b, W_x, b, Lam, y_t=ys[s_],
-                             algo=a.algo)
+        one(s_)
     e1.record(stream)
     torch.cuda.synchronize()
     ms_eager = e0.elapsed_time(e1) / steps
@@ -489,8 +546,7 @@ def run_decode(rg, dev, a, pk):
     with torch.cuda.stream(cap):
         with torch.cuda.graph(graph, stream=cap):
             for s_ in range(steps):
-                rg.rglru_decode_step(x[s_], ring, s_, h, conv_w, W_a, b, W_x, b, Lam,
-                                     y_t=ys[s_], algo=a.algo)
+                one(s_)
     stream.wait_stream(cap)
     graph.replay()
     torch.cuda.synchronize()
@@ -506,70 +562,46 @@ def run_decode(rg, dev, a, pk):
             "value": B * D / (ms / 1e3), "unit": "channel-tokens/s", "us_per_step": ms * 1e3,
             "timing": f"{steps} steps captured in one CUDA graph, replayed; CUDA events",
             "us_per_step_eager": ms_eager * 1e3,
+            "gpu_launches_per_step": rg.decode_launches(B, D, H, wl.dtype, a.algo),
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "traffic": None,
                          "algorithmic_bytes_per_launch": bytes_step},
-            "inputs": "seeded on the device with the workload's recipe",
+            "inputs": "the decode_batch workload's seeded draws (workloads.generate)",
             "l2": "state, ring and weights total 113 MB; the state is re-read each step "
                   "(L2 may hold part of it, as in real decoding)"}
 
 
 # ------------------------------------------------------------ CPU oracle --
 
-def oracle_sample(wl, t, seconds):
-    """Time the float64 oracle on the first rows of the workload, growing the
-    sample until it takes about `seconds` of wall time. Returns (chtok/s, desc)."""
-    from oracle import rglru_oracle as orc
-    rows, reps = 1, 1
-    Tcap = wl.T
-    while True:
-        xs = t["x"][:rows, :Tcap]
-        h0 = t["h0"][:rows] if t["h0"] is not None else None
-        t0 = time.perf_counter()
-        for _ in range(reps):
-            orc.rglru_fwd(xs, t["conv_w"], t["W_a"], t["b_a"], t["W_x"], t["b_x"],
-                          t["Lambda"], h0=h0)
-        dt = time.perf_counter() - t0
-        work = reps * rows * Tcap * wl.D
-        if dt >= 0.8 * seconds:
-            return work / dt, (f"{reps} x ({rows} of {wl.B} batch rows x {Tcap} tokens x "
-                               f"D={wl.D}), {dt:.1f} s wall, float64 numpy oracle")
-        grow = max(2, int(math.ceil(seconds / max(dt, 1e-3))))
-        if rows < wl.B:
-            rows = min(wl.B, rows * grow)
-        else:
-            reps *= grow
-
-
-def cpu_baseline(wl, t, seconds):
-    v, desc = oracle_sample(wl, t, seconds)
-    return {"value": v, "unit": "channel-tokens/s", "cores": 1, "kind": "oracle",
-            "sample": desc}
+def cpu_baseline(wl, seconds, t=None):
+    """The float64 oracle, as it stands, on every host core over a bounded sample of
+    the workload (independent (batch row, head) blocks; see oracle/timing.py)."""
+    from oracle import timing
+    return timing.measure(t if t is not None else generate(wl), wl, seconds)
 
 
 # -------------------------------------------------------- reference arm --
 
 def run_reference(a, ws, rank):
+    """The reference arm: the float64 oracle on the host's cores, the same metric
+    and config as our arm; nothing here loads the CUDA library."""
     if rank != 0:
         return None
     wl = WORKLOADS[a.workload]
     t = generate(wl)
-    per = []
-    desc = ""
+    from oracle import timing
     for _ in range(a.warmup):
-        oracle_sample(wl, t, 0.5)
-    for _ in range(a.steps):
-        v, desc = oracle_sample(wl, t, a.ref_seconds)
-        per.append(v)
-    v = statistics.median(per)
+        timing.measure(t, wl, 0.3)
+    per = [timing.measure(t, wl, a.ref_seconds) for _ in range(a.steps)]
+    v = statistics.median(p["value"] for p in per)
+    base = dict(per[-1])
+    base["value"] = v
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "channel-tokens/s",
             "n_gpus": ws, "steps": a.steps, "warmup": a.warmup, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded; recipe of the workload)",
-            "config": {"workload": f"{wl.name} B={wl.B} T={wl.T} D={wl.D} H={wl.H} "
-                                   f"bw={wl.bw} io={wl.io}", "seq_len": wl.T},
-            "cpu_baseline": {"value": v, "unit": "channel-tokens/s", "cores": 1,
-                             "kind": "oracle", "sample": desc},
+            "config": config_of(wl, ws, a.algo),
+            "cpu_baseline": base,
             "e2e": {"value": v, "unit": "channel-tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
@@ -580,19 +612,21 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="hawk_block", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="long_context", choices=sorted(WORKLOADS))
     ap.add_argument("--algo", default="auto", choices=["auto", "generic", "tensor"])
     ap.add_argument("--soak-s", type=float, default=1.5,
                     help="untimed seconds of the same steps before and after the timed "
                          "region, so the clock sampler sees the load")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-legs", dest="legs", action="store_false",
+                    help="skip the other forward workloads (hawk_block, griffin2b, ...)")
     ap.add_argument("--no-decode", dest="decode", action="store_false")
     ap.add_argument("--no-backward", dest="backward", action="store_false")
     ap.add_argument("--no-block", dest="block", action="store_false")
     ap.add_argument("--decode-steps", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--ref-seconds", type=float, default=5.0)
+    ap.add_argument("--ref-seconds", type=float, default=4.0)
     a = ap.parse_args(argv)
     if a.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

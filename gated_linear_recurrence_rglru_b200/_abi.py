@@ -193,27 +193,32 @@ def rglru_fwd(x, conv_w, W_a, b_a, W_x, b_x, Lambda, h0=None, conv_state_in=None
 
 
 def rglru_fwd_noalloc(x, conv_w, W_a, b_a, W_x, b_x, Lambda, h0=None, conv_state_in=None, *,
-                      y=None, h_T=None, conv_state_out=None, stream=None):
+                      y, h_T=None, conv_state_out=None, stream=None):
     """rglru_fwd without a workspace: the library's static device scratch is used.
 
-    For callers that cannot allocate device memory while running (output
-    buffers may be passed in). Returns (y, h_T, conv_state_out).
+    For callers that cannot allocate device memory while they run, so every
+    output buffer is the caller's: y (B, T, D) is required; h_T and
+    conv_state_out are written when given. The call runs with x's device
+    current and, unless `stream` is given, on that device's current stream.
+    Returns (y, h_T, conv_state_out).
     """
     B, T, D = x.shape
     H = W_a.shape[0]
     bw = D // H if H else 0
     dt = x.dtype
-    st = LIB.rglru_fwd_noalloc(
-        _ptr(x, "x", dt), _ptr(conv_w, "conv_w", dt, (4, D)),
-        _ptr(W_a, "W_a", dt, (H, bw, bw)), _ptr(b_a, "b_a", dt, (D,)),
-        _ptr(W_x, "W_x", dt, (H, bw, bw)), _ptr(b_x, "b_x", dt, (D,)),
-        _ptr(Lambda, "Lambda", torch.float32, (D,)),
-        _ptr(h0, "h0", torch.float32, (B, D), optional=True),
-        _ptr(conv_state_in, "conv_state_in", dt, (B, 3, D), optional=True),
-        _ptr(y, "y", dt, (B, T, D)),
-        _ptr(h_T, "h_T", torch.float32, (B, D), optional=True),
-        _ptr(conv_state_out, "conv_state_out", dt, (B, 3, D), optional=True),
-        B, T, D, H, _io_of(dt), _stream_handle(stream))
+    with torch.cuda.device(x.device):
+        st = LIB.rglru_fwd_noalloc(
+            _ptr(x, "x", dt), _ptr(conv_w, "conv_w", dt, (4, D)),
+            _ptr(W_a, "W_a", dt, (H, bw, bw)), _ptr(b_a, "b_a", dt, (D,)),
+            _ptr(W_x, "W_x", dt, (H, bw, bw)), _ptr(b_x, "b_x", dt, (D,)),
+            _ptr(Lambda, "Lambda", torch.float32, (D,)),
+            _ptr(h0, "h0", torch.float32, (B, D), optional=True),
+            _ptr(conv_state_in, "conv_state_in", dt, (B, 3, D), optional=True),
+            _ptr(y, "y", dt, (B, T, D)),
+            _ptr(h_T, "h_T", torch.float32, (B, D), optional=True),
+            _ptr(conv_state_out, "conv_state_out", dt, (B, 3, D), optional=True),
+            B, T, D, H, _io_of(dt),
+            (stream if stream is not None else torch.cuda.current_stream(x.device)).cuda_stream)
     if st != 0:
         raise RGLRUError(st, "rglru_fwd_noalloc")
     return y, h_T, conv_state_out

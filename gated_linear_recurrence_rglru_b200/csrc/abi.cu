@@ -7,6 +7,20 @@
 
 using namespace rglru;
 
+namespace rglru {
+
+int check_shape(int B, int T, int D, int H, int io) {
+  if (B < 1 || T < 1 || D < 1 || H < 1) return RGLRU_ERR_INVALID_ARG;
+  if (io != RGLRU_IO_F32 && io != RGLRU_IO_BF16) return RGLRU_ERR_INVALID_ARG;
+  if (D % H != 0 || D % 8 != 0) return RGLRU_ERR_INVALID_ARG;
+  if (D / H > 1024) return RGLRU_ERR_UNSUPPORTED;
+  if ((long long)B * D > (1ll << 31) - 1) return RGLRU_ERR_UNSUPPORTED;
+  if ((long long)B * T > (1ll << 31) - 1) return RGLRU_ERR_UNSUPPORTED;
+  return RGLRU_OK;
+}
+
+}  // namespace rglru
+
 namespace {
 
 constexpr int kVersion = 100;  // 0.1.0
@@ -19,16 +33,6 @@ bool overlap(const void *a, size_t na, const void *b, size_t nb) {
   if (a == nullptr || b == nullptr || na == 0 || nb == 0) return false;
   const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
   return a0 < b0 + nb && b0 < a0 + na;
-}
-
-int check_shape(int B, int T, int D, int H, int io) {
-  if (B < 1 || T < 1 || D < 1 || H < 1) return RGLRU_ERR_INVALID_ARG;
-  if (io != RGLRU_IO_F32 && io != RGLRU_IO_BF16) return RGLRU_ERR_INVALID_ARG;
-  if (D % H != 0 || D % 8 != 0) return RGLRU_ERR_INVALID_ARG;
-  if (D / H > 1024) return RGLRU_ERR_UNSUPPORTED;
-  if ((long long)B * D > (1ll << 31) - 1) return RGLRU_ERR_UNSUPPORTED;
-  if ((long long)B * T > (1ll << 31) - 1) return RGLRU_ERR_UNSUPPORTED;
-  return RGLRU_OK;
 }
 
 size_t io_bytes(int io) { return io == RGLRU_IO_F32 ? 4 : 2; }

@@ -1,7 +1,6 @@
 // Backward of the RG-LRU layer: the gradient of <dy, y> + <dh_T, h_T> with
-// respect to every input ("Griffin: Mixing Gated Linear Recurrences with Local
-// Attention for Efficient Language Models", section "Model Architecture"
-// defines the forward; the backward is the chain rule through it, run as
+// respect to every input (the forward is the layer's definition stated in
+// include/rglru.h; the backward is the chain rule through it, run as
 // linear scans in both time directions, the forward's scheme in S. De's
 // thread). fp32 arithmetic, except that for bf16 I/O with heads 32, 64 or
 // 128 wide the two in-loop gate contractions (z = u W in K1, d z W^T in K3),

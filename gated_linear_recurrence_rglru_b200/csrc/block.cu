@@ -1,7 +1,8 @@
-// The recurrent block around the RG-LRU layer ("Griffin: Mixing Gated Linear
-// Recurrences with Local Attention for Efficient Language Models", section
-// "Model Architecture": the recurrent block carries a temporal Conv1D and the
-// RG-LRU; the model's MLP is GeLU-gated). Read as two branches from the
+// The recurrent block around the RG-LRU layer (S. De's thread on Griffin: a
+// simple recurrent block with a temporal Conv1D and the RG-LRU, and gated MLP
+// blocks; "Beyond Transformer Architecture: Griffin and Google RecurrentGemma",
+// "Core Components of Griffin", 3. Architecture Design: a GeGeLU-like gated
+// MLP). The pages print no equation for it. Read as two branches from the
 // block input x (B, T, Dm):
 //   gate branch       g = GeLU(x W_gate)                      (B, T, D)
 //   recurrent branch  y = RG-LRU layer (Conv1D, gates, scan) of x W_in

@@ -1,10 +1,10 @@
 // Fused RG-LRU forward on the 5th-generation tensor core (sm_100a), bf16 I/O.
 //
-// One pass over HBM: x is read once (TMA), y written once. The layer
-// ("Griffin: Mixing Gated Linear Recurrences with Local Attention for Efficient
-// Language Models", section "Model Architecture"; gates independent of the
-// state, "Beyond Transformer Architecture: Griffin and Google RecurrentGemma",
-// "Core Components of Griffin", 1. RG-LRU) is split into
+// One pass over HBM: x is read once (TMA), y written once. The layer (its
+// definition in include/rglru.h; gates independent of the state, "Beyond
+// Transformer Architecture: Griffin and Google RecurrentGemma", "Core
+// Components of Griffin", 1. RG-LRU; a memory-bound layer whose kernel should
+// optimise HBM accesses, S. De's thread on Griffin) is split into
 //   unit = (batch row b, group of 128 output channels), tile = 64 tokens
 //   (32 tokens when a head is 256 wide, so that its weights fit on chip).
 // Per tile

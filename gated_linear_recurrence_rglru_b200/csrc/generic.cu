@@ -1,8 +1,7 @@
 // Generic RG-LRU kernels: fp32 arithmetic on CUDA cores for any I/O type.
 //
-// Forward over a sequence (the recurrence of "Griffin: Mixing Gated Linear
-// Recurrences with Local Attention for Efficient Language Models", section
-// "Model Architecture"; run as a linear scan, S. De's thread on Griffin):
+// Forward over a sequence (the layer's definition, include/rglru.h; run as a
+// linear scan, S. De's thread on Griffin):
 // time is cut into nseg segments so that B * H * nseg blocks fill the GPU.
 //   pass 1  aggregate: per (b, segment, channel) the segment's decay product
 //           A = prod a_t and its local state H (scan from zero);

@@ -41,6 +41,10 @@ struct DecArgs {
   int B, D, H;
 };
 
+// Shape checks shared by every entry point: an rglru_status (RGLRU_OK when the
+// sizes and the I/O type are well formed and supported).
+int check_shape(int B, int T, int D, int H, int io);
+
 struct GenericPlan {
   int nseg;  // time segments
   int L;     // tokens per segment (the last may be shorter)

@@ -1,7 +1,8 @@
 // Device helpers shared by the tensor-core kernels: fast gate math of the
-// RG-LRU ("Griffin: Mixing Gated Linear Recurrences with Local Attention for
-// Efficient Language Models", section "Model Architecture": r = sigmoid(z_a),
-// i = sigmoid(z_x), log a = -c r softplus(-Lambda), beta = sqrt(1 - a^2) i u),
+// RG-LRU (the layer's definition, include/rglru.h: r = sigmoid(z_a),
+// i = sigmoid(z_x), log a = -c r softplus(-Lambda), beta = sqrt(1 - a^2) i u;
+// gates that never read the state, "Beyond Transformer Architecture: Griffin
+// and Google RecurrentGemma", "Core Components of Griffin", 1. RG-LRU),
 // bf16 packing, and global-memory acquire/release accesses.
 #pragma once
 

@@ -5,9 +5,10 @@ arithmetic and is the one module that the CUDA path's callers (tests, bench,
 smoke) and the float64 oracle share: both sides receive the very same tensors.
 
 The five named workloads are the Griffin / Hawk recurrent-core shapes this
-library is measured on ("Griffin: Mixing Gated Linear Recurrences with Local
-Attention for Efficient Language Models", section "Model Architecture": the
-RG-LRU layer, whose recurrent block carries a temporal Conv1D):
+library is measured on (the RG-LRU layer with the temporal Conv1D of its
+recurrent block, S. De's thread on Griffin; training sequences of 2048 tokens
+and extrapolation to longer ones, "Beyond Transformer Architecture: Griffin and
+Google RecurrentGemma", "Technical Foundations of RecurrentGemma"):
 
   tiny_f32       B=1    T=256    D=256  H=4   fp32 I/O        a^8 ~ U[0.9, 0.999]
   hawk_block     B=8    T=2048   D=1024 H=16  bf16 I/O        a^8 ~ U[0.9, 0.999]

@@ -1,18 +1,23 @@
 /*
  * rglru.h -- C ABI of the B200 (sm_100a) RG-LRU library.
  *
- * The RG-LRU layer ("Griffin: Mixing Gated Linear Recurrences with Local
- * Attention for Efficient Language Models", section "Model Architecture"; the
- * recurrent gate added to a diagonal LRU and the temporal Conv1D of the
- * recurrent block are described in S. De's thread on Griffin, "how we got
- * there"; the gates do not read the recurrent state, "Beyond Transformer
- * Architecture: Griffin and Google RecurrentGemma", "Core Components of
- * Griffin", 1. RG-LRU):
+ * The RG-LRU layer, the recurrent core of Griffin / Hawk. The source pages
+ * describe its parts but print no formula for it; the equations below are the
+ * layer's definition as this library states it, and every page passage cited
+ * in this header supports only what it says:
+ *   - S. De's thread on Griffin ("how we got there"): the RG-LRU is the LRU, a
+ *     diagonal recurrence, with a recurrent gate added; the simple recurrent
+ *     block carries a temporal Conv1D; the layer is memory-bound, its kernel
+ *     optimises HBM accesses and runs a linear scan rather than a parallel one;
+ *   - "Beyond Transformer Architecture: Griffin and Google RecurrentGemma",
+ *     "Core Components of Griffin", 1. RG-LRU: the gates do not depend on the
+ *     recurrent state; "Key Strengths of RecurrentGemma", 1. Reduced Memory
+ *     Usage: the state has a fixed size, whatever the sequence length.
  *
  *   u_t     = sum_{k=0..3} conv_w[k] * x_{t-3+k}          causal depthwise Conv1D, width 4
  *   r_t     = sigmoid(u_t W_a + b_a)                       block-diagonal per head
  *   i_t     = sigmoid(u_t W_x + b_x)                       block-diagonal per head
- *   log a_t = -8 * r_t * softplus(-Lambda)
+ *   log a_t = -8 * r_t * softplus(-Lambda)                 a_t = sigmoid(Lambda)^(8 r_t)
  *   h_t     = a_t * h_{t-1} + sqrt(1 - a_t^2) * (i_t * u_t)
  *   y_t     = h_t
  *
@@ -86,7 +91,9 @@ size_t rglru_fwd_workspace_bytes(int B, int T, int D, int H, int io);
 int rglru_fwd_launches(int B, int T, int D, int H, int io, int algo);
 
 /*
- * Full-sequence forward of the layer.
+ * Full-sequence forward of the layer: every equation above over t = 0..T-1,
+ * the scan carried across time by a linear scan (S. De's thread: linear scans
+ * rather than parallel ones), split across thread blocks by tiles of time.
  *   x              (B, T, D)  io     input of the Conv1D
  *   conv_w         (4, D)     io
  *   W_a, W_x       (H, bw, bw) io    gate weights
@@ -113,7 +120,7 @@ int rglru_fwd(const void *x, const void *conv_w, const void *W_a, const void *b_
 
 /*
  * rglru_fwd with an explicit algorithm (rglru_algo). RGLRU_ALGO_TENSOR needs
- * io = RGLRU_IO_BF16, D % 128 == 0 and bw in {16, 32, 64, 128, 256}; otherwise
+ * io = RGLRU_IO_BF16, D % 128 == 0 and bw in {64, 128, 256}; otherwise
  * it returns RGLRU_ERR_UNSUPPORTED. Both algorithms compute the same layer.
  */
 int rglru_fwd_algo(const void *x, const void *conv_w, const void *W_a, const void *b_a,
@@ -181,16 +188,23 @@ int rglru_fwd_ex(const void *x, const void *conv_w, const void *W_a, const void 
  * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  *
  * Arguments, layouts and results are those of rglru_fwd without the
- * workspace and dev_status arguments. The stream must belong to the current
- * device. The first call on a device looks up that device's copy of the
- * static array (cudaGetSymbolAddress, once per device, with the device
- * current); make that first call before any stream capture. Problems whose
- * scratch would exceed RGLRU_NOALLOC_SCRATCH_BYTES (rglru_fwd_workspace_bytes
- * larger than it) are rejected with RGLRU_ERR_WORKSPACE before anything is
- * launched. All calls on a device share the one array, which keeps the last
- * call's contents (nothing in it needs to start at zero): calls that can
- * overlap on the GPU, from different streams or threads, race on it and
- * must be serialised by the caller.
+ * workspace and dev_status arguments; invalid sizes get the status that
+ * rglru_fwd gives them. The stream must belong to the current device. Each
+ * call made while the stream is not capturing looks up the current device's
+ * copy of the static array (cudaGetSymbolAddress, with that device current),
+ * so the address stays right after a device reset; a call made while the
+ * stream is capturing uses the address found by the last such call, so make
+ * a first call on each device before any stream capture. A problem whose
+ * scratch would exceed RGLRU_NOALLOC_SCRATCH_BYTES is rejected with
+ * RGLRU_ERR_WORKSPACE before anything is launched: the generic algorithm
+ * needs 12 bytes per (batch row, time segment, channel) when it splits time
+ * into segments (about 296 / (B * H) segments, each of at least 16 tokens),
+ * and none when it does not. The forward shapes measured by this library need
+ * well under 1 MiB (B=8 T=2048 D=1024 H=16: 0.29 MB; B=16 T=4096 D=2560
+ * H=10: 0.98 MB; B=1 T=131072 D=4096 H=16: 0.93 MB). All calls on a device
+ * share the one array, which keeps the last call's contents (nothing in it
+ * needs to start at zero): calls that can overlap on the GPU, from different
+ * streams or threads, race on it and must be serialised by the caller.
  */
 int rglru_fwd_noalloc(const void *x, const void *conv_w, const void *W_a, const void *b_a,
                       const void *W_x, const void *b_x, const float *Lambda, const float *h0,
@@ -198,7 +212,11 @@ int rglru_fwd_noalloc(const void *x, const void *conv_w, const void *W_a, const 
                       int B, int T, int D, int H, int io, void *stream);
 
 /*
- * One decode step for B independent sequences, state updated in place.
+ * One decode step for B independent sequences, state updated in place: the
+ * equations above for one t, from the fixed-size state (h and the last three
+ * inputs) rather than the sequence ("Beyond Transformer Architecture: Griffin
+ * and Google RecurrentGemma", "Key Strengths of RecurrentGemma", 1. Reduced
+ * Memory Usage: the memory needed stays constant whatever the length).
  *   x_t        (B, D)     io     this step's input
  *   conv_state (B, 3, D)  io     ring at step pos (read); slot pos%3 is overwritten with x_t
  *   pos        >= 0              step index that places the ring (see above)
@@ -226,9 +244,9 @@ int rglru_decode_step_algo(const void *x_t, void *conv_state, int pos, float *h,
 
 /*
  * Backward of the layer (the gradient of a scalar loss through one forward
- * call). The forward is the layer of "Griffin: Mixing Gated Linear
- * Recurrences with Local Attention for Efficient Language Models", section
- * "Model Architecture"; the backward is the chain rule through it: with
+ * call), the training side of the layer whose kernel S. De's thread reports a
+ * 3x training speed-up for. The backward is the chain rule through the
+ * equations above: with
  * dy = dL/dy (B, T, D) and dh_T = dL/dh_T (B, D, or NULL for zeros) it returns
  * the gradients of L with respect to every forward input, recomputing the
  * forward from its inputs (nothing is saved between the calls). Time is cut
@@ -272,10 +290,11 @@ int rglru_bwd(const void *x, const void *conv_w, const void *W_a, const void *b_
 int rglru_bwd_launches(int B, int T, int D, int H, int io);
 
 /*
- * Recurrent block around the layer ("Griffin: Mixing Gated Linear Recurrences
- * with Local Attention for Efficient Language Models", section "Model
- * Architecture": a temporal Conv1D and the RG-LRU inside a recurrent block;
- * the model's MLP is GeLU-gated). Read as two branches of the block
+ * Recurrent block around the layer (S. De's thread: a simple recurrent block
+ * with a temporal Conv1D and the RG-LRU, and gated MLP blocks; "Beyond
+ * Transformer Architecture: Griffin and Google RecurrentGemma", "Core
+ * Components of Griffin", 3. Architecture Design: the gated MLP is GeGLU-like).
+ * The pages print no equation for it; it is read as two branches of the block
  * input x (B, T, Dm):
  *   g   = GeLU(x W_gate)              GeLU(v) = v (1 + erf(v / sqrt 2)) / 2
  *   y   = rglru_fwd(x W_in)           the layer above, with h0 / conv_state_in

@@ -4,11 +4,10 @@ TEST INFRASTRUCTURE ONLY, like rglru_oracle (whose layer it calls): only
 tests/ and the bench's CPU legs may call it. It shares no code with the CUDA
 library.
 
-Sources: "Griffin: Mixing Gated Linear Recurrences with Local Attention for
-Efficient Language Models", section "Model Architecture" (the recurrent block
-holds a temporal Conv1D and the RG-LRU layer; the model's feedforward part is a
-GeLU-gated MLP), and S. De's thread (a simple recurrent block with a temporal
-Conv1D). The pages name the parts but print no equation for the block; the
+Sources: S. De's thread on Griffin (a simple recurrent block with a temporal
+Conv1D around the RG-LRU; gated MLP blocks) and "Beyond Transformer
+Architecture: Griffin and Google RecurrentGemma", "Core Components of Griffin",
+3. Architecture Design (the gated MLP is GeGeLU-like). The pages name the parts but print no equation for the block; the
 plainest reading, used here and listed in the design notes:
   g   = GeLU(x W_gate)          the gate branch (GeLU gating)
   v   = x W_in                  the recurrent branch's input projection

@@ -1,20 +1,38 @@
 """Error measure used to compare a result with the float64 oracle (test infrastructure).
 
-max relative error = max_i |g_i - o_i| / max(|o_i|, s_i), where s_i is the
-root-mean-square of the oracle's output over every batch row and time (or
-decode) step of the element's own channel. A pure elementwise relative error
-is undefined where h_t crosses zero; the floor at the channel's RMS keeps the
-measure relative to the scale of that channel's state, so a wrong term, sign
-or index still shows up as an O(1) error while a correct bf16 pipeline, whose
-absolute error is a small fraction of the channel's scale, does not. (One
-batch row's RMS alone is too small a floor for a few decode steps from a state
-that happens to be near zero: the step's increment then dominates the error.)
+max relative error = max_i |g_i - o_i| / max(|o_i|, s_i),  s_i = FLOOR * RMS_c,
+
+where RMS_c is the root-mean-square of the oracle's output over every batch
+row and time (or decode) step of element i's own channel c, and FLOOR = 0.75.
+
+Why a floor, and why this one. A pure elementwise relative error is undefined
+where h_t crosses zero, so some floor is needed. The floor is derived from the
+arithmetic that a bf16 tensor-core gate contraction performs, not chosen from
+a kernel's result: tests/test_bf16_operand_rounding.py runs the float64
+oracle with one change, the Conv1D output rounded to bf16 where it enters the
+gate contraction (and y stored in bf16), on the parity cases, and finds:
+  * its absolute error reaches about 2e-2 of the channel's RMS, so under a
+    floor of 1e-3 * RMS the designed arithmetic itself scores 2 to 10, over
+    100 times the 2e-2 bar: no bf16-operand contraction can meet that floor;
+  * with the RMS of one batch row as the scale, a 5-step decode case needs a
+    factor of at least 1.05 (a row whose state stays near zero for a few steps
+    has a small RMS while the step's increment, and its rounding, does not);
+  * with the channel's RMS over all rows and steps, every case meets the bar
+    from a factor of 0.59 (forward) or 0.52 (decode) up. FLOOR = 0.75 is the
+    tightest round factor above them with a margin of about 1.25.
+A wrong term, sign or index still shows up as an O(1) error under this floor
+(tests/test_oracle_mutants.py plants such mistakes). The GPU tests also compare
+the tensor-core path with the bf16-operand arithmetic itself: y agrees to the
+bf16 unit roundoff 2^-8 (its own output rounding, five times inside the bar)
+and h_T to 1e-4, so the error against the exact oracle is that rounding.
 """
 from __future__ import annotations
 
 import numpy as np
 
 TINY = 1e-30
+FLOOR = 0.75          # floor factor on the channel RMS (see above)
+SURVEY_FLOOR = 1e-3   # a floor too tight for any bf16-operand contraction; reported only
 
 
 def channel_rms(o: np.ndarray, time_axis: int = 1) -> np.ndarray:
@@ -28,8 +46,14 @@ def channel_rms(o: np.ndarray, time_axis: int = 1) -> np.ndarray:
     return np.sqrt(np.mean(o * o, axis=axes, keepdims=True))
 
 
-def max_rel_err(g, o, scale=None, time_axis: int = 1) -> float:
-    """max |g - o| / max(|o|, scale); scale defaults to the per-channel RMS of o."""
+def row_rms(o: np.ndarray, time_axis: int = 1) -> np.ndarray:
+    """RMS of o per (batch row, channel) over the time axis only; keepdims (reported only)."""
+    o = np.asarray(o, dtype=np.float64)
+    return np.sqrt(np.mean(o * o, axis=time_axis, keepdims=True))
+
+
+def max_rel_err(g, o, scale=None, time_axis: int = 1, floor: float = FLOOR) -> float:
+    """max |g - o| / max(|o|, floor * scale); scale defaults to the per-channel RMS of o."""
     g = np.asarray(g, dtype=np.float64)
     o = np.asarray(o, dtype=np.float64)
     if g.shape != o.shape:
@@ -38,7 +62,7 @@ def max_rel_err(g, o, scale=None, time_axis: int = 1) -> float:
         return 0.0
     if scale is None:
         scale = channel_rms(o, time_axis)
-    den = np.maximum(np.maximum(np.abs(o), scale), TINY)
+    den = np.maximum(np.maximum(np.abs(o), floor * np.asarray(scale)), TINY)
     err = np.abs(g - o) / den
     if not np.all(np.isfinite(g)):
         return float("inf")
@@ -52,3 +76,11 @@ def normwise_err(g, o) -> float:
     if o.size == 0:
         return 0.0
     return float(np.abs(g - o).max() / max(np.abs(o).max(), TINY))
+
+
+def error_report(g, o, time_axis: int = 1) -> dict:
+    """The same comparison under the three floors discussed above, for reporting."""
+    return {"floor_0.75_channel_rms": max_rel_err(g, o, time_axis=time_axis),
+            "floor_1e-3_channel_rms": max_rel_err(g, o, time_axis=time_axis, floor=SURVEY_FLOOR),
+            "floor_1_row_rms": max_rel_err(g, o, scale=row_rms(o, time_axis), floor=1.0),
+            "normwise": normwise_err(g, o)}

@@ -8,9 +8,8 @@ What it computes: the exact gradient of the scalar
     L = sum_{b,t,d} dy[b,t,d] * y[b,t,d] + sum_{b,d} dh_T[b,d] * h_T[b,d]
 with respect to every input of the forward layer (x, the conv taps, both gate
 weights and biases, Lambda, h0 and the conv history), i.e. the vector-Jacobian
-product of the layer defined in "Griffin: Mixing Gated Linear Recurrences with
-Local Attention for Efficient Language Models", section "Model Architecture"
-(the forward equations are restated in rglru_oracle). The sources give no
+product of the layer as defined in rglru_oracle (the layer's definition; the
+pages print no equation for it). The sources give no
 backward pass; this is the plain chain rule through the forward definition, in
 reverse order of its steps:
 

@@ -32,7 +32,7 @@ def main():
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "oracle_regression.txt")
     with open(path, "w") as f:
         f.write("# RG-LRU float64 oracle on workload tiny_f32 recipe with %s\n" % CASE)
-        f.write("# (Griffin, section 'Model Architecture': the RG-LRU layer with its width-4 Conv1D)\n")
+        f.write("# (the RG-LRU layer with its width-4 Conv1D, as defined in include/rglru.h)\n")
         f.write("# rows: y[b, t, :] for b, t in order, then h_T[b, :]\n")
         for b in range(CASE["B"]):
             for tt in range(CASE["T"]):

@@ -16,7 +16,7 @@ import torch.nn.functional as F
 
 from gated_linear_recurrence_rglru_b200.workloads import WORKLOADS, generate, lambda_from_ac
 from oracle import rglru_oracle as orc
-from oracle.compare import max_rel_err
+from oracle.compare import FLOOR, max_rel_err
 
 RNG = np.random.default_rng(1234)
 
@@ -304,7 +304,8 @@ def test_max_rel_err_measure():
     assert max_rel_err(g, o) == 0.0
     g[0, 1, 0] = 0.1                                      # error at a zero of o: floored by channel rms
     rms0 = math.sqrt((1.0 + 0.0) / 2)
-    assert max_rel_err(g, o) == pytest.approx(0.1 / rms0)
+    assert max_rel_err(g, o) == pytest.approx(0.1 / (FLOOR * rms0))
+    assert max_rel_err(g, o, floor=1.0) == pytest.approx(0.1 / rms0)
     g = o * 1.01
     assert max_rel_err(g, o) == pytest.approx(0.01)
     g[0, 0, 0] = np.nan

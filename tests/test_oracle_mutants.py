@@ -42,8 +42,23 @@ def _scan_off_by_one(a, beta, h0=None):
     return out
 
 
+def _ring_rotated_wrong(ring, pos):
+    ring = orc.as_f64(ring)
+    return ring[:, [(pos + 1 + k) % 3 for k in range(3)], :]
+
+
+def _decode_writes_wrong_slot(x_t, ring, pos, h, conv_w, W_a, b_a, W_x, b_x, Lambda,
+                              gate_operand=None):
+    y, h_new, ring_new = orc_decode(x_t, ring, pos, h, conv_w, W_a, b_a, W_x, b_x, Lambda,
+                                    gate_operand)
+    ring_new = orc.as_f64(ring).copy()
+    ring_new[:, (pos + 1) % 3, :] = orc.as_f64(x_t)
+    return y, h_new, ring_new
+
+
 orc_conv4 = orc.conv4
 orc_gate = orc.gate_preacts
+orc_decode = orc.rglru_decode_step
 
 MUTANTS = {
     "conv taps reversed": ("conv4", _flip_taps),
@@ -53,6 +68,8 @@ MUTANTS = {
     "sqrt(1 - a) normaliser": ("gated_input", _sqrt_one_minus_a),
     "input term drops u": ("gated_input", _drop_u),
     "scan uses a_{t-1}": ("linear_scan", _scan_off_by_one),
+    "decode ring read in the wrong order": ("ring_to_chronological", _ring_rotated_wrong),
+    "decode overwrites the wrong ring slot": ("rglru_decode_step", _decode_writes_wrong_slot),
 }
 
 PIN_TESTS = [
@@ -66,9 +83,24 @@ PIN_TESTS = [
     lambda: pins.test_chunked_and_sequential_scans_agree(7),
     pins.test_second_moment_is_preserved,
     pins.test_stationary_worst_case_bound,
-    pins.test_decode_steps_compose_with_fwd.__wrapped__ if hasattr(
-        pins.test_decode_steps_compose_with_fwd, "__wrapped__") else (lambda: None),
+    lambda: pins.test_decode_steps_compose_with_fwd(0),
+    lambda: pins.test_decode_steps_compose_with_fwd(3),
 ]
+
+
+def test_pins_pass_on_the_unchanged_oracle():
+    for pin in PIN_TESTS:
+        pin()
+
+
+@pytest.mark.parametrize("name", ["decode ring read in the wrong order",
+                                  "decode overwrites the wrong ring slot"])
+def test_decode_pin_alone_catches_ring_mutants(name, monkeypatch):
+    """The fwd/decode composition pin on its own catches both ring mistakes."""
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(orc, attr, fn)
+    with pytest.raises(AssertionError):
+        pins.test_decode_steps_compose_with_fwd(3)
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))

@@ -1,7 +1,9 @@
 """GPU parity: the CUDA library (through the C ABI) against the float64 oracle.
 
-Bars (max relative error, floored at the channel RMS, see oracle/compare.py):
-fp32 I/O 1e-4, bf16 I/O (fp32 state) 2e-2. The conv state outputs are copies
+Bars (max relative error, floored at 0.75 times the channel RMS, a floor derived
+in oracle/compare.py and tests/test_bf16_operand_rounding.py): fp32 I/O 1e-4,
+bf16 I/O (fp32 state) 2e-2. Output buffers start as NaN, so an element the
+kernels never write fails the comparison. The conv state outputs are copies
 of inputs and must match bit for bit. Small cases span several tiles and a
 ragged tail; the full-size workloads run in the bench's launch configuration
 and are checked on whole (batch row) or (head) blocks, which the layer keeps
@@ -41,9 +43,13 @@ def check_fwd(wl, algo, dev, with_csi=False, csi_seed=11):
         g = torch.Generator().manual_seed(csi_seed)
         csi = torch.randn(wl.B, 3, wl.D, generator=g).to(wl.dtype)
     g = to_dev(t, dev)
-    y, hT, cs = rg.rglru_fwd(g["x"], g["conv_w"], g["W_a"], g["b_a"], g["W_x"], g["b_x"],
-                             g["Lambda"], h0=g["h0"],
-                             conv_state_in=csi.to(dev) if csi is not None else None, algo=algo)
+    # outputs start as NaN: every element must be written
+    y = torch.full_like(g["x"], float("nan"))
+    hT = torch.full((wl.B, wl.D), float("nan"), device=dev)
+    cs = torch.full((wl.B, 3, wl.D), float("nan"), device=dev, dtype=wl.dtype)
+    rg.rglru_fwd(g["x"], g["conv_w"], g["W_a"], g["b_a"], g["W_x"], g["b_x"], g["Lambda"],
+                 h0=g["h0"], conv_state_in=csi.to(dev) if csi is not None else None, algo=algo,
+                 y=y, h_T=hT, conv_state_out=cs)
     torch.cuda.synchronize()
     yo, hTo, cso = orc.rglru_fwd(t["x"], t["conv_w"], t["W_a"], t["b_a"], t["W_x"], t["b_x"],
                                  t["Lambda"], h0=t["h0"], conv_state=csi)
@@ -114,7 +120,10 @@ def decode_run(wl, rows, dev, algo, steps):
     ring = g["conv_state"].clone()
     ys = []
     for s in range(steps):
-        ys.append(rg.rglru_decode_step(g["x_steps"][s], ring, s, h, *w_dev, algo=algo)[rows])
+        y_t = torch.full_like(g["x_steps"][s], float("nan"))    # must be fully written
+        rg.rglru_decode_step(g["x_steps"][s], ring, s, h, *w_dev, algo=algo, y_t=y_t)
+        assert bool(torch.isfinite(y_t.float()).all())
+        ys.append(y_t[rows])
     torch.cuda.synchronize()
     # oracle on the sampled rows only (rows never interact)
     w = {k: t[k] for k in ("conv_w", "W_a", "b_a", "W_x", "b_x", "Lambda")}
@@ -178,11 +187,13 @@ def full_fwd_sampled(name, dev, algo, sample):
     t = generate(wl)
     g = to_dev(t, dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
+    y = torch.full_like(g["x"], float("nan"))       # every element must be written
+    hT = torch.full((wl.B, wl.D), float("nan"), device=dev)
     y, hT, cs = rg.rglru_fwd(g["x"], g["conv_w"], g["W_a"], g["b_a"], g["W_x"], g["b_x"],
-                             g["Lambda"], h0=g["h0"], algo=algo, dev_status=status)
+                             g["Lambda"], h0=g["h0"], algo=algo, dev_status=status, y=y, h_T=hT)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
-    assert torch.isfinite(y.float()).all()
+    assert torch.isfinite(y.float()).all() and torch.isfinite(hT).all()
     errs = []
     for kind, idx in sample:
         if kind == "rows":
