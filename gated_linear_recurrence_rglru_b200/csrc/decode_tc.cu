@@ -449,7 +449,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
           if (fast) {
             gate_pair_fast(make_float2(za[2 * pr], za[2 * pr + 1]),
                            make_float2(zx[2 * pr], zx[2 * pr + 1]),
-                           make_float2(uu[2 * pr], uu[2 * pr + 1]), kc, a, beta, la);
+                           make_float2(uu[2 * pr], uu[2 * pr + 1]), kc, a, beta);
           } else {
             gate_one(za[2 * pr], zx[2 * pr], uu[2 * pr], kc, a.x, beta.x, la.x);
             gate_one(za[2 * pr + 1], zx[2 * pr + 1], uu[2 * pr + 1], kc, a.y, beta.y, la.y);

@@ -6,15 +6,20 @@
 // Components of Griffin", 1. RG-LRU; a memory-bound layer whose kernel should
 // optimise HBM accesses, S. De's thread on Griffin) is split into
 //   unit = (batch row b, group of 128 output channels), tile = 64 tokens
-//   (32 tokens when a head is 256 wide, so that its weights fit on chip).
+//   (32 tokens when a head is 256 wide).
 // Per tile
-//   1. the conv warpgroup computes the width-4 Conv1D token-major (4 channels x 8 tokens per step,
-//      vector shared-memory rows, packed fp32x2 FMAs) into the K-major bf16
-//      MMA operand and, for 128-wide channel ranges, an fp32 copy of u;
-//   2. (one thread of another warp issues tcgen05.mma with the gate weights as
-//      the A operand, M = 128 output channels, MN-major and loaded by TMA, and
-//      the conv output as B, N = tokens: TMEM lane m then holds channel m's
-//      two gate pre-activations along time);
+//   1. the conv warpgroup computes the width-4 Conv1D token-major (4 channels x
+//      4 tokens per step, vector shared-memory rows, packed fp32x2 FMAs) into
+//      the K-major bf16 MMA operand and an fp32 copy of the unit's own 128
+//      channels of u;
+//   2. one thread of another warp issues tcgen05.mma with the gate weights as
+//      the A operand (M = 128 output channels) and the conv output as B
+//      (N = tokens), so that TMEM lane m holds channel m's two gate
+//      pre-activations along time. The weights sit in shared memory for heads
+//      up to 128 wide (TMA, 128-byte swizzle, block-diagonal zeros for 64-wide
+//      heads) and in TMEM for 256-wide heads, where both gates (128 KB) would
+//      leave no shared memory for the pipeline (the conv warpgroup writes them
+//      there at each change of unit);
 //   3. an epilogue warpgroup, per lane (channel): sigmoid gates, log-space
 //      decay, sqrt(1 - a^2) and a local scan along time from a zero state,
 //      keeping the running products P_t = a_1 ... a_t and local states Hl_t
@@ -51,10 +56,16 @@ using namespace gates;
 constexpr int kM = 128;         // output channels per unit (MMA M, TMEM lanes)
 constexpr int kJQ = 8;          // job ring depth
 constexpr uint64_t kWaitNs = 2000000000ull;   // bound of any wait
+// predecessor carry words read per look-back round trip (one L2 latency each)
+#ifndef RGLRU_LOOKBACK_WORDS
+#define RGLRU_LOOKBACK_WORDS 4
+#endif
+constexpr int kLB = RGLRU_LOOKBACK_WORDS;
 constexpr uint64_t kDrainNs = 200000000ull;   // bound of the drain after an abort
 
 struct TcParams {
   const __nv_bfloat16 *conv_w, *b_a, *b_x;
+  const __nv_bfloat16 *W_a, *W_x;            // (H, bw, bw): read directly when A is in TMEM
   const float *Lambda, *h0;
   const __nv_bfloat16 *conv_state_in;
   __nv_bfloat16 *y;
@@ -76,17 +87,19 @@ struct Cfg {
   static constexpr int kThreads = (64 + 128 + NE * 128 + 127) / 128 * 128;
   static constexpr int kXRows = N + 3;
   static constexpr int kXBytes = ((kXRows * K * 2) + 1023) / 1024 * 1024;
-  static constexpr int kABytes = K * 256;          // one gate: 2 M-blocks x K rows x 128 B
+  // Gate weights (the MMA's A operand, M = 128 output channels x K): in shared
+  // memory for K = 128 (TMA, 128-byte swizzle; block-diagonal zeros for 64-wide
+  // heads), in TMEM for K = 256, where both gates (128 KB) would not leave
+  // shared memory for the pipeline (written by the conv warpgroup)
+  static constexpr bool kATmem = (K == 256);
+  static constexpr int kABytes = kATmem ? 0 : K * 256;     // one gate: 2 M-blocks x K rows x 128 B
   static constexpr int kBBytes = N * K * 2;        // K-major conv output, one slot
-  // fp32 u of the unit's own channels, token-major [N][128], for beta (K = 128
-  // only; with K = 256 the epilogue recomputes u from the x tile instead)
-  static constexpr bool kUTile = (K == 128);
-  static constexpr int kUBytes = kUTile ? N * kM * 4 : 0;
+  // fp32 u of the unit's own channels, channel-major [128][N], for beta
+  static constexpr int kUBytes = N * kM * 4;
   static constexpr int kNS = 2;                    // conv -> MMA slots (B operand)
   // conv -> epilogue slots (u tile); with three, the conv of job i waits for
-  // pass 1 of job i - 3 rather than of job i - 2 (which ran in the same
-  // epilogue warpgroup as job i and would chain conv, MMA and pass 1 serially)
-  static constexpr int kNU = kUTile ? NU : 1;
+  // pass 1 of job i - 3 rather than of job i - 2
+  static constexpr int kNU = NU;
   // TMEM slots: one per epilogue warpgroup and one for the MMA to run ahead
   static constexpr int kNT = NE + 1;
   static constexpr int kOffA = 0;
@@ -95,20 +108,21 @@ struct Cfg {
   static constexpr int kOffU = kOffB + kNS * kBBytes;
   static constexpr int kOffBar = kOffU + kNU * kUBytes;
   // job_full[JQ], job_empty[JQ], x_full[NX], x_empty[NX], w_full, w_free,
-  // b_full[NS], b_empty[NS], u_empty[NU], acc_full[NT], tmem_empty[NT]
-  static constexpr int kNumBars = 2 * kJQ + 2 * NX + 2 + 2 * kNS + kNU + 2 * kNT;
+  // b_full[NS], b_empty[NS], u_empty[NU], acc_full[NT], tmem_empty[NT], a_ready
+  static constexpr int kNumBars = 2 * kJQ + 2 * NX + 2 + 2 * kNS + kNU + 2 * kNT + 1;
   static constexpr int kOffJobs = (kOffBar + kNumBars * 8 + 15) / 16 * 16;
   static constexpr int kOffMisc = kOffJobs + kJQ * 16;
   // the dynamic shared memory base is declared 1024-byte aligned (the kernel
   // checks it), as the 128-byte swizzle of the TMA and MMA tiles needs
   static constexpr int kSmemBytes = kOffMisc + 64;
-  static constexpr int kSlotCols = 2 * N;                   // z_a | z_x, then a | beta
-  static constexpr int kTmemCols =
-      kNT * kSlotCols <= 128 ? 128 : (kNT * kSlotCols <= 256 ? 256 : 512);
+  static constexpr int kSlotCols = 2 * N;                   // z_a | z_x, then P | Hl
+  static constexpr int kACol = kNT * kSlotCols;             // TMEM A: gate a, then gate x
+  static constexpr int kUsedCols = kACol + (kATmem ? K : 0);
+  static constexpr int kTmemCols = kUsedCols <= 128 ? 128 : (kUsedCols <= 256 ? 256 : 512);
   static_assert((N * (K / 4)) % 128 == 0, "conv mapping");
-  static_assert(N % 16 == 0 && K % 128 == 0, "tile shape");
+  static_assert(N % 32 == 0 && K % 128 == 0, "tile shape");
   static_assert(kSmemBytes <= 232448, "shared memory");
-  static_assert(kNT * kSlotCols <= 512, "TMEM allocation");
+  static_assert(kUsedCols <= 512, "TMEM allocation");
 };
 
 __device__ void raise_abort(const TcParams &p, volatile int *cta_abort, int code) {
@@ -152,9 +166,9 @@ __device__ __forceinline__ uint32_t u_offset(int c, int jb) {
 // (no bank conflicts). The loop advances 4 tokens per iteration with a sliding
 // window of 4 input rows in registers (a compact loop: the conv shares the
 // instruction cache with the epilogue). Writes the bf16 B operand (K-major,
-// 128-byte swizzle) and, when kUTile, the fp32 u of the unit's own channels
+// 128-byte swizzle) and the fp32 u of the unit's own channels
 // channel-major into ut (see u_offset). w holds the 4 taps of the 4 channels.
-template <int K, int N, bool kUTile>
+template <int K, int N>
 __device__ __forceinline__ void conv_tile(const unsigned char *__restrict__ xs,
                                           unsigned char *__restrict__ bt,
                                           unsigned char *__restrict__ ut, const TcParams &p, int b,
@@ -230,7 +244,7 @@ __device__ __forceinline__ void conv_tile(const unsigned char *__restrict__ xs,
       uacc[2][q] = u[1].x;
       uacc[3][q] = u[1].y;
     }
-    if (kUTile && own) {
+    if (own) {
       const uint32_t blk = static_cast<uint32_t>((nb + jb) >> 2) << 4;
 #pragma unroll
       for (int k = 0; k < 4; ++k)
@@ -249,6 +263,39 @@ __device__ __forceinline__ void conv_tile(const unsigned char *__restrict__ xs,
         v = __ldg(reinterpret_cast<const uint2 *>(p.conv_state_in +
                                                    (static_cast<size_t>(b) * 3 + row) * p.D + chq));
       *reinterpret_cast<uint2 *>(p.conv_state_out + (static_cast<size_t>(b) * 3 + r) * p.D + chq) = v;
+    }
+  }
+}
+
+// Pass 2 of one tile for one channel (this thread's TMEM lane): y_t =
+// P_t h_in + Hl_t for the valid tokens, stored bf16 at a row stride of kD
+// channels (a compile-time stride for the common widths, so that the 16
+// stores of a chunk take immediate offsets; 0 = runtime D).
+template <int N, int kD>
+__device__ __forceinline__ void pass2_store(__nv_bfloat16 *yrow, int D, uint32_t t_lane,
+                                            int nvalid, float h_in) {
+  const size_t ld = kD > 0 ? static_cast<size_t>(kD) : static_cast<size_t>(D);
+#pragma unroll 1
+  for (int ch = 0; ch < N / 16; ++ch) {
+    if (ch * 16 >= nvalid) break;
+    float pv[16], hv[16];
+    tmem_ld16(t_lane + ch * 16, pv);
+    tmem_ld16(t_lane + N + ch * 16, hv);
+    tmem_wait_ld();
+    __nv_bfloat16 *yc = yrow + static_cast<size_t>(ch * 16) * ld;
+    if (ch * 16 + 16 <= nvalid) {
+#pragma unroll
+      for (int j = 0; j < 16; j += 2) {
+        const float2 v = __ffma2_rn(make_float2(pv[j], pv[j + 1]), f2(h_in),
+                                    make_float2(hv[j], hv[j + 1]));
+        yc[static_cast<size_t>(j) * ld] = __float2bfloat16_rn(v.x);
+        yc[static_cast<size_t>(j + 1) * ld] = __float2bfloat16_rn(v.y);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (ch * 16 + j < nvalid)
+          yc[static_cast<size_t>(j) * ld] = __float2bfloat16_rn(fmaf(pv[j], h_in, hv[j]));
     }
   }
 }
@@ -282,6 +329,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
   uint64_t *u_empty = b_empty + NS;                 // [NU] epilogue pass 1 -> conv
   uint64_t *acc_full = u_empty + NUS;               // [NT] MMA -> epilogue
   uint64_t *tmem_empty = acc_full + NT;             // [NT] epilogue pass 2 -> MMA
+  uint64_t *a_ready = tmem_empty + NT;              // conv warpgroup wrote TMEM weights -> MMA
   int4 *jobs = reinterpret_cast<int4 *>(sm + C::kOffJobs);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + C::kOffMisc);
   volatile int *cta_abort = reinterpret_cast<volatile int *>(sm + C::kOffMisc + 4);
@@ -311,6 +359,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
       mbar_init(&acc_full[i], 1);
       mbar_init(&tmem_empty[i], 4);                 // 4 epilogue warps
     }
+    mbar_init(a_ready, 4);                          // 4 conv warps
     *cta_abort = 0;
     fence_mbar_init();
     prefetch_tmap(&tmap_x);
@@ -416,7 +465,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
           break;
         }
         const int b = unit / p.n_cg, cg = unit % p.n_cg;
-        if (reload) {
+        if (reload && !C::kATmem) {
           if (i > 0) {
             // the MMA warp signals once the MMAs of job i-1 (the last readers of
             // the weights in shared memory) have completed
@@ -442,8 +491,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
               }
             }
           }
-          w_unit = unit;
         }
+        if (reload) w_unit = unit;
         const int kbase = p.bw <= 128 ? cg * kM : (cg >> 1) * 256;
         if (lane == 0) {
           mbar_arrive_expect_tx(&x_full[xb], static_cast<uint32_t>(C::kXRows * K * 2));
@@ -460,9 +509,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
   } else if (warp == 1) {
     // ============================== MMA issuer ==============================
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kM, N, true, false);
+      // A from shared memory is MN-major (loaded by TMA); A from TMEM is K-major
+      constexpr uint32_t idesc = idesc_bf16_f32(kM, N, !C::kATmem, false);
       const uint64_t ada0 = sdesc_sw128(smem_u32(sA), K * 128, 1024);
       const uint64_t adx0 = sdesc_sw128(smem_u32(sA + C::kABytes), K * 128, 1024);
+      const uint32_t ta_a = tmem_base + static_cast<uint32_t>(C::kACol);
+      const uint32_t ta_x = ta_a + static_cast<uint32_t>(K / 2);
       uint32_t w_phase = 0;
       int last_commit = -1;
       for (int i = 0;; ++i) {
@@ -471,13 +523,18 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
         const int4 job = jobs[js];
         if (job.x < 0) break;
         if (job.z) {
-          if (last_commit >= 0) {
-            // MMAs complete in order: job i-1 done => every read of the old weights done
-            const int lc = last_commit;
-            RG_WAIT_OR_ABORT(&acc_full[lc % NT], (lc / NT) & 1);
-            mbar_arrive(w_free);
+          if (C::kATmem) {
+            // the conv warpgroup has written this unit's weights into TMEM
+            RG_WAIT_OR_ABORT(a_ready, w_phase);
+          } else {
+            if (last_commit >= 0) {
+              // MMAs complete in order: job i-1 done => every read of the old weights done
+              const int lc = last_commit;
+              RG_WAIT_OR_ABORT(&acc_full[lc % NT], (lc / NT) & 1);
+              mbar_arrive(w_free);
+            }
+            RG_WAIT_OR_ABORT(w_full, w_phase);
           }
-          RG_WAIT_OR_ABORT(w_full, w_phase);
           w_phase ^= 1;
         }
         const int s = i % NS, ts = i % NT;
@@ -494,9 +551,14 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
 #pragma unroll
         for (int ks = 0; ks < K / 16; ++ks) {
           const uint64_t bd = bd0 + static_cast<uint64_t>(((ks >> 2) * (N * 128) + (ks & 3) * 32) >> 4);
-          const uint64_t astep = static_cast<uint64_t>((ks * 16 * 128) >> 4);
-          mma_bf16(d_a, ada0 + astep, bd, idesc, ks > 0 ? 1u : 0u);
-          mma_bf16(d_x, adx0 + astep, bd, idesc, ks > 0 ? 1u : 0u);
+          if (C::kATmem) {
+            mma_bf16_ts(d_a, ta_a + static_cast<uint32_t>(ks * 8), bd, idesc, ks > 0 ? 1u : 0u);
+            mma_bf16_ts(d_x, ta_x + static_cast<uint32_t>(ks * 8), bd, idesc, ks > 0 ? 1u : 0u);
+          } else {
+            const uint64_t astep = static_cast<uint64_t>((ks * 16 * 128) >> 4);
+            mma_bf16(d_a, ada0 + astep, bd, idesc, ks > 0 ? 1u : 0u);
+            mma_bf16(d_x, adx0 + astep, bd, idesc, ks > 0 ? 1u : 0u);
+          }
         }
         mma_commit(&acc_full[ts]);
         mma_commit(&b_empty[s]);
@@ -530,12 +592,46 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
           cwq[tap][0] = bf2_to_f2(raw.x);
           cwq[tap][1] = bf2_to_f2(raw.y);
         }
+        if (C::kATmem) {
+          // This unit's gate weights into TMEM (the A operand): lane m (output
+          // channel cg*128 + m) holds W[h][k][j] for k = 0..K-1, two per column.
+          // Every MMA of earlier jobs has read the old weights once the
+          // accumulator of job i-1 is complete (MMAs complete in issue order).
+          if (i > 0) RG_WAIT_OR_ABORT(&acc_full[(i - 1) % NT], ((i - 1) / NT) & 1);
+          const int qd = warp & 3;                  // this warp's TMEM lane quadrant
+          const int cout = cg * kM + qd * 32 + lane;
+          const int hh = cout / p.bw, jj = cout % p.bw;
+          const uint32_t tq = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) +
+                              static_cast<uint32_t>(C::kACol);
+#pragma unroll 1
+          for (int g = 0; g < 2; ++g) {
+            const unsigned short *Wg =
+                reinterpret_cast<const unsigned short *>(g == 0 ? p.W_a : p.W_x) +
+                static_cast<size_t>(hh) * p.bw * p.bw + jj;
+#pragma unroll 1
+            for (int cc = 0; cc < K / 64; ++cc) {
+              uint32_t v[32];
+#pragma unroll
+              for (int q = 0; q < 32; ++q) {
+                const int k = cc * 64 + 2 * q;
+                const uint32_t lo = __ldg(Wg + static_cast<size_t>(k) * p.bw);
+                const uint32_t hi = __ldg(Wg + static_cast<size_t>(k + 1) * p.bw);
+                v[q] = lo | (hi << 16);
+              }
+              tmem_st32u(tq + static_cast<uint32_t>(g * (K / 2) + cc * 32), v);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(a_ready);
+        }
       }
       const int s = i % NS, xb = i % NX, us = i % NUS;
       RG_WAIT_OR_ABORT(&x_full[xb], (i / NX) & 1);
       RG_WAIT_OR_ABORT(&b_empty[s], ((i / NS) & 1) ^ 1);
-      if (C::kUTile) RG_WAIT_OR_ABORT(&u_empty[us], ((i / NUS) & 1) ^ 1);
-      conv_tile<K, N, C::kUTile>(sX + xb * C::kXBytes, sB + s * C::kBBytes, sU + us * C::kUBytes,
+      RG_WAIT_OR_ABORT(&u_empty[us], ((i / NUS) & 1) ^ 1);
+      conv_tile<K, N>(sX + xb * C::kXBytes, sB + s * C::kBBytes, sU + us * C::kUBytes,
                                  p, b, kbase, own_lo, tile, nvalid, tile == p.n_tiles - 1, wt,
                                  cwq);
       // each warp hands its part over on its own: no barrier that an aborting
@@ -543,7 +639,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        if (C::kUTile) mbar_arrive(&x_empty[xb]);   // else the epilogue still reads x
+        mbar_arrive(&x_empty[xb]);
         mbar_arrive(&b_full[s]);
         mbar_arrive(&job_empty[js]);
       }
@@ -560,8 +656,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
     const int m = qd * 32 + lane;                 // TMEM lane == output channel in unit
     const uint32_t t_lane0 = tmem_base + (static_cast<uint32_t>(qd * 32) << 16);
     int cur_unit = -1;
-    ChanK kc{0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    float cwo[4] = {0.f, 0.f, 0.f, 0.f};          // own channel's conv taps (K = 256)
+    ChanK kc{};
     bool fast = true;
 
     for (int i = eg;; i += NE) {
@@ -572,86 +667,49 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
       if (unit < 0) break;
       const int b = unit / p.n_cg, cg = unit % p.n_cg;
       const int c = cg * kM + m;                  // own output channel
-      const int own_lo = p.bw <= 128 ? 0 : (cg & 1) * kM;
       const int nvalid = min(N, p.T - tile * N);
-      const int us = i % NUS, ts = i % NT, xb = i % NX;
+      const int us = i % NUS, ts = i % NT;
       const uint32_t t_lane = t_lane0 + static_cast<uint32_t>(ts * C::kSlotCols);
       if (unit != cur_unit) {
         cur_unit = unit;
         kc = chan_consts(__bfloat162float(p.b_a[c]), __bfloat162float(p.b_x[c]), p.Lambda[c]);
         fast = __all_sync(0xffffffffu, chan_fast(kc));
-        if (!C::kUTile) {
-#pragma unroll
-          for (int tap = 0; tap < 4; ++tap) cwo[tap] = __bfloat162float(p.conv_w[tap * p.D + c]);
-        }
       }
       RG_WAIT_OR_ABORT(&acc_full[ts], (i / NT) & 1);
       tc_fence_after();
-      // own channel's u: fp32 tile from the conv warpgroup (K = 128), or
-      // recomputed from the x tile (K = 256)
-      // this channel's row of the u tile and its block permutation (x 16 bytes)
+      // own channel's u: the fp32 tile from the conv warpgroup; this channel's
+      // row of it and its block permutation (x 16 bytes)
       const uint32_t urow = smem_u32(sU + us * C::kUBytes) + static_cast<uint32_t>(m * (N * 4));
       const uint32_t uperm = static_cast<uint32_t>((m & 7) ^ ((m >> 3) & 7)) << 4;
-      const __nv_bfloat16 *xown =
-          reinterpret_cast<const __nv_bfloat16 *>(sX + xb * C::kXBytes) + own_lo + m;
-      float xm3 = 0.f, xm2 = 0.f, xm1 = 0.f;
-      if (!C::kUTile) {
-        xm3 = __bfloat162float(xown[0]);
-        xm2 = __bfloat162float(xown[K]);
-        xm1 = __bfloat162float(xown[2 * K]);
-        if (tile == 0 && p.conv_state_in != nullptr) {
-          const __nv_bfloat16 *cs = p.conv_state_in + static_cast<size_t>(b) * 3 * p.D + c;
-          xm3 = __bfloat162float(cs[0]);
-          xm2 = __bfloat162float(cs[p.D]);
-          xm1 = __bfloat162float(cs[2 * p.D]);
-        }
-      }
       // ---- pass 1: gates, decay, local scan from zero; (P_t, Hl_t) -> TMEM ----
-      // Tokens past the end of the sequence (last tile) are computed like the
-      // others (their x rows read as zeros) and never used: the tile's
-      // aggregate is read back at the last valid token.
+      // 16 tokens per TMEM round trip, the gate math two tokens at a time in
+      // fp32x2 instructions. Tokens past the end of the sequence (last tile)
+      // are computed like the others (their x rows read as zeros) and never
+      // used: the tile's aggregate is read back at the last valid token.
       float Hl = 0.f, P = 1.f;
 #pragma unroll 1
       for (int ch = 0; ch < N / 16; ++ch) {
-        float za[16], zx[16];
+        float za[16], zx[16], uu[16];
         tmem_ld16(t_lane + ch * 16, za);
         tmem_ld16(t_lane + N + ch * 16, zx);
-        float uu[16];
-        if (C::kUTile) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float4 v = lds128f(urow + (static_cast<uint32_t>((ch * 4 + q) << 4) ^ uperm));
-            uu[4 * q] = v.x;
-            uu[4 * q + 1] = v.y;
-            uu[4 * q + 2] = v.z;
-            uu[4 * q + 3] = v.w;
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float xv = __bfloat162float(xown[(ch * 16 + j + 3) * K]);
-            uu[j] = fmaf(cwo[3], xv, fmaf(cwo[2], xm1, fmaf(cwo[1], xm2, cwo[0] * xm3)));
-            xm3 = xm2;
-            xm2 = xm1;
-            xm1 = xv;
-          }
+        for (int q = 0; q < 4; ++q) {
+          const float4 v = lds128f(urow + (static_cast<uint32_t>((ch * 4 + q) << 4) ^ uperm));
+          uu[4 * q] = v.x; uu[4 * q + 1] = v.y; uu[4 * q + 2] = v.z; uu[4 * q + 3] = v.w;
         }
         if (ch == N / 16 - 1) {
-          // the last reads of the u (x) tile are issued: hand the slot back
+          // the last reads of the u tile are issued: hand the slot back
           __syncwarp();
-          if (lane == 0) {
-            if (C::kUTile) mbar_arrive(&u_empty[us]);
-            else mbar_arrive(&x_empty[xb]);
-          }
+          if (lane == 0) mbar_arrive(&u_empty[us]);
         }
         tmem_wait_ld();
         if (fast) {
 #pragma unroll
           for (int pr = 0; pr < 8; ++pr) {
-            float2 a, beta, la;
+            float2 a, beta;
             gate_pair_fast(make_float2(za[2 * pr], za[2 * pr + 1]),
                            make_float2(zx[2 * pr], zx[2 * pr + 1]),
-                           make_float2(uu[2 * pr], uu[2 * pr + 1]), kc, a, beta, la);
+                           make_float2(uu[2 * pr], uu[2 * pr + 1]), kc, a, beta);
             Hl = fmaf(a.x, Hl, beta.x);
             P *= a.x;
             za[2 * pr] = P;
@@ -676,10 +734,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
         tmem_st16(t_lane + N + ch * 16, zx);
       }
       tmem_wait_st();
-      float A = P;
+      // the tile's aggregate over its valid tokens: (prod a, local state)
+      float A = P, Hag = Hl;
       if (nvalid < N) {
         A = tmem_ld1(t_lane + (nvalid - 1));
-        Hl = tmem_ld1(t_lane + N + (nvalid - 1));
+        Hag = tmem_ld1(t_lane + N + (nvalid - 1));
         tmem_wait_ld();
       }
       // publish this channel's word: inclusive for the first tile of a
@@ -690,9 +749,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
         if (!silent) {
           if (tile == 0) {
             const float h0v = p.h0 != nullptr ? p.h0[static_cast<size_t>(b) * p.D + c] : 0.f;
-            st_relaxed_u64(p.carry + wix, carry_inc(fmaf(A, h0v, Hl)));
+            st_relaxed_u64(p.carry + wix, carry_inc(fmaf(A, h0v, Hag)));
           } else {
-            st_relaxed_u64(p.carry + wix, carry_agg(A, Hl));
+            st_relaxed_u64(p.carry + wix, carry_agg(A, Hag));
           }
         }
       }
@@ -702,7 +761,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
       if (tile == 0) {
         if (p.h0 != nullptr) h_in = p.h0[static_cast<size_t>(b) * p.D + c];
       } else {
-        // Look back along this lane's channel, four words per round trip: fold
+        // Look back along this lane's channel, kLB words per round trip: fold
         // aggregates until an inclusive word; an unpublished word ends the
         // round and is read again in the next.
         float mult = 1.f, add = 0.f;
@@ -711,13 +770,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
         const uint64_t t0 = globaltimer_ns();
         for (;;) {
           if (!done) {
-            unsigned long long w[4];
+            unsigned long long w[kLB];
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
+            for (int q = 0; q < kLB; ++q)
               w[q] = (k - q >= 0) ? ld_relaxed_u64(cw + static_cast<size_t>(k - q) * kM) : 0ull;
             bool stop = false;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < kLB; ++q) {
               if (stop) continue;
               const uint32_t lo = static_cast<uint32_t>(w[q]);
               const float hi = __uint_as_float(static_cast<uint32_t>(w[q] >> 32));
@@ -746,31 +805,18 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
           __nanosleep(64);
         }
         if (!(unit == 0 && tile == p.fault_tile))
-          st_relaxed_u64(cw + static_cast<size_t>(tile) * kM, carry_inc(fmaf(A, h_in, Hl)));
+          st_relaxed_u64(cw + static_cast<size_t>(tile) * kM, carry_inc(fmaf(A, h_in, Hag)));
       }
       // ---- pass 2: y_t = P_t h_in + Hl_t ----
       __nv_bfloat16 *yrow = p.y + (static_cast<size_t>(b) * p.T + tile * N) * p.D + c;
-#pragma unroll 1
-      for (int ch = 0; ch < N / 16; ++ch) {
-        if (ch * 16 >= nvalid) break;
-        float pv[16], hv[16];
-        tmem_ld16(t_lane + ch * 16, pv);
-        tmem_ld16(t_lane + N + ch * 16, hv);
-        tmem_wait_ld();
-        __nv_bfloat16 *yc = yrow + static_cast<size_t>(ch * 16) * p.D;
-        if (ch * 16 + 16 <= nvalid) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            yc[static_cast<size_t>(j) * p.D] = __float2bfloat16_rn(fmaf(pv[j], h_in, hv[j]));
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (ch * 16 + j < nvalid)
-              yc[static_cast<size_t>(j) * p.D] = __float2bfloat16_rn(fmaf(pv[j], h_in, hv[j]));
-        }
+      switch (p.D) {
+        case 1024: pass2_store<N, 1024>(yrow, p.D, t_lane, nvalid, h_in); break;
+        case 2560: pass2_store<N, 2560>(yrow, p.D, t_lane, nvalid, h_in); break;
+        case 4096: pass2_store<N, 4096>(yrow, p.D, t_lane, nvalid, h_in); break;
+        default: pass2_store<N, 0>(yrow, p.D, t_lane, nvalid, h_in); break;
       }
       if (tile == p.n_tiles - 1 && p.h_T != nullptr)
-        p.h_T[static_cast<size_t>(b) * p.D + c] = fmaf(A, h_in, Hl);
+        p.h_T[static_cast<size_t>(b) * p.D + c] = fmaf(A, h_in, Hag);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -860,6 +906,8 @@ cudaError_t launch_tc_t(const FwdArgs &a, const TcLayout &L, void *ws, cudaStrea
   p.conv_w = static_cast<const __nv_bfloat16 *>(a.conv_w);
   p.b_a = static_cast<const __nv_bfloat16 *>(a.b_a);
   p.b_x = static_cast<const __nv_bfloat16 *>(a.b_x);
+  p.W_a = static_cast<const __nv_bfloat16 *>(a.W_a);
+  p.W_x = static_cast<const __nv_bfloat16 *>(a.W_x);
   p.Lambda = a.Lambda;
   p.h0 = a.h0;
   p.conv_state_in = static_cast<const __nv_bfloat16 *>(a.conv_state_in);
@@ -922,7 +970,7 @@ size_t tc_workspace_bytes(int B, int T, int D, int H) { return tc_layout(B, T, D
 cudaError_t launch_fwd_tc(const FwdArgs &a, void *ws, cudaStream_t st) {
   const int bw = a.D / a.H;
   const TcLayout L = tc_layout(a.B, a.T, a.D, a.H);
-  if (bw == 256) return launch_tc_t<256, 32, 3, 3, 1>(a, L, ws, st);
+  if (bw == 256) return launch_tc_t<256, 32, 3, 3, 3>(a, L, ws, st);
   return launch_tc_t<128, 64, 2, 3, 3>(a, L, ws, st);
 }
 

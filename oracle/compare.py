@@ -3,23 +3,27 @@
 max relative error = max_i |g_i - o_i| / max(|o_i|, s_i),  s_i = FLOOR * RMS_c,
 
 where RMS_c is the root-mean-square of the oracle's output over every batch
-row and time (or decode) step of element i's own channel c, and FLOOR = 0.75.
+row and time (or decode) step of element i's own channel c, and FLOOR = 1.
 
 Why a floor, and why this one. A pure elementwise relative error is undefined
 where h_t crosses zero, so some floor is needed. The floor is derived from the
 arithmetic that a bf16 tensor-core gate contraction performs, not chosen from
 a kernel's result: tests/test_bf16_operand_rounding.py runs the float64
 oracle with one change, the Conv1D output rounded to bf16 where it enters the
-gate contraction (and y stored in bf16), on the parity cases, and finds:
-  * its absolute error reaches about 2e-2 of the channel's RMS, so under a
+gate contraction (and y stored in bf16), on the shapes of the parity cases,
+and tests/test_backward_bf16_operands.py does the same for the backward's two
+rounded operands. They find:
+  * the absolute error reaches about 2e-2 of the channel's RMS, so under a
     floor of 1e-3 * RMS the designed arithmetic itself scores 2 to 10, over
     100 times the 2e-2 bar: no bf16-operand contraction can meet that floor;
   * with the RMS of one batch row as the scale, a 5-step decode case needs a
     factor of at least 1.05 (a row whose state stays near zero for a few steps
     has a small RMS while the step's increment, and its rounding, does not);
-  * with the channel's RMS over all rows and steps, every case meets the bar
-    from a factor of 0.59 (forward) or 0.52 (decode) up. FLOOR = 0.75 is the
-    tightest round factor above them with a margin of about 1.25.
+  * with the channel's RMS over all rows and steps, the bar is met from a
+    factor of 0.83 up in the worst forward case (long-memory channels,
+    a^8 up to 0.9999, T = 2000), 0.79 in the backward and 0.52 in the decode
+    step. FLOOR = 1 is the tightest round factor above them, with a margin of
+    at least 1.2.
 A wrong term, sign or index still shows up as an O(1) error under this floor
 (tests/test_oracle_mutants.py plants such mistakes). The GPU tests also compare
 the tensor-core path with the bf16-operand arithmetic itself: y agrees to the
@@ -31,7 +35,11 @@ from __future__ import annotations
 import numpy as np
 
 TINY = 1e-30
-FLOOR = 0.75          # floor factor on the channel RMS (see above)
+FLOOR = 1.0           # floor factor on the channel RMS (see above)
+# The backward rounds two operands to bf16 (u for z = u W and d z for d z W^T), and
+# its d u = own term + d z W^T can cancel: its designed arithmetic needs a factor of
+# 0.79 on the B=2 T=2048 D=1024 H=16 case (tests/test_backward_bf16_operands.py).
+BWD_FLOOR = FLOOR
 SURVEY_FLOOR = 1e-3   # a floor too tight for any bf16-operand contraction; reported only
 
 
@@ -80,7 +88,7 @@ def normwise_err(g, o) -> float:
 
 def error_report(g, o, time_axis: int = 1) -> dict:
     """The same comparison under the three floors discussed above, for reporting."""
-    return {"floor_0.75_channel_rms": max_rel_err(g, o, time_axis=time_axis),
+    return {"floor_1_channel_rms": max_rel_err(g, o, time_axis=time_axis),
             "floor_1e-3_channel_rms": max_rel_err(g, o, time_axis=time_axis, floor=SURVEY_FLOOR),
             "floor_1_row_rms": max_rel_err(g, o, scale=row_rms(o, time_axis), floor=1.0),
             "normwise": normwise_err(g, o)}

@@ -139,7 +139,9 @@ def test_tensor_path_is_the_designed_arithmetic(cuda_device, idx):
     ye, he, _ = _oracle(t, gate_operand="bf16")
     yo, ho, _ = _oracle(t)
     e_design = max_rel_err(yg, ye)
-    e_exact = max_rel_err(yg, yo)
     h_design = max_rel_err(hg, he, scale=channel_rms(ye, 1)[:, 0, :])
+    h_exact = max_rel_err(hg, ho, scale=channel_rms(yo, 1)[:, 0, :])
     assert e_design <= DESIGNED_TOL_Y and h_design <= DESIGNED_TOL_H, (e_design, h_design)
-    assert e_design < e_exact / 2, (e_design, e_exact)   # the rounding explains the error
+    # the operand rounding explains the error: h_T (fp32, no output rounding)
+    # is far closer to the designed arithmetic than to the exact oracle
+    assert h_design < h_exact / 10, (h_design, h_exact)
