@@ -267,8 +267,10 @@ def time_forward(rg, wl, dev, steps, warmup, algo, pk, soak_s=0.0, ws=1):
             step(i)
             i += 1
         torch.cuda.synchronize()
-    if int(status.item()) != 0:
-        raise SystemExit(f"device status {int(status.item())}: {rg.status_str(int(status.item()))}")
+    word = int(status.item())
+    if word != 0:
+        raise SystemExit(f"device status word {word:#x}: {rg.status_str(word & 0xFF)} "
+                         f"(wait site {(word >> 8) & 0xFF}, block {word >> 16})")
     chtok = B * T * D
     bytes_step = fwd_bytes_per_chtok(wl) * chtok
     kname, traffic = kernel_traffic(wl, algo)

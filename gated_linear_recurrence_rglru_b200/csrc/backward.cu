@@ -1253,10 +1253,16 @@ template <typename T>
 cudaError_t launch_bwd_io(const BwdArgs &p, void *ws, cudaStream_t st) {
   const int bw = p.D / p.H;
   if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-    // bf16 operands for the two in-loop gate contractions (tensor cores)
-    if (bw == 32) return launch_bwd_t<T, false, 256, 32>(p, ws, st);
-    if (bw == 64) return launch_bwd_t<T, false, 256, 64>(p, ws, st);
-    if (bw == 128) return launch_bwd_t<T, false, 512, 128>(p, ws, st);
+    // bf16 operands for the two in-loop gate contractions (tensor cores), from
+    // one 8-token group over all rows up: below that a channel has fewer than
+    // 8 samples, and the operands' rounding (2^-9 of u and of d z), against
+    // cancellation between d u's two terms, is no longer small next to the
+    // channel's own scale; those tiny problems take the fp32 operands below
+    if (static_cast<long long>(p.B) * p.T >= 8) {
+      if (bw == 32) return launch_bwd_t<T, false, 256, 32>(p, ws, st);
+      if (bw == 64) return launch_bwd_t<T, false, 256, 64>(p, ws, st);
+      if (bw == 128) return launch_bwd_t<T, false, 512, 128>(p, ws, st);
+    }
   }
   // both gate weights in shared memory (fp32) up to 128-wide heads: 2 x 129 x 128 x 4 B;
   // a segment's threads (bw rounded up to a warp) fit a 512-thread block up to 512-wide

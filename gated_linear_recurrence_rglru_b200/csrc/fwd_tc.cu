@@ -125,8 +125,19 @@ struct Cfg {
   static_assert(kUsedCols <= 512, "TMEM allocation");
 };
 
-__device__ void raise_abort(const TcParams &p, volatile int *cta_abort, int code) {
-  if (p.dev_status) atomicCAS(p.dev_status, 0, code);
+// Where a wait gave up, recorded in bits 8-15 of the status word (bits 16-31
+// hold the CTA index), so that an expiry names its wait.
+enum WaitSite : int {
+  kSiteProducer = 1,   // job ring / x slot / weights free (tile claims and TMA)
+  kSiteMma = 2,        // job / weights / B operand / TMEM slot (MMA issue)
+  kSiteConv = 3,       // job / x tile / B slot / u slot (Conv1D)
+  kSiteEpilogue = 4,   // job / accumulator (epilogue)
+  kSiteLookBack = 5    // a predecessor tile's carry word
+};
+
+__device__ void raise_abort(const TcParams &p, volatile int *cta_abort, int code, int site) {
+  if (p.dev_status)
+    atomicCAS(p.dev_status, 0, code | (site << 8) | (static_cast<int>(blockIdx.x) << 16));
   atomicExch(p.abort_flag, 1);
   *cta_abort = 1;
 }
@@ -381,14 +392,15 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
   const uint32_t tmem_base = *tmem_slot;
   const int R = p.bw <= 128 ? p.bw : 256;           // weight rows per TMA box
 
-#define RG_WAIT_OR_ABORT(bar, par)                                   \
-  if (!mbar_wait((bar), (par), cta_abort, p.wait_ns)) {                \
-    if (!*cta_abort) raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);   \
-    break;                                                           \
+#define RG_WAIT_OR_ABORT(bar, par)                                          \
+  if (!mbar_wait((bar), (par), cta_abort, p.wait_ns)) {                       \
+    if (!*cta_abort) raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT, wait_site); \
+    break;                                                                  \
   }
 
   if (warp == 0) {
     // =============================== producer ===============================
+    constexpr int wait_site = kSiteProducer;
     // The whole warp runs this loop (all decisions are warp-uniform): all
     // lanes wait on the ring barriers, lane 0 takes the counter, all lanes
     // scan the other units in parallel once the current unit is done, and
@@ -508,6 +520,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
     }
   } else if (warp == 1) {
     // ============================== MMA issuer ==============================
+    constexpr int wait_site = kSiteMma;
     if (lane == 0) {
       // A from shared memory is MN-major (loaded by TMA); A from TMEM is K-major
       constexpr uint32_t idesc = idesc_bf16_f32(kM, N, !C::kATmem, false);
@@ -570,6 +583,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
     }
   } else if (warp < 6) {
     // ============================ conv warpgroup ============================
+    constexpr int wait_site = kSiteConv;
     const int wt = tid - 64;                      // 0 .. 127
     int cur_unit = -1;
     float2 cwq[4][2];                             // conv taps of this thread's channel quad
@@ -646,6 +660,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
     }
   } else if (warp < 6 + 4 * NE) {
     // ========================== epilogue warpgroups ==========================
+    constexpr int wait_site = kSiteEpilogue;
     // Epilogue warpgroup e takes jobs e, e + NE, ...; each of its 4 warps owns
     // one TMEM quadrant (32 channels, one per lane) and works on its own: per
     // job, pass 1, the publication of each channel's aggregate, the carry
@@ -797,7 +812,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
           const bool give_up = *cta_abort || *(volatile const int *)p.abort_flag ||
                                (globaltimer_ns() - t0 > p.wait_ns);
           if (__any_sync(0xffffffffu, give_up)) {
-            if (lane == 0 && !*cta_abort) raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT);
+            if (lane == 0 && !*cta_abort)
+              raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT, kSiteLookBack);
             *cta_abort = 1;
             h_in = 0.f;
             break;

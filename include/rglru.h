@@ -107,9 +107,13 @@ int rglru_fwd_launches(int B, int T, int D, int H, int io, int algo);
  *                                    must not alias conv_state_in
  *   workspace      device scratch of at least rglru_fwd_workspace_bytes(...)
  *   dev_status     device int, or NULL. On a device-side failure a kernel
- *                  stores a nonzero rglru_status there (RGLRU_ERR_TIMEOUT when
- *                  a bounded wait for another block's carry expired; y is then
- *                  incomplete). The library never clears it.
+ *                  stores a nonzero word there (the first failure only): bits
+ *                  0-7 hold the rglru_status (RGLRU_ERR_TIMEOUT when a bounded
+ *                  wait expired; y is then incomplete); for a timeout of the
+ *                  tensor-core forward bits 8-15 name the wait that gave up
+ *                  (1 tile claims and input copies, 2 MMA issue, 3 Conv1D,
+ *                  4 epilogue, 5 a predecessor tile's carry) and bits 16-31
+ *                  the index of the thread block. The library never clears it.
  * Requirements: B, T >= 1; H >= 1; D % H == 0; D % 8 == 0; bw = D / H <= 1024.
  */
 int rglru_fwd(const void *x, const void *conv_w, const void *W_a, const void *b_a,
@@ -271,8 +275,9 @@ int rglru_decode_step_algo(const void *x_t, void *conv_state, int pos, float *h,
  * workspace: device memory of rglru_bwd_workspace_bytes(B, T, D, H, io) bytes,
  * 16-byte aligned, not shared with a concurrent call.
  * Arithmetic is fp32, except that for bf16 I/O with heads 32, 64 or 128 wide
- * the gate contractions z = u W and d z W^T (and U^T dZ for heads 64 or 128
- * wide) run on the tensor cores with bf16 operands and fp32 accumulation; any
+ * and B * T >= 8 the gate contractions z = u W and d z W^T (and U^T dZ for
+ * heads 64 or 128 wide) run on the tensor cores with bf16 operands and fp32
+ * accumulation (below 8 tokens over all rows the operands stay fp32); any
  * head width up to 1024 that divides D. Returns RGLRU_OK, INVALID_ARG (shapes, NULL required
  * pointers, alignment, overlaps), WORKSPACE or CUDA. Nothing in the backward
  * waits on another block, so it has no device-side status.
@@ -305,7 +310,8 @@ int rglru_bwd_launches(int B, int T, int D, int H, int io);
  * layer's, over D channels). Dm >= 8 and a multiple of 8.
  * The three projections are dense GEMMs run by cuBLAS with fp32 accumulation
  * (fp32 I/O: no TF32); x W_in, x W_gate and y are kept in the I/O dtype in
- * the workspace; GeLU and the product are one kernel of this library.
+ * the workspace; GeLU and the product are one memory-bound kernel of this
+ * library over 16-byte vectors.
  * workspace: rglru_block_fwd_workspace_bytes(...) bytes of device memory,
  * 16-byte aligned. out must not overlap x. dev_status as for rglru_fwd.
  * Returns RGLRU_OK, INVALID_ARG, UNSUPPORTED, WORKSPACE or CUDA (including a

@@ -32,7 +32,9 @@ def test_unpublished_tile_times_out_and_context_survives(cuda_device):
     t0 = time.time()
     rg.rglru_fwd(g["x"], *w, algo="tensor", dev_status=status, options=opts)
     torch.cuda.synchronize()
-    assert int(status.item()) == 4                  # RGLRU_ERR_TIMEOUT
+    word = int(status.item())
+    assert word & 0xFF == 4                         # RGLRU_ERR_TIMEOUT
+    assert (word >> 8) & 0xFF == 5                  # ... in the look-back for a carry word
     assert time.time() - t0 < 20.0
     # same context, normal call: correct again
     status.zero_()
