@@ -504,9 +504,10 @@ def run_block(rg, wl, dev, a, pk):
             "roofline": {"bound": "tensor", "achieved": tfs, "peak": pk["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": tfs / pk["bf16_tflops"], "traffic": None,
                          "algorithmic_flops_per_step": flops,
-                         "note": "three dense projections (cuBLAS, bf16, fp32 accumulate) "
-                                 "over the step time, which also holds the layer and the "
-                                 "GeLU gating (HBM-bound, about 45 and 15 us)"}}
+                         "note": "three dense projections (the library's tcgen05 GEMM, bf16 "
+                                 "operands, fp32 accumulation in TMEM; the GeLU gating fused "
+                                 "into the gate projection's epilogue) over the step time, "
+                                 "which also holds the layer (about 42 us)"}}
 
 
 def run_decode(rg, dev, a, pk):

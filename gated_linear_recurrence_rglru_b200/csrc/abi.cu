@@ -269,6 +269,17 @@ int rglru_block_fwd(const void *x, const void *W_in, const void *W_gate, const v
   void *xr = w + L.off_xr, *g = w + L.off_g, *y = w + L.off_y, *fw = w + L.off_fwd;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int M = B * T;
+  if (io == RGLRU_IO_BF16) {
+    // tensor-core GEMMs; the gating runs in the gate projection's epilogue, over y
+    if ((st = launch_gemm_tc(M, D, Dm, x, W_in, nullptr, xr, dev_status, s)) != RGLRU_OK)
+      return st;
+    st = rglru_fwd(xr, conv_w, W_a, b_a, W_x, b_x, Lambda, h0, conv_state_in, y, h_T,
+                   conv_state_out, B, T, D, H, io, fw, workspace_bytes - L.off_fwd, dev_status,
+                   stream);
+    if (st != RGLRU_OK) return st;
+    if ((st = launch_gemm_tc(M, D, Dm, x, W_gate, y, y, dev_status, s)) != RGLRU_OK) return st;
+    return launch_gemm_tc(M, Dm, D, y, W_out, nullptr, out, dev_status, s);
+  }
   if ((st = launch_block_gemm(io, M, D, Dm, x, W_in, xr, s)) != RGLRU_OK) return st;
   if ((st = launch_block_gemm(io, M, D, Dm, x, W_gate, g, s)) != RGLRU_OK) return st;
   st = rglru_fwd(xr, conv_w, W_a, b_a, W_x, b_x, Lambda, h0, conv_state_in, y, h_T,

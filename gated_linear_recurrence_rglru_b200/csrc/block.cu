@@ -9,11 +9,13 @@
 //   output            out = (y * g) W_out                      (B, T, Dm)
 // with GeLU(v) = v Phi(v) = v (1 + erf(v / sqrt 2)) / 2 (the exact form).
 //
-// The three projections are plain dense GEMMs (cuBLAS, fp32 accumulation;
-// fp32 I/O uses the pedantic fp32 compute type, no TF32). The layer is the
-// library's own forward, and y * GeLU(g) is one elementwise kernel over 16-byte
-// vectors, written over y. Intermediates x W_in, x W_gate and y are in the I/O
-// type in the caller's workspace.
+// bf16 I/O: the three projections run on the library's tcgen05 GEMM
+// (gemm_tc.cu), and the gating is fused into the gate projection's epilogue:
+// y * GeLU(x W_gate) is formed where x W_gate leaves the accumulator, written
+// over y. fp32 I/O: the projections run on cuBLAS with the pedantic fp32
+// compute type (no TF32: the exact fp32 reference of the block), and
+// y * GeLU(g) is one elementwise kernel over 16-byte vectors. Intermediates
+// are in the I/O type in the caller's workspace.
 #include <cublas_v2.h>
 
 #include "common.cuh"
@@ -47,10 +49,6 @@ cublasStatus_t gemm_rm(cublasHandle_t h, int io, int M, int N, int K, const void
       io == RGLRU_IO_F32 ? CUBLAS_COMPUTE_32F_PEDANTIC : CUBLAS_COMPUTE_32F;
   return cublasGemmEx(h, CUBLAS_OP_N, CUBLAS_OP_N, N, M, K, &one, B, t, N, A, t, K, &zero, C, t,
                       N, ct, CUBLAS_GEMM_DEFAULT);
-}
-
-__device__ __forceinline__ float gelu_exact(float v) {
-  return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
 }
 
 // y[i] *= GeLU(g[i]) over n elements, 16 bytes per thread per step.

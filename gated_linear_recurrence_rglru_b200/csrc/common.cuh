@@ -47,6 +47,12 @@ __device__ __forceinline__ void decay_and_input(float za, float zx, float u, flo
   beta = sqrtf(-expm1f(2.0f * log_a)) * (i * u);
 }
 
+// GeLU(v) = v Phi(v) = v (1 + erf(v / sqrt 2)) / 2, the exact form (the gating
+// of the recurrent block around the layer).
+__device__ __forceinline__ float gelu_exact(float v) {
+  return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
+}
+
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 

@@ -1,0 +1,315 @@
+// Dense bf16 GEMM on the 5th-generation tensor core (sm_100a) for the recurrent
+// block around the layer: C[M x N] = A[M x K] B[K x N], row-major, fp32
+// accumulation in TMEM, C stored bf16; optionally C = Y * GeLU(A B) with Y
+// (M x N, bf16) read in the epilogue (the block's gating of the layer output
+// by GeLU of the gate projection, fused where the gate projection is
+// produced; the pages describe the block's gated MLP as GeGeLU-like: "Beyond
+// Transformer Architecture: Griffin and Google RecurrentGemma", "Core
+// Components of Griffin", 3. Architecture Design).
+//
+// Tiles of 128 x 256 outputs, persistent CTAs over the tiles (tile i on CTA
+// i mod grid), K in steps of 64. Roles: warp 0 issues the TMA copies of A
+// (K-major, 128-byte swizzle, box 64 x 128) and B (MN-major, 128-byte swizzle,
+// four boxes of 64 columns x 64 rows) into a 4-stage ring; warp 1 issues
+// tcgen05.mma (M = 128, N = 256, K = 16) into one of two TMEM accumulators;
+// two epilogue warpgroups read the accumulator (warp w holds TMEM lanes = rows
+// 32 (w mod 4) .. +31, warpgroup g columns 128 g .. +127), convert, and store
+// 64 contiguous bytes per row and chunk. Every wait is bounded; on expiry the
+// kernel records RGLRU_ERR_TIMEOUT (wait site 6) in the status word, drains
+// what it issued and returns.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_primitives.cuh"
+
+namespace rglru {
+namespace {
+
+using namespace tc;
+
+constexpr int kBM = 128, kBN = 256, kBK = 64, kStages = 4, kNE = 2;
+constexpr int kThreads = 64 + kNE * 128 + 64;        // padded to whole warpgroups
+constexpr int kABytes = kBM * kBK * 2;                // 16 KB
+constexpr int kBBytes = kBK * kBN * 2;                // 32 KB (4 blocks of 64 columns)
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kOffBar = kStages * kStageBytes;
+constexpr int kNumBars = 2 * kStages + 4;             // full, empty, acc_full[2], acc_empty[2]
+constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kSmemBytes = kOffMisc + 64;
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr uint64_t kDrainNs = 200000000ull;
+constexpr int kSiteGemm = 6;
+static_assert(kSmemBytes <= 232448, "shared memory");
+
+struct GemmParams {
+  int M, N, K;
+  int n_mt, n_nt, n_tiles;
+  const __nv_bfloat16 *Y;    // (M, N) or null: C = Y * GeLU(A B)
+  __nv_bfloat16 *C;          // (M, N)
+  int *dev_status;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+               const GemmParams p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  if ((smem_u32(smem_raw) & 1023u) != 0u) {
+    if (threadIdx.x == 0 && p.dev_status) atomicCAS(p.dev_status, 0, RGLRU_ERR_UNSUPPORTED);
+    return;
+  }
+  unsigned char *sm = smem_raw;
+  uint64_t *full = reinterpret_cast<uint64_t *>(sm + kOffBar);
+  uint64_t *empty = full + kStages;
+  uint64_t *acc_full = empty + kStages;
+  uint64_t *acc_empty = acc_full + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kOffMisc);
+  volatile int *cta_abort = reinterpret_cast<volatile int *>(sm + kOffMisc + 4);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int k_steps = (p.K + kBK - 1) / kBK;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kNE * 4);
+    }
+    *cta_abort = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  auto give_up = [&]() {
+    if (!*cta_abort) {
+      if (p.dev_status) atomicCAS(p.dev_status, 0, RGLRU_ERR_TIMEOUT | (kSiteGemm << 8) |
+                                                      (static_cast<int>(blockIdx.x) << 16));
+      *cta_abort = 1;
+    }
+  };
+
+  if (warp == 0) {
+    // ============================ TMA producer ============================
+    if (lane == 0) {
+      int it = 0, last = -1;
+      for (int tile = blockIdx.x; tile < p.n_tiles && !*cta_abort; tile += gridDim.x) {
+        const int m0 = (tile / p.n_nt) * kBM, n0 = (tile % p.n_nt) * kBN;
+        int nb = 0;                                   // B boxes with any column inside N
+        while (nb < kBN / 64 && n0 + nb * 64 < p.N) ++nb;
+        for (int kb = 0; kb < k_steps; ++kb, ++it) {
+          const int s = it % kStages;
+          if (!mbar_wait(&empty[s], ((it / kStages) & 1) ^ 1, cta_abort, kWaitNs)) {
+            give_up();
+            break;
+          }
+          unsigned char *st = sm + s * kStageBytes;
+          mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kABytes + nb * 64 * kBK * 2));
+          tma_load_2d(st, &tmap_a, &full[s], kb * kBK, m0);
+          for (int j = 0; j < nb; ++j)
+            tma_load_2d(st + kABytes + j * (64 * kBK * 2), &tmap_b, &full[s], n0 + j * 64,
+                        kb * kBK);
+          last = it;
+        }
+      }
+      if (*cta_abort)
+        for (int j = last; j >= 0 && j > last - kStages; --j)
+          mbar_wait_drain(&full[j % kStages], (j / kStages) & 1, kDrainNs);
+    }
+  } else if (warp == 1) {
+    // ============================= MMA issuer =============================
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, false, true);
+      int it = 0, lt = 0, last = -1;
+      for (int tile = blockIdx.x; tile < p.n_tiles && !*cta_abort; tile += gridDim.x, ++lt) {
+        const int buf = lt & 1;
+        if (!mbar_wait(&acc_empty[buf], ((lt >> 1) & 1) ^ 1, cta_abort, kWaitNs)) {
+          give_up();
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(buf * kBN);
+        bool ok = true;
+        for (int kb = 0; kb < k_steps; ++kb, ++it) {
+          const int s = it % kStages;
+          if (!mbar_wait(&full[s], (it / kStages) & 1, cta_abort, kWaitNs)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(sm + s * kStageBytes);
+          // A: K-major rows of 128 B, 8-row groups 1024 B apart; a K step of 16
+          // moves 32 B along the row. B: MN-major, 64-column blocks of 64 K rows
+          // (8 KB apart), 8-row groups 1024 B apart; a K step moves 16 rows.
+          const uint64_t ad = sdesc_sw128(sa, 16, 1024);
+          const uint64_t bd = sdesc_sw128(sa + kABytes, 64 * kBK * 2, 1024);
+#pragma unroll
+          for (int ks = 0; ks < kBK / 16; ++ks)
+            mma_bf16(d, ad + static_cast<uint64_t>((ks * 32) >> 4),
+                     bd + static_cast<uint64_t>((ks * 16 * 128) >> 4), idesc,
+                     (kb > 0 || ks > 0) ? 1u : 0u);
+          mma_commit(&empty[s]);
+          last = it;
+        }
+        if (!ok) break;
+        mma_commit(&acc_full[buf]);
+      }
+      if (*cta_abort && last >= 0)
+        mbar_wait_drain(&empty[last % kStages], (last / kStages) & 1, kDrainNs);
+    }
+  } else if (warp < 2 + 4 * kNE) {
+    // ============================== epilogue ==============================
+    const int g = (warp - 2) >> 2;                  // column half of the tile
+    const int qd = warp & 3;                        // TMEM lane quadrant = row block
+    int lt = 0;
+    for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++lt) {
+      const int buf = lt & 1;
+      if (!mbar_wait(&acc_full[buf], (lt >> 1) & 1, cta_abort, kWaitNs)) {
+        give_up();
+        break;
+      }
+      tc_fence_after();
+      const int m0 = (tile / p.n_nt) * kBM, n0 = (tile % p.n_nt) * kBN;
+      const int row = m0 + qd * 32 + lane;
+      const uint32_t tl = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) +
+                          static_cast<uint32_t>(buf * kBN + g * 128);
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        const int c0 = n0 + g * 128 + ch * 32;     // first column of this chunk
+        float v[32];
+        __syncwarp();                               // tcgen05.ld is warp-collective
+        tmem_ld32(tl + static_cast<uint32_t>(ch * 32), v);
+        tmem_wait_ld();
+        if (row < p.M && c0 < p.N) {
+          const size_t off = static_cast<size_t>(row) * p.N + c0;
+          const int nq = min(4, (p.N - c0) / 8);   // whole 8-column vectors in range
+          if (p.Y != nullptr) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (q >= nq) break;
+              const uint4 yv = *reinterpret_cast<const uint4 *>(p.Y + off + q * 8);
+              const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float y0 = __uint_as_float(yw[e] << 16);
+                const float y1 = __uint_as_float(yw[e] & 0xFFFF0000u);
+                v[q * 8 + 2 * e] = y0 * gelu_exact(v[q * 8 + 2 * e]);
+                v[q * 8 + 2 * e + 1] = y1 * gelu_exact(v[q * 8 + 2 * e + 1]);
+              }
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (q >= nq) break;
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 h =
+                  __floats2bfloat162_rn(v[q * 8 + 2 * e], v[q * 8 + 2 * e + 1]);
+              w[e] = *reinterpret_cast<const uint32_t *>(&h);
+            }
+            *reinterpret_cast<uint4 *>(p.C + off + q * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, 512);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 gemm_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+}  // namespace
+
+bool gemm_tc_supported(int M, int N, int K) {
+  // TMA row strides must be multiples of 16 bytes; the epilogue stores 8-column vectors
+  return M >= 1 && N >= 8 && K >= 8 && N % 8 == 0 && K % 8 == 0;
+}
+
+int launch_gemm_tc(int M, int N, int K, const void *A, const void *B, const void *Y, void *C,
+                   int *dev_status, cudaStream_t st) {
+  if (!gemm_tc_supported(M, N, K)) return RGLRU_ERR_UNSUPPORTED;
+  auto enc = gemm_encode_fn();
+  if (enc == nullptr) return RGLRU_ERR_CUDA;
+  CUtensorMap ta, tb;
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    cuuint32_t box[2] = {kBK, kBM};
+    cuuint32_t es[2] = {1, 1};
+    if (enc(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(A), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return RGLRU_ERR_CUDA;
+  }
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(K)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
+    cuuint32_t box[2] = {64, kBK};
+    cuuint32_t es[2] = {1, 1};
+    if (enc(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(B), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return RGLRU_ERR_CUDA;
+  }
+  GemmParams p;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.n_mt = ceil_div(M, kBM);
+  p.n_nt = ceil_div(N, kBN);
+  p.n_tiles = p.n_mt * p.n_nt;
+  p.Y = static_cast<const __nv_bfloat16 *>(Y);
+  p.C = static_cast<__nv_bfloat16 *>(C);
+  p.dev_status = dev_status;
+  constexpr int kMaxDev = 64;
+  static std::atomic<int> sms_of[kMaxDev];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RGLRU_ERR_CUDA;
+  int sms = dev < kMaxDev ? sms_of[dev].load(std::memory_order_acquire) : 0;
+  if (sms == 0) {
+    if (cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes) != cudaSuccess)
+      return RGLRU_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return RGLRU_ERR_CUDA;
+    if (dev < kMaxDev) sms_of[dev].store(sms, std::memory_order_release);
+  }
+  const int grid = p.n_tiles < sms ? p.n_tiles : sms;
+  gemm_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(ta, tb, p);
+  return cudaGetLastError() == cudaSuccess ? RGLRU_OK : RGLRU_ERR_CUDA;
+}
+
+}  // namespace rglru

@@ -67,6 +67,11 @@ BlockLayout block_layout(int B, int T, int D, int io, size_t fwd_ws);
 int launch_block_gemm(int io, int M, int N, int K, const void *A, const void *B, void *C,
                       cudaStream_t st);
 cudaError_t launch_gelu_gate(int io, void *y, const void *g, size_t n, cudaStream_t st);
+// Row-major bf16 C[M x N] = A[M x K] B[K x N] on the tensor core (gemm_tc.cu);
+// with Y (M x N bf16, may alias C) non-null, C = Y * GeLU(A B). An RGLRU_* status.
+bool gemm_tc_supported(int M, int N, int K);
+int launch_gemm_tc(int M, int N, int K, const void *A, const void *B, const void *Y, void *C,
+                   int *dev_status, cudaStream_t st);
 cudaError_t launch_fwd_generic(const FwdArgs &p, int io, void *ws, cudaStream_t st);
 cudaError_t launch_decode_generic(const DecArgs &p, int io, cudaStream_t st);
 

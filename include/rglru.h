@@ -308,10 +308,14 @@ int rglru_bwd_launches(int B, int T, int D, int H, int io);
  * W_out (D, Dm), out (B, T, Dm); the layer's parameters, h0, conv_state_in,
  * h_T and conv_state_out as for rglru_fwd (the state and conv history are the
  * layer's, over D channels). Dm >= 8 and a multiple of 8.
- * The three projections are dense GEMMs run by cuBLAS with fp32 accumulation
- * (fp32 I/O: no TF32); x W_in, x W_gate and y are kept in the I/O dtype in
- * the workspace; GeLU and the product are one memory-bound kernel of this
- * library over 16-byte vectors.
+ * bf16 I/O: the three projections run on the library's tcgen05 GEMM (bf16
+ * operands, fp32 accumulation in TMEM), and GeLU and the product are fused
+ * into the gate projection's epilogue (y * GeLU(x W_gate) is formed where
+ * x W_gate leaves the accumulator and written over y). fp32 I/O: the
+ * projections run on cuBLAS with the pedantic fp32 compute type (no TF32),
+ * and GeLU and the product are one memory-bound kernel of this library.
+ * x W_in and y are kept in the I/O dtype in the workspace (and x W_gate for
+ * fp32 I/O).
  * workspace: rglru_block_fwd_workspace_bytes(...) bytes of device memory,
  * 16-byte aligned. out must not overlap x. dev_status as for rglru_fwd.
  * Returns RGLRU_OK, INVALID_ARG, UNSUPPORTED, WORKSPACE or CUDA (including a
