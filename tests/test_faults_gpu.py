@@ -46,6 +46,32 @@ def test_unpublished_tile_times_out_and_context_survives(cuda_device):
     assert max_rel_err(y.float().cpu().numpy(), yo) <= 2e-2
 
 
+def test_unpublished_tile_times_out_with_wide_heads(cuda_device):
+    """The same with 256-wide heads (32-token tiles, gate weights in TMEM, two
+    units per head): the stalled tile's look-back names the failure and the
+    next call is correct."""
+    wl = WORKLOADS["hawk_block"].with_shape(B=1, T=32 * 12, D=512, H=2, seed=73)
+    t = generate(wl)
+    g = {k: (v.to(cuda_device) if v is not None else None) for k, v in t.items()}
+    w = [g[k] for k in ("conv_w", "W_a", "b_a", "W_x", "b_x", "Lambda")]
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    opts = FwdOptions(wait_limit_ns=50_000_000, fault_unpublished_tile=4)
+    t0 = time.time()
+    rg.rglru_fwd(g["x"], *w, algo="tensor", dev_status=status, options=opts)
+    torch.cuda.synchronize()
+    word = int(status.item())
+    assert word & 0xFF == 4
+    assert (word >> 8) & 0xFF == 5
+    assert time.time() - t0 < 20.0
+    status.zero_()
+    y, _, _ = rg.rglru_fwd(g["x"], *w, algo="tensor", dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    yo, _, _ = orc.rglru_fwd(t["x"], t["conv_w"], t["W_a"], t["b_a"], t["W_x"], t["b_x"],
+                             t["Lambda"])
+    assert max_rel_err(y.float().cpu().numpy(), yo) <= 2e-2
+
+
 def test_too_short_wait_limit_is_refused(cuda_device):
     _, g = _inputs(cuda_device)
     w = [g[k] for k in ("conv_w", "W_a", "b_a", "W_x", "b_x", "Lambda")]

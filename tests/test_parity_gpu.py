@@ -76,6 +76,10 @@ SMALL = [
     WORKLOADS["hawk_block"].with_shape(B=2, T=1, D=128, H=2, h0_var=1.0, seed=38),
     WORKLOADS["hawk_block"].with_shape(B=2, T=64, D=256, H=4, seed=39),
     WORKLOADS["hawk_block"].with_shape(B=2, T=65, D=256, H=2, h0_var=1.0, seed=40),
+    # 256-wide heads: a sequence shorter than the Conv1D history; one token past
+    # a 32-token tile with several rows and heads
+    WORKLOADS["hawk_block"].with_shape(B=2, T=2, D=512, H=2, h0_var=1.0, seed=43),
+    WORKLOADS["hawk_block"].with_shape(B=3, T=33, D=1024, H=4, bias_std=0.5, seed=44),
 ]
 
 
@@ -90,6 +94,15 @@ def test_fwd_small(cuda_device, algo, idx):
 def test_fwd_with_conv_state_in(cuda_device, algo, io):
     wl = WORKLOADS["hawk_block"].with_shape(B=2, T=70, D=256, H=4, io=io, h0_var=0.3, seed=41)
     check_fwd(wl, algo, cuda_device, with_csi=True)
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("T", [2, 70])
+def test_fwd_with_conv_state_in_wide_heads(cuda_device, algo, T):
+    """conv_state_in / conv_state_out with 256-wide heads, where a unit's
+    Conv1D covers the head's 256 channels and writes its own 128 to the state."""
+    wl = WORKLOADS["hawk_block"].with_shape(B=2, T=T, D=512, H=2, h0_var=0.3, seed=45)
+    check_fwd(wl, algo, cuda_device, with_csi=True, csi_seed=12)
 
 
 @pytest.mark.parametrize("algo", ALGOS)
