@@ -47,6 +47,7 @@ constexpr uint64_t kDrainNs = 200000000ull;
 
 struct DecTcParams {
   const __nv_bfloat16 *conv_w, *b_a, *b_x;
+  const __nv_bfloat16 *W_a, *W_x;            // (H, bw, bw): read directly when A is in TMEM
   const float *Lambda;
   __nv_bfloat16 *ring;
   const __nv_bfloat16 *x_t;
@@ -61,7 +62,11 @@ template <int K, int N>
 struct DCfg {
   static constexpr int NE = 2;                     // epilogue warpgroups
   static constexpr int kThreads = 64 + 128 + NE * 128;
-  static constexpr int kABytes = K * 256;          // one gate: 2 M-blocks x K rows x 128 B
+  // Gate weights (the MMA's A operand): in shared memory for K = 128 (TMA),
+  // in TMEM for K = 256, where the tensor core would otherwise re-read 128 KB
+  // of shared memory for every 16-row job (written by the conv warpgroup)
+  static constexpr bool kATmem = (K == 256);
+  static constexpr int kABytes = kATmem ? 0 : K * 256;   // one gate: 2 M-blocks x K rows x 128 B
   static constexpr int kInBytes = N * K * 2;       // one input tile: N rows x K channels, bf16
   static constexpr int kXBytes = 4 * kInBytes;     // x_t and ring slots pos, pos+1, pos+2 (mod 3)
   static constexpr int kNX = 2;                    // input slots
@@ -75,14 +80,17 @@ struct DCfg {
   static constexpr int kOffU = kOffB + kNS * kBBytes;
   static constexpr int kOffBar = kOffU + kNS * kUBytes;
   // job_full[JQ], job_empty[JQ], x_full[NX], x_empty[NX], w_full, w_free,
-  // b_full[NS], b_empty[NS], u_empty[NS], acc_full[NT], tmem_empty[NT]
-  static constexpr int kNumBars = 2 * kJQ + 2 * kNX + 2 + 3 * kNS + 2 * kNT;
+  // b_full[NS], b_empty[NS], u_empty[NS], acc_full[NT], tmem_empty[NT], a_ready
+  static constexpr int kNumBars = 2 * kJQ + 2 * kNX + 2 + 3 * kNS + 2 * kNT + 1;
   static constexpr int kOffJobs = (kOffBar + kNumBars * 8 + 15) / 16 * 16;
   static constexpr int kOffMisc = kOffJobs + kJQ * 16;
   // the dynamic shared memory base is declared 1024-byte aligned (checked)
   static constexpr int kSmemBytes = kOffMisc + 64;
   static constexpr int kSlotCols = 2 * N;
-  static constexpr int kTmemCols = kNT * kSlotCols <= 128 ? 128 : (kNT * kSlotCols <= 256 ? 256 : 512);
+  static constexpr int kACol = kNT * kSlotCols;             // TMEM A: gate a, then gate x
+  static constexpr int kUsedCols = kACol + (kATmem ? K : 0);
+  static constexpr int kTmemCols = kUsedCols <= 128 ? 128 : (kUsedCols <= 256 ? 256 : 512);
+  static_assert(kUsedCols <= 512, "TMEM allocation");
   static constexpr int NQ = K / 4;                 // conv: channel quads
   static constexpr int SEG = N * NQ / 128;         // conv: rows per thread
   static_assert(kSmemBytes <= 232448, "shared memory");
@@ -188,6 +196,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
   uint64_t *u_empty = b_empty + NS;
   uint64_t *acc_full = u_empty + NS;
   uint64_t *tmem_empty = acc_full + NT;
+  uint64_t *a_ready = tmem_empty + NT;              // conv warpgroup wrote TMEM weights -> MMA
   int4 *jobs = reinterpret_cast<int4 *>(sm + C::kOffJobs);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + C::kOffMisc);
   volatile int *cta_abort = reinterpret_cast<volatile int *>(sm + C::kOffMisc + 4);
@@ -218,6 +227,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
       mbar_init(&acc_full[i], 1);
       mbar_init(&tmem_empty[i], 4);
     }
+    mbar_init(a_ready, 4);                          // 4 conv warps
     *cta_abort = 0;
     fence_mbar_init();
     prefetch_tmap(&tmap_wa);
@@ -267,7 +277,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
         jobs[js] = make_int4(unit, tile, reload, 0);
         mbar_arrive(&job_full[js]);
         const int cg = unit;
-        if (reload) {
+        if (reload && !C::kATmem) {
           if (i > 0) {
             RG_WAIT_OR_ABORT(w_free, wfree_phase);
             wfree_phase ^= 1;
@@ -288,8 +298,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
                             (cg >> 1) * 256);
             }
           }
-          w_unit = unit;
         }
+        if (reload) w_unit = unit;
         // the job's inputs: x_t rows, then ring slots pos % 3 (x_{t-3}),
         // (pos + 1) % 3 (x_{t-2}), (pos + 2) % 3 (x_{t-1}); rows past B read as zeros
         const int xb = i % NX;
@@ -311,9 +321,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
   } else if (warp == 1) {
     // ============================== MMA issuer ==============================
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kM, N, true, false);
+      // A from shared memory is MN-major (loaded by TMA); A from TMEM is K-major
+      constexpr uint32_t idesc = idesc_bf16_f32(kM, N, !C::kATmem, false);
       const uint64_t ada0 = sdesc_sw128(smem_u32(sA), K * 128, 1024);
       const uint64_t adx0 = sdesc_sw128(smem_u32(sA + C::kABytes), K * 128, 1024);
+      const uint32_t ta_a = tmem_base + static_cast<uint32_t>(C::kACol);
+      const uint32_t ta_x = ta_a + static_cast<uint32_t>(K / 2);
       uint32_t w_phase = 0;
       int last_commit = -1;
       for (int i = 0;; ++i) {
@@ -322,12 +335,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
         const int4 job = jobs[js];
         if (job.x < 0) break;
         if (job.z) {
-          if (last_commit >= 0) {
-            const int lc = last_commit;
-            RG_WAIT_OR_ABORT(&acc_full[lc % NT], (lc / NT) & 1);
-            mbar_arrive(w_free);
+          if (C::kATmem) {
+            // the conv warpgroup has written this unit's weights into TMEM
+            RG_WAIT_OR_ABORT(a_ready, w_phase);
+          } else {
+            if (last_commit >= 0) {
+              const int lc = last_commit;
+              RG_WAIT_OR_ABORT(&acc_full[lc % NT], (lc / NT) & 1);
+              mbar_arrive(w_free);
+            }
+            RG_WAIT_OR_ABORT(w_full, w_phase);
           }
-          RG_WAIT_OR_ABORT(w_full, w_phase);
           w_phase ^= 1;
         }
         const int s = i % NS, ts = i % NT;
@@ -344,9 +362,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
 #pragma unroll
         for (int ks = 0; ks < K / 16; ++ks) {
           const uint64_t bd = bd0 + static_cast<uint64_t>(((ks >> 2) * (N * 128) + (ks & 3) * 32) >> 4);
-          const uint64_t astep = static_cast<uint64_t>((ks * 16 * 128) >> 4);
-          mma_bf16(d_a, ada0 + astep, bd, idesc, ks > 0 ? 1u : 0u);
-          mma_bf16(d_x, adx0 + astep, bd, idesc, ks > 0 ? 1u : 0u);
+          if (C::kATmem) {
+            mma_bf16_ts(d_a, ta_a + static_cast<uint32_t>(ks * 8), bd, idesc, ks > 0 ? 1u : 0u);
+            mma_bf16_ts(d_x, ta_x + static_cast<uint32_t>(ks * 8), bd, idesc, ks > 0 ? 1u : 0u);
+          } else {
+            const uint64_t astep = static_cast<uint64_t>((ks * 16 * 128) >> 4);
+            mma_bf16(d_a, ada0 + astep, bd, idesc, ks > 0 ? 1u : 0u);
+            mma_bf16(d_x, adx0 + astep, bd, idesc, ks > 0 ? 1u : 0u);
+          }
         }
         mma_commit(&acc_full[ts]);
         mma_commit(&b_empty[s]);
@@ -378,6 +401,40 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
           const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(p.conv_w + tap * p.D + chq));
           cwq[tap][0] = bf2_to_f2(raw.x);
           cwq[tap][1] = bf2_to_f2(raw.y);
+        }
+        if (C::kATmem) {
+          // This unit's gate weights into TMEM (the A operand): lane m (output
+          // channel cg*128 + m) holds W[h][k][j] for k = 0..K-1, two per column.
+          // Every MMA of earlier jobs has read the old weights once the
+          // accumulator of job i-1 is complete (MMAs complete in issue order).
+          if (i > 0) RG_WAIT_OR_ABORT(&acc_full[(i - 1) % NT], ((i - 1) / NT) & 1);
+          const int qd = warp & 3;                  // this warp's TMEM lane quadrant
+          const int cout = cg * kM + qd * 32 + lane;
+          const int hh = cout / p.bw, jj = cout % p.bw;
+          const uint32_t tq = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) +
+                              static_cast<uint32_t>(C::kACol);
+#pragma unroll 1
+          for (int g = 0; g < 2; ++g) {
+            const unsigned short *Wg =
+                reinterpret_cast<const unsigned short *>(g == 0 ? p.W_a : p.W_x) +
+                static_cast<size_t>(hh) * p.bw * p.bw + jj;
+#pragma unroll 1
+            for (int cc = 0; cc < K / 64; ++cc) {
+              uint32_t v[32];
+#pragma unroll
+              for (int q = 0; q < 32; ++q) {
+                const int k = cc * 64 + 2 * q;
+                const uint32_t lo = __ldg(Wg + static_cast<size_t>(k) * p.bw);
+                const uint32_t hi = __ldg(Wg + static_cast<size_t>(k + 1) * p.bw);
+                v[q] = lo | (hi << 16);
+              }
+              tmem_st32u(tq + static_cast<uint32_t>(g * (K / 2) + cc * 32), v);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(a_ready);
         }
       }
       const int s = i % NS, xb = i % NX;
@@ -559,6 +616,8 @@ cudaError_t launch_dec_t(const DecArgs &a, cudaStream_t st) {
   p.conv_w = static_cast<const __nv_bfloat16 *>(a.conv_w);
   p.b_a = static_cast<const __nv_bfloat16 *>(a.b_a);
   p.b_x = static_cast<const __nv_bfloat16 *>(a.b_x);
+  p.W_a = static_cast<const __nv_bfloat16 *>(a.W_a);
+  p.W_x = static_cast<const __nv_bfloat16 *>(a.W_x);
   p.Lambda = a.Lambda;
   p.ring = static_cast<__nv_bfloat16 *>(a.conv_state);
   p.h = a.h;
