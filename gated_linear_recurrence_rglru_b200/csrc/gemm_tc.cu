@@ -7,16 +7,25 @@
 // Transformer Architecture: Griffin and Google RecurrentGemma", "Core
 // Components of Griffin", 3. Architecture Design).
 //
-// Tiles of 128 x 256 outputs, persistent CTAs over the tiles (tile i on CTA
-// i mod grid), K in steps of 64. Roles: warp 0 issues the TMA copies of A
-// (K-major, 128-byte swizzle, box 64 x 128) and B (MN-major, 128-byte swizzle,
-// four boxes of 64 columns x 64 rows) into a 4-stage ring; warp 1 issues
-// tcgen05.mma (M = 128, N = 256, K = 16) into one of two TMEM accumulators;
-// two epilogue warpgroups read the accumulator (warp w holds TMEM lanes = rows
-// 32 (w mod 4) .. +31, warpgroup g columns 128 g .. +127), convert, and store
-// 64 contiguous bytes per row and chunk. Every wait is bounded; on expiry the
-// kernel records RGLRU_ERR_TIMEOUT (wait site 6) in the status word, drains
-// what it issued and returns.
+// Two kernels, the same roles: warp 0 issues the TMA copies of A (K-major,
+// 128-byte swizzle, boxes of 64 K x 128 rows) and B (MN-major, 128-byte
+// swizzle, boxes of 64 columns x 64 K rows) into a ring of stages; warp 1
+// issues tcgen05.mma (K = 16 per instruction) into one of two TMEM
+// accumulators; two epilogue warpgroups read the accumulator (warp w holds
+// TMEM lanes = rows 32 (w mod 4) .. +31, warpgroup g columns 128 g .. +127),
+// convert, and store 64 contiguous bytes per row and chunk. Persistent over
+// the tiles, K in steps of 64.
+//  - gemm_tc2_kernel, when M and N are multiples of 256: clusters of two CTAs
+//    share 256 x 256 tiles through the pair MMA (tcgen05 cta_group::2, M =
+//    256): each CTA loads 128 rows of A and 128 columns of B per stage, both
+//    CTAs' loads complete on the even CTA's barrier, whose MMA thread issues
+//    for the pair and commits stage and accumulator releases to both CTAs;
+//    each CTA's epilogue stores its 128 rows. Per CTA and stage 32 KB, six
+//    stages; a tile's operands cross L2 once per pair, a third less traffic
+//    per flop than 128 x 256 tiles on one CTA.
+//  - gemm_tc_kernel otherwise: 128 x 256 tiles on one CTA, four stages.
+// Every wait is bounded; on expiry the kernel records RGLRU_ERR_TIMEOUT (wait
+// site 6) in the status word, drains what it issued and returns.
 #include <cudaTypedefs.h>
 
 #include <atomic>
@@ -31,8 +40,17 @@ namespace {
 
 using namespace tc;
 
-constexpr int kBM = 128, kBN = 256, kBK = 64, kStages = 4, kNE = 2;
-constexpr int kThreads = 64 + kNE * 128 + 64;        // padded to whole warpgroups
+#ifndef RGLRU_GEMM_NE
+#define RGLRU_GEMM_NE 2
+#endif
+constexpr int kBM = 128, kBN = 256, kBK = 64, kStages = 4;
+constexpr int kNE = RGLRU_GEMM_NE;                    // epilogue warpgroups (256 / kNE columns each)
+constexpr int kEpiCols = 256 / kNE;
+#ifndef RGLRU_GEMM_GELU
+#define RGLRU_GEMM_GELU gelu_as7126
+#endif
+// warps 0 (TMA) and 1 (MMA), the epilogue warpgroups; padded to whole warpgroups
+constexpr int kThreads = (64 + kNE * 128 + 127) / 128 * 128;
 constexpr int kABytes = kBM * kBK * 2;                // 16 KB
 constexpr int kBBytes = kBK * kBN * 2;                // 32 KB (4 blocks of 64 columns)
 constexpr int kStageBytes = kABytes + kBBytes;
@@ -52,6 +70,68 @@ struct GemmParams {
   __nv_bfloat16 *C;          // (M, N)
   int *dev_status;
 };
+
+// Y operand of one warp's epilogue: this lane's row, kEpiCols columns from
+// c_first, loaded as 8-column vectors before the accumulator is ready (the
+// loads then overlap the tile's MMAs instead of the epilogue's arithmetic).
+struct EpiY {
+  uint4 v[kEpiCols / 8];
+};
+
+__device__ __forceinline__ void epilogue_load_y(const GemmParams &p, int row, int c_first,
+                                                EpiY &y) {
+  if (p.Y == nullptr || row >= p.M) return;
+  const __nv_bfloat16 *yr = p.Y + static_cast<size_t>(row) * p.N;
+#pragma unroll
+  for (int q = 0; q < kEpiCols / 8; ++q)
+    if (c_first + q * 8 < p.N) y.v[q] = *reinterpret_cast<const uint4 *>(yr + c_first + q * 8);
+}
+
+// Epilogue of one warp: kEpiCols accumulator columns of this lane's row (TMEM
+// address tl: the warp's lane quadrant, the first column), converted to bf16
+// (times Y * GeLU when Y is given, from y) and stored from column c_first on,
+// in chunks of 32 columns (64 contiguous bytes per row and chunk).
+__device__ __forceinline__ void epilogue_rows(const GemmParams &p, uint32_t tl, int row,
+                                              int c_first, const EpiY &y) {
+#pragma unroll
+  for (int ch = 0; ch < kEpiCols / 32; ++ch) {
+    const int c0 = c_first + ch * 32;               // first column of this chunk
+    float v[32];
+    __syncwarp();                                   // tcgen05.ld is warp-collective
+    tmem_ld32(tl + static_cast<uint32_t>(ch * 32), v);
+    tmem_wait_ld();
+    if (row < p.M && c0 < p.N) {
+      const size_t off = static_cast<size_t>(row) * p.N + c0;
+      const int nq = min(4, (p.N - c0) / 8);       // whole 8-column vectors in range
+      if (p.Y != nullptr) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (q >= nq) break;
+          const uint4 yv = y.v[ch * 4 + q];
+          const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float y0 = __uint_as_float(yw[e] << 16);
+            const float y1 = __uint_as_float(yw[e] & 0xFFFF0000u);
+            v[q * 8 + 2 * e] = y0 * RGLRU_GEMM_GELU(v[q * 8 + 2 * e]);
+            v[q * 8 + 2 * e + 1] = y1 * RGLRU_GEMM_GELU(v[q * 8 + 2 * e + 1]);
+          }
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (q >= nq) break;
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat162 h = __floats2bfloat162_rn(v[q * 8 + 2 * e], v[q * 8 + 2 * e + 1]);
+          w[e] = *reinterpret_cast<const uint32_t *>(&h);
+        }
+        *reinterpret_cast<uint4 *>(p.C + off + q * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  }
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
@@ -173,59 +253,23 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
     }
   } else if (warp < 2 + 4 * kNE) {
     // ============================== epilogue ==============================
-    const int g = (warp - 2) >> 2;                  // column half of the tile
+    const int g = (warp - 2) >> 2;                  // column group of the tile
     const int qd = warp & 3;                        // TMEM lane quadrant = row block
     int lt = 0;
     for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++lt) {
       const int buf = lt & 1;
+      const int m0 = (tile / p.n_nt) * kBM, n0 = (tile % p.n_nt) * kBN;
+      const int row = m0 + qd * 32 + lane;
+      EpiY y;
+      epilogue_load_y(p, row, n0 + g * kEpiCols, y);
       if (!mbar_wait(&acc_full[buf], (lt >> 1) & 1, cta_abort, kWaitNs)) {
         give_up();
         break;
       }
       tc_fence_after();
-      const int m0 = (tile / p.n_nt) * kBM, n0 = (tile % p.n_nt) * kBN;
-      const int row = m0 + qd * 32 + lane;
       const uint32_t tl = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) +
-                          static_cast<uint32_t>(buf * kBN + g * 128);
-#pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        const int c0 = n0 + g * 128 + ch * 32;     // first column of this chunk
-        float v[32];
-        __syncwarp();                               // tcgen05.ld is warp-collective
-        tmem_ld32(tl + static_cast<uint32_t>(ch * 32), v);
-        tmem_wait_ld();
-        if (row < p.M && c0 < p.N) {
-          const size_t off = static_cast<size_t>(row) * p.N + c0;
-          const int nq = min(4, (p.N - c0) / 8);   // whole 8-column vectors in range
-          if (p.Y != nullptr) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              if (q >= nq) break;
-              const uint4 yv = *reinterpret_cast<const uint4 *>(p.Y + off + q * 8);
-              const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float y0 = __uint_as_float(yw[e] << 16);
-                const float y1 = __uint_as_float(yw[e] & 0xFFFF0000u);
-                v[q * 8 + 2 * e] = y0 * gelu_exact(v[q * 8 + 2 * e]);
-                v[q * 8 + 2 * e + 1] = y1 * gelu_exact(v[q * 8 + 2 * e + 1]);
-              }
-            }
-          }
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (q >= nq) break;
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const __nv_bfloat162 h =
-                  __floats2bfloat162_rn(v[q * 8 + 2 * e], v[q * 8 + 2 * e + 1]);
-              w[e] = *reinterpret_cast<const uint32_t *>(&h);
-            }
-            *reinterpret_cast<uint4 *>(p.C + off + q * 8) = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        }
-      }
+                          static_cast<uint32_t>(buf * kBN + g * kEpiCols);
+      epilogue_rows(p, tl, row, n0 + g * kEpiCols, y);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
@@ -235,6 +279,180 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, 512);
+}
+
+// ------------------------------------------------------------ CTA pairs ----
+
+constexpr int kPM = 128;                              // rows of A and D per CTA
+constexpr int kPN = 128;                              // columns of B per CTA (N = 256 per pair)
+constexpr int kPStages = 6;
+constexpr int kPABytes = kPM * kBK * 2;               // 16 KB
+constexpr int kPBBytes = kBK * kPN * 2;               // 16 KB (2 blocks of 64 columns)
+constexpr int kPStageBytes = kPABytes + kPBBytes;
+constexpr int kPOffBar = kPStages * kPStageBytes;
+constexpr int kPNumBars = 2 * kPStages + 4;           // full, empty, acc_full[2], acc_empty[2]
+constexpr int kPOffMisc = kPOffBar + kPNumBars * 8;
+constexpr int kPSmemBytes = kPOffMisc + 64;
+static_assert(kPSmemBytes <= 232448, "shared memory");
+
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                const GemmParams p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // the alignment is the same in both CTAs, so both return here or neither does
+  if ((smem_u32(smem_raw) & 1023u) != 0u) {
+    if (threadIdx.x == 0 && p.dev_status) atomicCAS(p.dev_status, 0, RGLRU_ERR_UNSUPPORTED);
+    return;
+  }
+  unsigned char *sm = smem_raw;
+  uint64_t *full = reinterpret_cast<uint64_t *>(sm + kPOffBar);
+  uint64_t *empty = full + kPStages;
+  uint64_t *acc_full = empty + kPStages;
+  uint64_t *acc_empty = acc_full + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kPOffMisc);
+  volatile int *cta_abort = reinterpret_cast<volatile int *>(sm + kPOffMisc + 4);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();            // 0: issues the pair's MMAs
+  const int cid = static_cast<int>(blockIdx.x) >> 1, n_clusters = static_cast<int>(gridDim.x) >> 1;
+  const int k_steps = p.K / kBK;
+  const uint32_t peer_abort = mapa_shared(smem_u32(const_cast<int *>(cta_abort)), rank ^ 1u);
+
+  if (tid == 0) {
+    for (int s = 0; s < kPStages; ++s) {
+      mbar_init(&full[s], 1);                         // the even CTA's expect_tx (both CTAs' bytes)
+      mbar_init(&empty[s], 1);                        // the pair MMA's commit
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 2 * kNE * 4);          // epilogue warps of both CTAs
+    }
+    *cta_abort = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();                                     // barriers of both CTAs initialised
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  auto give_up = [&]() {
+    if (!*cta_abort) {
+      if (p.dev_status) atomicCAS(p.dev_status, 0, RGLRU_ERR_TIMEOUT | (kSiteGemm << 8) |
+                                                      (static_cast<int>(blockIdx.x) << 16));
+      *cta_abort = 1;
+      st_cluster_u32(peer_abort, 1u);                 // the partner stops at its next wait
+    }
+  };
+
+  if (warp == 0) {
+    // ============================ TMA producer ============================
+    if (lane == 0) {
+      const uint32_t full0 = mapa_shared(smem_u32(full), 0u);   // the even CTA's barriers
+      int it = 0;
+      for (int tile = cid; tile < p.n_tiles && !*cta_abort; tile += n_clusters) {
+        const int m0 = (tile / p.n_nt) * (2 * kPM) + static_cast<int>(rank) * kPM;
+        const int n0 = (tile % p.n_nt) * (2 * kPN) + static_cast<int>(rank) * kPN;
+        for (int kb = 0; kb < k_steps; ++kb, ++it) {
+          const int s = it % kPStages;
+          if (!mbar_wait(&empty[s], ((it / kPStages) & 1) ^ 1, cta_abort, kWaitNs)) {
+            give_up();
+            break;
+          }
+          unsigned char *st = sm + s * kPStageBytes;
+          if (rank == 0u) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(2 * kPStageBytes));
+          const uint32_t fb = full0 + static_cast<uint32_t>(s * 8);
+          tma_load_2d_pair(st, &tmap_a, fb, kb * kBK, m0);
+          for (int j = 0; j < kPN / 64; ++j)
+            tma_load_2d_pair(st + kPABytes + j * (64 * kBK * 2), &tmap_b, fb, n0 + j * 64, kb * kBK);
+        }
+      }
+      // the pair MMA's last stage releases arrive here by multicast: let them
+      // land before this CTA can exit (bounded)
+      for (int j = it - 1; j >= 0 && j >= it - kPStages; --j)
+        mbar_wait_drain(&empty[j % kPStages], ((j / kPStages) & 1), kDrainNs);
+    }
+  } else if (warp == 1) {
+    // ============================= MMA issuer =============================
+    if (lane == 0 && rank == 0u) {
+      constexpr uint32_t idesc = idesc_bf16_f32(2 * kPM, 2 * kPN, false, true);
+      int it = 0, lt = 0;
+      for (int tile = cid; tile < p.n_tiles && !*cta_abort; tile += n_clusters, ++lt) {
+        const int buf = lt & 1;
+        if (!mbar_wait(&acc_empty[buf], ((lt >> 1) & 1) ^ 1, cta_abort, kWaitNs)) {
+          give_up();
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(buf * 2 * kPN);
+        bool ok = true;
+        for (int kb = 0; kb < k_steps; ++kb, ++it) {
+          const int s = it % kPStages;
+          if (!mbar_wait(&full[s], (it / kPStages) & 1, cta_abort, kWaitNs)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(sm + s * kPStageBytes);
+          // A: K-major rows of 128 B, 8-row groups 1024 B apart, a K step of 16
+          // moves 32 B along the row; B: MN-major, 64-column blocks of 64 K
+          // rows (8 KB apart), a K step moves 16 rows. The same offsets in the
+          // odd CTA hold its rows of A and its columns of B.
+          const uint64_t ad = sdesc_sw128(sa, 16, 1024);
+          const uint64_t bd = sdesc_sw128(sa + kPABytes, 64 * kBK * 2, 1024);
+#pragma unroll
+          for (int ks = 0; ks < kBK / 16; ++ks)
+            mma_bf16_pair(d, ad + static_cast<uint64_t>((ks * 32) >> 4),
+                          bd + static_cast<uint64_t>((ks * 16 * 128) >> 4), idesc,
+                          (kb > 0 || ks > 0) ? 1u : 0u);
+          mma_commit_pair(&empty[s], 0x3);
+        }
+        if (!ok) break;
+        mma_commit_pair(&acc_full[buf], 0x3);
+      }
+    }
+  } else if (warp < 2 + 4 * kNE) {
+    // ============================== epilogue ==============================
+    const int g = (warp - 2) >> 2;                  // column group of the tile
+    const int qd = warp & 3;                        // TMEM lane quadrant = row block
+    const uint32_t acc_empty0 = mapa_shared(smem_u32(acc_empty), 0u);
+    int lt = 0;
+    for (int tile = cid; tile < p.n_tiles; tile += n_clusters, ++lt) {
+      const int buf = lt & 1;
+      const int m0 = (tile / p.n_nt) * (2 * kPM) + static_cast<int>(rank) * kPM;
+      const int n0 = (tile % p.n_nt) * (2 * kPN);
+      const int row = m0 + qd * 32 + lane;
+      EpiY y;
+      epilogue_load_y(p, row, n0 + g * kEpiCols, y);
+      if (!mbar_wait(&acc_full[buf], (lt >> 1) & 1, cta_abort, kWaitNs)) {
+        give_up();
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tl = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) +
+                          static_cast<uint32_t>(buf * 2 * kPN + g * kEpiCols);
+      epilogue_rows(p, tl, row, n0 + g * kEpiCols, y);
+      tc_fence_before();
+      __syncwarp();
+      // the accumulator's reads are complete (tcgen05.wait::ld): a relaxed
+      // signal to the MMA thread suffices
+      if (lane == 0) {
+        if (rank == 0u)
+          mbar_arrive(&acc_empty[buf]);
+        else
+          mbar_arrive_cluster_relaxed(acc_empty0 + static_cast<uint32_t>(buf * 8));
+      }
+    }
+  }
+  tc_fence_before();
+  cluster_sync();                                     // neither CTA exits while the other works
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, 512);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 gemm_encode_fn() {
@@ -284,28 +502,61 @@ int launch_gemm_tc(int M, int N, int K, const void *A, const void *B, const void
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return RGLRU_ERR_CUDA;
   }
+  const bool pair = M % (2 * kPM) == 0 && N % (2 * kPN) == 0 && K % kBK == 0;
   GemmParams p;
   p.M = M;
   p.N = N;
   p.K = K;
-  p.n_mt = ceil_div(M, kBM);
-  p.n_nt = ceil_div(N, kBN);
+  p.n_mt = pair ? M / (2 * kPM) : ceil_div(M, kBM);
+  p.n_nt = pair ? N / (2 * kPN) : ceil_div(N, kBN);
   p.n_tiles = p.n_mt * p.n_nt;
   p.Y = static_cast<const __nv_bfloat16 *>(Y);
   p.C = static_cast<__nv_bfloat16 *>(C);
   p.dev_status = dev_status;
+  // per device, once: the shared-memory opt-ins, the SM count and how many CTA
+  // pairs are resident at once
   constexpr int kMaxDev = 64;
-  static std::atomic<int> sms_of[kMaxDev];
+  static std::atomic<int> sms_of[kMaxDev], pairs_of[kMaxDev];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return RGLRU_ERR_CUDA;
   int sms = dev < kMaxDev ? sms_of[dev].load(std::memory_order_acquire) : 0;
+  int pairs = dev < kMaxDev ? pairs_of[dev].load(std::memory_order_acquire) : 0;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kPSmemBytes;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (sms == 0) {
     if (cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSmemBytes) != cudaSuccess)
+                             kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kPSmemBytes) != cudaSuccess)
       return RGLRU_ERR_CUDA;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return RGLRU_ERR_CUDA;
-    if (dev < kMaxDev) sms_of[dev].store(sms, std::memory_order_release);
+    cfg.gridDim = dim3(2 * (sms / 2));
+    if (cudaOccupancyMaxActiveClusters(&pairs, gemm_tc2_kernel, &cfg) != cudaSuccess)
+      return RGLRU_ERR_CUDA;
+    if (dev < kMaxDev) {
+      pairs_of[dev].store(pairs, std::memory_order_release);
+      sms_of[dev].store(sms, std::memory_order_release);
+    }
+  }
+  if (pair && pairs > 0) {
+    cfg.gridDim = dim3(2 * (p.n_tiles < pairs ? p.n_tiles : pairs));
+    if (cudaLaunchKernelEx(&cfg, gemm_tc2_kernel, ta, tb, p) != cudaSuccess) return RGLRU_ERR_CUDA;
+    return RGLRU_OK;
+  }
+  if (pair) {                                          // no pair fits: one-CTA tiles
+    p.n_mt = ceil_div(M, kBM);
+    p.n_nt = ceil_div(N, kBN);
+    p.n_tiles = p.n_mt * p.n_nt;
   }
   const int grid = p.n_tiles < sms ? p.n_tiles : sms;
   gemm_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(ta, tb, p);

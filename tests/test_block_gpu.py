@@ -30,6 +30,12 @@ CASES = [
     (WORKLOADS["hawk_block"].with_shape(B=1, T=700, D=384, H=6, h0_var=0.1, seed=63), 512),
     # the bench's block shape at two batch rows
     (WORKLOADS["hawk_block"].with_shape(B=2, seed=64), 1024),
+    # B*T, D and Dm multiples of 256: every projection on CTA-pair 256 x 256 tiles,
+    # with widths other than the bench's
+    (WORKLOADS["hawk_block"].with_shape(B=2, T=256, D=512, H=2, h0_var=0.3, seed=66), 768),
+    # D = 384: the input and gate projections on one-CTA tiles, the output
+    # projection (N = Dm = 256, K = 384) on CTA pairs
+    (WORKLOADS["hawk_block"].with_shape(B=1, T=512, D=384, H=3, seed=67), 256),
 ]
 
 

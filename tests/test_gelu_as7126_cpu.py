@@ -1,0 +1,76 @@
+"""The GeLU of the recurrent block's tensor-core GEMM epilogue takes erf from
+Abramowitz and Stegun, Handbook of Mathematical Functions, formula 7.1.26
+(|error| <= 1.5e-7 for x >= 0). These tests read the coefficients as they are
+written in the CUDA header and check the formula against math.erf in float64
+over the whole range, the published bound, and the GeLU assembled from it the
+way the kernel assembles it (Phi(-|v|) = erfc(|v| / sqrt 2) / 2, no
+cancellation for negative v). A one-digit slip in any coefficient fails."""
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+HEADER = os.path.join(os.path.dirname(__file__), os.pardir, "gated_linear_recurrence_rglru_b200",
+                      "csrc", "common.cuh")
+NAMES = ("kP", "kA1", "kA2", "kA3", "kA4", "kA5")
+
+
+def header_coefficients() -> dict:
+    text = open(HEADER).read()
+    block = text[text.index("namespace erf_as7126"):]
+    block = block[:block.index("}  // namespace erf_as7126")]
+    out = {}
+    for name in NAMES:
+        m = re.search(rf"constexpr float {name} = (-?[0-9.]+)f;", block)
+        assert m, f"{name} not found in the header"
+        out[name] = float(m.group(1))
+    return out
+
+
+def erf_as(x, c):
+    t = 1.0 / (1.0 + c["kP"] * x)
+    poly = t * (c["kA1"] + t * (c["kA2"] + t * (c["kA3"] + t * (c["kA4"] + t * c["kA5"]))))
+    return 1.0 - poly * np.exp(-x * x)
+
+
+def gelu_as(v, c):
+    x = np.abs(v) / math.sqrt(2.0)
+    phi_neg = 0.5 * (1.0 - erf_as(x, c))          # = erfc(x) / 2 as the kernel forms it
+    return v * np.where(v >= 0, 1.0 - phi_neg, phi_neg)
+
+
+ERF = np.vectorize(math.erf)
+
+
+def test_coefficients_meet_the_published_bound():
+    c = header_coefficients()
+    x = np.linspace(0.0, 8.0, 200001)
+    err = np.abs(erf_as(x, c) - ERF(x))
+    assert err.max() <= 1.5e-7, err.max()
+    # the bound is nearly attained: the coefficients are the minimax ones, not a
+    # looser fit that happens to pass
+    assert err.max() > 0.5e-7
+
+
+def test_gelu_from_the_formula_against_the_exact_gelu():
+    c = header_coefficients()
+    v = np.linspace(-12.0, 12.0, 240001)
+    exact = 0.5 * v * (1.0 + ERF(v / math.sqrt(2.0)))
+    got = gelu_as(v, c)
+    # |Phi error| <= 7.5e-8, so |GeLU error| <= 7.5e-8 |v|
+    assert np.all(np.abs(got - exact) <= 7.5e-8 * np.abs(v) + 1e-300)
+    # far tails: exactly v for large v, and tiny (not a cancelled 0 or garbage)
+    # values for large negative v
+    assert got[-1] == pytest.approx(12.0, rel=1e-15)
+    neg = v < -6
+    assert np.all(np.abs(got[neg]) <= np.abs(v[neg]) * 1e-8)
+
+
+@pytest.mark.parametrize("name", NAMES)
+def test_a_slip_in_any_coefficient_breaks_the_bound(name):
+    c = header_coefficients()
+    c[name] = c[name] * (1.0 + 1e-4)               # a slip in the fifth significant digit
+    x = np.linspace(0.0, 8.0, 20001)
+    assert np.abs(erf_as(x, c) - ERF(x)).max() > 1.5e-7
