@@ -32,8 +32,9 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "gelu_as7126.cuh"
 #include "kernels.h"
-#include "tc_primitives.cuh"
+#include "tc_pair.cuh"
 
 namespace rglru {
 namespace {

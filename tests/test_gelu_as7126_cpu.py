@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 
 HEADER = os.path.join(os.path.dirname(__file__), os.pardir, "gated_linear_recurrence_rglru_b200",
-                      "csrc", "common.cuh")
+                      "csrc", "gelu_as7126.cuh")
 NAMES = ("kP", "kA1", "kA2", "kA3", "kA4", "kA5")
 
 
