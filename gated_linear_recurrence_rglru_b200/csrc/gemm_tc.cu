@@ -66,7 +66,8 @@ static_assert(kSmemBytes <= 232448, "shared memory");
 
 struct GemmParams {
   int M, N, K;
-  int n_mt, n_nt, n_tiles;
+  int n_mt, n_nt, n_tiles;   // CTA pairs: n_tiles work items, the first n_full whole tiles
+  int n_full;                // (see pair_item)
   const __nv_bfloat16 *Y;    // (M, N) or null: C = Y * GeLU(A B)
   __nv_bfloat16 *C;          // (M, N)
   int *dev_status;
@@ -80,22 +81,25 @@ struct EpiY {
 };
 
 __device__ __forceinline__ void epilogue_load_y(const GemmParams &p, int row, int c_first,
-                                                EpiY &y) {
+                                                EpiY &y, int ncols = kEpiCols) {
   if (p.Y == nullptr || row >= p.M) return;
   const __nv_bfloat16 *yr = p.Y + static_cast<size_t>(row) * p.N;
 #pragma unroll
   for (int q = 0; q < kEpiCols / 8; ++q)
-    if (c_first + q * 8 < p.N) y.v[q] = *reinterpret_cast<const uint4 *>(yr + c_first + q * 8);
+    if (q * 8 < ncols && c_first + q * 8 < p.N)
+      y.v[q] = *reinterpret_cast<const uint4 *>(yr + c_first + q * 8);
 }
 
-// Epilogue of one warp: kEpiCols accumulator columns of this lane's row (TMEM
-// address tl: the warp's lane quadrant, the first column), converted to bf16
-// (times Y * GeLU when Y is given, from y) and stored from column c_first on,
-// in chunks of 32 columns (64 contiguous bytes per row and chunk).
+// Epilogue of one warp: ncols (a multiple of 32, at most kEpiCols) accumulator
+// columns of this lane's row (TMEM address tl: the warp's lane quadrant, the
+// first column), converted to bf16 (times Y * GeLU when Y is given, from y) and
+// stored from column c_first on, in chunks of 32 columns (64 contiguous bytes
+// per row and chunk).
 __device__ __forceinline__ void epilogue_rows(const GemmParams &p, uint32_t tl, int row,
-                                              int c_first, const EpiY &y) {
+                                              int c_first, const EpiY &y, int ncols = kEpiCols) {
 #pragma unroll
   for (int ch = 0; ch < kEpiCols / 32; ++ch) {
+    if (ch * 32 >= ncols) break;
     const int c0 = c_first + ch * 32;               // first column of this chunk
     float v[32];
     __syncwarp();                                   // tcgen05.ld is warp-collective
@@ -296,6 +300,25 @@ constexpr int kPOffMisc = kPOffBar + kPNumBars * 8;
 constexpr int kPSmemBytes = kPOffMisc + 64;
 static_assert(kPSmemBytes <= 232448, "shared memory");
 
+// Work item w of the pair kernel: whole 256 x 256 tiles first (w < n_full, a
+// whole number of waves over the pairs), then each remaining tile as two
+// 256 x 128 halves, so that the last wave runs twice as many items of half the
+// length. Tiles are numbered with N fastest. Returns the first row, the first
+// column and the width (256 or 128).
+struct PairItem {
+  int m0, n0, nw;
+};
+
+__device__ __forceinline__ PairItem pair_item(const GemmParams &p, int w) {
+  int f = w, nw = 2 * kPN, half = 0;
+  if (w >= p.n_full) {
+    f = p.n_full + (w - p.n_full) / 2;
+    half = (w - p.n_full) & 1;
+    nw = kPN;
+  }
+  return {(f / p.n_nt) * (2 * kPM), (f % p.n_nt) * (2 * kPN) + half * kPN, nw};
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                 const GemmParams p) {
@@ -356,8 +379,11 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
       const uint32_t full0 = mapa_shared(smem_u32(full), 0u);   // the even CTA's barriers
       int it = 0;
       for (int tile = cid; tile < p.n_tiles && !*cta_abort; tile += n_clusters) {
-        const int m0 = (tile / p.n_nt) * (2 * kPM) + static_cast<int>(rank) * kPM;
-        const int n0 = (tile % p.n_nt) * (2 * kPN) + static_cast<int>(rank) * kPN;
+        const PairItem w = pair_item(p, tile);
+        // this CTA's rows of A and its half of the item's columns of B
+        const int m0 = w.m0 + static_cast<int>(rank) * kPM;
+        const int n0 = w.n0 + static_cast<int>(rank) * (w.nw / 2);
+        const int nb = w.nw / 128;                    // 64-column B boxes per CTA
         for (int kb = 0; kb < k_steps; ++kb, ++it) {
           const int s = it % kPStages;
           if (!mbar_wait(&empty[s], ((it / kPStages) & 1) ^ 1, cta_abort, kWaitNs)) {
@@ -365,10 +391,11 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
             break;
           }
           unsigned char *st = sm + s * kPStageBytes;
-          if (rank == 0u) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(2 * kPStageBytes));
+          if (rank == 0u)
+            mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(2 * (kPABytes + nb * 64 * kBK * 2)));
           const uint32_t fb = full0 + static_cast<uint32_t>(s * 8);
           tma_load_2d_pair(st, &tmap_a, fb, kb * kBK, m0);
-          for (int j = 0; j < kPN / 64; ++j)
+          for (int j = 0; j < nb; ++j)
             tma_load_2d_pair(st + kPABytes + j * (64 * kBK * 2), &tmap_b, fb, n0 + j * 64, kb * kBK);
         }
       }
@@ -380,9 +407,11 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
   } else if (warp == 1) {
     // ============================= MMA issuer =============================
     if (lane == 0 && rank == 0u) {
-      constexpr uint32_t idesc = idesc_bf16_f32(2 * kPM, 2 * kPN, false, true);
+      constexpr uint32_t idesc_whole = idesc_bf16_f32(2 * kPM, 2 * kPN, false, true);
+      constexpr uint32_t idesc_half = idesc_bf16_f32(2 * kPM, kPN, false, true);
       int it = 0, lt = 0;
       for (int tile = cid; tile < p.n_tiles && !*cta_abort; tile += n_clusters, ++lt) {
+        const uint32_t idesc = pair_item(p, tile).nw == 2 * kPN ? idesc_whole : idesc_half;
         const int buf = lt & 1;
         if (!mbar_wait(&acc_empty[buf], ((lt >> 1) & 1) ^ 1, cta_abort, kWaitNs)) {
           give_up();
@@ -425,19 +454,19 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
     int lt = 0;
     for (int tile = cid; tile < p.n_tiles; tile += n_clusters, ++lt) {
       const int buf = lt & 1;
-      const int m0 = (tile / p.n_nt) * (2 * kPM) + static_cast<int>(rank) * kPM;
-      const int n0 = (tile % p.n_nt) * (2 * kPN);
-      const int row = m0 + qd * 32 + lane;
+      const PairItem w = pair_item(p, tile);
+      const int row = w.m0 + static_cast<int>(rank) * kPM + qd * 32 + lane;
+      const int ncols = w.nw / kNE;                 // this warpgroup's columns of the item
       EpiY y;
-      epilogue_load_y(p, row, n0 + g * kEpiCols, y);
+      epilogue_load_y(p, row, w.n0 + g * ncols, y, ncols);
       if (!mbar_wait(&acc_full[buf], (lt >> 1) & 1, cta_abort, kWaitNs)) {
         give_up();
         break;
       }
       tc_fence_after();
       const uint32_t tl = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) +
-                          static_cast<uint32_t>(buf * 2 * kPN + g * kEpiCols);
-      epilogue_rows(p, tl, row, n0 + g * kEpiCols, y);
+                          static_cast<uint32_t>(buf * 2 * kPN + g * ncols);
+      epilogue_rows(p, tl, row, w.n0 + g * ncols, y, ncols);
       tc_fence_before();
       __syncwarp();
       // the accumulator's reads are complete (tcgen05.wait::ld): a relaxed
@@ -511,6 +540,7 @@ int launch_gemm_tc(int M, int N, int K, const void *A, const void *B, const void
   p.n_mt = pair ? M / (2 * kPM) : ceil_div(M, kBM);
   p.n_nt = pair ? N / (2 * kPN) : ceil_div(N, kBN);
   p.n_tiles = p.n_mt * p.n_nt;
+  p.n_full = p.n_tiles;
   p.Y = static_cast<const __nv_bfloat16 *>(Y);
   p.C = static_cast<__nv_bfloat16 *>(C);
   p.dev_status = dev_status;
@@ -550,7 +580,15 @@ int launch_gemm_tc(int M, int N, int K, const void *A, const void *B, const void
     }
   }
   if (pair && pairs > 0) {
-    cfg.gridDim = dim3(2 * (p.n_tiles < pairs ? p.n_tiles : pairs));
+    const int clusters = p.n_tiles < pairs ? p.n_tiles : pairs;
+    // whole tiles in whole waves; the rest as halves when they then fit one wave
+    const int rest = p.n_tiles % clusters;
+    p.n_full = p.n_tiles;
+    if (rest > 0 && 2 * rest <= clusters) {
+      p.n_full = p.n_tiles - rest;
+      p.n_tiles = p.n_full + 2 * rest;
+    }
+    cfg.gridDim = dim3(2 * clusters);
     if (cudaLaunchKernelEx(&cfg, gemm_tc2_kernel, ta, tb, p) != cudaSuccess) return RGLRU_ERR_CUDA;
     return RGLRU_OK;
   }

@@ -36,6 +36,9 @@ CASES = [
     # D = 384: the input and gate projections on one-CTA tiles, the output
     # projection (N = Dm = 256, K = 384) on CTA pairs
     (WORKLOADS["hawk_block"].with_shape(B=1, T=512, D=384, H=3, seed=67), 256),
+    # B*T = 5120: 80 tiles of 256 x 256 per projection, more than a wave of CTA
+    # pairs on a B200 (74): the tiles past the last whole wave run as halves
+    (WORKLOADS["hawk_block"].with_shape(B=5, T=1024, h0_var=0.2, seed=68), 1024),
 ]
 
 
