@@ -68,10 +68,27 @@ struct GemmParams {
   int M, N, K;
   int n_mt, n_nt, n_tiles;   // CTA pairs: n_tiles work items, the first n_full whole tiles
   int n_full;                // (see pair_item)
+  int c_v8, y_v8;            // 1: C (Y) rows may be accessed 32 bytes at a time (N % 16 == 0
+                             // and a 32-byte aligned base)
   const __nv_bfloat16 *Y;    // (M, N) or null: C = Y * GeLU(A B)
   __nv_bfloat16 *C;          // (M, N)
   int *dev_status;
 };
+
+// 32 bytes at a 32-byte aligned global address (sm_100 256-bit accesses: one
+// whole sector per lane).
+__device__ __forceinline__ void st_global_v8(void *ptr, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(ptr), "r"(w[0]),
+               "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
+__device__ __forceinline__ void ld_global_v8(const void *ptr, uint4 &a, uint4 &b) {
+  asm volatile("ld.global.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z),
+                 "=r"(b.w)
+               : "l"(ptr));
+}
 
 // Y operand of one warp's epilogue: this lane's row, kEpiCols columns from
 // c_first, loaded as 8-column vectors before the accumulator is ready (the
@@ -84,6 +101,13 @@ __device__ __forceinline__ void epilogue_load_y(const GemmParams &p, int row, in
                                                 EpiY &y, int ncols = kEpiCols) {
   if (p.Y == nullptr || row >= p.M) return;
   const __nv_bfloat16 *yr = p.Y + static_cast<size_t>(row) * p.N;
+  if (p.y_v8 && c_first % 16 == 0 && c_first + ncols <= p.N) {
+    // whole 16-column (32-byte) pieces, 32-byte aligned: one sector per load
+#pragma unroll
+    for (int q = 0; q < kEpiCols / 8; q += 2)
+      if (q * 8 < ncols) ld_global_v8(yr + c_first + q * 8, y.v[q], y.v[q + 1]);
+    return;
+  }
 #pragma unroll
   for (int q = 0; q < kEpiCols / 8; ++q)
     if (q * 8 < ncols && c_first + q * 8 < p.N)
@@ -123,16 +147,33 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams &p, uint32_t tl, 
           }
         }
       }
+      if (nq == 4 && p.c_v8) {
+        // a whole chunk at a 32-byte aligned address (c0 is a multiple of 32
+        // columns): two 256-bit stores, each one whole sector
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (q >= nq) break;
-        uint32_t w[4];
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t w[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const __nv_bfloat162 h = __floats2bfloat162_rn(v[q * 8 + 2 * e], v[q * 8 + 2 * e + 1]);
-          w[e] = *reinterpret_cast<const uint32_t *>(&h);
+          for (int e = 0; e < 8; ++e) {
+            const __nv_bfloat162 h =
+                __floats2bfloat162_rn(v[h2 * 16 + 2 * e], v[h2 * 16 + 2 * e + 1]);
+            w[e] = *reinterpret_cast<const uint32_t *>(&h);
+          }
+          st_global_v8(p.C + off + h2 * 16, w);
         }
-        *reinterpret_cast<uint4 *>(p.C + off + q * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (q >= nq) break;
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 h =
+                __floats2bfloat162_rn(v[q * 8 + 2 * e], v[q * 8 + 2 * e + 1]);
+            w[e] = *reinterpret_cast<const uint32_t *>(&h);
+          }
+          *reinterpret_cast<uint4 *>(p.C + off + q * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
       }
     }
   }
@@ -543,6 +584,8 @@ int launch_gemm_tc(int M, int N, int K, const void *A, const void *B, const void
   p.n_full = p.n_tiles;
   p.Y = static_cast<const __nv_bfloat16 *>(Y);
   p.C = static_cast<__nv_bfloat16 *>(C);
+  p.c_v8 = (N % 16 == 0 && (reinterpret_cast<uintptr_t>(C) & 31u) == 0) ? 1 : 0;
+  p.y_v8 = (Y != nullptr && N % 16 == 0 && (reinterpret_cast<uintptr_t>(Y) & 31u) == 0) ? 1 : 0;
   p.dev_status = dev_status;
   // per device, once: the shared-memory opt-ins, the SM count and how many CTA
   // pairs are resident at once
