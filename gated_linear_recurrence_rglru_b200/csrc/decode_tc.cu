@@ -62,11 +62,12 @@ template <int K, int N>
 struct DCfg {
   static constexpr int NE = 2;                     // epilogue warpgroups
   static constexpr int kThreads = 64 + 128 + NE * 128;
-  // Gate weights (the MMA's A operand): in shared memory for K = 128 (TMA),
-  // in TMEM for K = 256, where the tensor core would otherwise re-read 128 KB
-  // of shared memory for every 16-row job (written by the conv warpgroup)
+  // Gate weights (the MMA's A operand), TMA-loaded into shared memory at each
+  // change of unit: the MMA reads them there for K = 128; for K = 256 the conv
+  // warpgroup copies them into TMEM once per unit, where the tensor core would
+  // otherwise re-read 128 KB of shared memory for every 16-row job
   static constexpr bool kATmem = (K == 256);
-  static constexpr int kABytes = kATmem ? 0 : K * 256;   // one gate: 2 M-blocks x K rows x 128 B
+  static constexpr int kABytes = K * 256;          // one gate: 2 M-blocks x K rows x 128 B
   static constexpr int kInBytes = N * K * 2;       // one input tile: N rows x K channels, bf16
   static constexpr int kXBytes = 4 * kInBytes;     // x_t and ring slots pos, pos+1, pos+2 (mod 3)
   static constexpr int kNX = 2;                    // input slots
@@ -96,6 +97,13 @@ struct DCfg {
   static_assert(kSmemBytes <= 232448, "shared memory");
   static_assert(N % 16 == 0 && (N * NQ) % 128 == 0 && SEG % 4 == 0, "conv mapping");
 };
+
+// One 16-bit shared-memory load (zero-extended).
+__device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a) : "memory");
+  return v;
+}
 
 // Offset (bytes) of (own channel c, 4-row block jb) in the fp32 u tile:
 // channel-major rows of N floats whose 16-byte blocks are XOR-permuted so that
@@ -217,7 +225,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
       mbar_init(&x_empty[i], 4);                    // 4 conv warps
     }
     mbar_init(w_full, 1);
-    mbar_init(w_free, 1);
+    mbar_init(w_free, C::kATmem ? 4 : 1);          // the conv warps' TMEM copy, or the MMA
     for (int i = 0; i < NS; ++i) {
       mbar_init(&b_full[i], 4);                     // 4 conv warps
       mbar_init(&b_empty[i], 1);
@@ -235,7 +243,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
     prefetch_tmap(&tmap_xt);
     prefetch_tmap(&tmap_ring);
   }
-  {
+  if (!C::kATmem) {
+    // block-diagonal zeros of 64-wide heads (the TMA fills 256-wide heads' tiles whole)
     uint4 *a4 = reinterpret_cast<uint4 *>(sA);
     for (int i = tid; i < 2 * C::kABytes / 16; i += C::kThreads) a4[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
@@ -277,7 +286,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
         jobs[js] = make_int4(unit, tile, reload, 0);
         mbar_arrive(&job_full[js]);
         const int cg = unit;
-        if (reload && !C::kATmem) {
+        if (reload) {
           if (i > 0) {
             RG_WAIT_OR_ABORT(w_free, wfree_phase);
             wfree_phase ^= 1;
@@ -383,6 +392,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
     // ============================== conv warpgroup ==============================
     const int wt = tid - 64;
     int cur_unit = -1;
+    uint32_t wfull_phase = 0;
     float2 cwq[4][2];
     for (int i = 0;; ++i) {
       const int js = i % kJQ;
@@ -404,28 +414,33 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
         }
         if (C::kATmem) {
           // This unit's gate weights into TMEM (the A operand): lane m (output
-          // channel cg*128 + m) holds W[h][k][j] for k = 0..K-1, two per column.
-          // Every MMA of earlier jobs has read the old weights once the
-          // accumulator of job i-1 is complete (MMAs complete in issue order).
+          // channel cg*128 + m) holds W[h][k][j] for k = 0..K-1, two per column,
+          // copied from the TMA-loaded shared-memory tiles (128-byte swizzle,
+          // MN-major: per 64-channel block ma, row k of 128 B, 16-byte chunk
+          // (m % 64) / 8 stored at chunk ^ (k % 8); a warp's 32 channels read
+          // 64 bytes of one row: no bank conflicts). Every MMA of earlier jobs
+          // has read the old TMEM weights once the accumulator of job i-1 is
+          // complete (MMAs complete in issue order).
+          RG_WAIT_OR_ABORT(w_full, wfull_phase);
+          wfull_phase ^= 1;
           if (i > 0) RG_WAIT_OR_ABORT(&acc_full[(i - 1) % NT], ((i - 1) / NT) & 1);
           const int qd = warp & 3;                  // this warp's TMEM lane quadrant
-          const int cout = cg * kM + qd * 32 + lane;
-          const int hh = cout / p.bw, jj = cout % p.bw;
+          const int m = qd * 32 + lane;             // output channel within the unit
           const uint32_t tq = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) +
                               static_cast<uint32_t>(C::kACol);
+          const uint32_t mcol = static_cast<uint32_t>((m >> 6) * (K * 128) + ((m & 7) << 1));
+          const uint32_t mchunk = static_cast<uint32_t>((m & 63) >> 3);
 #pragma unroll 1
           for (int g = 0; g < 2; ++g) {
-            const unsigned short *Wg =
-                reinterpret_cast<const unsigned short *>(g == 0 ? p.W_a : p.W_x) +
-                static_cast<size_t>(hh) * p.bw * p.bw + jj;
+            const uint32_t ag = smem_u32(sA + g * C::kABytes) + mcol;
 #pragma unroll 1
             for (int cc = 0; cc < K / 64; ++cc) {
               uint32_t v[32];
 #pragma unroll
               for (int q = 0; q < 32; ++q) {
-                const int k = cc * 64 + 2 * q;
-                const uint32_t lo = __ldg(Wg + static_cast<size_t>(k) * p.bw);
-                const uint32_t hi = __ldg(Wg + static_cast<size_t>(k + 1) * p.bw);
+                const uint32_t k = static_cast<uint32_t>(cc * 64 + 2 * q);   // even: k % 8 = 2q % 8
+                const uint32_t lo = lds_u16(ag + k * 128 + ((mchunk ^ (k & 7)) << 4));
+                const uint32_t hi = lds_u16(ag + (k + 1) * 128 + ((mchunk ^ ((k + 1) & 7)) << 4));
                 v[q] = lo | (hi << 16);
               }
               tmem_st32u(tq + static_cast<uint32_t>(g * (K / 2) + cc * 32), v);
@@ -434,7 +449,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(a_ready);
+          if (lane == 0) {
+            mbar_arrive(a_ready);
+            mbar_arrive(w_free);                    // the shared-memory tiles may be reloaded
+          }
         }
       }
       const int s = i % NS, xb = i % NX;
