@@ -154,7 +154,10 @@ def decode_run(wl, rows, dev, algo, steps):
 
 
 @pytest.mark.parametrize("algo", DEC_ALGOS)
-@pytest.mark.parametrize("shape", [(70, 256, 4), (33, 256, 2), (45, 512, 2), (1, 128, 1)])
+# (2560, 512, 2): 256-wide heads, 2 heads x 160 row tiles = 320 (head, tile) pairs over the
+# CTAs, so that CTA ranges hold several pairs and some cross the head boundary
+@pytest.mark.parametrize("shape", [(70, 256, 4), (33, 256, 2), (45, 512, 2), (1, 128, 1),
+                                   (2560, 512, 2)])
 def test_decode_shapes_bf16(cuda_device, algo, shape):
     B, D, H = shape
     wl = WORKLOADS["decode_batch"].with_shape(B=B, D=D, H=H, decode_steps=5, bias_std=0.3,
