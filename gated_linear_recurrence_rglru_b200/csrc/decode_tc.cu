@@ -22,9 +22,13 @@
 // epilogue warpgroups take the jobs alternately and load their rows' h before
 // waiting for the MMA.
 //
-// Heads 256 wide are split over two channel groups whose CTAs both read all
-// 256 channels of the ring's slot pos % 3; that slot is then rewritten by a
-// separate small kernel after this one (ring_update_kernel) instead of here.
+// Heads 256 wide run as CTA pairs (a cluster of 2): the two 128-channel units
+// of a head take the same row tiles; each CTA loads x_t and the ring slots of
+// its own 128 channels only, computes their Conv1D, and sends its half of the
+// MMA's B operand (all 256 input channels) to the partner by a bulk copy that
+// completes on the partner's barrier; the MMA releases a B slot to both CTAs.
+// Each CTA is then the only reader of its channels' ring slot and rewrites it
+// with x_t itself, so a step is one launch for every head width.
 #include <cudaTypedefs.h>
 
 #include <atomic>
@@ -32,6 +36,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_gates.cuh"
+#include "tc_pair.cuh"
 #include "tc_primitives.cuh"
 
 namespace rglru {
@@ -68,9 +73,14 @@ struct DCfg {
   // otherwise re-read 128 KB of shared memory for every 16-row job
   static constexpr bool kATmem = (K == 256);
   static constexpr int kABytes = K * 256;          // one gate: 2 M-blocks x K rows x 128 B
-  static constexpr int kInBytes = N * K * 2;       // one input tile: N rows x K channels, bf16
+  // 256-wide heads run as CTA pairs (a cluster of 2, one per 128-channel unit of
+  // the head, on the same rows): each CTA loads and convolves only its own 128
+  // channels and sends its half of the B operand to the partner
+  static constexpr bool kPair = (K == 256);
+  static constexpr int kXK = kPair ? kM : K;       // channels of an input tile
+  static constexpr int kInBytes = N * kXK * 2;     // one input tile: N rows x kXK channels, bf16
   static constexpr int kXBytes = 4 * kInBytes;     // x_t and ring slots pos, pos+1, pos+2 (mod 3)
-  static constexpr int kNX = 2;                    // input slots
+  static constexpr int kNX = kPair ? 4 : 2;        // input slots
   static constexpr int kBBytes = N * K * 2;
   static constexpr int kUBytes = N * kM * 4;
   static constexpr int kNS = 2;
@@ -92,7 +102,7 @@ struct DCfg {
   static constexpr int kUsedCols = kACol + (kATmem ? K : 0);
   static constexpr int kTmemCols = kUsedCols <= 128 ? 128 : (kUsedCols <= 256 ? 256 : 512);
   static_assert(kUsedCols <= 512, "TMEM allocation");
-  static constexpr int NQ = K / 4;                 // conv: channel quads
+  static constexpr int NQ = kXK / 4;               // conv: channel quads
   static constexpr int SEG = N * NQ / 128;         // conv: rows per thread
   static_assert(kSmemBytes <= 232448, "shared memory");
   static_assert(N % 16 == 0 && (N * NQ) % 128 == 0 && SEG % 4 == 0, "conv mapping");
@@ -117,36 +127,38 @@ __device__ __forceinline__ uint32_t u_off(int c, int jb) {
   return static_cast<uint32_t>(c * (N * 4) + ((jb ^ perm) << 4));
 }
 
-// Conv1D of N rows x K channels from the input tile in shared memory (row-major
-// [N][K] per array: x_t, then the ring slots holding x_{t-3}, x_{t-2}, x_{t-1}).
-// Thread t covers channel quad q (4 channels) and SEG consecutive rows. Writes
-// the bf16 K-major B operand (128-byte swizzle), the fp32 u of the own channels
-// (channel-major, see u_off) and, when asked, the ring update of the own channels.
+// Conv1D of N rows x kXK channels from the input tile in shared memory
+// (row-major [N][kXK] per array: x_t, then the ring slots holding x_{t-3},
+// x_{t-2}, x_{t-1}). Thread t covers channel quad q (4 channels) and SEG
+// consecutive rows. Writes the bf16 K-major B operand (128-byte swizzle) at K
+// rows koff + channel, the fp32 u of the own channels (channel-major, see
+// u_off) and, when asked, the ring update of the own channels.
 template <int K, int N>
 __device__ __forceinline__ void dec_conv(const DecTcParams &p, const unsigned char *__restrict__ xin,
                                          unsigned char *__restrict__ bt,
                                          unsigned char *__restrict__ ut, int kbase, int own_lo,
-                                         int r0, int t, const float2 (&w)[4][2]) {
+                                         int koff, int r0, int t, const float2 (&w)[4][2]) {
   using C = DCfg<K, N>;
-  constexpr int NQ = C::NQ, SEG = C::SEG;
+  constexpr int NQ = C::NQ, SEG = C::SEG, XK = C::kXK;
   const int qd = t % NQ, sg = t / NQ;
   const int kq = qd * 4, nb = sg * SEG;
   const bool own = (kq >= own_lo) && (kq < own_lo + kM);
   const int chq = kbase + kq;
   const int s0 = p.pos % 3;
-  const unsigned char *xq = xin + kq * 2;          // + array * kInBytes + row * K * 2
-  unsigned char *bq = bt + (kq >> 6) * N * 128 + ((kq & 7) << 1);
-  const int chunk = (kq & 63) >> 3;
+  const int kk = koff + kq;                        // K row of the quad in the B operand
+  const unsigned char *xq = xin + kq * 2;          // + array * kInBytes + row * XK * 2
+  unsigned char *bq = bt + (kk >> 6) * N * 128 + ((kk & 7) << 1);
+  const int chunk = (kk & 63) >> 3;
 #pragma unroll
   for (int j0 = 0; j0 < SEG; j0 += 4) {
     float uacc[4][4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int n = nb + j0 + j;
-      const uint2 xv = *reinterpret_cast<const uint2 *>(xq + n * K * 2);
-      const uint2 r0v = *reinterpret_cast<const uint2 *>(xq + C::kInBytes + n * K * 2);
-      const uint2 r1v = *reinterpret_cast<const uint2 *>(xq + 2 * C::kInBytes + n * K * 2);
-      const uint2 r2v = *reinterpret_cast<const uint2 *>(xq + 3 * C::kInBytes + n * K * 2);
+      const uint2 xv = *reinterpret_cast<const uint2 *>(xq + n * XK * 2);
+      const uint2 r0v = *reinterpret_cast<const uint2 *>(xq + C::kInBytes + n * XK * 2);
+      const uint2 r1v = *reinterpret_cast<const uint2 *>(xq + 2 * C::kInBytes + n * XK * 2);
+      const uint2 r2v = *reinterpret_cast<const uint2 *>(xq + 3 * C::kInBytes + n * XK * 2);
       float2 u[2];
 #pragma unroll
       for (int pp = 0; pp < 2; ++pp) {
@@ -211,9 +223,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  // this CTA's contiguous, balanced range of jobs (job = unit * n_tiles + tile)
-  const int j_begin = static_cast<int>(static_cast<long>(p.n_jobs) * blockIdx.x / gridDim.x);
-  const int j_end = static_cast<int>(static_cast<long>(p.n_jobs) * (blockIdx.x + 1) / gridDim.x);
+  constexpr bool kPair = C::kPair;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+  // this CTA's (pair's) contiguous, balanced range of work items: jobs (unit *
+  // n_tiles + tile), or for CTA pairs (head * n_tiles + tile), the CTA of rank r
+  // taking unit 2 head + r
+  const int n_items = kPair ? p.n_jobs / 2 : p.n_jobs;
+  const int n_grp = kPair ? static_cast<int>(gridDim.x) / 2 : static_cast<int>(gridDim.x);
+  const int grp = kPair ? static_cast<int>(blockIdx.x) / 2 : static_cast<int>(blockIdx.x);
+  const int j_begin = static_cast<int>(static_cast<long>(n_items) * grp / n_grp);
+  const int j_end = static_cast<int>(static_cast<long>(n_items) * (grp + 1) / n_grp);
 
   if (tid == 0) {
     for (int i = 0; i < kJQ; ++i) {
@@ -227,8 +246,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
     mbar_init(w_full, 1);
     mbar_init(w_free, C::kATmem ? 4 : 1);          // the conv warps' TMEM copy, or the MMA
     for (int i = 0; i < NS; ++i) {
-      mbar_init(&b_full[i], 4);                     // 4 conv warps
-      mbar_init(&b_empty[i], 1);
+      // 4 conv warps; for a pair each also expects the bytes of the partner's
+      // matching warp (bulk copies of its half of the B operand)
+      mbar_init(&b_full[i], 4);
+      mbar_init(&b_empty[i], kPair ? 2 : 1);        // MMA commit (of each CTA of a pair)
       mbar_init(&u_empty[i], 4);
     }
     for (int i = 0; i < NT; ++i) {
@@ -254,15 +275,22 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  // a pair's barriers are initialised before either CTA arrives on the other's
+  if (kPair)
+    cluster_sync();
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int R = p.bw <= 128 ? p.bw : 256;
+  const uint32_t peer_abort =
+      kPair ? mapa_shared(smem_u32(const_cast<int *>(cta_abort)), rank ^ 1u) : 0u;
 
-#define RG_WAIT_OR_ABORT(bar, par)                   \
-  if (!mbar_wait((bar), (par), cta_abort, kWaitNs)) { \
-    *cta_abort = 1;                                  \
-    break;                                           \
+#define RG_WAIT_OR_ABORT(bar, par)                        \
+  if (!mbar_wait((bar), (par), cta_abort, kWaitNs)) {      \
+    *cta_abort = 1;                                       \
+    if (kPair) st_cluster_u32(peer_abort, 1u);            \
+    break;                                                \
   }
 
   if (warp == 0) {
@@ -280,8 +308,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
           mbar_arrive(&job_full[js]);
           continue;
         }
-        const int job = j_begin + i;
-        const int unit = job / p.n_tiles, tile = job % p.n_tiles;
+        const int item = j_begin + i;
+        const int unit = kPair ? 2 * (item / p.n_tiles) + static_cast<int>(rank) : item / p.n_tiles;
+        const int tile = item % p.n_tiles;
         const int reload = unit != w_unit ? 1 : 0;
         jobs[js] = make_int4(unit, tile, reload, 0);
         mbar_arrive(&job_full[js]);
@@ -313,7 +342,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
         // (pos + 1) % 3 (x_{t-2}), (pos + 2) % 3 (x_{t-1}); rows past B read as zeros
         const int xb = i % NX;
         RG_WAIT_OR_ABORT(&x_empty[xb], ((i / NX) & 1) ^ 1);
-        const int kbase = p.bw <= 128 ? cg * kM : (cg >> 1) * 256;
+        // input channels of the job: the unit's own 128 (CTA pairs, heads up to
+        // 128 wide), else the head's 256
+        const int kbase = (kPair || p.bw <= 128) ? cg * kM : (cg >> 1) * 256;
         unsigned char *dst = sX + xb * C::kXBytes;
         mbar_arrive_expect_tx(&x_full[xb], static_cast<uint32_t>(C::kXBytes));
         tma_load_2d(dst, &tmap_xt, &x_full[xb], kbase, tile * N);
@@ -381,7 +412,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
           }
         }
         mma_commit(&acc_full[ts]);
-        mma_commit(&b_empty[s]);
+        // the B slot is free once the MMAs of both CTAs of a pair have read it
+        if (kPair)
+          mma_commit_multicast(&b_empty[s], 0x3);
+        else
+          mma_commit(&b_empty[s]);
         last_commit = i;
         mbar_arrive(&job_empty[js]);
       }
@@ -394,18 +429,27 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
     int cur_unit = -1;
     uint32_t wfull_phase = 0;
     float2 cwq[4][2];
-    for (int i = 0;; ++i) {
+    // CTA pairs: the partner's B slots and b_full barriers (shared::cluster), and
+    // this warp's rows of the B operand (see dec_conv: SEG rows per warp)
+    const uint32_t sB_peer = kPair ? mapa_shared(smem_u32(sB), rank ^ 1u) : 0u;
+    const uint32_t bfull_peer = kPair ? mapa_shared(smem_u32(b_full), rank ^ 1u) : 0u;
+    const uint32_t seg_off = static_cast<uint32_t>((wt >> 5) * C::SEG * 128);
+    int i = 0;
+    for (;; ++i) {
       const int js = i % kJQ;
       RG_WAIT_OR_ABORT(&job_full[js], (i / kJQ) & 1);
       const int4 job = jobs[js];
       const int unit = job.x, tile = job.y;
       if (unit < 0) break;
       const int cg = unit;
-      const int kbase = p.bw <= 128 ? cg * kM : (cg >> 1) * 256;
-      const int own_lo = p.bw <= 128 ? 0 : (cg & 1) * kM;
+      // the input channels convolved here (the unit's own 128 for pairs and
+      // heads up to 128 wide), the own ones among them, and their K rows in B
+      const int kbase = (kPair || p.bw <= 128) ? cg * kM : (cg >> 1) * 256;
+      const int own_lo = (kPair || p.bw <= 128) ? 0 : (cg & 1) * kM;
+      const int koff = kPair ? (cg & 1) * kM : 0;
       if (unit != cur_unit) {
         cur_unit = unit;
-        const int chq = kbase + (wt % (K / 4)) * 4;
+        const int chq = kbase + (wt % C::NQ) * 4;
 #pragma unroll
         for (int tap = 0; tap < 4; ++tap) {
           const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(p.conv_w + tap * p.D + chq));
@@ -460,14 +504,36 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
       RG_WAIT_OR_ABORT(&b_empty[s], ((i / NS) & 1) ^ 1);
       RG_WAIT_OR_ABORT(&u_empty[s], ((i / NS) & 1) ^ 1);
       dec_conv<K, N>(p, sX + xb * C::kXBytes, sB + s * C::kBBytes, sU + s * C::kUBytes, kbase,
-                     own_lo, tile * N, wt, cwq);
+                     own_lo, koff, tile * N, wt, cwq);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {                              // per warp: no barrier to strand an aborting warp at
         mbar_arrive(&x_empty[xb]);
-        mbar_arrive(&b_full[s]);
+        if (kPair) {
+          // this warp's rows of both 64-channel blocks of the unit go to the
+          // same place in the partner's slot by bulk copy, completing there on
+          // b_full; here the arrival expects the partner's matching rows
+          constexpr uint32_t kRowBytes = C::SEG * 128;
+#pragma unroll
+          for (int kb = 0; kb < 2; ++kb) {
+            const uint32_t off =
+                static_cast<uint32_t>(s * C::kBBytes + ((koff >> 6) + kb) * N * 128) + seg_off;
+            bulk_copy_to_cluster(sB_peer + off, smem_u32(sB) + off, kRowBytes,
+                                 bfull_peer + static_cast<uint32_t>(s * 8));
+          }
+          mbar_arrive_expect_tx(&b_full[s], 2u * kRowBytes);
+        } else {
+          mbar_arrive(&b_full[s]);
+        }
         mbar_arrive(&job_empty[js]);
       }
+    }
+    if (kPair) {
+      // the last B slots' releases are commits of both CTAs' MMAs arriving here
+      // (and they follow the partner's reads of this CTA's copies): let them
+      // land before this CTA can exit
+      for (int j = i - NS > 0 ? i - NS : 0; j < i; ++j)
+        mbar_wait_drain(&b_empty[j % NS], (j / NS) & 1, kDrainNs);
     }
   } else if (warp < 6 + 4 * NE) {
     // ============================ epilogue warpgroups ============================
@@ -554,23 +620,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
 #undef RG_WAIT_OR_ABORT
 
   tc_fence_before();
-  __syncthreads();
+  // neither CTA of a pair exits while the other may still copy into its
+  // shared memory or arrive on its barriers
+  if (kPair)
+    cluster_sync();
+  else
+    __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
-}
-
-// ring[:, pos % 3, :] <- x_t, 8 channels per thread (heads 256 wide).
-__global__ void ring_update_kernel(const __nv_bfloat16 *__restrict__ x_t,
-                                   __nv_bfloat16 *__restrict__ ring, int B, int D, int pos) {
-  const size_t n8 = static_cast<size_t>(B) * D / 8;
-  const int s0 = pos % 3;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const size_t e = i * 8;
-    const size_t b = e / D, d = e - b * D;
-    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(x_t) + i);
-    *reinterpret_cast<uint4 *>(ring + (b * 3 + s0) * D + d) = v;
-  }
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 dec_encode_fn() {
@@ -597,10 +654,10 @@ cudaError_t launch_dec_t(const DecArgs &a, cudaStream_t st) {
   const int R = bw <= 128 ? bw : 256;
   CUtensorMap twa, twx, txt, tring;
   {
-    // x_t (B, D): box K channels x N rows
+    // x_t (B, D): box kXK channels x N rows
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.D), static_cast<cuuint64_t>(a.B)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.D) * 2};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(K), static_cast<cuuint32_t>(N)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(C::kXK), static_cast<cuuint32_t>(N)};
     cuuint32_t es[2] = {1, 1};
     if (enc(&txt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(a.x_t), dims, strides,
             box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -608,10 +665,10 @@ cudaError_t launch_dec_t(const DecArgs &a, cudaStream_t st) {
       return cudaErrorInvalidValue;
   }
   {
-    // ring (B, 3, D): box K channels x 1 slot x N rows
+    // ring (B, 3, D): box kXK channels x 1 slot x N rows
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(a.D), 3, static_cast<cuuint64_t>(a.B)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(a.D) * 2, static_cast<cuuint64_t>(a.D) * 6};
-    cuuint32_t box[3] = {static_cast<cuuint32_t>(K), 1, static_cast<cuuint32_t>(N)};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(C::kXK), 1, static_cast<cuuint32_t>(N)};
     cuuint32_t es[3] = {1, 1, 1};
     if (enc(&tring, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.conv_state, dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -648,40 +705,57 @@ cudaError_t launch_dec_t(const DecArgs &a, cudaStream_t st) {
   p.n_cg = a.D / kM;
   p.n_tiles = ceil_div(a.B, N);
   p.n_jobs = p.n_cg * p.n_tiles;
-  p.write_ring = bw <= 128 ? 1 : 0;
+  // every CTA is the only reader of its own channels' ring slot (heads up to
+  // 128 wide, and CTA pairs), so it rewrites that slot itself
+  p.write_ring = 1;
   auto kern = decode_tc_kernel<K, N>;
-  // per device, once: the kernel's shared-memory opt-in and the SM count (no
-  // attribute call on later steps, which may be captured in a CUDA graph)
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = st;
+  if (C::kPair) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  // per device, once: the kernel's shared-memory opt-in and how many CTAs (CTA
+  // pairs) are resident at once (no attribute call on later steps, which may be
+  // captured in a CUDA graph)
   constexpr int kMaxDev = 64;
-  static std::atomic<int> sms_of[kMaxDev];
+  static std::atomic<int> slots_of[kMaxDev];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  int sms = dev < kMaxDev ? sms_of[dev].load(std::memory_order_acquire) : 0;
-  if (sms == 0) {
+  int slots = dev < kMaxDev ? slots_of[dev].load(std::memory_order_acquire) : 0;
+  if (slots == 0) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
+    int sms = 0;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
       return e;
-    if (dev < kMaxDev) sms_of[dev].store(sms, std::memory_order_release);
+    slots = sms;
+    if (C::kPair) {
+      cfg.gridDim = dim3(2 * (sms / 2));
+      if ((e = cudaOccupancyMaxActiveClusters(&slots, kern, &cfg)) != cudaSuccess) return e;
+      if (slots < 1) return cudaErrorNotSupported;
+    }
+    if (dev < kMaxDev) slots_of[dev].store(slots, std::memory_order_release);
   }
-  const int grid = p.n_jobs < sms ? p.n_jobs : sms;
-  kern<<<grid, C::kThreads, C::kSmemBytes, st>>>(twa, twx, txt, tring, p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess || p.write_ring) return e;
-  const size_t n8 = static_cast<size_t>(a.B) * a.D / 8;
-  const int blocks = static_cast<int>((n8 + 255) / 256 < 4 * static_cast<size_t>(sms)
-                                          ? (n8 + 255) / 256
-                                          : 4 * static_cast<size_t>(sms));
-  ring_update_kernel<<<blocks, 256, 0, st>>>(p.x_t, p.ring, a.B, a.D, a.pos);
-  return cudaGetLastError();
+  const int items = C::kPair ? p.n_jobs / 2 : p.n_jobs;
+  const int groups = items < slots ? items : slots;
+  cfg.gridDim = dim3(C::kPair ? 2 * groups : groups);
+  return cudaLaunchKernelEx(&cfg, kern, twa, twx, txt, tring, p);
 }
 
 }  // namespace
 
 bool tc_decode_supported(int B, int D, int H, int io) { return tc_supported(B, 1, D, H, io); }
 
-int tc_decode_launches(int D, int H) { return D / H == 256 ? 2 : 1; }
+int tc_decode_launches(int D, int H) { return D > 0 && H > 0 ? 1 : 0; }
 
 cudaError_t launch_decode_tc(const DecArgs &a, cudaStream_t st) {
   const int bw = a.D / a.H;

@@ -40,6 +40,29 @@ __device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t caddr) {
                : "memory");
 }
 
+// Bulk copy (async proxy) of `bytes` from this CTA's shared memory to a CTA of
+// the cluster (dst: shared::cluster address); the destination's mbarrier (bar,
+// shared::cluster address in that CTA) receives complete_tx of the bytes.
+// Addresses 16-byte aligned, bytes a multiple of 16. The source must have been
+// written before a fence_proxy_async_smem.
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, uint32_t src, uint32_t bytes,
+                                                     uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst), "r"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// As mma_commit (one CTA's own MMAs, cta_group::1), arriving on the mbarrier at
+// `bar`'s offset in every CTA of `cta_mask` (bit r = cluster rank r).
+__device__ __forceinline__ void mma_commit_multicast(uint64_t *bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
+}
+
 // Every thread of both CTAs arrives (release) and waits (acquire); the
 // non-aligned form, so that a warp's threads need not be converged.
 __device__ __forceinline__ void cluster_sync() {
