@@ -583,6 +583,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
           uu[4 * q + 3] = v.w;
         }
         tmem_wait_ld();
+        if (ch == N / 16 - 1) {
+          // the job's accumulator and u tile are in registers: hand both slots
+          // back before the gate math and the global stores
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&u_empty[s]);
+            mbar_arrive(&tmem_empty[ts]);
+          }
+        }
 #pragma unroll
         for (int pr = 0; pr < 8; ++pr) {
           const int n = ch * 16 + 2 * pr;
@@ -608,13 +618,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_wa,
           }
         }
       }
-      tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&u_empty[s]);
-        mbar_arrive(&tmem_empty[ts]);
-        mbar_arrive(&job_empty[js]);
-      }
+      if (lane == 0) mbar_arrive(&job_empty[js]);
     }
   }
 #undef RG_WAIT_OR_ABORT
