@@ -80,10 +80,11 @@ struct DCfg {
   static constexpr int kXK = kPair ? kM : K;       // channels of an input tile
   static constexpr int kInBytes = N * kXK * 2;     // one input tile: N rows x kXK channels, bf16
   static constexpr int kXBytes = 4 * kInBytes;     // x_t and ring slots pos, pos+1, pos+2 (mod 3)
-  static constexpr int kNX = kPair ? 4 : 2;        // input slots
+  static constexpr int kNX = kPair ? 3 : 2;        // input slots
   static constexpr int kBBytes = N * K * 2;
   static constexpr int kUBytes = N * kM * 4;
-  static constexpr int kNS = 2;
+  // B operand and u tile slots (a pair's third slot absorbs the partner's lag)
+  static constexpr int kNS = kPair ? 3 : 2;
   static constexpr int kNT = NE + 1;
   static constexpr int kOffA = 0;
   static constexpr int kOffX = 2 * kABytes;
