@@ -42,7 +42,7 @@ namespace {
 using namespace tc;
 
 #ifndef RGLRU_GEMM_NE
-#define RGLRU_GEMM_NE 2
+#define RGLRU_GEMM_NE 4
 #endif
 constexpr int kBM = 128, kBN = 256, kBK = 64, kStages = 4;
 constexpr int kNE = RGLRU_GEMM_NE;                    // epilogue warpgroups (256 / kNE columns each)
