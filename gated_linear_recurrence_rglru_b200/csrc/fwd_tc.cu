@@ -93,6 +93,8 @@ struct Cfg {
   // shared memory for the pipeline (written by the conv warpgroup)
   static constexpr bool kATmem = (K == 256);
   static constexpr int kABytes = kATmem ? 0 : K * 256;     // one gate: 2 M-blocks x K rows x 128 B
+  // staging of one gate's weights (TMA, 128-byte swizzle) on its way into TMEM
+  static constexpr int kWBytes = kATmem ? K * 256 : 0;
   static constexpr int kBBytes = N * K * 2;        // K-major conv output, one slot
   // fp32 u of the unit's own channels, channel-major [128][N], for beta
   static constexpr int kUBytes = N * kM * 4;
@@ -103,13 +105,14 @@ struct Cfg {
   // TMEM slots: one per epilogue warpgroup and one for the MMA to run ahead
   static constexpr int kNT = NE + 1;
   static constexpr int kOffA = 0;
-  static constexpr int kOffX = 2 * kABytes;
+  static constexpr int kOffW = 2 * kABytes;
+  static constexpr int kOffX = kOffW + kWBytes;
   static constexpr int kOffB = kOffX + NX * kXBytes;
   static constexpr int kOffU = kOffB + kNS * kBBytes;
   static constexpr int kOffBar = kOffU + kNU * kUBytes;
   // job_full[JQ], job_empty[JQ], x_full[NX], x_empty[NX], w_full, w_free,
-  // b_full[NS], b_empty[NS], u_empty[NU], acc_full[NT], tmem_empty[NT], a_ready
-  static constexpr int kNumBars = 2 * kJQ + 2 * NX + 2 + 2 * kNS + kNU + 2 * kNT + 1;
+  // b_full[NS], b_empty[NS], u_empty[NU], acc_full[NT], tmem_empty[NT], a_ready, w_mid
+  static constexpr int kNumBars = 2 * kJQ + 2 * NX + 2 + 2 * kNS + kNU + 2 * kNT + 2;
   static constexpr int kOffJobs = (kOffBar + kNumBars * 8 + 15) / 16 * 16;
   static constexpr int kOffMisc = kOffJobs + kJQ * 16;
   // the dynamic shared memory base is declared 1024-byte aligned (the kernel
@@ -278,6 +281,13 @@ __device__ __forceinline__ void conv_tile(const unsigned char *__restrict__ xs,
   }
 }
 
+// One 16-bit shared-memory load (zero-extended).
+__device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a) : "memory");
+  return v;
+}
+
 // Pass 2 of one tile for one channel (this thread's TMEM lane): y_t =
 // P_t h_in + Hl_t for the valid tokens, stored bf16 at a row stride of kD
 // channels (a compile-time stride for the common widths, so that the 16
@@ -325,6 +335,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
   }
   unsigned char *sm = smem_raw;
   unsigned char *sA = sm + C::kOffA;
+  unsigned char *sW = sm + C::kOffW;
   unsigned char *sX = sm + C::kOffX;
   unsigned char *sB = sm + C::kOffB;
   unsigned char *sU = sm + C::kOffU;
@@ -341,10 +352,14 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
   uint64_t *acc_full = u_empty + NUS;               // [NT] MMA -> epilogue
   uint64_t *tmem_empty = acc_full + NT;             // [NT] epilogue pass 2 -> MMA
   uint64_t *a_ready = tmem_empty + NT;              // conv warpgroup wrote TMEM weights -> MMA
+  uint64_t *w_mid = a_ready + 1;                    // staged gate a read (TMEM weights)
   int4 *jobs = reinterpret_cast<int4 *>(sm + C::kOffJobs);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + C::kOffMisc);
   volatile int *cta_abort = reinterpret_cast<volatile int *>(sm + C::kOffMisc + 4);
   volatile int *bcast = reinterpret_cast<volatile int *>(sm + C::kOffMisc + 8);  // [NE][2]
+  // phases of w_full armed so far (producer and conv warpgroup): an aborting CTA
+  // waits for the last one before it exits, so that no weight copy is in flight
+  int *w_armed = reinterpret_cast<int *>(sm + C::kOffMisc + 48);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -360,7 +375,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
       mbar_init(&x_empty[i], 4);                    // 4 conv warps, or 4 epilogue warps
     }
     mbar_init(w_full, 1);
-    mbar_init(w_free, 1);
+    // shared-memory weights: the MMA thread; TMEM weights: the conv warps' copy
+    mbar_init(w_free, C::kATmem ? 4 : 1);
     for (int i = 0; i < NS; ++i) {
       mbar_init(&b_full[i], 4);                     // 4 conv warps
       mbar_init(&b_empty[i], 1);
@@ -371,7 +387,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
       mbar_init(&tmem_empty[i], 4);                 // 4 epilogue warps
     }
     mbar_init(a_ready, 4);                          // 4 conv warps
+    mbar_init(w_mid, 4);                            // 4 conv warps
     *cta_abort = 0;
+    *w_armed = 0;
     fence_mbar_init();
     prefetch_tmap(&tmap_x);
     prefetch_tmap(&tmap_wa);
@@ -485,6 +503,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
             wfree_phase ^= 1;
           }
           if (lane == 0) {
+            atomicAdd(w_armed, 1);
             mbar_arrive_expect_tx(w_full, 2u * 2u * static_cast<uint32_t>(R) * 128u);
             for (int g = 0; g < 2; ++g) {
               const CUtensorMap *tm = g == 0 ? &tmap_wa : &tmap_wx;
@@ -502,6 +521,21 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
                               (cg >> 1) * 256);
               }
             }
+          }
+        }
+        if (reload && C::kATmem) {
+          // gate a of the new unit into the staging buffer, ahead of its job; the
+          // conv warpgroup copies it into TMEM, then stages gate x itself
+          if (i > 0) {
+            RG_WAIT_OR_ABORT(w_free, wfree_phase);  // the previous unit's staging is copied
+            wfree_phase ^= 1;
+          }
+          if (lane == 0) {
+            atomicAdd(w_armed, 1);
+            mbar_arrive_expect_tx(w_full, static_cast<uint32_t>(C::kWBytes));
+            for (int ma = 0; ma < 2; ++ma)
+              tma_load_2d(sW + ma * (K * 128), &tmap_wa, w_full, (cg & 1) * 128 + 64 * ma,
+                          (cg >> 1) * 256);
           }
         }
         if (reload) w_unit = unit;
@@ -586,6 +620,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
     constexpr int wait_site = kSiteConv;
     const int wt = tid - 64;                      // 0 .. 127
     int cur_unit = -1;
+    uint32_t wfull_phase = 0, wmid_phase = 0;     // staged-weight barriers (TMEM weights)
     float2 cwq[4][2];                             // conv taps of this thread's channel quad
     for (int i = 0;; ++i) {
       const int js = i % kJQ;
@@ -609,36 +644,72 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
         if (C::kATmem) {
           // This unit's gate weights into TMEM (the A operand): lane m (output
           // channel cg*128 + m) holds W[h][k][j] for k = 0..K-1, two per column.
-          // Every MMA of earlier jobs has read the old weights once the
-          // accumulator of job i-1 is complete (MMAs complete in issue order).
+          // Each gate comes through the staging buffer (TMA, 128-byte swizzle,
+          // MN-major: per 64-channel block ma, row k of 128 B, 16-byte chunk
+          // (m % 64) / 8 stored at chunk ^ (k % 8); a warp's 32 channels read 64
+          // bytes of one row: no bank conflicts): gate a was staged by the tile
+          // claimer ahead of this job, gate x is staged here once every warp has
+          // copied gate a. Every MMA of earlier jobs has read the old weights once
+          // the accumulator of job i-1 is complete (MMAs complete in issue order).
+          RG_WAIT_OR_ABORT(w_full, wfull_phase);        // gate a staged
+          wfull_phase ^= 1;
           if (i > 0) RG_WAIT_OR_ABORT(&acc_full[(i - 1) % NT], ((i - 1) / NT) & 1);
           const int qd = warp & 3;                  // this warp's TMEM lane quadrant
-          const int cout = cg * kM + qd * 32 + lane;
-          const int hh = cout / p.bw, jj = cout % p.bw;
+          const int m = qd * 32 + lane;             // output channel within the unit
           const uint32_t tq = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) +
                               static_cast<uint32_t>(C::kACol);
+          const uint32_t wsrc = smem_u32(sW) +
+                                static_cast<uint32_t>((m >> 6) * (K * 128) + ((m & 7) << 1));
+          const uint32_t mchunk = static_cast<uint32_t>((m & 63) >> 3);
+          bool ok = true;
 #pragma unroll 1
-          for (int g = 0; g < 2; ++g) {
-            const unsigned short *Wg =
-                reinterpret_cast<const unsigned short *>(g == 0 ? p.W_a : p.W_x) +
-                static_cast<size_t>(hh) * p.bw * p.bw + jj;
+          for (int g = 0; g < 2 && ok; ++g) {
+            if (g == 1) {
+              // every warp has read gate a: one thread stages gate x
+              __syncwarp();
+              if (lane == 0) mbar_arrive(w_mid);
+              if (warp == 2 && lane == 0) {
+                if (mbar_wait(w_mid, wmid_phase, cta_abort, p.wait_ns)) {
+                  atomicAdd(w_armed, 1);
+                  mbar_arrive_expect_tx(w_full, static_cast<uint32_t>(C::kWBytes));
+                  for (int ma = 0; ma < 2; ++ma)
+                    tma_load_2d(sW + ma * (K * 128), &tmap_wx, w_full, (cg & 1) * 128 + 64 * ma,
+                                (cg >> 1) * 256);
+                } else if (!*cta_abort) {
+                  raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT, wait_site);
+                }
+              }
+              __syncwarp();                         // warp 2's lane 0 rejoins its warp
+              wmid_phase ^= 1;
+              ok = mbar_wait(w_full, wfull_phase, cta_abort, p.wait_ns);   // gate x staged
+              wfull_phase ^= 1;
+              if (!ok) break;
+            }
+            __syncwarp();                           // tcgen05.st is warp-collective
 #pragma unroll 1
             for (int cc = 0; cc < K / 64; ++cc) {
               uint32_t v[32];
 #pragma unroll
               for (int q = 0; q < 32; ++q) {
-                const int k = cc * 64 + 2 * q;
-                const uint32_t lo = __ldg(Wg + static_cast<size_t>(k) * p.bw);
-                const uint32_t hi = __ldg(Wg + static_cast<size_t>(k + 1) * p.bw);
+                const uint32_t k = static_cast<uint32_t>(cc * 64 + 2 * q);   // even: k % 8 = 2q % 8
+                const uint32_t lo = lds_u16(wsrc + k * 128 + ((mchunk ^ (k & 7)) << 4));
+                const uint32_t hi = lds_u16(wsrc + (k + 1) * 128 + ((mchunk ^ ((k + 1) & 7)) << 4));
                 v[q] = lo | (hi << 16);
               }
               tmem_st32u(tq + static_cast<uint32_t>(g * (K / 2) + cc * 32), v);
             }
           }
+          if (!ok) {
+            if (!*cta_abort) raise_abort(p, cta_abort, RGLRU_ERR_TIMEOUT, wait_site);
+            break;
+          }
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(a_ready);
+          if (lane == 0) {
+            mbar_arrive(a_ready);
+            mbar_arrive(w_free);                    // the staging buffer may be reloaded
+          }
         }
       }
       const int s = i % NS, xb = i % NX, us = i % NUS;
@@ -848,6 +919,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (tid == 0 && *cta_abort && *w_armed > 0)
+    mbar_wait_drain(w_full, static_cast<uint32_t>(*w_armed - 1) & 1u, kDrainNs);
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
 }
 
