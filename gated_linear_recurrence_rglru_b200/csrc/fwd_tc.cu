@@ -74,6 +74,7 @@ struct TcParams {
   int B, T, D, H, bw;
   int n_cg, n_units, n_tiles;
   int *counters, *abort_flag;
+  int *workers;                    // per unit: CTAs currently claiming its tiles (a heuristic)
   unsigned long long *carry;       // [unit][tile][128] carry words (see carry_word)
   int *dev_status;
   uint64_t wait_ns;                // bound of every wait
@@ -429,6 +430,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
     {
       int unit = blockIdx.x % p.n_units, w_unit = -1;
       int i = 0, last_x_job = -1;
+      if (lane == 0) atomicAdd(&p.workers[unit], 1);
       uint32_t wfree_phase = 0;
       for (;; ++i) {
         const int js = i % kJQ, xb = i % NX;
@@ -443,26 +445,31 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
             tile = t;
             break;
           }
-          // this unit is done: continue on the unit with the most tiles left,
-          // ties broken by distance from a per-CTA starting point so that the
-          // CTAs that run out at the same time spread over the units (the
-          // counters are read from L2 without ordering: a stale value only
-          // makes a worse choice, the claim itself is the atomic)
+          // this unit is done: join the unit that would finish last, the one
+          // with the most tiles left per CTA claiming it (with this one), so
+          // that units end together and CTAs change unit (a TMEM weight reload
+          // and a pipeline drain for 256-wide heads) as rarely as possible;
+          // ties broken by distance from a per-CTA starting point. Counters and
+          // worker counts are read from L2 without ordering: a stale value only
+          // makes a worse choice, the claim itself is the atomic.
+          if (lane == 0) atomicSub(&p.workers[unit], 1);
           const int rot = static_cast<int>((blockIdx.x * 37u) % static_cast<unsigned>(p.n_units));
-          unsigned key = 0;                       // (tiles left << 16) | (65535 - distance)
+          unsigned key = 0;                       // (16 x tiles left per CTA << 16) | (65535 - distance)
           for (int u0 = 0; u0 < p.n_units; u0 += 128) {
-            int l[4];
+            int l[4], wk[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const int u = u0 + q * 32 + lane;
               l[q] = u < p.n_units ? p.n_tiles - __ldcg(p.counters + u) : 0;
+              wk[q] = u < p.n_units ? __ldcg(p.workers + u) : 0;
             }
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const int u = u0 + q * 32 + lane;
               if (l[q] > 0) {
                 const int dist = u >= rot ? u - rot : u + p.n_units - rot;
-                const unsigned k = (static_cast<unsigned>(min(l[q], 32767)) << 16) |
+                const int per = min(l[q] * 16 / (max(wk[q], 0) + 1), 65535);
+                const unsigned k = (static_cast<unsigned>(per) << 16) |
                                    static_cast<unsigned>(65535 - min(dist, 65535));
                 key = max(key, k);
               }
@@ -474,6 +481,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
           } else {
             const int dist = 65535 - static_cast<int>(key & 0xFFFFu);
             unit = rot + dist < p.n_units ? rot + dist : rot + dist - p.n_units;
+            if (lane == 0) atomicAdd(&p.workers[unit], 1);
           }
         }
         unit = __shfl_sync(0xffffffffu, *cta_abort ? -1 : unit, 0);
@@ -944,7 +952,7 @@ int tile_tokens(int bw) { return bw == 256 ? 32 : 64; }
 
 struct TcLayout {
   int n_cg, n_units, n_tiles;
-  size_t off_counters, off_abort, off_carry, total;
+  size_t off_counters, off_workers, off_abort, off_carry, total;
 };
 
 TcLayout tc_layout(int B, int T, int D, int H) {
@@ -954,7 +962,8 @@ TcLayout tc_layout(int B, int T, int D, int H) {
   L.n_units = B * L.n_cg;
   L.n_tiles = ceil_div(T, tile_tokens(bw));
   L.off_counters = 0;
-  L.off_abort = static_cast<size_t>(L.n_units) * 4;
+  L.off_workers = static_cast<size_t>(L.n_units) * 4;
+  L.off_abort = L.off_workers + static_cast<size_t>(L.n_units) * 4;
   L.off_carry = align_up(L.off_abort + 4, 256);
   // one 8-byte carry word per (unit, tile, channel); all of it starts at zero
   L.total = align_up(L.off_carry + static_cast<size_t>(L.n_units) * L.n_tiles * kM * 8, 256);
@@ -1015,6 +1024,7 @@ cudaError_t launch_tc_t(const FwdArgs &a, const TcLayout &L, void *ws, cudaStrea
   p.n_tiles = L.n_tiles;
   p.counters = reinterpret_cast<int *>(w + L.off_counters);
   p.abort_flag = reinterpret_cast<int *>(w + L.off_abort);
+  p.workers = reinterpret_cast<int *>(w + L.off_workers);
   p.carry = reinterpret_cast<unsigned long long *>(w + L.off_carry);
   p.dev_status = a.dev_status;
   p.wait_ns = a.wait_ns ? a.wait_ns : kWaitNs;
