@@ -18,8 +18,9 @@
 //      pre-activations along time. The weights sit in shared memory for heads
 //      up to 128 wide (TMA, 128-byte swizzle, block-diagonal zeros for 64-wide
 //      heads) and in TMEM for 256-wide heads, where both gates (128 KB) would
-//      leave no shared memory for the pipeline (the conv warpgroup writes them
-//      there at each change of unit);
+//      leave no shared memory for the pipeline (at each change of unit each gate
+//      comes through a 64 KB shared-memory staging buffer by TMA and the conv
+//      warpgroup copies it into TMEM);
 //   3. an epilogue warpgroup, per lane (channel): sigmoid gates, log-space
 //      decay, sqrt(1 - a^2) and a local scan along time from a zero state,
 //      keeping the running products P_t = a_1 ... a_t and local states Hl_t
@@ -30,8 +31,9 @@
 //      parallel scans"), parallel across tiles;
 //   5. writes y_t = P_t h_in + Hl_t from the carried state h_in (pass 2, no
 //      dependency between tokens).
-// Roles: warp 0 claims tiles (per-unit counters in time order, stealing from
-// other units once its own is done) and issues TMA; warp 1 owns TMEM and
+// Roles: warp 0 claims tiles (per-unit counters in time order; once its own
+// unit is done, joining the unit with the most tiles left per CTA claiming it)
+// and issues TMA; warp 1 owns TMEM and
 // issues the MMAs; warps 2-5 compute the Conv1D of every job; NE epilogue
 // warpgroups take the jobs round robin, connected by mbarriers. Tiles
 // of a unit are claimed in time order by running CTAs only, so every
