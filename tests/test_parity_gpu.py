@@ -80,6 +80,9 @@ SMALL = [
     # a 32-token tile with several rows and heads
     WORKLOADS["hawk_block"].with_shape(B=2, T=2, D=512, H=2, h0_var=1.0, seed=43),
     WORKLOADS["hawk_block"].with_shape(B=3, T=33, D=1024, H=4, bias_std=0.5, seed=44),
+    # 256-wide heads, 144 units of 7 tiles on 148 CTAs: CTAs steal from one another's
+    # units and reload the staged TMEM weights many times
+    WORKLOADS["griffin2b"].with_shape(B=24, T=200, D=768, H=3, bias_std=0.5, seed=46),
 ]
 
 
