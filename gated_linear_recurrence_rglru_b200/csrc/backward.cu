@@ -539,7 +539,17 @@ __global__ void bwd_carry_kernel(int B, int D, int nseg, const float *__restrict
 // of time (sza, szx, sdy: this thread's channel at token 0 of the group, rows
 // sstride elements apart, zeros past t1); else they are read from the
 // workspace and dy in global memory, with an L1 prefetch of the next group.
-template <typename T, bool kStaged, typename Sink>
+// d W tiles: 64 x 64 (i, j) per block (both d W kernels)
+constexpr int kDwTile = 64;
+
+// bf16 copies of u, d z_a and d z_x for the tensor-core d W (which reads its
+// operands as bf16): stored by K3 with the same round-to-nearest, so d W is the
+// same while these streams move half the bytes of fp32 ones.
+struct Bf16Streams {
+  __nv_bfloat16 *u, *dza, *dzx;
+};
+
+template <typename T, bool kStaged, bool kB16, typename Sink>
 __device__ __forceinline__ void final_group(const BwdThread &th, const ChanC &c, const T *xb,
                                             const T *cs_in_b, const T *dyb, size_t orow, int D,
                                             int tb, size_t go, float h_in,
@@ -549,7 +559,7 @@ __device__ __forceinline__ void final_group(const BwdThread &th, const ChanC &c,
                                             float *__restrict__ ws_u, float &gc, float &acc_q,
                                             float &acc_ba, float &acc_bx, float (&dub)[kTB],
                                             const float *sza, const float *szx, const T *sdy,
-                                            int sstride, Sink sink) {
+                                            int sstride, const Bf16Streams &b16, Sink sink) {
   const float neg_c_sp = -kDecayC * c.sp, csp = kDecayC * c.sp;
   if (!kStaged && tb - kTB >= th.t0) {
     // the group processed next (8 tokens earlier): its z and dy rows
@@ -580,7 +590,12 @@ __device__ __forceinline__ void final_group(const BwdThread &th, const ChanC &c,
       za = in ? ws_za[o] : 0.f;
       zx = in ? ws_zx[o] : 0.f;
     }
-    if (in) ws_u[o] = u[k];
+    if (in) {
+      if constexpr (kB16)
+        b16.u[o] = __float2bfloat16_rn(u[k]);
+      else
+        ws_u[o] = u[k];
+    }
     const TokGates tg = tok_gates(za, zx, neg_c_sp);
     const float r = tg.r, ig = tg.i, a = tg.a, gg = tg.g, rog = tg.rog;
     const float q = a * (a * ig * u[k] * rog - hh * r);
@@ -609,8 +624,13 @@ __device__ __forceinline__ void final_group(const BwdThread &th, const ChanC &c,
       acc_ba += dza;
       acc_bx += dzx;
       gc = fa[k] * G;
-      ws_za[o] = dza;
-      ws_zx[o] = dzx;
+      if constexpr (kB16) {
+        b16.dza[o] = __float2bfloat16_rn(dza);
+        b16.dzx[o] = __float2bfloat16_rn(dzx);
+      } else {
+        ws_za[o] = dza;
+        ws_zx[o] = dzx;
+      }
     }
     sink(k, dza, dzx);
   }
@@ -658,9 +678,10 @@ bwd_final_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
     float dub[kTB];
     if (live) {
       const size_t go = ((size_t)b * ngt + tb / kTB) * D + th.d;
-      final_group<T, false>(th, c, xb, cs_in_b, dyb, orow, D, tb, go, h_in, ws_gP, ws_gH, ws_za,
-                            ws_zx, ws_u, gc, acc_q, acc_ba, acc_bx, dub, nullptr, nullptr,
-                            nullptr, 0, [&](int k, float dza, float dzx) {
+      final_group<T, false, false>(th, c, xb, cs_in_b, dyb, orow, D, tb, go, h_in, ws_gP, ws_gH,
+                                   ws_za, ws_zx, ws_u, gc, acc_q, acc_ba, acc_bx, dub, nullptr,
+                                   nullptr, nullptr, 0, Bf16Streams{},
+                                   [&](int k, float dza, float dzx) {
                               dza_row[k] = dza;
                               dzx_row[k] = dzx;
                             });
@@ -708,7 +729,7 @@ bwd_final_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
 // its channel's 8 tokens to its own part of d u.
 template <int kBW>
 __global__ void __launch_bounds__(TcGeo<kBW>::kThreads, kBW == 128 ? 1 : 2)
-bwd_final_tc_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
+bwd_final_tc_kernel(BwdArgs p, BwdPlan pl, Bf16Streams b16, const float *__restrict__ ws_hin,
                     const float *__restrict__ ws_C, const float *__restrict__ ws_gP,
                     const float *__restrict__ ws_gH, float *__restrict__ ws_za,
                     float *__restrict__ ws_zx, float *__restrict__ ws_u,
@@ -803,9 +824,11 @@ bwd_final_tc_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
     if (live) {
       const size_t go = ((size_t)b * ngt + tb / kTB) * D + th.d;
       const int srow = ((buf * G::S + th.sl) * kTB) * kBW + th.j;
-      final_group<T, true>(th, c, xb, cs_in_b, dyb, orow, D, tb, go, h_in, ws_gP, ws_gH, ws_za,
-                           ws_zx, ws_u, gc, acc_q, acc_ba, acc_bx, dub, za_st + srow,
-                           zx_st + srow, dy_st + srow, kBW, [&](int k, float dza, float dzx) {
+      final_group<T, true, kBW % kDwTile == 0>(th, c, xb, cs_in_b, dyb, orow, D, tb, go, h_in,
+                                               ws_gP, ws_gH, ws_za, ws_zx, ws_u, gc, acc_q,
+                                               acc_ba, acc_bx, dub, za_st + srow, zx_st + srow,
+                                               dy_st + srow, kBW, b16,
+                                               [&](int k, float dza, float dzx) {
                              dza_col[k * G::kStride] = __float2bfloat16_rn(dza);
                              dzx_col[k * G::kStride] = __float2bfloat16_rn(dzx);
                            });
@@ -867,7 +890,7 @@ bwd_final_tc_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
 // tokens: a 64 x 64 tile of (i, j) of one gate and head per block, 4 x 4 per
 // thread, 32 tokens of both operands staged in shared memory at a time (the
 // next 32 already in flight to registers).
-constexpr int kDwTile = 64, kDwRows = 32, kDwThreads = 256;
+constexpr int kDwRows = 32, kDwThreads = 256;
 
 __global__ void __launch_bounds__(kDwThreads)
 bwd_dw_kernel(const float *__restrict__ U, const float *__restrict__ dZa,
@@ -944,13 +967,6 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&a)[4]) {
                : "r"(addr));
 }
 
-__device__ __forceinline__ uint2 f4_to_bf16x4(float4 v) {
-  const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
-  const __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
-  return make_uint2(*reinterpret_cast<const uint32_t *>(&lo),
-                    *reinterpret_cast<const uint32_t *>(&hi));
-}
-
 // d W on the tensor cores (bf16 I/O, heads a multiple of 64 wide): the same
 // 64 x 64 (i, j) tiles and token chunks as bwd_dw_kernel, 4 warps each a
 // 32 x 32 quarter. 32 tokens of U and dZ are staged as bf16 token-major rows
@@ -961,9 +977,9 @@ __device__ __forceinline__ uint2 f4_to_bf16x4(float4 v) {
 constexpr int kDwTcThreads = 128, kDwTcStride = kDwTile + 8;
 
 __global__ void __launch_bounds__(kDwTcThreads)
-bwd_dw_tc_kernel(const float *__restrict__ U, const float *__restrict__ dZa,
-                 const float *__restrict__ dZx, float *__restrict__ dWa, float *__restrict__ dWx,
-                 int N, int D, int H, int chunk) {
+bwd_dw_tc_kernel(const __nv_bfloat16 *__restrict__ U, const __nv_bfloat16 *__restrict__ dZa,
+                 const __nv_bfloat16 *__restrict__ dZx, float *__restrict__ dWa,
+                 float *__restrict__ dWx, int N, int D, int H, int chunk) {
   __shared__ __align__(16) __nv_bfloat16 us[kDwRows][kDwTcStride];
   __shared__ __align__(16) __nv_bfloat16 zs[kDwRows][kDwTcStride];
   const int bw = D / H;
@@ -972,24 +988,24 @@ bwd_dw_tc_kernel(const float *__restrict__ U, const float *__restrict__ dZa,
   const int gate = tile & 1;
   tile >>= 1;
   const int ti = tile % tiles, tj = (tile / tiles) % tiles, h = tile / (tiles * tiles);
-  const float *Z = gate == 0 ? dZa : dZx;
+  const __nv_bfloat16 *Z = gate == 0 ? dZa : dZx;
   float *dW = gate == 0 ? dWa : dWx;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int wi = (warp & 1) * 32, wj = (warp >> 1) * 32;
   const int i0 = ti * kDwTile, j0 = tj * kDwTile;
-  // loader: rows lr + 8 q, columns lc .. lc + 3 (16-byte fp32 loads)
+  // loader: rows lr + 8 q, columns lc .. lc + 3 (8-byte bf16 loads)
   const int lr = tid >> 4, lc = (tid & 15) * 4;
-  const float *Uc = U + (size_t)h * bw + i0 + lc;
-  const float *Zc = Z + (size_t)h * bw + j0 + lc;
+  const __nv_bfloat16 *Uc = U + (size_t)h * bw + i0 + lc;
+  const __nv_bfloat16 *Zc = Z + (size_t)h * bw + j0 + lc;
   const int n_begin = blockIdx.y * chunk, n_end = min(N, n_begin + chunk);
-  float4 pu[kDwRows / 8], pz[kDwRows / 8];
+  uint2 pu[kDwRows / 8], pz[kDwRows / 8];
   auto fetch = [&](int n0) {
 #pragma unroll
     for (int q = 0; q < kDwRows / 8; ++q) {
       const int n = n0 + lr + 8 * q;
       const bool ok = n < n_end;
-      pu[q] = ok ? *reinterpret_cast<const float4 *>(Uc + (size_t)n * D) : make_float4(0, 0, 0, 0);
-      pz[q] = ok ? *reinterpret_cast<const float4 *>(Zc + (size_t)n * D) : make_float4(0, 0, 0, 0);
+      pu[q] = ok ? *reinterpret_cast<const uint2 *>(Uc + (size_t)n * D) : make_uint2(0, 0);
+      pz[q] = ok ? *reinterpret_cast<const uint2 *>(Zc + (size_t)n * D) : make_uint2(0, 0);
     }
   };
   // ldmatrix lane rows: A blocks (n-block q / 2, i-block q % 2), B blocks (n-block q % 2,
@@ -1009,8 +1025,8 @@ bwd_dw_tc_kernel(const float *__restrict__ U, const float *__restrict__ dZa,
   for (int n0 = n_begin; n0 < n_end; n0 += kDwRows) {
 #pragma unroll
     for (int q = 0; q < kDwRows / 8; ++q) {
-      *reinterpret_cast<uint2 *>(&us[lr + 8 * q][lc]) = f4_to_bf16x4(pu[q]);
-      *reinterpret_cast<uint2 *>(&zs[lr + 8 * q][lc]) = f4_to_bf16x4(pz[q]);
+      *reinterpret_cast<uint2 *>(&us[lr + 8 * q][lc]) = pu[q];
+      *reinterpret_cast<uint2 *>(&zs[lr + 8 * q][lc]) = pz[q];
     }
     __syncthreads();
     if (n0 + kDwRows < n_end) fetch(n0 + kDwRows);
@@ -1133,7 +1149,9 @@ bwd_conv_kernel(BwdArgs p, const float *__restrict__ du) {
 }
 
 struct BwdLayout {
-  size_t off_A, off_H, off_R, off_hin, off_C, off_gP, off_gH, off_za, off_zx, off_u, off_du, total;
+  size_t off_A, off_H, off_R, off_hin, off_C, off_gP, off_gH, off_za, off_zx, off_u, off_du;
+  size_t off_dzx16;   // bf16 d z_x for the tensor-core d W (bf16 u and d z_a share u's region)
+  size_t total;
 };
 
 BwdLayout bwd_layout(int B, int T, int D, int H) {
@@ -1153,7 +1171,8 @@ BwdLayout bwd_layout(int B, int T, int D, int H) {
   L.off_zx = L.off_za + tok;
   L.off_u = L.off_zx + tok;
   L.off_du = L.off_u + tok;
-  L.total = L.off_du + tok;
+  L.off_dzx16 = L.off_du + tok;
+  L.total = L.off_dzx16 + align_up((size_t)B * T * D * 2, 256);
   return L;
 }
 
@@ -1168,6 +1187,10 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
   float *A = at(Ly.off_A), *Hh = at(Ly.off_H), *R = at(Ly.off_R);
   float *hin = at(Ly.off_hin), *C = at(Ly.off_C), *gP = at(Ly.off_gP), *gH = at(Ly.off_gH);
   float *za = at(Ly.off_za), *zx = at(Ly.off_zx), *U = at(Ly.off_u), *du = at(Ly.off_du);
+  // bf16 u, d z_a (in u's fp32 region, two halves) and d z_x for the tensor-core d W
+  const size_t ntok = (size_t)p.B * p.T * p.D;
+  Bf16Streams b16{reinterpret_cast<__nv_bfloat16 *>(U), reinterpret_cast<__nv_bfloat16 *>(U) + ntok,
+                  reinterpret_cast<__nv_bfloat16 *>(w + Ly.off_dzx16)};
   const size_t D = p.D;
   cudaError_t e;
   // the accumulated gradients start at zero
@@ -1204,8 +1227,8 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
     bwd_carry_kernel<<<ceil_div(bd, 256), 256, 0, st>>>(p.B, p.D, pl.nseg, A, Hh, R, p.h0,
                                                         p.dh_T, hin, C, p.dh0);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    bwd_final_tc_kernel<kTcBW><<<grid, G::kThreads, smem3, st>>>(p, pl, hin, C, gP, gH, za, zx,
-                                                                  U, du);
+    bwd_final_tc_kernel<kTcBW><<<grid, G::kThreads, smem3, st>>>(p, pl, b16, hin, C, gP, gH, za,
+                                                                  zx, U, du);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   } else {
     const size_t wsm = kSW ? 2 * (size_t)bw * (bw + 1) * sizeof(float) : 0;
@@ -1236,9 +1259,9 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
   const int tile_blocks = 2 * tiles * tiles * p.H;
   const int nchunk = ceil_div(8 * 148, tile_blocks);
   const int chunk = ceil_div(ceil_div(N, nchunk), kDwRows) * kDwRows;
-  if (kTcBW > 0 && bw % kDwTile == 0)
+  if (kTcBW > 0 && kTcBW % kDwTile == 0)
     bwd_dw_tc_kernel<<<dim3(tile_blocks, ceil_div(N, chunk)), kDwTcThreads, 0, st>>>(
-        U, za, zx, p.dW_a, p.dW_x, N, p.D, p.H, chunk);
+        b16.u, b16.dza, b16.dzx, p.dW_a, p.dW_x, N, p.D, p.H, chunk);
   else
     bwd_dw_kernel<<<dim3(tile_blocks, ceil_div(N, chunk)), kDwThreads, 0, st>>>(
         U, za, zx, p.dW_a, p.dW_x, N, p.D, p.H, chunk);
