@@ -236,6 +236,10 @@ __device__ __forceinline__ void cp_async_commit() {
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
+// all but this thread's most recently committed group complete
+__device__ __forceinline__ void cp_async_wait_one_pending() {
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
 
 // Gate math of the backward in fp32 with about 1e-6 relative error: sigmoid
 // and exp through the hardware base-2 exponential, approximate reciprocal and
@@ -275,14 +279,17 @@ __device__ __forceinline__ TokGates tok_gates(float za, float zx, float neg_c_sp
 }
 
 // The post-contraction part of a K1 group: decay, input, the local scan and
-// the running R; z_a, z_x of the live tokens to the workspace.
+// the running R; z_a, z_x of the live tokens to the workspace. sdy: the
+// group's dy rows staged in shared memory (this thread's channel at token 0,
+// rows sstride apart), or nullptr to read dy from global memory.
 template <typename T>
 __device__ __forceinline__ void gates_scan_group(const float (&za)[kTB], const float (&zx)[kTB],
                                                  const float (&u)[kTB], int tb, int t1,
                                                  float neg_c_sp, const T *dyb, size_t orow,
                                                  int D, float &P, float &Hl, float &R,
                                                  float *__restrict__ ws_za,
-                                                 float *__restrict__ ws_zx) {
+                                                 float *__restrict__ ws_zx,
+                                                 const T *sdy = nullptr, int sstride = 0) {
 #pragma unroll
   for (int k = 0; k < kTB; ++k) {
     const int t = tb + k;
@@ -291,7 +298,7 @@ __device__ __forceinline__ void gates_scan_group(const float (&za)[kTB], const f
       Hl = fmaf(q.a, Hl, q.g * (q.i * u[k]));
       P *= q.a;
       const size_t o = orow + (size_t)t * D;
-      R = fmaf(P, ldg_f32(dyb + o), R);
+      R = fmaf(P, sdy != nullptr ? to_f32<T>(sdy[k * sstride]) : ldg_f32(dyb + o), R);
       ws_za[o] = za[k];
       ws_zx[o] = zx[k];
     }
@@ -377,7 +384,8 @@ bwd_gates_kernel(BwdArgs p, BwdPlan pl, float *__restrict__ ws_A, float *__restr
 // warp multiplies its two 16-token m-tiles by its 8 columns of W_a and W_x
 // (fragments held in registers for the whole kernel), scatters the fp32
 // results into (segment, channel) rows, and each thread reads back its own
-// channel's 8 tokens for the scan.
+// channel's 8 tokens for the scan. The x and dy rows of a group arrive in
+// shared memory by cp.async two groups ahead of use.
 template <int kBW>
 __global__ void __launch_bounds__(TcGeo<kBW>::kThreads, kBW == 128 ? 1 : 3)
 bwd_gates_tc_kernel(BwdArgs p, BwdPlan pl, float *__restrict__ ws_A, float *__restrict__ ws_H,
@@ -389,6 +397,11 @@ bwd_gates_tc_kernel(BwdArgs p, BwdPlan pl, float *__restrict__ ws_A, float *__re
   extern __shared__ float4 smem_gt[];
   float *z_s = reinterpret_cast<float *>(smem_gt);                        // [S][2][kBW][kRow]
   T *u_s = reinterpret_cast<T *>(z_s + G::S * 2 * kBW * kRow);            // [M][kStride]
+  // x rows tb-3 .. tb+7 and dy rows tb .. tb+7 of each segment's group, a ring of
+  // three slots filled two groups ahead: [3][S][kTB + 3][kBW], [3][S][kTB][kBW]
+  constexpr int XR = kTB + 3;
+  T *xs_st = u_s + G::M * G::kStride;
+  T *dys_st = xs_st + 3 * G::S * XR * kBW;
   const int D = p.D, h = blockIdx.y, b = blockIdx.z;
   const BwdThread th = bwd_thread(p, pl, kBW);
   const T *xb = static_cast<const T *>(p.x) + (size_t)b * p.T * D;
@@ -426,22 +439,70 @@ bwd_gates_tc_kernel(BwdArgs p, BwdPlan pl, float *__restrict__ ws_A, float *__re
   const float *zx_row = z_s + ((th.sl * 2 + 1) * kBW + th.j) * kRow;
   T *u_col = u_s + th.sl * kTB * G::kStride + th.j;
   float P = 1.f, Hl = 0.f, R = 0.f;
+  // Staging of group g into ring slot buf: 16-byte copies (kBW / 8 per row) spread
+  // over the block. x rows before t = 0 come from the conv history (zeros without
+  // one), rows past a segment's end are zero-filled, and segments with no live
+  // token in the group are skipped. Every thread commits one group per call
+  // (possibly empty), so that cp_async_wait_one_pending always refers to the same
+  // group on every thread.
+  constexpr int CX = kBW / 8;
+  auto stage = [&](int g, int buf) {
+    for (int ci = threadIdx.x; ci < G::S * (XR + kTB) * CX; ci += G::kThreads) {
+      const int rowid = ci / CX, w = ci - rowid * CX;
+      const int sl = rowid / (XR + kTB), r = rowid - sl * (XR + kTB);
+      const int s0 = min(p.T, (blockIdx.x * G::S + sl) * pl.L), s1 = min(p.T, s0 + pl.L);
+      const int tb = s0 + g * kTB;
+      if (tb >= s1) continue;
+      const T *src = xb + (size_t)tb * D + (size_t)h * kBW + w * 8;   // a valid address
+      bool full = false;
+      T *dst;
+      if (r < XR) {                                   // x row t = tb - 3 + r
+        const int t = tb - 3 + r;
+        dst = xs_st + ((buf * G::S + sl) * XR + r) * kBW + w * 8;
+        if (t >= 0 && t < s1) {
+          src = xb + (size_t)t * D + (size_t)h * kBW + w * 8;
+          full = true;
+        } else if (t < 0 && cs_in_b != nullptr) {
+          src = cs_in_b + (size_t)(3 + t) * D + (size_t)h * kBW + w * 8;
+          full = true;
+        }
+      } else {                                        // dy row t = tb + k
+        const int k = r - XR, t = tb + k;
+        dst = dys_st + ((buf * G::S + sl) * kTB + k) * kBW + w * 8;
+        if (t < s1) {
+          src = dyb + ((size_t)b * p.T + t) * D + (size_t)h * kBW + w * 8;
+          full = true;
+        }
+      }
+      cp_async16(dst, src, full);
+    }
+    cp_async_commit();
+  };
   const int ng = pl.L / kTB;
+  stage(0, 0);
+  stage(1, 1);
+  cp_async_wait_one_pending();
+  __syncthreads();
   for (int g = 0; g < ng; ++g) {
     const int tb = th.t0 + g * kTB;
     const bool live = th.active && tb < th.t1;
+    const int buf = g % 3;
     float u[kTB];
     if (live) {
       const size_t go = ((size_t)b * ngt + tb / kTB) * D + th.d;
       ws_gP[go] = P;
       ws_gH[go] = Hl;
-      conv_group<T>(xb, cs_in_b, D, th.d, tb, th.t1, c, u);
-      // this group's dy rows and the next group's x rows
+      // Conv1D from the staged rows (the operation order of conv_group):
+      // u_t = w0 x_{t-3} + w1 x_{t-2} + w2 x_{t-1} + w3 x_t, rows k .. k + 3
+      const T *xr = xs_st + (buf * G::S + th.sl) * XR * kBW + th.j;
+      float xw[XR];
 #pragma unroll
-      for (int k = 0; k < kTB; ++k) {
-        if (tb + k < th.t1) prefetch_l1(dyb + orow + (size_t)(tb + k) * D);
-        if (tb + kTB + k < th.t1) prefetch_l1(xb + (size_t)(tb + kTB + k) * D + th.d);
-      }
+      for (int r = 0; r < XR; ++r) xw[r] = to_f32<T>(xr[r * kBW]);
+#pragma unroll
+      for (int k = 0; k < kTB; ++k)
+        u[k] = tb + k < th.t1
+                   ? fmaf(c.w3, xw[k + 3], fmaf(c.w2, xw[k + 2], fmaf(c.w1, xw[k + 1], c.w0 * xw[k])))
+                   : 0.f;
     } else {
 #pragma unroll
       for (int k = 0; k < kTB; ++k) u[k] = 0.f;
@@ -449,6 +510,9 @@ bwd_gates_tc_kernel(BwdArgs p, BwdPlan pl, float *__restrict__ ws_A, float *__re
 #pragma unroll
     for (int k = 0; k < kTB; ++k) u_col[k * G::kStride] = __float2bfloat16_rn(u[k]);
     __syncthreads();
+    // ring slot (g + 2) % 3 = (g - 1) % 3 was last read in group g - 1 (its dy rows
+    // after that group's second barrier): every thread has passed the barrier above
+    stage(g + 2, (g + 2) % 3);
     float acc[2][2][4];
 #pragma unroll
     for (int mi = 0; mi < 2; ++mi)
@@ -472,6 +536,7 @@ bwd_gates_tc_kernel(BwdArgs p, BwdPlan pl, float *__restrict__ ws_A, float *__re
         z_s[(((r >> 3) * 2 + 0) * kBW + col) * kRow + (r & 7)] = acc[mi][0][e];
         z_s[(((r >> 3) * 2 + 1) * kBW + col) * kRow + (r & 7)] = acc[mi][1][e];
       }
+    cp_async_wait_one_pending();   // group g + 1's rows: published by the barrier below
     __syncthreads();
     if (live) {
       float za[kTB], zx[kTB];
@@ -488,9 +553,11 @@ bwd_gates_tc_kernel(BwdArgs p, BwdPlan pl, float *__restrict__ ws_A, float *__re
         zx[4 * q + 2] = vx.z + c.bx;
         zx[4 * q + 3] = vx.w + c.bx;
       }
-      gates_scan_group<T>(za, zx, u, tb, th.t1, neg_c_sp, dyb, orow, D, P, Hl, R, ws_za, ws_zx);
+      gates_scan_group<T>(za, zx, u, tb, th.t1, neg_c_sp, dyb, orow, D, P, Hl, R, ws_za, ws_zx,
+                          dys_st + (buf * G::S + th.sl) * kTB * kBW + th.j, kBW);
     }
   }
+  cp_async_wait_all();   // no copy outlives the block
   if (!th.active) return;
   const size_t o = ((size_t)b * pl.nseg + th.s) * D + th.d;
   ws_A[o] = P;
@@ -1206,11 +1273,13 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
   const int bd = p.B * p.D;
   if constexpr (kTcBW > 0) {
     using G = TcGeo<kTcBW>;
-    // K1: fp32 z rows [S][2][bw][kRow] and bf16 u rows [M][kStride];
+    // K1: fp32 z rows [S][2][bw][kRow], bf16 u rows [M][kStride] and the staged
+    //     x and dy rows (bf16) [3][S][2 kTB + 3][bw];
     // K3: fp32 d u rows [S][bw][kRow], bf16 d z_a, d z_x rows [2][M][kStride],
     //     bf16 W_a, W_x rows [2][bw][kStride] and the staged z_a, z_x (fp32) and dy
     //     (bf16) rows [2][S][kTB][bw]
-    const size_t smem1 = (size_t)G::S * 2 * kTcBW * kRow * 4 + (size_t)G::M * G::kStride * 2;
+    const size_t smem1 = (size_t)G::S * 2 * kTcBW * kRow * 4 + (size_t)G::M * G::kStride * 2 +
+                         3 * (size_t)G::S * (2 * kTB + 3) * kTcBW * 2;
     const size_t smem3 = (size_t)G::S * kTcBW * kRow * 4 + 2 * (size_t)G::M * G::kStride * 2 +
                          2 * (size_t)kTcBW * G::kStride * 2 +   // + bf16 W_a, W_x rows
                          2 * (size_t)G::S * kTB * kTcBW * (4 + 4 + 2);   // + staged rows
