@@ -21,7 +21,8 @@
 //                 H = local end state and R = sum_t P_t dy_t with
 //                 P_t = a_t0 ... a_t (the segment's contribution to the state
 //                 gradient that leaves it leftwards);
-//   K2 carry      per (b, channel): h_in of each segment in time order from h0,
+//   K2 carry      per (b, channel), as a two-level scan over parts of the
+//                 segments: h_in of each segment in time order from h0,
 //                 and C_s, the state gradient entering segment s from the right
 //                 (dh_T for the last), in reverse order: C_{s-1} = R_s + A_s C_s,
 //                 dh0 = R_0 + A_0 C_0;
@@ -565,29 +566,72 @@ bwd_gates_tc_kernel(BwdArgs p, BwdPlan pl, float *__restrict__ ws_A, float *__re
   ws_R[o] = R;
 }
 
-__global__ void bwd_carry_kernel(int B, int D, int nseg, const float *__restrict__ ws_A,
-                                 const float *__restrict__ ws_H, const float *__restrict__ ws_R,
-                                 const float *__restrict__ h0, const float *__restrict__ dh_T,
-                                 float *__restrict__ ws_hin, float *__restrict__ ws_C,
-                                 float *__restrict__ dh0) {
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= B * D) return;
-  const int b = idx / D, d = idx - (idx / D) * D;
-  float hh = h0 ? h0[idx] : 0.f;
-#pragma unroll 8
-  for (int s = 0; s < nseg; ++s) {
-    const size_t o = ((size_t)b * nseg + s) * D + d;
-    ws_hin[o] = hh;
-    hh = fmaf(ws_A[o], hh, ws_H[o]);
-  }
-  float cc = dh_T ? dh_T[idx] : 0.f;
-#pragma unroll 8
-  for (int s = nseg - 1; s >= 0; --s) {
-    const size_t o = ((size_t)b * nseg + s) * D + d;
-    ws_C[o] = cc;
-    cc = fmaf(ws_A[o], cc, ws_R[o]);
-  }
-  if (dh0) dh0[idx] = cc;
+// K2: the two carries as two-level scans of affine maps. A block covers
+// kCarryCh channels (one per lane) and splits each channel's segments into
+// kCarryParts contiguous parts (one warp per part). Each part composes its
+// segments' maps (h -> A h + H forward, c -> A c + R backward) with loads that
+// do not depend on one another, the parts' entry values come from folding the
+// earlier parts' maps (shared memory), and each part then walks its own
+// segments storing h_in and C. The same recurrences as one sequential walk,
+// reassociated: the chains are nseg / kCarryParts long instead of nseg.
+constexpr int kCarryCh = 32, kCarryParts = 8;
+__global__ void __launch_bounds__(kCarryCh * kCarryParts)
+bwd_carry_kernel(int B, int D, int nseg, const float *__restrict__ ws_A,
+                 const float *__restrict__ ws_H, const float *__restrict__ ws_R,
+                 const float *__restrict__ h0, const float *__restrict__ dh_T,
+                 float *__restrict__ ws_hin, float *__restrict__ ws_C, float *__restrict__ dh0) {
+  __shared__ float mA[kCarryParts][kCarryCh], mV[kCarryParts][kCarryCh];
+  const int cl = threadIdx.x % kCarryCh, part = threadIdx.x / kCarryCh;
+  const int idx = blockIdx.x * kCarryCh + cl;
+  const bool on = idx < B * D;                 // no early return: the block meets at barriers
+  const int b = on ? idx / D : 0, d = on ? idx - b * D : 0;
+  const int q = ceil_div(nseg, kCarryParts);
+  const int s0 = min(nseg, part * q), s1 = min(nseg, s0 + q);
+  const size_t base = (size_t)b * nseg * D + d;
+  // forward: this part's map h -> Ap h + Vp, then the state entering it
+  float Ap = 1.f, Vp = 0.f;
+  if (on)
+    for (int s = s0; s < s1; ++s) {
+      const size_t o = base + (size_t)s * D;
+      const float a = ws_A[o];
+      Vp = fmaf(a, Vp, ws_H[o]);
+      Ap *= a;
+    }
+  mA[part][cl] = Ap;
+  mV[part][cl] = Vp;
+  __syncthreads();
+  float hh = (on && h0) ? h0[idx] : 0.f;
+  for (int r = 0; r < part; ++r) hh = fmaf(mA[r][cl], hh, mV[r][cl]);
+  if (on)
+    for (int s = s0; s < s1; ++s) {
+      const size_t o = base + (size_t)s * D;
+      ws_hin[o] = hh;
+      hh = fmaf(ws_A[o], hh, ws_H[o]);
+    }
+  __syncthreads();                             // every part has read mA, mV
+  // backward: this part's map c -> Ap c + Vp over its segments last to first,
+  // then the gradient entering it from the right
+  Ap = 1.f;
+  Vp = 0.f;
+  if (on)
+    for (int s = s1 - 1; s >= s0; --s) {
+      const size_t o = base + (size_t)s * D;
+      const float a = ws_A[o];
+      Vp = fmaf(a, Vp, ws_R[o]);
+      Ap *= a;
+    }
+  mA[part][cl] = Ap;
+  mV[part][cl] = Vp;
+  __syncthreads();
+  float cc = (on && dh_T) ? dh_T[idx] : 0.f;
+  for (int r = kCarryParts - 1; r > part; --r) cc = fmaf(mA[r][cl], cc, mV[r][cl]);
+  if (on)
+    for (int s = s1 - 1; s >= s0; --s) {
+      const size_t o = base + (size_t)s * D;
+      ws_C[o] = cc;
+      cc = fmaf(ws_A[o], cc, ws_R[o]);
+    }
+  if (on && part == 0 && dh0) dh0[idx] = cc;
 }
 
 // The per-thread part of a K3 group (a live thread only): the group's start
@@ -1293,8 +1337,8 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
       return e;
     bwd_gates_tc_kernel<kTcBW><<<grid, G::kThreads, smem1, st>>>(p, pl, A, Hh, R, gP, gH, za, zx);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    bwd_carry_kernel<<<ceil_div(bd, 256), 256, 0, st>>>(p.B, p.D, pl.nseg, A, Hh, R, p.h0,
-                                                        p.dh_T, hin, C, p.dh0);
+    bwd_carry_kernel<<<ceil_div(bd, kCarryCh), kCarryCh * kCarryParts, 0, st>>>(
+        p.B, p.D, pl.nseg, A, Hh, R, p.h0, p.dh_T, hin, C, p.dh0);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     bwd_final_tc_kernel<kTcBW><<<grid, G::kThreads, smem3, st>>>(p, pl, b16, hin, C, gP, gH, za,
                                                                   zx, U, du);
@@ -1315,8 +1359,8 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
     bwd_gates_kernel<T, kSW, kMaxT><<<grid, threads, smem1, st>>>(p, pl, A, Hh, R, gP, gH, za,
                                                                    zx);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    bwd_carry_kernel<<<ceil_div(bd, 256), 256, 0, st>>>(p.B, p.D, pl.nseg, A, Hh, R, p.h0,
-                                                        p.dh_T, hin, C, p.dh0);
+    bwd_carry_kernel<<<ceil_div(bd, kCarryCh), kCarryCh * kCarryParts, 0, st>>>(
+        p.B, p.D, pl.nseg, A, Hh, R, p.h0, p.dh_T, hin, C, p.dh0);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     bwd_final_kernel<T, kSW, kMaxT><<<grid, threads, smem3, st>>>(p, pl, hin, C, gP, gH, za, zx,
                                                                    U, du);
