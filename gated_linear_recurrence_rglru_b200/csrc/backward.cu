@@ -670,7 +670,8 @@ __device__ __forceinline__ void final_group(const BwdThread &th, const ChanC &c,
                                             float *__restrict__ ws_u, float &gc, float &acc_q,
                                             float &acc_ba, float &acc_bx, float (&dub)[kTB],
                                             const float *sza, const float *szx, const T *sdy,
-                                            int sstride, const Bf16Streams &b16, Sink sink) {
+                                            const T *sx, const float *sg, int sstride,
+                                            const Bf16Streams &b16, Sink sink) {
   const float neg_c_sp = -kDecayC * c.sp, csp = kDecayC * c.sp;
   if (!kStaged && tb - kTB >= th.t0) {
     // the group processed next (8 tokens earlier): its z and dy rows
@@ -684,10 +685,24 @@ __device__ __forceinline__ void final_group(const BwdThread &th, const ChanC &c,
       prefetch_l1(pdy + (size_t)k * D);
     }
   }
-  float u[kTB];
-  conv_group<T>(xb, cs_in_b, D, th.d, tb, th.t1, c, u);
+  float u[kTB], hh;
+  if constexpr (kStaged) {
+    // the staged x rows tb - 3 .. tb + 7 (conv_group's operation order) and the
+    // group's start pair (prod a, local state)
+    float xw[kTB + 3];
+#pragma unroll
+    for (int r = 0; r < kTB + 3; ++r) xw[r] = to_f32<T>(sx[r * sstride]);
+#pragma unroll
+    for (int k = 0; k < kTB; ++k)
+      u[k] = tb + k < th.t1
+                 ? fmaf(c.w3, xw[k + 3], fmaf(c.w2, xw[k + 2], fmaf(c.w1, xw[k + 1], c.w0 * xw[k])))
+                 : 0.f;
+    hh = fmaf(sg[0], h_in, sg[sstride]);
+  } else {
+    conv_group<T>(xb, cs_in_b, D, th.d, tb, th.t1, c, u);
+    hh = fmaf(ws_gP[go], h_in, ws_gH[go]);
+  }
   float fa[kTB], fza[kTB], fq[kTB], fzx[kTB], fu[kTB];
-  float hh = fmaf(ws_gP[go], h_in, ws_gH[go]);
 #pragma unroll
   for (int k = 0; k < kTB; ++k) {
     const int t = tb + k;
@@ -791,7 +806,7 @@ bwd_final_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
       const size_t go = ((size_t)b * ngt + tb / kTB) * D + th.d;
       final_group<T, false, false>(th, c, xb, cs_in_b, dyb, orow, D, tb, go, h_in, ws_gP, ws_gH,
                                    ws_za, ws_zx, ws_u, gc, acc_q, acc_ba, acc_bx, dub, nullptr,
-                                   nullptr, nullptr, 0, Bf16Streams{},
+                                   nullptr, nullptr, nullptr, nullptr, 0, Bf16Streams{},
                                    [&](int k, float dza, float dzx) {
                               dza_row[k] = dza;
                               dzx_row[k] = dzx;
@@ -851,10 +866,15 @@ bwd_final_tc_kernel(BwdArgs p, BwdPlan pl, Bf16Streams b16, const float *__restr
   float *du_s = reinterpret_cast<float *>(smem_ft);                  // [S][kBW][kRow]
   T *a_s = reinterpret_cast<T *>(du_s + G::S * kBW * kRow);          // [2][M][kStride]
   T *w_s = a_s + 2 * G::M * G::kStride;                              // [2][kBW][kStride]
-  // z_a, z_x and dy rows of a group, double-buffered: [2][S][kTB][kBW]
+  // z_a, z_x and dy rows of a group, double-buffered: [2][S][kTB][kBW]; then its
+  // x rows tb-3 .. tb+7 [2][S][kTB + 3][kBW] and its start pair (prod a, local
+  // state) [2][S][2][kBW]
+  constexpr int XR = kTB + 3;
   float *za_st = reinterpret_cast<float *>(w_s + 2 * kBW * G::kStride);
   float *zx_st = za_st + 2 * G::S * kTB * kBW;
   T *dy_st = reinterpret_cast<T *>(zx_st + 2 * G::S * kTB * kBW);
+  T *xs_st = dy_st + 2 * G::S * kTB * kBW;
+  float *gs_st = reinterpret_cast<float *>(xs_st + 2 * G::S * XR * kBW);
   const int D = p.D, h = blockIdx.y, b = blockIdx.z;
   const BwdThread th = bwd_thread(p, pl, kBW);
   const T *xb = static_cast<const T *>(p.x) + (size_t)b * p.T * D;
@@ -901,9 +921,11 @@ bwd_final_tc_kernel(BwdArgs p, BwdPlan pl, Bf16Streams b16, const float *__restr
   float acc_q = 0.f, acc_ba = 0.f, acc_bx = 0.f;
   // Staging of group g's rows into buffer buf: 16-byte copies spread over the
   // block (per segment and token: kBW/4 chunks of z_a, kBW/4 of z_x, kBW/8 of
-  // dy). Rows past a segment's end are zero-filled; segments with no live
-  // token in the group are skipped (no thread reads them).
-  constexpr int CZ = kBW / 4, CY = kBW / 8, CR = 2 * CZ + CY;
+  // dy; per segment: 11 x rows of kBW/8 chunks and 2 start-pair rows of kBW/4).
+  // Rows past a segment's end are zero-filled, x rows before t = 0 come from the
+  // conv history (zeros without one); segments with no live token in the group
+  // are skipped (no thread reads them).
+  constexpr int CZ = kBW / 4, CY = kBW / 8, CR = 2 * CZ + CY, CXG = XR * CY + 2 * CZ;
   auto stage = [&](int g, int buf) {
     for (int ci = threadIdx.x; ci < G::S * kTB * CR; ci += G::kThreads) {
       const int rowid = ci / CR, w = ci - rowid * CR;
@@ -917,6 +939,31 @@ bwd_final_tc_kernel(BwdArgs p, BwdPlan pl, Bf16Streams b16, const float *__restr
       if (w < CZ) cp_async16(za_st + slot + w * 4, ws_za + grow + w * 4, in);
       else if (w < 2 * CZ) cp_async16(zx_st + slot + (w - CZ) * 4, ws_zx + grow + (w - CZ) * 4, in);
       else cp_async16(dy_st + slot + (w - 2 * CZ) * 8, dyb + grow + (w - 2 * CZ) * 8, in);
+    }
+    for (int ci = threadIdx.x; ci < G::S * CXG; ci += G::kThreads) {
+      const int sl = ci / CXG, w = ci - sl * CXG;
+      const int s0 = min(p.T, (blockIdx.x * G::S + sl) * pl.L), s1 = min(p.T, s0 + pl.L);
+      const int tb = s0 + g * kTB;
+      if (tb >= s1) continue;
+      if (w < XR * CY) {                              // x row t = tb - 3 + r
+        const int r = w / CY, cx = w - r * CY, t = tb - 3 + r;
+        const size_t col = (size_t)h * kBW + cx * 8;
+        const T *src = xb + (size_t)tb * D + col;     // a valid address
+        bool full = false;
+        if (t >= 0 && t < s1) {
+          src = xb + (size_t)t * D + col;
+          full = true;
+        } else if (t < 0 && cs_in_b != nullptr) {
+          src = cs_in_b + (size_t)(3 + t) * D + col;
+          full = true;
+        }
+        cp_async16(xs_st + ((buf * G::S + sl) * XR + r) * kBW + cx * 8, src, full);
+      } else {                                        // prod a (row 0), local state (row 1)
+        const int w2 = w - XR * CY, which = w2 / CZ, cz = w2 - which * CZ;
+        const size_t go = ((size_t)b * ngt + tb / kTB) * D + (size_t)h * kBW + cz * 4;
+        cp_async16(gs_st + ((buf * G::S + sl) * 2 + which) * kBW + cz * 4,
+                   (which ? ws_gH : ws_gP) + go, true);
+      }
     }
     cp_async_commit();
   };
@@ -938,7 +985,10 @@ bwd_final_tc_kernel(BwdArgs p, BwdPlan pl, Bf16Streams b16, const float *__restr
       final_group<T, true, kBW % kDwTile == 0>(th, c, xb, cs_in_b, dyb, orow, D, tb, go, h_in,
                                                ws_gP, ws_gH, ws_za, ws_zx, ws_u, gc, acc_q,
                                                acc_ba, acc_bx, dub, za_st + srow, zx_st + srow,
-                                               dy_st + srow, kBW, b16,
+                                               dy_st + srow,
+                                               xs_st + (buf * G::S + th.sl) * XR * kBW + th.j,
+                                               gs_st + (buf * G::S + th.sl) * 2 * kBW + th.j,
+                                               kBW, b16,
                                                [&](int k, float dza, float dzx) {
                              dza_col[k * G::kStride] = __float2bfloat16_rn(dza);
                              dzx_col[k * G::kStride] = __float2bfloat16_rn(dzx);
@@ -1320,13 +1370,16 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
     // K1: fp32 z rows [S][2][bw][kRow], bf16 u rows [M][kStride] and the staged
     //     x and dy rows (bf16) [3][S][2 kTB + 3][bw];
     // K3: fp32 d u rows [S][bw][kRow], bf16 d z_a, d z_x rows [2][M][kStride],
-    //     bf16 W_a, W_x rows [2][bw][kStride] and the staged z_a, z_x (fp32) and dy
-    //     (bf16) rows [2][S][kTB][bw]
+    //     bf16 W_a, W_x rows [2][bw][kStride], the staged z_a, z_x (fp32) and dy
+    //     (bf16) rows [2][S][kTB][bw], x rows (bf16) [2][S][kTB + 3][bw] and start
+    //     pairs (fp32) [2][S][2][bw]
     const size_t smem1 = (size_t)G::S * 2 * kTcBW * kRow * 4 + (size_t)G::M * G::kStride * 2 +
                          3 * (size_t)G::S * (2 * kTB + 3) * kTcBW * 2;
     const size_t smem3 = (size_t)G::S * kTcBW * kRow * 4 + 2 * (size_t)G::M * G::kStride * 2 +
                          2 * (size_t)kTcBW * G::kStride * 2 +   // + bf16 W_a, W_x rows
-                         2 * (size_t)G::S * kTB * kTcBW * (4 + 4 + 2);   // + staged rows
+                         2 * (size_t)G::S * kTB * kTcBW * (4 + 4 + 2) +   // + staged rows
+                         2 * (size_t)G::S * (kTB + 3) * kTcBW * 2 +       // + staged x rows
+                         2 * (size_t)G::S * 2 * kTcBW * 4;                // + start pairs
     if ((e = cudaFuncSetAttribute(bwd_gates_tc_kernel<kTcBW>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1)) !=
         cudaSuccess)
