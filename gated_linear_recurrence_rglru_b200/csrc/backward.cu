@@ -447,35 +447,37 @@ bwd_gates_tc_kernel(BwdArgs p, BwdPlan pl, float *__restrict__ ws_A, float *__re
   // (possibly empty), so that cp_async_wait_one_pending always refers to the same
   // group on every thread.
   constexpr int CX = kBW / 8;
+  // the dy rows come to exactly one chunk per thread; x rows in a loop of their own,
+  // so that a warp's copies stay on one branch
+  static_assert(G::S * kTB * CX == G::kThreads, "dy chunks per thread");
   auto stage = [&](int g, int buf) {
-    for (int ci = threadIdx.x; ci < G::S * (XR + kTB) * CX; ci += G::kThreads) {
+    {                                                 // dy row t = tb + k
+      const int rowid = threadIdx.x / CX, w = threadIdx.x - rowid * CX;
+      const int sl = rowid / kTB, k = rowid - sl * kTB;
+      const int s0 = min(p.T, (blockIdx.x * G::S + sl) * pl.L), s1 = min(p.T, s0 + pl.L);
+      const int tb = s0 + g * kTB, t = tb + k;
+      if (tb < s1)
+        cp_async16(dys_st + ((buf * G::S + sl) * kTB + k) * kBW + w * 8,
+                   dyb + ((size_t)b * p.T + (t < s1 ? t : tb)) * D + (size_t)h * kBW + w * 8,
+                   t < s1);
+    }
+    for (int ci = threadIdx.x; ci < G::S * XR * CX; ci += G::kThreads) {
       const int rowid = ci / CX, w = ci - rowid * CX;
-      const int sl = rowid / (XR + kTB), r = rowid - sl * (XR + kTB);
+      const int sl = rowid / XR, r = rowid - sl * XR;
       const int s0 = min(p.T, (blockIdx.x * G::S + sl) * pl.L), s1 = min(p.T, s0 + pl.L);
       const int tb = s0 + g * kTB;
       if (tb >= s1) continue;
+      const int t = tb - 3 + r;                       // x row t = tb - 3 + r
       const T *src = xb + (size_t)tb * D + (size_t)h * kBW + w * 8;   // a valid address
       bool full = false;
-      T *dst;
-      if (r < XR) {                                   // x row t = tb - 3 + r
-        const int t = tb - 3 + r;
-        dst = xs_st + ((buf * G::S + sl) * XR + r) * kBW + w * 8;
-        if (t >= 0 && t < s1) {
-          src = xb + (size_t)t * D + (size_t)h * kBW + w * 8;
-          full = true;
-        } else if (t < 0 && cs_in_b != nullptr) {
-          src = cs_in_b + (size_t)(3 + t) * D + (size_t)h * kBW + w * 8;
-          full = true;
-        }
-      } else {                                        // dy row t = tb + k
-        const int k = r - XR, t = tb + k;
-        dst = dys_st + ((buf * G::S + sl) * kTB + k) * kBW + w * 8;
-        if (t < s1) {
-          src = dyb + ((size_t)b * p.T + t) * D + (size_t)h * kBW + w * 8;
-          full = true;
-        }
+      if (t >= 0 && t < s1) {
+        src = xb + (size_t)t * D + (size_t)h * kBW + w * 8;
+        full = true;
+      } else if (t < 0 && cs_in_b != nullptr) {
+        src = cs_in_b + (size_t)(3 + t) * D + (size_t)h * kBW + w * 8;
+        full = true;
       }
-      cp_async16(dst, src, full);
+      cp_async16(xs_st + ((buf * G::S + sl) * XR + r) * kBW + w * 8, src, full);
     }
     cp_async_commit();
   };
@@ -925,10 +927,17 @@ bwd_final_tc_kernel(BwdArgs p, BwdPlan pl, Bf16Streams b16, const float *__restr
   // Rows past a segment's end are zero-filled, x rows before t = 0 come from the
   // conv history (zeros without one); segments with no live token in the group
   // are skipped (no thread reads them).
-  constexpr int CZ = kBW / 4, CY = kBW / 8, CR = 2 * CZ + CY, CXG = XR * CY + 2 * CZ;
+  constexpr int CZ = kBW / 4, CY = kBW / 8, CXG = XR * CY + 2 * CZ;
+  // z_a and z_x rows come to exactly two chunks per thread each, dy rows to one;
+  // one loop per stream keeps a warp's copies on one branch
+  static_assert(G::S * kTB * CZ == 2 * G::kThreads && G::S * kTB * CY == G::kThreads,
+                "chunks per thread");
   auto stage = [&](int g, int buf) {
-    for (int ci = threadIdx.x; ci < G::S * kTB * CR; ci += G::kThreads) {
-      const int rowid = ci / CR, w = ci - rowid * CR;
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+      const int ci = threadIdx.x + (q < 2 ? q : 0) * G::kThreads;
+      const int cpr = q < 2 ? CZ : CY;                // chunks per row (powers of two)
+      const int rowid = ci / cpr, w = ci - rowid * cpr;
       const int sl = rowid / kTB, k = rowid - sl * kTB;
       const int s0 = min(p.T, (blockIdx.x * G::S + sl) * pl.L), s1 = min(p.T, s0 + pl.L);
       const int tb = s0 + g * kTB;
@@ -936,9 +945,12 @@ bwd_final_tc_kernel(BwdArgs p, BwdPlan pl, Bf16Streams b16, const float *__restr
       const bool in = tb + k < s1;
       const size_t grow = ((size_t)b * p.T + (in ? tb + k : tb)) * D + (size_t)h * kBW;
       const int slot = ((buf * G::S + sl) * kTB + k) * kBW;
-      if (w < CZ) cp_async16(za_st + slot + w * 4, ws_za + grow + w * 4, in);
-      else if (w < 2 * CZ) cp_async16(zx_st + slot + (w - CZ) * 4, ws_zx + grow + (w - CZ) * 4, in);
-      else cp_async16(dy_st + slot + (w - 2 * CZ) * 8, dyb + grow + (w - 2 * CZ) * 8, in);
+      if (q < 2) {
+        cp_async16(za_st + slot + w * 4, ws_za + grow + w * 4, in);
+        cp_async16(zx_st + slot + w * 4, ws_zx + grow + w * 4, in);
+        continue;
+      }
+      cp_async16(dy_st + slot + w * 8, dyb + grow + w * 8, in);
     }
     for (int ci = threadIdx.x; ci < G::S * CXG; ci += G::kThreads) {
       const int sl = ci / CXG, w = ci - sl * CXG;

@@ -49,6 +49,9 @@ CASES = [
     # gate contractions (bf16 operands would exceed the bar here by design: see
     # tests/test_backward_bf16_operands.py)
     WORKLOADS["hawk_block"].with_shape(B=2, T=1, D=128, H=2, h0_var=1.0, seed=51),
+    # the tensor-core kernels with T shorter than one group (B*T = 12): one segment per
+    # sequence whose staged rows are mostly past its end or in the conv history
+    WORKLOADS["hawk_block"].with_shape(B=4, T=3, D=256, H=4, h0_var=0.5, bias_std=0.3, seed=54),
 ]
 
 
