@@ -1142,19 +1142,22 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&a)[4]) {
 
 // d W on the tensor cores (bf16 I/O, heads a multiple of 64 wide): the same
 // 64 x 64 (i, j) tiles and token chunks as bwd_dw_kernel, 4 warps each a
-// 32 x 32 quarter. 32 tokens of U and dZ are staged as bf16 token-major rows
+// 32 x 32 quarter. kDwTcRows tokens of U and dZ are staged as bf16 token-major rows
 // (padded by 8 elements); with A[i][n] = U[n][i] and B[n][j] = dZ[n][j], both
 // fragments come from ldmatrix .trans of those rows (a thread receives stored
 // elements (2q, g) and (2q + 1, g) of each 8 x 8 block: the k pairs of column
-// g). The next 32 tokens are in flight to registers during the MMAs.
+// g). The next kDwTcRows tokens are in flight to registers during the MMAs.
 constexpr int kDwTcThreads = 128, kDwTcStride = kDwTile + 8;
+// tokens per step of the tensor-core d W: 64, so that a block's loads of the next step
+// cover twice the bytes of the CUDA-core kernel's 32-token steps
+constexpr int kDwTcRows = 64;
 
 __global__ void __launch_bounds__(kDwTcThreads)
 bwd_dw_tc_kernel(const __nv_bfloat16 *__restrict__ U, const __nv_bfloat16 *__restrict__ dZa,
                  const __nv_bfloat16 *__restrict__ dZx, float *__restrict__ dWa,
                  float *__restrict__ dWx, int N, int D, int H, int chunk) {
-  __shared__ __align__(16) __nv_bfloat16 us[kDwRows][kDwTcStride];
-  __shared__ __align__(16) __nv_bfloat16 zs[kDwRows][kDwTcStride];
+  __shared__ __align__(16) __nv_bfloat16 us[kDwTcRows][kDwTcStride];
+  __shared__ __align__(16) __nv_bfloat16 zs[kDwTcRows][kDwTcStride];
   const int bw = D / H;
   const int tiles = bw / kDwTile;
   int tile = blockIdx.x;
@@ -1171,10 +1174,10 @@ bwd_dw_tc_kernel(const __nv_bfloat16 *__restrict__ U, const __nv_bfloat16 *__res
   const __nv_bfloat16 *Uc = U + (size_t)h * bw + i0 + lc;
   const __nv_bfloat16 *Zc = Z + (size_t)h * bw + j0 + lc;
   const int n_begin = blockIdx.y * chunk, n_end = min(N, n_begin + chunk);
-  uint2 pu[kDwRows / 8], pz[kDwRows / 8];
+  uint2 pu[kDwTcRows / 8], pz[kDwTcRows / 8];
   auto fetch = [&](int n0) {
 #pragma unroll
-    for (int q = 0; q < kDwRows / 8; ++q) {
+    for (int q = 0; q < kDwTcRows / 8; ++q) {
       const int n = n0 + lr + 8 * q;
       const bool ok = n < n_end;
       pu[q] = ok ? *reinterpret_cast<const uint2 *>(Uc + (size_t)n * D) : make_uint2(0, 0);
@@ -1195,16 +1198,16 @@ bwd_dw_tc_kernel(const __nv_bfloat16 *__restrict__ U, const __nv_bfloat16 *__res
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[mi][nt][e] = 0.f;
   fetch(n_begin);
-  for (int n0 = n_begin; n0 < n_end; n0 += kDwRows) {
+  for (int n0 = n_begin; n0 < n_end; n0 += kDwTcRows) {
 #pragma unroll
-    for (int q = 0; q < kDwRows / 8; ++q) {
+    for (int q = 0; q < kDwTcRows / 8; ++q) {
       *reinterpret_cast<uint2 *>(&us[lr + 8 * q][lc]) = pu[q];
       *reinterpret_cast<uint2 *>(&zs[lr + 8 * q][lc]) = pz[q];
     }
     __syncthreads();
-    if (n0 + kDwRows < n_end) fetch(n0 + kDwRows);
+    if (n0 + kDwTcRows < n_end) fetch(n0 + kDwTcRows);
 #pragma unroll
-    for (int ks = 0; ks < kDwRows / 16; ++ks) {
+    for (int ks = 0; ks < kDwTcRows / 16; ++ks) {
       uint32_t a[2][4], b[2][4];
 #pragma unroll
       for (int mi = 0; mi < 2; ++mi) ldsm_x4_trans(a_lane + ks * 16 * kRowBytes + mi * 32, a[mi]);
@@ -1436,8 +1439,10 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
   const int tiles = ceil_div(bw, kDwTile);
   const int tile_blocks = 2 * tiles * tiles * p.H;
   const int nchunk = ceil_div(8 * 148, tile_blocks);
-  const int chunk = ceil_div(ceil_div(N, nchunk), kDwRows) * kDwRows;
-  if (kTcBW > 0 && kTcBW % kDwTile == 0)
+  const bool dw_tc = kTcBW > 0 && kTcBW % kDwTile == 0;
+  const int dw_rows = dw_tc ? kDwTcRows : kDwRows;   // tokens per step
+  const int chunk = ceil_div(ceil_div(N, nchunk), dw_rows) * dw_rows;
+  if (dw_tc)
     bwd_dw_tc_kernel<<<dim3(tile_blocks, ceil_div(N, chunk)), kDwTcThreads, 0, st>>>(
         b16.u, b16.dza, b16.dzx, p.dW_a, p.dW_x, N, p.D, p.H, chunk);
   else
