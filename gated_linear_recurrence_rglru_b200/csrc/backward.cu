@@ -15,7 +15,7 @@
 // contractions; MMA fragments in registers in K1, bf16 rows in shared memory
 // in K3 for the tensor-core ones):
 //   K1 gates      per segment, in time order: Conv1D u, both gate
-//                 pre-activations (z_a, z_x -> fp32 workspace), the local scan
+//                 pre-activations and gates (r, i -> fp32 workspace), the local scan
 //                 from zero, whose (prod a, state) at each group start also go
 //                 to the workspace, and the aggregates A = prod a_t,
 //                 H = local end state and R = sum_t P_t dy_t with
@@ -27,14 +27,15 @@
 //                 (dh_T for the last), in reverse order: C_{s-1} = R_s + A_s C_s,
 //                 dh0 = R_0 + A_0 C_0;
 //   K3 final      per segment, groups in reverse order: the group's start state
-//                 (prod a) h_in + (local state) and its stored z_a, z_x give
+//                 (prod a) h_in + (local state) and its stored r, i give
 //                 h_{t-1}, a and beta for its 8 tokens; then G_t = dy_t +
 //                 a_{t+1} G_{t+1} from C_s and d a = G h_{t-1}, d beta = G,
 //                 g = sqrt(1 - a^2), d g = G i u, d i = G g u,
 //                 d u = G g i + d z_a W_a^T + d z_x W_x^T,
-//                 d la = d a a - d g a^2 / g, la = -c r sp, z -> r, i by sigmoid;
+//                 d la = d a a - d g a^2 / g, la = -c r sp, d z from r, i;
 //                 it accumulates d b_a, d b_x and d Lambda per channel and writes
-//                 u, d z_a, d z_x (over z_a, z_x) and d u to the workspace;
+//                 u, d z_a, d z_x (over r, i; bf16 for the tensor-core d W) and
+//                 d u to the workspace;
 //   K4 weights    d W[h] = U_h^T dZ_h for both gates (64 x 64 tiles, the token
 //                 sum split over blocks and combined with atomics; tensor cores
 //                 or 4 x 4 FFMA tiles per thread);
@@ -266,10 +267,11 @@ struct TokGates {
   float r, i, a, g, rog;
 };
 
-__device__ __forceinline__ TokGates tok_gates(float za, float zx, float neg_c_sp) {
+// The same from the gates r = sigmoid(z_a) and i = sigmoid(z_x) themselves.
+__device__ __forceinline__ TokGates tok_gates_ri(float r, float i, float neg_c_sp) {
   TokGates t;
-  t.r = sigmoid_fast(za);
-  t.i = sigmoid_fast(zx);
+  t.r = r;
+  t.i = i;
   const float la = neg_c_sp * t.r;
   t.a = __expf(la);
   const float om = neg_expm1_fast(2.0f * la);
@@ -279,8 +281,13 @@ __device__ __forceinline__ TokGates tok_gates(float za, float zx, float neg_c_sp
   return t;
 }
 
+__device__ __forceinline__ TokGates tok_gates(float za, float zx, float neg_c_sp) {
+  return tok_gates_ri(sigmoid_fast(za), sigmoid_fast(zx), neg_c_sp);
+}
+
 // The post-contraction part of a K1 group: decay, input, the local scan and
-// the running R; z_a, z_x of the live tokens to the workspace. sdy: the
+// the running R; the gates r and i of the live tokens to the workspace (K3
+// needs z_a and z_x only through them). sdy: the
 // group's dy rows staged in shared memory (this thread's channel at token 0,
 // rows sstride apart), or nullptr to read dy from global memory.
 template <typename T>
@@ -288,8 +295,8 @@ __device__ __forceinline__ void gates_scan_group(const float (&za)[kTB], const f
                                                  const float (&u)[kTB], int tb, int t1,
                                                  float neg_c_sp, const T *dyb, size_t orow,
                                                  int D, float &P, float &Hl, float &R,
-                                                 float *__restrict__ ws_za,
-                                                 float *__restrict__ ws_zx,
+                                                 float *__restrict__ ws_ga,
+                                                 float *__restrict__ ws_gx,
                                                  const T *sdy = nullptr, int sstride = 0) {
 #pragma unroll
   for (int k = 0; k < kTB; ++k) {
@@ -300,8 +307,8 @@ __device__ __forceinline__ void gates_scan_group(const float (&za)[kTB], const f
       P *= q.a;
       const size_t o = orow + (size_t)t * D;
       R = fmaf(P, sdy != nullptr ? to_f32<T>(sdy[k * sstride]) : ldg_f32(dyb + o), R);
-      ws_za[o] = za[k];
-      ws_zx[o] = zx[k];
+      ws_ga[o] = q.r;
+      ws_gx[o] = q.i;
     }
   }
 }
@@ -310,7 +317,7 @@ template <typename T, bool kSW, int kMaxT>
 __global__ void __launch_bounds__(kMaxT, kMaxT == 256 ? 3 : 1)
 bwd_gates_kernel(BwdArgs p, BwdPlan pl, float *__restrict__ ws_A, float *__restrict__ ws_H,
                  float *__restrict__ ws_R, float *__restrict__ ws_gP, float *__restrict__ ws_gH,
-                 float *__restrict__ ws_za, float *__restrict__ ws_zx) {
+                 float *__restrict__ ws_ga, float *__restrict__ ws_gx) {
   extern __shared__ float4 smem_g[];
   const int bw = p.D / p.H, D = p.D, h = blockIdx.y, b = blockIdx.z;
   const int seg_floats = pl.S * bw * kRow;
@@ -370,7 +377,7 @@ bwd_gates_kernel(BwdArgs p, BwdPlan pl, float *__restrict__ ws_A, float *__restr
           zx[k] = fmaf(uv[k], wx, zx[k]);
         }
       }
-      gates_scan_group<T>(za, zx, u, tb, th.t1, neg_c_sp, dyb, orow, D, P, Hl, R, ws_za, ws_zx);
+      gates_scan_group<T>(za, zx, u, tb, th.t1, neg_c_sp, dyb, orow, D, P, Hl, R, ws_ga, ws_gx);
     }
   }
   if (!th.active) return;
@@ -391,8 +398,8 @@ template <int kBW>
 __global__ void __launch_bounds__(TcGeo<kBW>::kThreads, kBW == 128 ? 1 : 3)
 bwd_gates_tc_kernel(BwdArgs p, BwdPlan pl, float *__restrict__ ws_A, float *__restrict__ ws_H,
                     float *__restrict__ ws_R, float *__restrict__ ws_gP,
-                    float *__restrict__ ws_gH, float *__restrict__ ws_za,
-                    float *__restrict__ ws_zx) {
+                    float *__restrict__ ws_gH, float *__restrict__ ws_ga,
+                    float *__restrict__ ws_gx) {
   using T = __nv_bfloat16;
   using G = TcGeo<kBW>;
   extern __shared__ float4 smem_gt[];
@@ -556,7 +563,7 @@ bwd_gates_tc_kernel(BwdArgs p, BwdPlan pl, float *__restrict__ ws_A, float *__re
         zx[4 * q + 2] = vx.z + c.bx;
         zx[4 * q + 3] = vx.w + c.bx;
       }
-      gates_scan_group<T>(za, zx, u, tb, th.t1, neg_c_sp, dyb, orow, D, P, Hl, R, ws_za, ws_zx,
+      gates_scan_group<T>(za, zx, u, tb, th.t1, neg_c_sp, dyb, orow, D, P, Hl, R, ws_ga, ws_gx,
                           dys_st + (buf * G::S + th.sl) * kTB * kBW + th.j, kBW);
     }
   }
@@ -637,7 +644,7 @@ bwd_carry_kernel(int B, int D, int nseg, const float *__restrict__ ws_A,
 }
 
 // The per-thread part of a K3 group (a live thread only): the group's start
-// state from (prod a, local state) and h_in, the stored z, then the reverse
+// state from (prod a, local state) and h_in, the stored gates r and i, then the reverse
 // chain over its tokens. With G_t the state gradient at token t, every
 // gradient of the token is G_t times a factor known in time order:
 //   d z_a = G c sp (1 - r) Q,  d Lambda-sum term = G c Q,
@@ -648,8 +655,8 @@ bwd_carry_kernel(int B, int D, int nseg, const float *__restrict__ ws_A,
 // each token's (d z_a, d z_x) to sink(k, ...) (zeros past t1), leaves the own
 // part of d u in dub and advances gc and the per-channel sums (acc_q sums
 // G Q; the caller scales it by c).
-// kStaged: the group's z_a, z_x and dy rows were copied to shared memory ahead
-// of time (sza, szx, sdy: this thread's channel at token 0 of the group, rows
+// kStaged: the group's r, i and dy rows were copied to shared memory ahead
+// of time (sr, si, sdy: this thread's channel at token 0 of the group, rows
 // sstride elements apart, zeros past t1); else they are read from the
 // workspace and dy in global memory, with an L1 prefetch of the next group.
 // d W tiles: 64 x 64 (i, j) per block (both d W kernels)
@@ -668,22 +675,22 @@ __device__ __forceinline__ void final_group(const BwdThread &th, const ChanC &c,
                                             int tb, size_t go, float h_in,
                                             const float *__restrict__ ws_gP,
                                             const float *__restrict__ ws_gH,
-                                            float *__restrict__ ws_za, float *__restrict__ ws_zx,
+                                            float *__restrict__ ws_ga, float *__restrict__ ws_gx,
                                             float *__restrict__ ws_u, float &gc, float &acc_q,
                                             float &acc_ba, float &acc_bx, float (&dub)[kTB],
-                                            const float *sza, const float *szx, const T *sdy,
+                                            const float *sr, const float *si, const T *sdy,
                                             const T *sx, const float *sg, int sstride,
                                             const Bf16Streams &b16, Sink sink) {
   const float neg_c_sp = -kDecayC * c.sp, csp = kDecayC * c.sp;
   if (!kStaged && tb - kTB >= th.t0) {
-    // the group processed next (8 tokens earlier): its z and dy rows
-    const float *pza = ws_za + orow + (size_t)(tb - kTB) * D;
-    const float *pzx = ws_zx + orow + (size_t)(tb - kTB) * D;
+    // the group processed next (8 tokens earlier): its r, i and dy rows
+    const float *pga = ws_ga + orow + (size_t)(tb - kTB) * D;
+    const float *pgx = ws_gx + orow + (size_t)(tb - kTB) * D;
     const T *pdy = dyb + orow + (size_t)(tb - kTB) * D;
 #pragma unroll
     for (int k = 0; k < kTB; ++k) {
-      prefetch_l1(pza + (size_t)k * D);
-      prefetch_l1(pzx + (size_t)k * D);
+      prefetch_l1(pga + (size_t)k * D);
+      prefetch_l1(pgx + (size_t)k * D);
       prefetch_l1(pdy + (size_t)k * D);
     }
   }
@@ -710,13 +717,13 @@ __device__ __forceinline__ void final_group(const BwdThread &th, const ChanC &c,
     const int t = tb + k;
     const size_t o = orow + (size_t)t * D;
     const bool in = t < th.t1;
-    float za, zx;
+    float rv, iv;                                 // the gates r and i stored by K1
     if constexpr (kStaged) {
-      za = sza[k * sstride];
-      zx = szx[k * sstride];
+      rv = sr[k * sstride];
+      iv = si[k * sstride];
     } else {
-      za = in ? ws_za[o] : 0.f;
-      zx = in ? ws_zx[o] : 0.f;
+      rv = in ? ws_ga[o] : 0.f;
+      iv = in ? ws_gx[o] : 0.f;
     }
     if (in) {
       if constexpr (kB16)
@@ -724,7 +731,7 @@ __device__ __forceinline__ void final_group(const BwdThread &th, const ChanC &c,
       else
         ws_u[o] = u[k];
     }
-    const TokGates tg = tok_gates(za, zx, neg_c_sp);
+    const TokGates tg = tok_gates_ri(rv, iv, neg_c_sp);
     const float r = tg.r, ig = tg.i, a = tg.a, gg = tg.g, rog = tg.rog;
     const float q = a * (a * ig * u[k] * rog - hh * r);
     fa[k] = a;
@@ -756,8 +763,8 @@ __device__ __forceinline__ void final_group(const BwdThread &th, const ChanC &c,
         b16.dza[o] = __float2bfloat16_rn(dza);
         b16.dzx[o] = __float2bfloat16_rn(dzx);
       } else {
-        ws_za[o] = dza;
-        ws_zx[o] = dzx;
+        ws_ga[o] = dza;
+        ws_gx[o] = dzx;
       }
     }
     sink(k, dza, dzx);
@@ -768,8 +775,8 @@ template <typename T, bool kSW, int kMaxT>
 __global__ void __launch_bounds__(kMaxT, kMaxT == 256 ? 3 : 1)
 bwd_final_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
                  const float *__restrict__ ws_C, const float *__restrict__ ws_gP,
-                 const float *__restrict__ ws_gH, float *__restrict__ ws_za,
-                 float *__restrict__ ws_zx, float *__restrict__ ws_u,
+                 const float *__restrict__ ws_gH, float *__restrict__ ws_ga,
+                 float *__restrict__ ws_gx, float *__restrict__ ws_u,
                  float *__restrict__ ws_du) {
   extern __shared__ float4 smem_f[];
   const int bw = p.D / p.H, D = p.D, h = blockIdx.y, b = blockIdx.z;
@@ -807,7 +814,7 @@ bwd_final_kernel(BwdArgs p, BwdPlan pl, const float *__restrict__ ws_hin,
     if (live) {
       const size_t go = ((size_t)b * ngt + tb / kTB) * D + th.d;
       final_group<T, false, false>(th, c, xb, cs_in_b, dyb, orow, D, tb, go, h_in, ws_gP, ws_gH,
-                                   ws_za, ws_zx, ws_u, gc, acc_q, acc_ba, acc_bx, dub, nullptr,
+                                   ws_ga, ws_gx, ws_u, gc, acc_q, acc_ba, acc_bx, dub, nullptr,
                                    nullptr, nullptr, nullptr, nullptr, 0, Bf16Streams{},
                                    [&](int k, float dza, float dzx) {
                               dza_row[k] = dza;
@@ -859,8 +866,8 @@ template <int kBW>
 __global__ void __launch_bounds__(TcGeo<kBW>::kThreads, kBW == 128 ? 1 : 2)
 bwd_final_tc_kernel(BwdArgs p, BwdPlan pl, Bf16Streams b16, const float *__restrict__ ws_hin,
                     const float *__restrict__ ws_C, const float *__restrict__ ws_gP,
-                    const float *__restrict__ ws_gH, float *__restrict__ ws_za,
-                    float *__restrict__ ws_zx, float *__restrict__ ws_u,
+                    const float *__restrict__ ws_gH, float *__restrict__ ws_ga,
+                    float *__restrict__ ws_gx, float *__restrict__ ws_u,
                     float *__restrict__ ws_du) {
   using T = __nv_bfloat16;
   using G = TcGeo<kBW>;
@@ -868,13 +875,13 @@ bwd_final_tc_kernel(BwdArgs p, BwdPlan pl, Bf16Streams b16, const float *__restr
   float *du_s = reinterpret_cast<float *>(smem_ft);                  // [S][kBW][kRow]
   T *a_s = reinterpret_cast<T *>(du_s + G::S * kBW * kRow);          // [2][M][kStride]
   T *w_s = a_s + 2 * G::M * G::kStride;                              // [2][kBW][kStride]
-  // z_a, z_x and dy rows of a group, double-buffered: [2][S][kTB][kBW]; then its
+  // r, i and dy rows of a group, double-buffered: [2][S][kTB][kBW]; then its
   // x rows tb-3 .. tb+7 [2][S][kTB + 3][kBW] and its start pair (prod a, local
   // state) [2][S][2][kBW]
   constexpr int XR = kTB + 3;
-  float *za_st = reinterpret_cast<float *>(w_s + 2 * kBW * G::kStride);
-  float *zx_st = za_st + 2 * G::S * kTB * kBW;
-  T *dy_st = reinterpret_cast<T *>(zx_st + 2 * G::S * kTB * kBW);
+  float *ra_st = reinterpret_cast<float *>(w_s + 2 * kBW * G::kStride);
+  float *ix_st = ra_st + 2 * G::S * kTB * kBW;
+  T *dy_st = reinterpret_cast<T *>(ix_st + 2 * G::S * kTB * kBW);
   T *xs_st = dy_st + 2 * G::S * kTB * kBW;
   float *gs_st = reinterpret_cast<float *>(xs_st + 2 * G::S * XR * kBW);
   const int D = p.D, h = blockIdx.y, b = blockIdx.z;
@@ -946,8 +953,8 @@ bwd_final_tc_kernel(BwdArgs p, BwdPlan pl, Bf16Streams b16, const float *__restr
       const size_t grow = ((size_t)b * p.T + (in ? tb + k : tb)) * D + (size_t)h * kBW;
       const int slot = ((buf * G::S + sl) * kTB + k) * kBW;
       if (q < 2) {
-        cp_async16(za_st + slot + w * 4, ws_za + grow + w * 4, in);
-        cp_async16(zx_st + slot + w * 4, ws_zx + grow + w * 4, in);
+        cp_async16(ra_st + slot + w * 4, ws_ga + grow + w * 4, in);
+        cp_async16(ix_st + slot + w * 4, ws_gx + grow + w * 4, in);
         continue;
       }
       cp_async16(dy_st + slot + w * 8, dyb + grow + w * 8, in);
@@ -995,8 +1002,8 @@ bwd_final_tc_kernel(BwdArgs p, BwdPlan pl, Bf16Streams b16, const float *__restr
       const size_t go = ((size_t)b * ngt + tb / kTB) * D + th.d;
       const int srow = ((buf * G::S + th.sl) * kTB) * kBW + th.j;
       final_group<T, true, kBW % kDwTile == 0>(th, c, xb, cs_in_b, dyb, orow, D, tb, go, h_in,
-                                               ws_gP, ws_gH, ws_za, ws_zx, ws_u, gc, acc_q,
-                                               acc_ba, acc_bx, dub, za_st + srow, zx_st + srow,
+                                               ws_gP, ws_gH, ws_ga, ws_gx, ws_u, gc, acc_q,
+                                               acc_ba, acc_bx, dub, ra_st + srow, ix_st + srow,
                                                dy_st + srow,
                                                xs_st + (buf * G::S + th.sl) * XR * kBW + th.j,
                                                gs_st + (buf * G::S + th.sl) * 2 * kBW + th.j,
@@ -1325,7 +1332,7 @@ bwd_conv_kernel(BwdArgs p, const float *__restrict__ du) {
 }
 
 struct BwdLayout {
-  size_t off_A, off_H, off_R, off_hin, off_C, off_gP, off_gH, off_za, off_zx, off_u, off_du;
+  size_t off_A, off_H, off_R, off_hin, off_C, off_gP, off_gH, off_ga, off_gx, off_u, off_du;
   size_t off_dzx16;   // bf16 d z_x for the tensor-core d W (bf16 u and d z_a share u's region)
   size_t total;
 };
@@ -1343,9 +1350,9 @@ BwdLayout bwd_layout(int B, int T, int D, int H) {
   L.off_C = L.off_hin + seg;
   L.off_gP = L.off_C + seg;
   L.off_gH = L.off_gP + grp;
-  L.off_za = L.off_gH + grp;
-  L.off_zx = L.off_za + tok;
-  L.off_u = L.off_zx + tok;
+  L.off_ga = L.off_gH + grp;
+  L.off_gx = L.off_ga + tok;
+  L.off_u = L.off_gx + tok;
   L.off_du = L.off_u + tok;
   L.off_dzx16 = L.off_du + tok;
   L.total = L.off_dzx16 + align_up((size_t)B * T * D * 2, 256);
@@ -1362,7 +1369,9 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
   auto at = [w](size_t off) { return reinterpret_cast<float *>(w + off); };
   float *A = at(Ly.off_A), *Hh = at(Ly.off_H), *R = at(Ly.off_R);
   float *hin = at(Ly.off_hin), *C = at(Ly.off_C), *gP = at(Ly.off_gP), *gH = at(Ly.off_gH);
-  float *za = at(Ly.off_za), *zx = at(Ly.off_zx), *U = at(Ly.off_u), *du = at(Ly.off_du);
+  // ga, gx: the gates r and i per token from K1; K3 writes d z_a and d z_x over them
+  // for the CUDA-core d W
+  float *ga = at(Ly.off_ga), *gx = at(Ly.off_gx), *U = at(Ly.off_u), *du = at(Ly.off_du);
   // bf16 u, d z_a (in u's fp32 region, two halves) and d z_x for the tensor-core d W
   const size_t ntok = (size_t)p.B * p.T * p.D;
   Bf16Streams b16{reinterpret_cast<__nv_bfloat16 *>(U), reinterpret_cast<__nv_bfloat16 *>(U) + ntok,
@@ -1385,7 +1394,7 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
     // K1: fp32 z rows [S][2][bw][kRow], bf16 u rows [M][kStride] and the staged
     //     x and dy rows (bf16) [3][S][2 kTB + 3][bw];
     // K3: fp32 d u rows [S][bw][kRow], bf16 d z_a, d z_x rows [2][M][kStride],
-    //     bf16 W_a, W_x rows [2][bw][kStride], the staged z_a, z_x (fp32) and dy
+    //     bf16 W_a, W_x rows [2][bw][kStride], the staged r, i (fp32) and dy
     //     (bf16) rows [2][S][kTB][bw], x rows (bf16) [2][S][kTB + 3][bw] and start
     //     pairs (fp32) [2][S][2][bw]
     const size_t smem1 = (size_t)G::S * 2 * kTcBW * kRow * 4 + (size_t)G::M * G::kStride * 2 +
@@ -1403,13 +1412,13 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3)) !=
         cudaSuccess)
       return e;
-    bwd_gates_tc_kernel<kTcBW><<<grid, G::kThreads, smem1, st>>>(p, pl, A, Hh, R, gP, gH, za, zx);
+    bwd_gates_tc_kernel<kTcBW><<<grid, G::kThreads, smem1, st>>>(p, pl, A, Hh, R, gP, gH, ga, gx);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     bwd_carry_kernel<<<ceil_div(bd, kCarryCh), kCarryCh * kCarryParts, 0, st>>>(
         p.B, p.D, pl.nseg, A, Hh, R, p.h0, p.dh_T, hin, C, p.dh0);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    bwd_final_tc_kernel<kTcBW><<<grid, G::kThreads, smem3, st>>>(p, pl, b16, hin, C, gP, gH, za,
-                                                                  zx, U, du);
+    bwd_final_tc_kernel<kTcBW><<<grid, G::kThreads, smem3, st>>>(p, pl, b16, hin, C, gP, gH, ga,
+                                                                  gx, U, du);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   } else {
     const size_t wsm = kSW ? 2 * (size_t)bw * (bw + 1) * sizeof(float) : 0;
@@ -1424,13 +1433,13 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3)) !=
         cudaSuccess)
       return e;
-    bwd_gates_kernel<T, kSW, kMaxT><<<grid, threads, smem1, st>>>(p, pl, A, Hh, R, gP, gH, za,
-                                                                   zx);
+    bwd_gates_kernel<T, kSW, kMaxT><<<grid, threads, smem1, st>>>(p, pl, A, Hh, R, gP, gH, ga,
+                                                                   gx);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     bwd_carry_kernel<<<ceil_div(bd, kCarryCh), kCarryCh * kCarryParts, 0, st>>>(
         p.B, p.D, pl.nseg, A, Hh, R, p.h0, p.dh_T, hin, C, p.dh0);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    bwd_final_kernel<T, kSW, kMaxT><<<grid, threads, smem3, st>>>(p, pl, hin, C, gP, gH, za, zx,
+    bwd_final_kernel<T, kSW, kMaxT><<<grid, threads, smem3, st>>>(p, pl, hin, C, gP, gH, ga, gx,
                                                                    U, du);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -1447,7 +1456,7 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
         b16.u, b16.dza, b16.dzx, p.dW_a, p.dW_x, N, p.D, p.H, chunk);
   else
     bwd_dw_kernel<<<dim3(tile_blocks, ceil_div(N, chunk)), kDwThreads, 0, st>>>(
-        U, za, zx, p.dW_a, p.dW_x, N, p.D, p.H, chunk);
+        U, ga, gx, p.dW_a, p.dW_x, N, p.D, p.H, chunk);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   bwd_conv_kernel<T><<<dim3(ceil_div(p.D, 2 * kConvThreads), p.B,
                             ceil_div(p.T + 3, kConvChunk)),
