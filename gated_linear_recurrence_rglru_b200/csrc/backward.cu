@@ -1263,21 +1263,50 @@ template <>
 __device__ __forceinline__ void st_pair<__nv_bfloat16>(__nv_bfloat16 *p, float2 v) {
   *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(v.x, v.y);
 }
+// A pair as it lies in memory (two bf16 in one word, or two floats) as floats.
+template <typename T>
+__device__ __forceinline__ float2 pair_to_f2(
+    typename std::conditional<sizeof(T) == 2, uint32_t, float2>::type v);
+template <>
+__device__ __forceinline__ float2 pair_to_f2<float>(float2 v) {
+  return v;
+}
+template <>
+__device__ __forceinline__ float2 pair_to_f2<__nv_bfloat16>(uint32_t v) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&v));
+}
 
 // d x (and the conv history's gradient) from d u, and d w per channel, for one
 // chunk of kConvChunk extended positions m (x_{m-3}) of one batch row; thread
-// per two adjacent channels (paired 8-byte d u and 4- or 8-byte x loads), the
-// last three d u values in registers:
+// per two adjacent channels, the last three d u values in registers:
 //   d x_{m-3} = sum_k w[k] d u_{m-k},  d w[k] += x_{m-3} d u_{m-k}  (0 <= m-k < T).
-constexpr int kConvChunk = 64, kConvThreads = 256;
+// Each thread streams its own d u pairs (8 B) and x pairs (4 or 8 B) through a
+// private ring of kConvStages batches of kConvBatch positions in shared memory
+// (cp.async, kConvStages - 1 batches ahead): many loads in flight per thread at
+// no register cost, and no block barrier, as no thread reads another's slots.
+constexpr int kConvChunk = 64, kConvThreads = 256, kConvBatch = 8, kConvStages = 2;
+
+// cp.async of n = 4 or 8 bytes (.ca), zero-filled when !full (src must still be
+// a valid address); completed by cp.async.wait_group on the issuing thread.
+template <int n>
+__device__ __forceinline__ void cp_async_small(void *dst, const void *src, bool full) {
+  static_assert(n == 4 || n == 8, "cp.async .ca size");
+  asm volatile("cp.async.ca.shared.global [%0], [%1], %2, %3;" ::"r"(shared_addr(dst)),
+               "l"(src), "n"(n), "r"(full ? n : 0)
+               : "memory");
+}
 
 template <typename T>
 __global__ void __launch_bounds__(kConvThreads)
 bwd_conv_kernel(BwdArgs p, const float *__restrict__ du) {
+  using X2 = typename std::conditional<sizeof(T) == 2, uint32_t, float2>::type;  // an x pair
+  extern __shared__ float2 conv_sm[];
+  float2 *s_du = conv_sm;                                         // [stage][batch][thread]
+  X2 *s_x = reinterpret_cast<X2 *>(s_du + kConvStages * kConvBatch * kConvThreads);
   const int D = p.D;
   const int d = 2 * (blockIdx.x * kConvThreads + threadIdx.x);   // D is a multiple of 8
   const int b = blockIdx.y;
-  if (d >= D) return;
+  if (d >= D) return;                 // no barriers below: each thread works on its own
   const int m_begin = blockIdx.z * kConvChunk, m_end = min(p.T + 3, m_begin + kConvChunk);
   const T *cw = static_cast<const T *>(p.conv_w);
   float2 w[4];
@@ -1293,37 +1322,71 @@ bwd_conv_kernel(BwdArgs p, const float *__restrict__ du) {
     return (t >= 0 && t < p.T) ? __ldg(reinterpret_cast<const float2 *>(dub + (size_t)t * D))
                                : make_float2(0.f, 0.f);
   };
-  auto x_at = [&](int t) {   // x_t, t >= -3 (t < 0: the conv history, or zeros)
-    if (t >= 0) return ldg_pair<T>(xb + (size_t)t * D);
-    if (csb != nullptr) return ldg_pair<T>(csb + (size_t)(3 + t) * D);
-    return make_float2(0.f, 0.f);
+  // batch j of the chunk into ring stage j % kConvStages: d u_m and x_{m-3} for its
+  // positions m (zeros past T, the conv history or zeros before t = 0); one commit
+  // per call, also when the batch lies past the chunk
+  auto issue = [&](int j) {
+    const int stg = j % kConvStages;
+#pragma unroll
+    for (int i = 0; i < kConvBatch; ++i) {
+      const int m = m_begin + j * kConvBatch + i;
+      if (m >= m_end) break;
+      const int slot = (stg * kConvBatch + i) * kConvThreads + threadIdx.x;
+      const bool gin = m < p.T;
+      cp_async_small<8>(s_du + slot, gin ? dub + (size_t)m * D : dub, gin);
+      const int t = m - 3;
+      const T *xs = xb;
+      bool xin = false;
+      if (t >= 0) {
+        xs = xb + (size_t)t * D;
+        xin = true;
+      } else if (csb != nullptr) {
+        xs = csb + (size_t)(3 + t) * D;
+        xin = true;
+      }
+      cp_async_small<sizeof(X2)>(s_x + slot, xs, xin);
+    }
+    cp_async_commit();
   };
   float2 g1 = du_at(m_begin - 1), g2 = du_at(m_begin - 2), g3 = du_at(m_begin - 3);
   float2 dw[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) dw[k] = make_float2(0.f, 0.f);
-#pragma unroll 8
-  for (int m = m_begin; m < m_end; ++m) {
-    const float2 g0 = du_at(m);
-    const float2 xv = x_at(m - 3);
-    float2 acc;
-    acc.x = fmaf(w[0].x, g0.x, fmaf(w[1].x, g1.x, fmaf(w[2].x, g2.x, w[3].x * g3.x)));
-    acc.y = fmaf(w[0].y, g0.y, fmaf(w[1].y, g1.y, fmaf(w[2].y, g2.y, w[3].y * g3.y)));
-    dw[0].x = fmaf(xv.x, g0.x, dw[0].x);
-    dw[0].y = fmaf(xv.y, g0.y, dw[0].y);
-    dw[1].x = fmaf(xv.x, g1.x, dw[1].x);
-    dw[1].y = fmaf(xv.y, g1.y, dw[1].y);
-    dw[2].x = fmaf(xv.x, g2.x, dw[2].x);
-    dw[2].y = fmaf(xv.y, g2.y, dw[2].y);
-    dw[3].x = fmaf(xv.x, g3.x, dw[3].x);
-    dw[3].y = fmaf(xv.y, g3.y, dw[3].y);
-    if (m >= 3) st_pair<T>(dxb + (size_t)(m - 3) * D, acc);
-    else if (p.dconv_state_in)
-      *reinterpret_cast<float2 *>(p.dconv_state_in + ((size_t)b * 3 + m) * D + d) = acc;
-    g3 = g2;
-    g2 = g1;
-    g1 = g0;
+  const int nb = ceil_div(m_end - m_begin, kConvBatch);
+#pragma unroll
+  for (int j = 0; j < kConvStages - 1; ++j) issue(j);
+  for (int j = 0; j < nb; ++j) {
+    // stage (j + kConvStages - 1) % kConvStages was read by this thread in batch j - 1
+    issue(j + kConvStages - 1);
+    asm volatile("cp.async.wait_group %0;" ::"n"(kConvStages - 1) : "memory");  // batch j landed
+    const int stg = j % kConvStages;
+#pragma unroll
+    for (int i = 0; i < kConvBatch; ++i) {
+      const int m = m_begin + j * kConvBatch + i;
+      if (m >= m_end) break;
+      const int slot = (stg * kConvBatch + i) * kConvThreads + threadIdx.x;
+      const float2 g0 = s_du[slot];
+      const float2 xv = pair_to_f2<T>(s_x[slot]);
+      float2 acc;
+      acc.x = fmaf(w[0].x, g0.x, fmaf(w[1].x, g1.x, fmaf(w[2].x, g2.x, w[3].x * g3.x)));
+      acc.y = fmaf(w[0].y, g0.y, fmaf(w[1].y, g1.y, fmaf(w[2].y, g2.y, w[3].y * g3.y)));
+      dw[0].x = fmaf(xv.x, g0.x, dw[0].x);
+      dw[0].y = fmaf(xv.y, g0.y, dw[0].y);
+      dw[1].x = fmaf(xv.x, g1.x, dw[1].x);
+      dw[1].y = fmaf(xv.y, g1.y, dw[1].y);
+      dw[2].x = fmaf(xv.x, g2.x, dw[2].x);
+      dw[2].y = fmaf(xv.y, g2.y, dw[2].y);
+      dw[3].x = fmaf(xv.x, g3.x, dw[3].x);
+      dw[3].y = fmaf(xv.y, g3.y, dw[3].y);
+      if (m >= 3) st_pair<T>(dxb + (size_t)(m - 3) * D, acc);
+      else if (p.dconv_state_in)
+        *reinterpret_cast<float2 *>(p.dconv_state_in + ((size_t)b * 3 + m) * D + d) = acc;
+      g3 = g2;
+      g2 = g1;
+      g1 = g0;
+    }
   }
+  cp_async_wait_all();   // the empty groups past the chunk
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     atomicAdd(p.dconv_w + (size_t)k * D + d, dw[k].x);
@@ -1458,9 +1521,13 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
     bwd_dw_kernel<<<dim3(tile_blocks, ceil_div(N, chunk)), kDwThreads, 0, st>>>(
         U, ga, gx, p.dW_a, p.dW_x, N, p.D, p.H, chunk);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const size_t smem_conv = (size_t)kConvStages * kConvBatch * kConvThreads * (8 + 2 * sizeof(T));
+  if ((e = cudaFuncSetAttribute(bwd_conv_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem_conv)) != cudaSuccess)
+    return e;
   bwd_conv_kernel<T><<<dim3(ceil_div(p.D, 2 * kConvThreads), p.B,
                             ceil_div(p.T + 3, kConvChunk)),
-                       kConvThreads, 0, st>>>(p, du);
+                       kConvThreads, smem_conv, st>>>(p, du);
   return cudaGetLastError();
 }
 
