@@ -1153,18 +1153,21 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&a)[4]) {
 // (padded by 8 elements); with A[i][n] = U[n][i] and B[n][j] = dZ[n][j], both
 // fragments come from ldmatrix .trans of those rows (a thread receives stored
 // elements (2q, g) and (2q + 1, g) of each 8 x 8 block: the k pairs of column
-// g). The next kDwTcRows tokens are in flight to registers during the MMAs.
+// g). The rows arrive by 16-byte cp.async through a ring of kDwTcStages steps
+// (kDwTcStages - 1 steps in flight during the MMAs), with no staging registers.
 constexpr int kDwTcThreads = 128, kDwTcStride = kDwTile + 8;
 // tokens per step of the tensor-core d W: 64, so that a block's loads of the next step
 // cover twice the bytes of the CUDA-core kernel's 32-token steps
-constexpr int kDwTcRows = 64;
+constexpr int kDwTcRows = 64, kDwTcStages = 3;
 
 __global__ void __launch_bounds__(kDwTcThreads)
 bwd_dw_tc_kernel(const __nv_bfloat16 *__restrict__ U, const __nv_bfloat16 *__restrict__ dZa,
                  const __nv_bfloat16 *__restrict__ dZx, float *__restrict__ dWa,
                  float *__restrict__ dWx, int N, int D, int H, int chunk) {
-  __shared__ __align__(16) __nv_bfloat16 us[kDwTcRows][kDwTcStride];
-  __shared__ __align__(16) __nv_bfloat16 zs[kDwTcRows][kDwTcStride];
+  extern __shared__ uint4 dw_sm[];
+  // [kDwTcStages][kDwTcRows][kDwTcStride] bf16 each
+  __nv_bfloat16 *us = reinterpret_cast<__nv_bfloat16 *>(dw_sm);
+  __nv_bfloat16 *zs = us + kDwTcStages * kDwTcRows * kDwTcStride;
   const int bw = D / H;
   const int tiles = bw / kDwTile;
   int tile = blockIdx.x;
@@ -1176,27 +1179,39 @@ bwd_dw_tc_kernel(const __nv_bfloat16 *__restrict__ U, const __nv_bfloat16 *__res
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int wi = (warp & 1) * 32, wj = (warp >> 1) * 32;
   const int i0 = ti * kDwTile, j0 = tj * kDwTile;
-  // loader: rows lr + 8 q, columns lc .. lc + 3 (8-byte bf16 loads)
-  const int lr = tid >> 4, lc = (tid & 15) * 4;
-  const __nv_bfloat16 *Uc = U + (size_t)h * bw + i0 + lc;
-  const __nv_bfloat16 *Zc = Z + (size_t)h * bw + j0 + lc;
+  const __nv_bfloat16 *Ub = U + (size_t)h * bw + i0;
+  const __nv_bfloat16 *Zb = Z + (size_t)h * bw + j0;
   const int n_begin = blockIdx.y * chunk, n_end = min(N, n_begin + chunk);
-  uint2 pu[kDwTcRows / 8], pz[kDwTcRows / 8];
-  auto fetch = [&](int n0) {
+  // step s (tokens n_begin + s * kDwTcRows ...) into ring stage s % kDwTcStages:
+  // 8 chunks of 16 bytes per row and operand, rows past n_end zero-filled; one
+  // commit per call, also for steps past the chunk
+  constexpr int kChunks = kDwTcRows * 8 / kDwTcThreads;
+  static_assert(kDwTcRows * 8 % kDwTcThreads == 0, "chunks per thread");
+  auto issue = [&](int step) {
+    const int n0 = n_begin + step * kDwTcRows, stg = step % kDwTcStages;
+    if (n0 < n_end) {
 #pragma unroll
-    for (int q = 0; q < kDwTcRows / 8; ++q) {
-      const int n = n0 + lr + 8 * q;
-      const bool ok = n < n_end;
-      pu[q] = ok ? *reinterpret_cast<const uint2 *>(Uc + (size_t)n * D) : make_uint2(0, 0);
-      pz[q] = ok ? *reinterpret_cast<const uint2 *>(Zc + (size_t)n * D) : make_uint2(0, 0);
+      for (int q = 0; q < kChunks; ++q) {
+        const int c = tid + q * kDwTcThreads, r = c >> 3, col = (c & 7) * 8;
+        const int n = n0 + r;
+        const bool ok = n < n_end;
+        const size_t row = (size_t)(ok ? n : n_begin) * D + col;
+        const int dst = (stg * kDwTcRows + r) * kDwTcStride + col;
+        cp_async16(us + dst, Ub + row, ok);
+        cp_async16(zs + dst, Zb + row, ok);
+      }
     }
+    cp_async_commit();
   };
   // ldmatrix lane rows: A blocks (n-block q / 2, i-block q % 2), B blocks (n-block q % 2,
   // j-block q / 2), q = lane / 8
   const int lq = lane >> 3, lrow = lane & 7;
-  const uint32_t a_lane = shared_addr(&us[lrow + (lq >> 1) * 8][wi + (lq & 1) * 8]);
-  const uint32_t b_lane = shared_addr(&zs[lrow + (lq & 1) * 8][wj + (lq >> 1) * 8]);
+  const uint32_t a_lane0 =
+      shared_addr(us + (lrow + (lq >> 1) * 8) * kDwTcStride + wi + (lq & 1) * 8);
+  const uint32_t b_lane0 =
+      shared_addr(zs + (lrow + (lq & 1) * 8) * kDwTcStride + wj + (lq >> 1) * 8);
   constexpr uint32_t kRowBytes = kDwTcStride * 2;
+  constexpr uint32_t kStageBytes = kDwTcRows * kRowBytes;
   float acc[2][4][4];
 #pragma unroll
   for (int mi = 0; mi < 2; ++mi)
@@ -1204,15 +1219,17 @@ bwd_dw_tc_kernel(const __nv_bfloat16 *__restrict__ U, const __nv_bfloat16 *__res
     for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[mi][nt][e] = 0.f;
-  fetch(n_begin);
-  for (int n0 = n_begin; n0 < n_end; n0 += kDwTcRows) {
+  const int nsteps = n_end > n_begin ? ceil_div(n_end - n_begin, kDwTcRows) : 0;
 #pragma unroll
-    for (int q = 0; q < kDwTcRows / 8; ++q) {
-      *reinterpret_cast<uint2 *>(&us[lr + 8 * q][lc]) = pu[q];
-      *reinterpret_cast<uint2 *>(&zs[lr + 8 * q][lc]) = pz[q];
-    }
+  for (int st = 0; st < kDwTcStages - 1; ++st) issue(st);
+  for (int it = 0; it < nsteps; ++it) {
+    // stage (it + kDwTcStages - 1) % kDwTcStages was last read in step it - 1, before
+    // that step's closing barrier
+    issue(it + kDwTcStages - 1);
+    asm volatile("cp.async.wait_group %0;" ::"n"(kDwTcStages - 1) : "memory");  // step it
     __syncthreads();
-    if (n0 + kDwTcRows < n_end) fetch(n0 + kDwTcRows);
+    const uint32_t a_lane = a_lane0 + (it % kDwTcStages) * kStageBytes;
+    const uint32_t b_lane = b_lane0 + (it % kDwTcStages) * kStageBytes;
 #pragma unroll
     for (int ks = 0; ks < kDwTcRows / 16; ++ks) {
       uint32_t a[2][4], b[2][4];
@@ -1228,6 +1245,7 @@ bwd_dw_tc_kernel(const __nv_bfloat16 *__restrict__ U, const __nv_bfloat16 *__res
     }
     __syncthreads();
   }
+  cp_async_wait_all();   // the empty groups past the chunk
   const int fg = lane >> 2, fq = lane & 3;
 #pragma unroll
   for (int mi = 0; mi < 2; ++mi)
@@ -1510,14 +1528,20 @@ cudaError_t launch_bwd_t(const BwdArgs &p, void *ws, cudaStream_t st) {
   const int N = p.B * p.T;
   const int tiles = ceil_div(bw, kDwTile);
   const int tile_blocks = 2 * tiles * tiles * p.H;
-  const int nchunk = ceil_div(8 * 148, tile_blocks);
   const bool dw_tc = kTcBW > 0 && kTcBW % kDwTile == 0;
+  // token chunks for about 8 blocks per SM, 4 for the tensor-core kernel (its ring
+  // of shared memory holds 4 per SM): one wave
+  const int nchunk = ceil_div((dw_tc ? 4 : 8) * 148, tile_blocks);
   const int dw_rows = dw_tc ? kDwTcRows : kDwRows;   // tokens per step
   const int chunk = ceil_div(ceil_div(N, nchunk), dw_rows) * dw_rows;
-  if (dw_tc)
-    bwd_dw_tc_kernel<<<dim3(tile_blocks, ceil_div(N, chunk)), kDwTcThreads, 0, st>>>(
+  if (dw_tc) {
+    const size_t smem_dw = (size_t)kDwTcStages * 2 * kDwTcRows * kDwTcStride * 2;
+    if ((e = cudaFuncSetAttribute(bwd_dw_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem_dw)) != cudaSuccess)
+      return e;
+    bwd_dw_tc_kernel<<<dim3(tile_blocks, ceil_div(N, chunk)), kDwTcThreads, smem_dw, st>>>(
         b16.u, b16.dza, b16.dzx, p.dW_a, p.dW_x, N, p.D, p.H, chunk);
-  else
+  } else
     bwd_dw_kernel<<<dim3(tile_blocks, ceil_div(N, chunk)), kDwThreads, 0, st>>>(
         U, ga, gx, p.dW_a, p.dW_x, N, p.D, p.H, chunk);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
