@@ -43,6 +43,18 @@
 //                 gradient) and d w[k] = sum_t x_{t-3+k} d u_t.
 // The path of d z_a through g carries r / g, which tends to 0 with r
 // (1 - a^2 ~ 2 c sp r); it is formed as that ratio (0 where g = 0).
+//
+// Loads reach the arithmetic through shared memory, copied by cp.async ahead
+// of use, so that no warp waits on a global load in its inner loop:
+//   K1 (tensor-core version): the x and dy rows of each segment's group, a
+//      ring of three slots filled two groups ahead;
+//   K3 (tensor-core version): r, i, dy, the x rows of the Conv1D recompute and
+//      the group-start pair, double-buffered one group ahead;
+//   K4 (tensor-core version): U and d Z rows, a three-stage ring of 64-token
+//      steps;
+//   K5: each thread's own d u and x pairs, a private two-batch ring (no block
+//      barrier: no thread reads another's slots).
+// The CUDA-core versions of K1 and K3 issue L1 prefetches of the next group.
 #include <type_traits>
 
 #include "common.cuh"
