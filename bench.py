@@ -459,8 +459,9 @@ def run_backward(rg, wl, dev, a, pk):
                                  "contractions (2 bw MACs per channel-token each) on the "
                                  "tensor cores (bf16 operands, fp32 accumulate) for bf16 I/O "
                                  "with 64/128-wide heads, the rest fp32 on CUDA cores; "
-                                 "fp32 intermediates in a workspace (z_a, z_x, u, d u: 16 B "
-                                 "per channel-token written and re-read) are not algorithmic"}}
+                                 "the intermediates in a workspace (the gates r, i and d u in "
+                                 "fp32, u, d z_a, d z_x in bf16: 18 B per channel-token "
+                                 "written and re-read) are not algorithmic"}}
 
 
 def run_block(rg, wl, dev, a, pk):
