@@ -40,7 +40,7 @@ FLOOR = 1.0           # floor factor on the channel RMS (see above)
 # its d u = own term + d z W^T can cancel: its designed arithmetic needs a factor of
 # 0.79 on the B=2 T=2048 D=1024 H=16 case (tests/test_backward_bf16_operands.py).
 BWD_FLOOR = FLOOR
-SURVEY_FLOOR = 1e-3   # a floor too tight for any bf16-operand contraction; reported only
+TIGHT_FLOOR = 1e-3   # a floor too tight for any bf16-operand contraction; reported only
 
 
 def channel_rms(o: np.ndarray, time_axis: int = 1) -> np.ndarray:
@@ -89,6 +89,6 @@ def normwise_err(g, o) -> float:
 def error_report(g, o, time_axis: int = 1) -> dict:
     """The same comparison under the three floors discussed above, for reporting."""
     return {"floor_1_channel_rms": max_rel_err(g, o, time_axis=time_axis),
-            "floor_1e-3_channel_rms": max_rel_err(g, o, time_axis=time_axis, floor=SURVEY_FLOOR),
+            "floor_1e-3_channel_rms": max_rel_err(g, o, time_axis=time_axis, floor=TIGHT_FLOOR),
             "floor_1_row_rms": max_rel_err(g, o, scale=row_rms(o, time_axis), floor=1.0),
             "normwise": normwise_err(g, o)}
