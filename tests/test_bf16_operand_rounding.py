@@ -147,7 +147,7 @@ def measured():
     return out
 
 
-def test_survey_floor_is_out_of_reach_of_bf16_operands(measured):
+def test_tight_floor_is_out_of_reach_of_bf16_operands(measured):
     """Under 1e-3 * RMS the designed arithmetic itself is far above the bar."""
     worst = max(m["at_tight_floor"] for m in measured)
     assert worst > 50 * BAR, worst
